@@ -1,0 +1,182 @@
+"""Pins of the oracle's stage 0, GQA routing, stage 2 and the end-to-end forward.
+
+Cited page: "DashAttention: Differentiable and Adaptive Sparse Hierarchical
+Attention" (gist.science explainer), technical summary, sections "Stage 0:
+local chunk summary", "Stage 1: entmax chunk routing" (GQA handling) and
+"Stage 2: prior-induced sparse softmax".  The independent references here are
+hand-computed values, library routines (numpy means, torch's
+scaled_dot_product_attention in fp64, scipy's optimiser) and invariances.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+from scipy.optimize import minimize
+
+from oracle.dash_oracle import (
+    block_summaries,
+    decode_pair,
+    diagonal_bias,
+    forward,
+    forward_row,
+    prior_softmax_attend,
+    route_row,
+)
+
+
+# --------------------------------------------------------------------------
+# Stage 0
+
+
+def test_block_mean_hand_example():
+    # two blocks of 2 tokens, d = 2, W_s = I: means by hand
+    k = np.array([[1.0, 2.0], [3.0, 6.0], [-1.0, 0.0], [5.0, 4.0], [7.0, 7.0]])
+    s = block_summaries(k, np.eye(2), block=2, n_tokens=5)
+    np.testing.assert_array_equal(s, [[2.0, 4.0], [2.0, 2.0], [7.0, 7.0]])
+
+
+def test_block_mean_matches_numpy_and_orientation():
+    rng = np.random.default_rng(0)
+    L, d, B = 640, 16, 64
+    k = rng.normal(size=(L, d))
+    s = block_summaries(k, np.eye(d), B, L)
+    np.testing.assert_allclose(s, k.reshape(L // B, B, d).mean(axis=1), atol=1e-14)
+    # row vector times matrix: a permutation W_s (W[i, pi(i)] = 1) moves
+    # coordinate i of the mean to position pi(i); the transpose would not.
+    perm = rng.permutation(d)
+    w = np.zeros((d, d))
+    w[np.arange(d), perm] = 1.0
+    s2 = block_summaries(k, w, B, L)
+    np.testing.assert_allclose(s2[:, perm], s, atol=1e-14)
+    # a partial trailing block is averaged over its valid tokens only
+    s3 = block_summaries(k, np.eye(d), B, 600)
+    np.testing.assert_allclose(s3[-1], k[576:600].mean(axis=0), atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Stage 1: GQA average
+
+
+def test_gqa_average_hand_example():
+    # d = 4, gamma = 1/2.  Head 0 is one-hot on block 0, head 1 on block 2.
+    summaries = np.eye(4)[:3] * 10.0
+    q = np.array([[1.0, 0, 0, 0], [0, 0, 1.0, 0]])
+    r = route_row(q, summaries, alpha=1.5)
+    np.testing.assert_allclose(r["p"], [[1, 0, 0], [0, 0, 1]], atol=0)
+    np.testing.assert_allclose(r["pbar"], [0.5, 0.0, 0.5])
+    np.testing.assert_array_equal(r["idx"], [0, 2])
+    np.testing.assert_allclose(r["logp"], [math.log(0.5)] * 2)
+    # z = gamma q.s with gamma = 1/sqrt(d)
+    np.testing.assert_allclose(r["z"][0], [5.0, 0.0, 0.0])
+
+
+# --------------------------------------------------------------------------
+# Stage 2
+
+
+def test_prior_softmax_is_the_variational_maximiser():
+    """softmax(l + log g) maximises <p, l> - KL(p || g) (scipy cross-check)."""
+    rng = np.random.default_rng(1)
+    n, d = 6, 8
+    q = rng.normal(size=d)
+    keys = rng.normal(size=(n, d))
+    g = rng.dirichlet(np.ones(n))
+    logits = keys @ q / math.sqrt(d)
+    # with values = identity rows the output is the attention distribution
+    p = prior_softmax_attend(q, keys, np.eye(n), np.log(g))
+
+    def obj(u):
+        u = np.clip(u, 1e-300, None)
+        return float(u @ logits - np.sum(u * np.log(u / g)))
+
+    res = minimize(lambda u: -obj(u), np.full(n, 1.0 / n), method="SLSQP",
+                   bounds=[(1e-12, 1.0)] * n,
+                   constraints=[{"type": "eq", "fun": lambda u: u.sum() - 1.0}],
+                   options={"ftol": 1e-15, "maxiter": 1000})
+    np.testing.assert_allclose(p, res.x, atol=1e-5)
+    assert obj(p) >= -res.fun - 1e-12
+
+
+def test_bias_shift_and_masking():
+    rng = np.random.default_rng(2)
+    n, d = 40, 16
+    q, keys, vals = rng.normal(size=d), rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    bias = rng.normal(size=n)
+    o = prior_softmax_attend(q, keys, vals, bias)
+    np.testing.assert_allclose(prior_softmax_attend(q, keys, vals, bias + 3.5), o, atol=1e-14)
+    # a -inf prior (g = 0) removes the token exactly
+    bias_m = bias.copy()
+    bias_m[5:15] = -np.inf
+    keep = np.r_[0:5, 15:n]
+    np.testing.assert_allclose(prior_softmax_attend(q, keys, vals, bias_m),
+                               prior_softmax_attend(q, keys[keep], vals[keep], bias[keep]), atol=1e-14)
+
+
+def _sdpa(q, k, v, causal):
+    """torch fp64 scaled_dot_product_attention; q [S,H,d], k/v [S,Hkv,d]."""
+    S, H, d = q.shape
+    G = H // k.shape[1]
+    qt = torch.from_numpy(q).permute(1, 0, 2)
+    kt = torch.from_numpy(np.repeat(k, G, axis=1)).permute(1, 0, 2)
+    vt = torch.from_numpy(np.repeat(v, G, axis=1)).permute(1, 0, 2)
+    return F.scaled_dot_product_attention(qt, kt, vt, is_causal=causal).permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_zero_w_s_is_full_attention(causal):
+    """W_s = 0 makes every score 0, entmax uniform over the N candidates, every
+    prior log(1/N) equal to the diagonal prior: the forward is plain attention."""
+    rng = np.random.default_rng(3)
+    S, H, Hkv, d, B = 203, 4, 2, 16, 16  # ragged tail: 203 = 12 * 16 + 11
+    q, k, v = rng.normal(size=(S, H, d)), rng.normal(size=(S, Hkv, d)), rng.normal(size=(S, Hkv, d))
+    res = forward(q, k, v, np.zeros((d, d)), alpha=1.5, block=B, causal=causal)
+    np.testing.assert_allclose(res["out"], _sdpa(q, k, v, causal), atol=1e-12)
+    for (pos, g), r in res["routes"].items():
+        assert len(r["blocks"]) == len(r["cand"])
+        assert r["beta"] == diagonal_bias(len(r["cand"]))
+
+
+def test_first_block_rows_attend_within_the_block():
+    rng = np.random.default_rng(4)
+    S, d, B = 64, 8, 32
+    q, k, v = rng.normal(size=(S, 1, d)), rng.normal(size=(S, 1, d)), rng.normal(size=(S, 1, d))
+    w = rng.normal(size=(d, d))
+    res = forward(q, k, v, w, alpha=1.5, block=B, rows=range(B))
+    np.testing.assert_allclose(res["out"], _sdpa(q[:B], k[:B], v[:B], True), atol=1e-12)
+
+
+def test_unselected_values_do_not_matter():
+    """Perturbing V inside blocks with zero routing mass leaves the output unchanged."""
+    rng = np.random.default_rng(5)
+    S, d, B = 512, 16, 32
+    q, k, v = rng.normal(size=(S, 1, d)), rng.normal(size=(S, 1, d)), rng.normal(size=(S, 1, d))
+    e = np.eye(d)[3]
+    k[64:96, 0] += 6.0 * e  # block 2 planted
+    q[480:, 0] += 6.0 * e
+    w = np.eye(d)
+    pos = 500
+    summ = block_summaries(k[:, 0], w, B, S)
+    r = forward_row(q[pos], k[:, 0], v[:, 0], summ, pos, S, B, 1.5)
+    assert 2 in r["blocks"] and len(r["blocks"]) < len(r["cand"])
+    unsel = [c for c in r["cand"] if c not in set(r["blocks"].tolist())]
+    v2 = v.copy()
+    for c in unsel:
+        v2[c * B:(c + 1) * B] += rng.normal(size=(B, 1, d)) * 100.0
+    r2 = forward_row(q[pos], k[:, 0], v2[:, 0], summ, pos, S, B, 1.5)
+    np.testing.assert_array_equal(r2["out"], r["out"])
+
+
+def test_decode_pair_zero_w_s_is_attention_over_context():
+    rng = np.random.default_rng(6)
+    L, d, B, G = 300, 16, 32, 2
+    q = rng.normal(size=(G, d))
+    k, v = rng.normal(size=(L + 50, d)), rng.normal(size=(L + 50, d))
+    r = decode_pair(q, k, v, np.zeros((d, d)), seqlen=L, block=B, alpha=2.0)
+    logits = q @ k[:L].T / math.sqrt(d)
+    w = np.exp(logits - logits.max(axis=1, keepdims=True))
+    ref = (w / w.sum(axis=1, keepdims=True)) @ v[:L]
+    np.testing.assert_allclose(r["out"], ref, atol=1e-12)
+    assert len(r["cand"]) == (L - 1) // B
