@@ -52,11 +52,13 @@ class Config:
         return replace(self, **kw)
 
 
-# Plant strengths calibrated so that the block-weighted mean sparsity lands
-# near 75% (prefill, decode) and so that needle heads route to their planted
-# blocks (long prefill).
-_PREFILL_KEY_STRENGTH = 4.0
-_NEEDLE_KEY_STRENGTH = 4.0
+# Plant strengths (calibrated with oracle/calibrate.py on a row subsample).
+# prefill: 4 -> 67.2%, 6 -> 73.1%, 8 -> 74.2% block-weighted sparsity; the
+# ceiling is 75% (one topic in four), approached as N grows.
+# long prefill needle heads: 6 -> 3.7%, 24 -> 94.5%, 32 -> 96.7% (the
+# diffuse heads stay at 0%).
+_PREFILL_KEY_STRENGTH = 8.0
+_NEEDLE_KEY_STRENGTH = 24.0
 
 CONFIGS: dict[str, Config] = {
     # 1K-token single-head fp32 case that the oracle runs in full.

@@ -1,0 +1,208 @@
+/*
+ * dashattn.h -- C ABI of libdashattn, the B200 (sm_100a) forward of
+ * DashAttention sparse hierarchical attention.
+ *
+ * Source of the method: "DashAttention: Differentiable and Adaptive Sparse
+ * Hierarchical Attention" (gist.science explainer of arXiv 2605.18753),
+ * technical summary, sections "Stage 0: local chunk summary",
+ * "Stage 1: entmax chunk routing" and "Stage 2: prior-induced sparse
+ * softmax".  alpha-entmax as in Peters, Niculae & Martins (2019).
+ *
+ * What the library computes, per batch element b and KV head g (G = H/Hkv
+ * query heads share g), for a query at position pos in block t = pos / B:
+ *   stage 0  s_c = mean_{j in block c} k_j @ W_s                 (fp32)
+ *   stage 1  z_{h,c} = q_h . s_c / sqrt(d);  p_h = alpha-entmax(z_h) over the
+ *            N candidate blocks (causal: the complete blocks c < t);
+ *            p_bar = mean over the G heads; selected = {c : p_bar_c > 0}
+ *   stage 2  o_h = sum_j softmax_j(q_h . k_j / sqrt(d) + bias_j) v_j over the
+ *            tokens of the selected blocks (bias log p_bar_c) and of the
+ *            diagonal block t (tokens <= pos when causal; bias log(1/N),
+ *            0 when N = 0).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are described by dash_tensor_t: a DEVICE pointer with extents
+ *    (b, s, h, d) and element strides for b, s and h; the d dimension is
+ *    contiguous.  Base pointers and the b/s/h strides (in bytes) must be
+ *    multiples of 16 bytes.  q and out are [B, S, H, d]; k and v are
+ *    [B, S, Hkv, d] (FlashAttention layout).
+ *  - q, k and v share one dtype: DASH_F32, DASH_F16 or DASH_BF16.  f16/bf16
+ *    use tensor cores with fp32 accumulation; f32 runs an fp32 CUDA-core
+ *    path.  Summaries, routing weights and thresholds are always fp32.
+ *  - Supported: d in {64, 128}; block in {64, 128}; G = H / Hkv in
+ *    {1, 2, 4, 8}; 1 < alpha <= 2.
+ *  - Ownership: the caller allocates every buffer (inputs, outputs,
+ *    workspace) and keeps it alive until the stream work completes.  The
+ *    library allocates no memory.
+ *  - Asynchrony: work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) of the current device; nothing synchronises.
+ *  - Errors: invalid arguments are detected on the host before anything is
+ *    launched and return a non-zero dash_status_t; dash_attn_last_error()
+ *    then gives a message (thread-local).  A failed launch returns
+ *    DASH_ERR_CUDA.  Device-side waits are bounded: if one gives up, the
+ *    kernel records DASH_ERR_DEVICE_TIMEOUT in the workspace status word,
+ *    which dash_attn_get_device_status() reads.
+ */
+#ifndef DASHATTN_H_
+#define DASHATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dash_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  DASH_OK = 0,
+  DASH_ERR_INVALID_ARGUMENT = 1,
+  DASH_ERR_UNSUPPORTED = 2,
+  DASH_ERR_WORKSPACE_TOO_SMALL = 3,
+  DASH_ERR_CUDA = 4,
+  DASH_ERR_DEVICE_TIMEOUT = 5
+} dash_status_t;
+
+typedef enum { DASH_F32 = 0, DASH_F16 = 1, DASH_BF16 = 2 } dash_dtype_t;
+
+typedef struct {
+  void* data;     /* device pointer to element (0, 0, 0, 0) */
+  int32_t dtype;  /* dash_dtype_t */
+  int32_t reserved;
+  int64_t b, s, h, d;                   /* extents */
+  int64_t stride_b, stride_s, stride_h; /* element strides; d is contiguous */
+} dash_tensor_t;
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int dash_attn_version(void);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* dash_attn_last_error(void);
+
+/*
+ * Bytes of workspace dash_attn_fwd needs for q [B, S, H, d], k [B, S, Hkv, d]
+ * and `block`.  Holds the stage-0 summaries [B, Hkv, T, d] fp32 (T =
+ * ceil(S / block)), the per-row routing lists [B, Hkv, S, T] (int32 block
+ * ids and fp32 log p_bar), the counts [B, Hkv, S], the per-tile union lists
+ * and a status word.  Returns 0 for arguments dash_attn_fwd would reject.
+ */
+size_t dash_attn_fwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t* k, int block);
+
+/*
+ * Full prefill forward: stages 0, 1 and 2 ("Stage 0" to "Stage 2" of the
+ * cited technical summary) over q [B, S, H, d], k, v [B, S, Hkv, d].
+ *   w_s       device fp32 [d, d] row-major; summaries are mean(k) @ w_s.
+ *   alpha     entmax alpha, 1 < alpha <= 2.
+ *   block     block (chunk) size B, 64 or 128.
+ *   causal    1: candidates are the complete blocks before the query's own
+ *             block, which is included with a causal mask.  0: every other
+ *             block is a candidate (a trailing partial block is pooled over
+ *             its valid tokens) and the own block is included whole.
+ *   out       [B, S, H, d], same dtype as q; written once per element.
+ *   workspace device buffer of at least dash_attn_fwd_workspace_size()
+ *             bytes, 256-byte aligned; its contents on return are the
+ *             routing lists of the call (readable with the layout above).
+ */
+dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                            const float* w_s, float alpha, int block, int causal, dash_tensor_t* out,
+                            void* workspace, size_t workspace_bytes, dash_stream_t stream);
+
+/*
+ * Stage 0 alone ("Stage 0: local chunk summary"; a summary is fixed and
+ * cached once its chunk is complete): summaries[b, g, c, :] =
+ * mean_{j in block c, j < n_b} k[b, j, g, :] @ w_s for blocks
+ * first_block <= c < ceil(n_b / block), where n_b = seqlens[b] (or k->s when
+ * seqlens is NULL).  A trailing partial block is averaged over its valid
+ * tokens; a decode step never reads it (it is the query's diagonal block).
+ *   seqlens         device int32 [B] or NULL.
+ *   summaries       device fp32 [B, Hkv, t_cap, d], contiguous.
+ *   t_cap           block capacity of `summaries`; must be >= ceil(k->s / block).
+ *   first_block     first block to (re)compute; 0 for all.  Decoding calls
+ *                   this again with the first block that has just completed.
+ */
+dash_status_t dash_attn_summarize(const dash_tensor_t* k, const int32_t* seqlens, const float* w_s,
+                                  int block, float* summaries, int64_t t_cap, int64_t first_block,
+                                  dash_stream_t stream);
+
+/*
+ * Bytes of workspace dash_attn_decode needs for q [B, 1, H, d] against a KV
+ * cache [B, Lmax, Hkv, d] with summaries of capacity t_cap blocks.
+ */
+size_t dash_attn_decode_workspace_size(const dash_tensor_t* q, const dash_tensor_t* kcache, int block,
+                                       int64_t t_cap);
+
+/*
+ * One decode step (stages 1 and 2 for a single new query token per
+ * sequence; "supports prefill and incremental decoding" in the cited
+ * technical summary).  The query of sequence b sits at position
+ * pos = seqlens[b] - 1; its candidates are the complete blocks
+ * c < pos / block, read from the cached summaries; the diagonal block holds
+ * tokens [ (pos / block) * block, pos ].
+ *   q          [B, 1, H, d]; kcache, vcache [B, Lmax, Hkv, d] (same dtype).
+ *   seqlens    device int32 [B], 1 <= seqlens[b] <= Lmax.
+ *   summaries  device fp32 [B, Hkv, t_cap, d] from dash_attn_summarize.
+ *   out        [B, 1, H, d].
+ */
+dash_status_t dash_attn_decode(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,
+                               const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha,
+                               int block, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                               dash_stream_t stream);
+
+/*
+ * Stage 1 alone ("Stage 1: entmax chunk routing", including GQA handling),
+ * for parity checks and for callers that bring their own stage 2.
+ * Prefill mode (seqlens == NULL): q is [B, S, H, d], the query at row i sits
+ * at position i and the context holds S tokens.  Decode mode: q is
+ * [B, 1, H, d] and the query of sequence b sits at seqlens[b] - 1 (always
+ * causal; seqlens[b] <= t_cap * block).
+ *   summaries  device fp32 [B, kv_heads, t_cap, d].
+ *   idx, logp  device [B, kv_heads, Sq, t_cap]: for each query row the
+ *              selected block ids in ascending order and log p_bar of each;
+ *              entries past cnt are left untouched.
+ *   cnt        device int32 [B, kv_heads, Sq]: number of selected blocks.
+ *   tau        optional device fp32 [B, H, Sq]: entmax threshold of each
+ *              head on the (alpha - 1) * z scale (0 when N = 0).
+ *   p_dense    optional device fp32 [B, H, Sq, t_cap]: per-head entmax
+ *              weight of every block (0 for non-candidates).
+ *   workspace  decode mode only: dash_attn_route_workspace_size() bytes,
+ *              256-byte aligned (the per-head logits); NULL in prefill mode.
+ */
+size_t dash_attn_route_workspace_size(const dash_tensor_t* q, int64_t kv_heads, int64_t t_cap, int decode);
+
+dash_status_t dash_attn_route(const dash_tensor_t* q, const float* summaries, int64_t kv_heads, int64_t t_cap,
+                              const int32_t* seqlens, float alpha, int block, int causal, int32_t* idx,
+                              float* logp, int32_t* cnt, float* tau, float* p_dense, void* workspace,
+                              size_t workspace_bytes, dash_stream_t stream);
+
+/*
+ * Bytes of workspace dash_attn_sparse needs (per-tile union lists and a
+ * status word).
+ */
+size_t dash_attn_sparse_workspace_size(const dash_tensor_t* q, const dash_tensor_t* k, int block, int64_t t_cap);
+
+/*
+ * Stage 2 alone ("Stage 2: prior-induced sparse softmax") on caller-given
+ * routing in the layout dash_attn_route writes (idx/logp/cnt with block
+ * capacity t_cap).  The diagonal block is always added with bias log(1/N).
+ * Selecting every candidate with logp = log(1/N) reproduces full attention.
+ */
+dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                               const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap,
+                               int block, int causal, dash_tensor_t* out, void* workspace,
+                               size_t workspace_bytes, dash_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the device status word of a workspace
+ * last used by dash_attn_fwd / dash_attn_decode / dash_attn_sparse /
+ * dash_attn_route (each call clears it when it starts).  Returns DASH_OK,
+ * DASH_ERR_DEVICE_TIMEOUT (a bounded device wait expired; outputs of that
+ * call are not valid), DASH_ERR_INVALID_ARGUMENT (a device-side value such
+ * as seqlens[b] was out of range; it was clamped) or DASH_ERR_CUDA.
+ */
+dash_status_t dash_attn_get_device_status(void* workspace, dash_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DASHATTN_H_ */

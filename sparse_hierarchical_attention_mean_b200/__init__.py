@@ -1,0 +1,287 @@
+"""Python binding of libdashattn (the DashAttention forward for B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/dashattn.h``.  PyTorch is used
+for device memory and the current CUDA stream.  The library must have been
+built (``python -m sparse_hierarchical_attention_mean_b200._build``); loading
+fails loudly otherwise -- there is no fallback implementation.
+
+Layouts (FlashAttention convention, last dim contiguous):
+q, out [B, S, H, d]; k, v [B, S, Hkv, d]; summaries [B, Hkv, T, d] fp32.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdashattn.so")
+
+DASH_OK = 0
+_STATUS = {
+    0: "DASH_OK",
+    1: "DASH_ERR_INVALID_ARGUMENT",
+    2: "DASH_ERR_UNSUPPORTED",
+    3: "DASH_ERR_WORKSPACE_TOO_SMALL",
+    4: "DASH_ERR_CUDA",
+    5: "DASH_ERR_DEVICE_TIMEOUT",
+}
+_DTYPE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+# Every symbol include/dashattn.h declares.
+EXPORTED = (
+    "dash_attn_version",
+    "dash_attn_last_error",
+    "dash_attn_fwd_workspace_size",
+    "dash_attn_fwd",
+    "dash_attn_summarize",
+    "dash_attn_decode_workspace_size",
+    "dash_attn_decode",
+    "dash_attn_route_workspace_size",
+    "dash_attn_route",
+    "dash_attn_sparse_workspace_size",
+    "dash_attn_sparse",
+    "dash_attn_get_device_status",
+)
+
+
+class DashError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class DashTensor(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p),
+        ("dtype", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("b", ctypes.c_int64),
+        ("s", ctypes.c_int64),
+        ("h", ctypes.c_int64),
+        ("d", ctypes.c_int64),
+        ("stride_b", ctypes.c_int64),
+        ("stride_s", ctypes.c_int64),
+        ("stride_h", ctypes.c_int64),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with `python -m sparse_hierarchical_attention_mean_b200._build`"
+        )
+    lib = ctypes.CDLL(_LIB_PATH)
+    T = ctypes.POINTER(DashTensor)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "dash_attn_version": (i32, []),
+        "dash_attn_last_error": (ctypes.c_char_p, []),
+        "dash_attn_fwd_workspace_size": (sz, [T, T, i32]),
+        "dash_attn_fwd": (i32, [T, T, T, vp, f32, i32, i32, T, vp, sz, vp]),
+        "dash_attn_summarize": (i32, [T, vp, vp, i32, vp, i64, i64, vp]),
+        "dash_attn_decode_workspace_size": (sz, [T, T, i32, i64]),
+        "dash_attn_decode": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp, sz, vp]),
+        "dash_attn_route_workspace_size": (sz, [T, i64, i64, i32]),
+        "dash_attn_route": (i32, [T, vp, i64, i64, vp, f32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "dash_attn_sparse_workspace_size": (sz, [T, T, i32, i64]),
+        "dash_attn_sparse": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, vp]),
+        "dash_attn_get_device_status": (i32, [vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+class _Lazy:
+    """Loads the library on first use (so the build step can import this package)."""
+
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _Lazy._cdll is None:
+            _Lazy._cdll = _load()
+        return getattr(_Lazy._cdll, name)
+
+
+_lib = _Lazy()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Loads (once) and returns the library; raises ImportError if it is missing."""
+    _lib.dash_attn_version  # noqa: B018
+    return _Lazy._cdll
+
+
+def version() -> int:
+    return _lib.dash_attn_version()
+
+
+def _check(status: int) -> None:
+    if status != DASH_OK:
+        raise DashError(status, _lib.dash_attn_last_error().decode())
+
+
+def _desc(t: torch.Tensor) -> DashTensor:
+    if t.dim() != 4:
+        raise ValueError("expected a [B, S, H, d] tensor")
+    if not t.is_cuda:
+        raise ValueError("tensors must be CUDA device tensors")
+    if t.stride(3) != 1:
+        raise ValueError("the last dimension must be contiguous")
+    if t.dtype not in _DTYPE:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    b, s, h, d = t.shape
+    return DashTensor(t.data_ptr(), _DTYPE[t.dtype], 0, b, s, h, d, t.stride(0), t.stride(1), t.stride(2))
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _workspace(nbytes: int, device, given: torch.Tensor | None) -> torch.Tensor:
+    if given is not None:
+        return given
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def n_blocks(seq: int, block: int) -> int:
+    return -(-seq // block)
+
+
+# ------------------------------------------------------------------ stage 0
+
+
+def summarize(k: torch.Tensor, w_s: torch.Tensor, block: int, seqlens: torch.Tensor | None = None,
+              summaries: torch.Tensor | None = None, first_block: int = 0, stream=None) -> torch.Tensor:
+    """Block summaries [B, Hkv, t_cap, d] fp32 (see dash_attn_summarize)."""
+    B, S, Hkv, d = k.shape
+    if summaries is None:
+        summaries = torch.zeros((B, Hkv, n_blocks(S, block), d), dtype=torch.float32, device=k.device)
+    assert summaries.is_contiguous() and summaries.dtype == torch.float32
+    kd = _desc(k)
+    _check(_lib.dash_attn_summarize(ctypes.byref(kd), _ptr(seqlens), w_s.data_ptr(), block,
+                                    summaries.data_ptr(), summaries.shape[2], first_block, _stream(stream)))
+    return summaries
+
+
+# ------------------------------------------------------------------ stage 1
+
+
+def route_workspace_size(q: torch.Tensor, kv_heads: int, t_cap: int, decode: bool) -> int:
+    qd = _desc(q)
+    return _lib.dash_attn_route_workspace_size(ctypes.byref(qd), kv_heads, t_cap, 1 if decode else 0)
+
+
+def route(q: torch.Tensor, summaries: torch.Tensor, alpha: float, block: int, causal: bool = True,
+          seqlens: torch.Tensor | None = None, want_tau: bool = False, want_p: bool = False,
+          idx=None, logp=None, cnt=None, workspace=None, stream=None) -> dict:
+    """Stage 1 alone; returns idx, logp [B, Hkv, Sq, t_cap], cnt [B, Hkv, Sq] (+ tau, p).
+
+    idx / logp / cnt / workspace may be passed in to reuse buffers.
+    """
+    B, Sq, H, d = q.shape
+    _, Hkv, t_cap, _ = summaries.shape
+    dev = q.device
+    if idx is None:
+        idx = torch.full((B, Hkv, Sq, t_cap), -1, dtype=torch.int32, device=dev)
+    if logp is None:
+        logp = torch.zeros((B, Hkv, Sq, t_cap), dtype=torch.float32, device=dev)
+    if cnt is None:
+        cnt = torch.zeros((B, Hkv, Sq), dtype=torch.int32, device=dev)
+    tau = torch.zeros((B, H, Sq), dtype=torch.float32, device=dev) if want_tau else None
+    p = torch.zeros((B, H, Sq, t_cap), dtype=torch.float32, device=dev) if want_p else None
+    ws = None
+    if seqlens is not None:
+        ws = _workspace(route_workspace_size(q, Hkv, t_cap, True), dev, workspace)
+    qd = _desc(q)
+    _check(_lib.dash_attn_route(ctypes.byref(qd), summaries.data_ptr(), Hkv, t_cap, _ptr(seqlens), alpha, block,
+                                1 if causal else 0, idx.data_ptr(), logp.data_ptr(), cnt.data_ptr(), _ptr(tau),
+                                _ptr(p), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return {"idx": idx, "logp": logp, "cnt": cnt, "tau": tau, "p": p, "workspace": ws}
+
+
+# ------------------------------------------------------------------ stage 2
+
+
+def sparse_workspace_size(q: torch.Tensor, k: torch.Tensor, block: int, t_cap: int) -> int:
+    qd, kd = _desc(q), _desc(k)
+    return _lib.dash_attn_sparse_workspace_size(ctypes.byref(qd), ctypes.byref(kd), block, t_cap)
+
+
+def sparse(q, k, v, idx, logp, cnt, block: int, causal: bool = True, out=None, workspace=None,
+           stream=None) -> torch.Tensor:
+    """Stage 2 alone on caller-given routing (layout of :func:`route`)."""
+    out = torch.empty_like(q) if out is None else out
+    t_cap = idx.shape[-1]
+    ws = _workspace(sparse_workspace_size(q, k, block, t_cap), q.device, workspace)
+    qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
+    _check(_lib.dash_attn_sparse(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), idx.data_ptr(),
+                                 logp.data_ptr(), cnt.data_ptr(), t_cap, block, 1 if causal else 0,
+                                 ctypes.byref(od), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ full forward
+
+
+def fwd_workspace_size(q: torch.Tensor, k: torch.Tensor, block: int) -> int:
+    qd, kd = _desc(q), _desc(k)
+    n = _lib.dash_attn_fwd_workspace_size(ctypes.byref(qd), ctypes.byref(kd), block)
+    if n == 0:
+        raise DashError(1, "arguments rejected by dash_attn_fwd_workspace_size")
+    return n
+
+
+def fwd(q, k, v, w_s, alpha: float, block: int, causal: bool = True, out=None, workspace=None,
+        stream=None) -> torch.Tensor:
+    """Full prefill forward (stages 0-2); see dash_attn_fwd."""
+    out = torch.empty_like(q) if out is None else out
+    ws = _workspace(fwd_workspace_size(q, k, block), q.device, workspace)
+    qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
+    _check(_lib.dash_attn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), w_s.data_ptr(), alpha, block,
+                              1 if causal else 0, ctypes.byref(od), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ decode
+
+
+def decode_workspace_size(q: torch.Tensor, kcache: torch.Tensor, block: int, t_cap: int) -> int:
+    qd, kd = _desc(q), _desc(kcache)
+    n = _lib.dash_attn_decode_workspace_size(ctypes.byref(qd), ctypes.byref(kd), block, t_cap)
+    if n == 0:
+        raise DashError(1, "arguments rejected by dash_attn_decode_workspace_size")
+    return n
+
+
+def decode(q, kcache, vcache, seqlens, summaries, alpha: float, block: int, out=None, workspace=None,
+           stream=None) -> torch.Tensor:
+    """One decode step for q [B, 1, H, d] (see dash_attn_decode)."""
+    out = torch.empty_like(q) if out is None else out
+    t_cap = summaries.shape[2]
+    ws = _workspace(decode_workspace_size(q, kcache, block, t_cap), q.device, workspace)
+    qd, kd, vd, od = _desc(q), _desc(kcache), _desc(vcache), _desc(out)
+    _check(_lib.dash_attn_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), seqlens.data_ptr(),
+                                 summaries.data_ptr(), t_cap, alpha, block, ctypes.byref(od), ws.data_ptr(),
+                                 ws.numel(), _stream(stream)))
+    return out
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Status word of the last call that used ``workspace`` (synchronises)."""
+    return _lib.dash_attn_get_device_status(workspace.data_ptr(), _stream(stream))
+

@@ -1,0 +1,508 @@
+// C ABI of libdashattn: argument checks, workspace carving and launches.
+// Every entry point validates on the host before launching anything and
+// allocates no memory; work goes to the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/dashattn.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+dash_status_t fail(dash_status_t st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+dash_status_t fail(dash_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+dash_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(DASH_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+dash_status_t ok() {
+  g_last_error.clear();
+  return DASH_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int elt_size(int dtype) { return dtype == DASH_F32 ? 4 : 2; }
+
+// Checks one tensor descriptor.  `name` is used in messages.
+dash_status_t check_tensor(const dash_tensor_t* t, const char* name) {
+  if (!t) return fail(DASH_ERR_INVALID_ARGUMENT, "%s: null descriptor", name);
+  if (!t->data) return fail(DASH_ERR_INVALID_ARGUMENT, "%s: null data pointer", name);
+  if (t->dtype != DASH_F32 && t->dtype != DASH_F16 && t->dtype != DASH_BF16)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, t->dtype);
+  if (t->b <= 0 || t->s <= 0 || t->h <= 0 || t->d <= 0)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "%s: extents must be positive (b=%lld s=%lld h=%lld d=%lld)", name,
+                (long long)t->b, (long long)t->s, (long long)t->h, (long long)t->d);
+  if (t->d != 64 && t->d != 128) return fail(DASH_ERR_UNSUPPORTED, "%s: head dim %lld not in {64, 128}", name, (long long)t->d);
+  if (t->s > (1LL << 30) || t->b > 65535 || t->h > 65535)
+    return fail(DASH_ERR_UNSUPPORTED, "%s: extents too large", name);
+  const int es = elt_size(t->dtype);
+  if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "%s: data pointer not 16-byte aligned", name);
+  if ((t->stride_b * es) % 16 || (t->stride_s * es) % 16 || (t->stride_h * es) % 16)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "%s: strides must be multiples of 16 bytes", name);
+  if (t->stride_b < 0 || t->stride_s < 0 || t->stride_h < 0)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "%s: negative strides are not supported", name);
+  return DASH_OK;
+}
+
+dash_status_t check_common(float alpha, int block) {
+  if (!(alpha > 1.0f && alpha <= 2.0f)) return fail(DASH_ERR_INVALID_ARGUMENT, "alpha %g not in (1, 2]", alpha);
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  return DASH_OK;
+}
+
+dash_status_t check_group(int64_t H, int64_t Hkv) {
+  if (Hkv <= 0 || H % Hkv) return fail(DASH_ERR_INVALID_ARGUMENT, "heads %lld not a multiple of kv heads %lld", (long long)H, (long long)Hkv);
+  const int64_t G = H / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(DASH_ERR_UNSUPPORTED, "group size %lld not in {1, 2, 4, 8}", (long long)G);
+  return DASH_OK;
+}
+
+dash::View view(const dash_tensor_t* t) { return dash::View{t->data, t->stride_b, t->stride_s, t->stride_h}; }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Workspace of dash_attn_fwd.
+struct FwdLayout {
+  size_t status, summ, idx, logp, cnt, ulist, ucnt, total;
+  int64_t T, n_tiles;
+  int tile_pos;
+};
+
+FwdLayout fwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, int block) {
+  FwdLayout L{};
+  const int64_t G = H / Hkv;
+  L.T = (S + block - 1) / block;
+  L.tile_pos = dash::sparse_tile_positions((int)G, block);
+  L.n_tiles = (S + L.tile_pos - 1) / L.tile_pos;
+  size_t off = 0;
+  L.status = off;
+  off = align256(off + sizeof(dash::DeviceStatus));
+  L.summ = off;
+  off = align256(off + (size_t)B * Hkv * L.T * D * 4);
+  L.idx = off;
+  off = align256(off + (size_t)B * Hkv * S * L.T * 4);
+  L.logp = off;
+  off = align256(off + (size_t)B * Hkv * S * L.T * 4);
+  L.cnt = off;
+  off = align256(off + (size_t)B * Hkv * S * 4);
+  L.ulist = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * L.T * 4);
+  L.ucnt = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
+  L.total = off;
+  return L;
+}
+
+struct SparseLayout {
+  size_t status, ulist, ucnt, total;
+  int64_t n_tiles;
+  int tile_pos;
+};
+
+SparseLayout sparse_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int block, int64_t t_cap) {
+  SparseLayout L{};
+  L.tile_pos = dash::sparse_tile_positions((int)(H / Hkv), block);
+  L.n_tiles = (S + L.tile_pos - 1) / L.tile_pos;
+  size_t off = 0;
+  L.status = off;
+  off = align256(off + sizeof(dash::DeviceStatus));
+  L.ulist = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * t_cap * 4);
+  L.ucnt = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
+  L.total = off;
+  return L;
+}
+
+struct DecodeLayout {
+  size_t status, scores, idx, logp, cnt, items, n_items, pair_base, part_o, part_ml, total;
+  int64_t max_items;
+  int chunk;
+};
+
+DecodeLayout decode_layout(int64_t B, int64_t H, int64_t Hkv, int64_t D, int block, int64_t t_cap) {
+  DecodeLayout L{};
+  const int64_t G = H / Hkv;
+  L.chunk = block == 64 ? 16 : 8;
+  L.max_items = dash::decode_max_items(B, Hkv, t_cap, L.chunk);
+  size_t off = 0;
+  L.status = off;
+  off = align256(off + sizeof(dash::DeviceStatus));
+  L.scores = off;
+  off = align256(off + (size_t)B * Hkv * G * t_cap * 4);
+  L.idx = off;
+  off = align256(off + (size_t)B * Hkv * t_cap * 4);
+  L.logp = off;
+  off = align256(off + (size_t)B * Hkv * t_cap * 4);
+  L.cnt = off;
+  off = align256(off + (size_t)B * Hkv * 4);
+  L.items = off;
+  off = align256(off + (size_t)L.max_items * 2 * 4);
+  L.n_items = off;
+  off = align256(off + 4);
+  L.pair_base = off;
+  off = align256(off + (size_t)B * Hkv * 4);
+  L.part_o = off;
+  off = align256(off + (size_t)L.max_items * G * D * 4);
+  L.part_ml = off;
+  off = align256(off + (size_t)L.max_items * G * 2 * 4);
+  L.total = off;
+  return L;
+}
+
+template <typename P>
+P* at(void* base, size_t off) {
+  return reinterpret_cast<P*>(static_cast<char*>(base) + off);
+}
+
+dash_status_t check_fwd_shapes(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                               const dash_tensor_t* out) {
+  dash_status_t st;
+  if ((st = check_tensor(q, "q")) || (st = check_tensor(k, "k")) || (st = check_tensor(v, "v")) ||
+      (st = check_tensor(out, "out")))
+    return st;
+  if (q->dtype != k->dtype || q->dtype != v->dtype || q->dtype != out->dtype)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "q, k, v and out must share one dtype");
+  if (k->b != q->b || v->b != q->b || out->b != q->b) return fail(DASH_ERR_INVALID_ARGUMENT, "batch mismatch");
+  if (k->d != q->d || v->d != q->d || out->d != q->d) return fail(DASH_ERR_INVALID_ARGUMENT, "head dim mismatch");
+  if (k->h != v->h) return fail(DASH_ERR_INVALID_ARGUMENT, "k and v head counts differ");
+  if (out->h != q->h || out->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "out must have q's shape");
+  return check_group(q->h, k->h);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dash_attn_version(void) { return 100; }
+
+const char* dash_attn_last_error(void) { return g_last_error.c_str(); }
+
+size_t dash_attn_fwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t* k, int block) {
+  if (check_tensor(q, "q") || check_tensor(k, "k") || (block != 64 && block != 128) || check_group(q->h, k->h))
+    return 0;
+  return fwd_layout(q->b, q->s, q->h, k->h, q->d, block).total;
+}
+
+dash_status_t dash_attn_summarize(const dash_tensor_t* k, const int32_t* seqlens, const float* w_s, int block,
+                                  float* summaries, int64_t t_cap, int64_t first_block, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_tensor(k, "k"))) return st;
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  if (!w_s || !summaries) return fail(DASH_ERR_INVALID_ARGUMENT, "null w_s or summaries");
+  if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
+  const int64_t T = (k->s + block - 1) / block;
+  if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block) = %lld", (long long)t_cap, (long long)T);
+  if (first_block < 0) return fail(DASH_ERR_INVALID_ARGUMENT, "first_block < 0");
+  dash::PoolParams p{};
+  p.k = view(k);
+  p.dtype = k->dtype;
+  p.B = (int)k->b;
+  p.S = (int)k->s;
+  p.Hkv = (int)k->h;
+  p.D = (int)k->d;
+  p.block = block;
+  p.seqlens = seqlens;
+  p.w_s = w_s;
+  p.summaries = summaries;
+  p.t_cap = t_cap;
+  p.first_block = first_block;
+  cudaError_t e = dash::launch_pool(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "summarize");
+  return ok();
+}
+
+size_t dash_attn_route_workspace_size(const dash_tensor_t* q, int64_t kv_heads, int64_t t_cap, int decode) {
+  if (check_tensor(q, "q") || check_group(q->h, kv_heads) || t_cap <= 0) return 0;
+  if (!decode) return 0;
+  return decode_layout(q->b, q->h, kv_heads, q->d, 64, t_cap).idx;  // status + per-head logits
+}
+
+dash_status_t dash_attn_route(const dash_tensor_t* q, const float* summaries, int64_t kv_heads, int64_t t_cap,
+                              const int32_t* seqlens, float alpha, int block, int causal, int32_t* idx, float* logp,
+                              int32_t* cnt, float* tau, float* p_dense, void* workspace, size_t workspace_bytes,
+                              dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_tensor(q, "q")) || (st = check_common(alpha, block)) || (st = check_group(q->h, kv_heads))) return st;
+  if (!summaries || !idx || !logp || !cnt) return fail(DASH_ERR_INVALID_ARGUMENT, "null summaries/idx/logp/cnt");
+  if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
+  const int G = (int)(q->h / kv_heads);
+  if (!seqlens) {
+    const int64_t T = (q->s + block - 1) / block;
+    if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block)", (long long)t_cap);
+    if (T > 4096) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per sequence");
+    dash::RouteParams p{};
+    p.q = view(q);
+    p.dtype = q->dtype;
+    p.B = (int)q->b;
+    p.S = (int)q->s;
+    p.H = (int)q->h;
+    p.Hkv = (int)kv_heads;
+    p.G = G;
+    p.D = (int)q->d;
+    p.block = block;
+    p.causal = causal ? 1 : 0;
+    p.alpha = alpha;
+    p.summaries = summaries;
+    p.t_cap = t_cap;
+    p.idx = idx;
+    p.logp = logp;
+    p.cnt = cnt;
+    p.tau = tau;
+    p.p_dense = p_dense;
+    cudaError_t e = dash::launch_route_prefill(p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "route");
+    return ok();
+  }
+  if (q->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode-mode route needs q with s == 1");
+  if (!causal) return fail(DASH_ERR_UNSUPPORTED, "decode-mode route is causal");
+  if (t_cap > 4096) return fail(DASH_ERR_UNSUPPORTED, "t_cap above 4096");
+  const DecodeLayout L = decode_layout(q->b, q->h, kv_heads, q->d, block, t_cap);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "decode-mode route needs a 256-byte aligned workspace");
+  if (workspace_bytes < L.idx)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.idx);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  dash::DecodeParams p{};
+  p.q = view(q);
+  p.dtype = q->dtype;
+  p.B = (int)q->b;
+  p.Lmax = (int)(t_cap * block);
+  p.H = (int)q->h;
+  p.Hkv = (int)kv_heads;
+  p.G = G;
+  p.D = (int)q->d;
+  p.block = block;
+  p.alpha = alpha;
+  p.seqlens = seqlens;
+  p.summaries = summaries;
+  p.t_cap = t_cap;
+  p.scores = at<float>(workspace, L.scores);
+  p.idx = idx;
+  p.logp = logp;
+  p.cnt = cnt;
+  p.tau = tau;
+  p.p_dense = p_dense;
+  p.status = at<dash::DeviceStatus>(workspace, L.status);
+  e = dash::launch_decode_route(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode route");
+  return ok();
+}
+
+size_t dash_attn_sparse_workspace_size(const dash_tensor_t* q, const dash_tensor_t* k, int block, int64_t t_cap) {
+  if (check_tensor(q, "q") || check_tensor(k, "k") || (block != 64 && block != 128) || check_group(q->h, k->h))
+    return 0;
+  return sparse_layout(q->b, q->s, q->h, k->h, block, t_cap).total;
+}
+
+static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                                const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                                int causal, dash_tensor_t* out, int32_t* ulist, int32_t* ucnt, int tile_pos,
+                                int64_t n_tiles, dash::DeviceStatus* status, cudaStream_t stream) {
+  if (q->dtype != DASH_F32) {
+    dash::UnionParams u{};
+    u.B = (int)q->b;
+    u.S = (int)q->s;
+    u.Hkv = (int)k->h;
+    u.block = block;
+    u.tile_pos = tile_pos;
+    u.n_tiles = (int)n_tiles;
+    u.t_cap = t_cap;
+    u.idx = idx;
+    u.cnt = cnt;
+    u.ulist = ulist;
+    u.ucnt = ucnt;
+    u.causal = causal ? 1 : 0;
+    u.status = status;
+    cudaError_t e = dash::launch_union(u, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "union");
+  }
+  dash::SparseParams p{};
+  p.q = view(q);
+  p.k = view(k);
+  p.v = view(v);
+  p.out = view(out);
+  p.dtype = q->dtype;
+  p.B = (int)q->b;
+  p.S = (int)q->s;
+  p.H = (int)q->h;
+  p.Hkv = (int)k->h;
+  p.G = (int)(q->h / k->h);
+  p.D = (int)q->d;
+  p.block = block;
+  p.causal = causal ? 1 : 0;
+  p.t_cap = t_cap;
+  p.idx = idx;
+  p.logp = logp;
+  p.cnt = cnt;
+  p.ulist = ulist;
+  p.ucnt = ucnt;
+  p.tile_pos = tile_pos;
+  p.n_tiles = (int)n_tiles;
+  p.status = status;
+  cudaError_t e = dash::launch_sparse_prefill(p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
+  return DASH_OK;
+}
+
+dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                               const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                               int causal, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                               dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_fwd_shapes(q, k, v, out))) return st;
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  if (k->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "prefill needs k and q of equal length");
+  if (!idx || !logp || !cnt) return fail(DASH_ERR_INVALID_ARGUMENT, "null routing lists");
+  const int64_t T = (q->s + block - 1) / block;
+  if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block)", (long long)t_cap);
+  const SparseLayout L = sparse_layout(q->b, q->s, q->h, k->h, block, t_cap);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < L.total)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, out, at<int32_t>(workspace, L.ulist),
+                  at<int32_t>(workspace, L.ucnt), L.tile_pos, L.n_tiles, at<dash::DeviceStatus>(workspace, L.status), s);
+  return st ? st : ok();
+}
+
+dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v, const float* w_s,
+                            float alpha, int block, int causal, dash_tensor_t* out, void* workspace,
+                            size_t workspace_bytes, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_fwd_shapes(q, k, v, out)) || (st = check_common(alpha, block))) return st;
+  if (k->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "prefill needs k and q of equal length");
+  if (!w_s) return fail(DASH_ERR_INVALID_ARGUMENT, "null w_s");
+  const FwdLayout L = fwd_layout(q->b, q->s, q->h, k->h, q->d, block);
+  if (L.T > 4096) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per sequence");
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < L.total)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  float* summ = at<float>(workspace, L.summ);
+  if ((st = dash_attn_summarize(k, nullptr, w_s, block, summ, L.T, 0, stream))) return st;
+  int32_t* idx = at<int32_t>(workspace, L.idx);
+  float* logp = at<float>(workspace, L.logp);
+  int32_t* cnt = at<int32_t>(workspace, L.cnt);
+  if ((st = dash_attn_route(q, summ, k->h, L.T, nullptr, alpha, block, causal, idx, logp, cnt, nullptr, nullptr,
+                            nullptr, 0, stream)))
+    return st;
+  st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, out, at<int32_t>(workspace, L.ulist),
+                  at<int32_t>(workspace, L.ucnt), L.tile_pos, L.n_tiles, at<dash::DeviceStatus>(workspace, L.status), s);
+  return st ? st : ok();
+}
+
+size_t dash_attn_decode_workspace_size(const dash_tensor_t* q, const dash_tensor_t* kcache, int block, int64_t t_cap) {
+  if (check_tensor(q, "q") || check_tensor(kcache, "kcache") || (block != 64 && block != 128) ||
+      check_group(q->h, kcache->h) || t_cap <= 0)
+    return 0;
+  return decode_layout(q->b, q->h, kcache->h, q->d, block, t_cap).total;
+}
+
+dash_status_t dash_attn_decode(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,
+                               const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha, int block,
+                               dash_tensor_t* out, void* workspace, size_t workspace_bytes, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_tensor(q, "q")) || (st = check_tensor(kcache, "kcache")) || (st = check_tensor(vcache, "vcache")) ||
+      (st = check_tensor(out, "out")) || (st = check_common(alpha, block)) || (st = check_group(q->h, kcache->h)))
+    return st;
+  if (q->s != 1 || out->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode takes one query token (s == 1)");
+  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "decode supports f16 and bf16");
+  if (q->dtype != kcache->dtype || q->dtype != vcache->dtype || q->dtype != out->dtype)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "q, caches and out must share one dtype");
+  if (kcache->b != q->b || vcache->b != q->b || out->b != q->b) return fail(DASH_ERR_INVALID_ARGUMENT, "batch mismatch");
+  if (kcache->d != q->d || vcache->d != q->d || out->d != q->d) return fail(DASH_ERR_INVALID_ARGUMENT, "head dim mismatch");
+  if (vcache->h != kcache->h || vcache->s != kcache->s) return fail(DASH_ERR_INVALID_ARGUMENT, "kcache and vcache differ");
+  if (out->h != q->h) return fail(DASH_ERR_INVALID_ARGUMENT, "out must have q's shape");
+  if (!seqlens || !summaries) return fail(DASH_ERR_INVALID_ARGUMENT, "null seqlens or summaries");
+  if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
+  const int64_t T = (kcache->s + block - 1) / block;
+  if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(Lmax / block)", (long long)t_cap);
+  if (t_cap > 4096) return fail(DASH_ERR_UNSUPPORTED, "t_cap above 4096");
+  const DecodeLayout L = decode_layout(q->b, q->h, kcache->h, q->d, block, t_cap);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < L.total)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(at<char>(workspace, L.n_items), 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  dash::DecodeParams p{};
+  p.q = view(q);
+  p.k = view(kcache);
+  p.v = view(vcache);
+  p.out = view(out);
+  p.dtype = q->dtype;
+  p.B = (int)q->b;
+  p.Lmax = (int)kcache->s;
+  p.H = (int)q->h;
+  p.Hkv = (int)kcache->h;
+  p.G = (int)(q->h / kcache->h);
+  p.D = (int)q->d;
+  p.block = block;
+  p.alpha = alpha;
+  p.seqlens = seqlens;
+  p.summaries = summaries;
+  p.t_cap = t_cap;
+  p.scores = at<float>(workspace, L.scores);
+  p.idx = at<int32_t>(workspace, L.idx);
+  p.logp = at<float>(workspace, L.logp);
+  p.cnt = at<int32_t>(workspace, L.cnt);
+  p.items = at<int32_t>(workspace, L.items);
+  p.n_items = at<int32_t>(workspace, L.n_items);
+  p.pair_base = at<int32_t>(workspace, L.pair_base);
+  p.part_o = at<float>(workspace, L.part_o);
+  p.part_ml = at<float>(workspace, L.part_ml);
+  p.max_items = L.max_items;
+  p.chunk_blocks = L.chunk;
+  p.status = at<dash::DeviceStatus>(workspace, L.status);
+  e = dash::launch_decode_route(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode route");
+  e = dash::launch_decode_attend(p, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode attend");
+  return ok();
+}
+
+dash_status_t dash_attn_get_device_status(void* workspace, dash_stream_t stream) {
+  if (!workspace) return fail(DASH_ERR_INVALID_ARGUMENT, "null workspace");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  dash::DeviceStatus st{};
+  e = cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (st.code == 0) return ok();
+  return fail((dash_status_t)st.code, "device reported status %d (detail %d)", st.code, st.detail);
+}
+
+}  // extern "C"

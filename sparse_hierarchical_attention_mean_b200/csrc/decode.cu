@@ -1,0 +1,516 @@
+// Decode step: stage 1 against cached summaries and the split-KV stage 2.
+//
+// "Stage 0: local chunk summary" (a chunk's summary is cached once the chunk
+// is complete, so decoding never recomputes it), "Stage 1: entmax chunk
+// routing" and "Stage 2: prior-induced sparse softmax" of the DashAttention
+// technical summary, for one new query token per sequence; the pages report
+// decoding speed "in the memory-bound regime", which is what these kernels
+// are shaped for: every byte of the cached summaries and of the selected
+// K/V blocks is read once.
+//
+//  score_decode      (b, g, 64-block chunk) CTAs; a warp reads 8 summary
+//                    rows (coalesced fp32) and dots them with the G query
+//                    heads; a warp reduce-scatter finishes the G*8 sums.
+//  entmax_decode     one CTA per (b, g): tau per head (warp per head), GQA
+//                    mean, ballot/popc compaction, and the split-KV work
+//                    items (chunks of selected blocks) appended with one
+//                    atomic per (b, g).
+//  attend_decode     persistent CTAs over the work items: K/V rows of the
+//                    selected blocks stream through a cp.async double
+//                    buffer; each warp owns 16 tokens of a 64-token step,
+//                    computes the G x 16 logits with a reduce-scatter, keeps
+//                    an online softmax per head and accumulates P V; the 4
+//                    warps merge into one (m, l, o) partial per item.
+//  combine_decode    log-sum-exp merge of the partials of each (b, g).
+#include "common.cuh"
+#include "internal.h"
+
+namespace dash {
+namespace {
+
+__device__ __forceinline__ int clamp_len(const int32_t* seqlens, int b, int lmax, DeviceStatus* st) {
+  int L = seqlens[b];
+  if (L < 1 || L > lmax) {
+    raise_status(st, 1 /* DASH_ERR_INVALID_ARGUMENT */, 100 + b);
+    L = L < 1 ? 1 : lmax;
+  }
+  return L;
+}
+
+// ------------------------------------------------------------------ scores
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(256) score_decode_kernel(DecodeParams p) {
+  constexpr int DL = D / 32;
+  constexpr int NV = 8 * G;
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int L = clamp_len(p.seqlens, b, p.Lmax, p.status);
+  const int N = (L - 1) / p.block;
+  const int c0 = blockIdx.x * 64 + warp * 8;
+  if (c0 >= N) return;
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  float qv[G][DL];
+  const T* q = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb;
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < DL; ++e) qv[h][e] = Elt<T>::load1(q + (int64_t)(g * G + h) * p.q.sh + lane * DL + e);
+  float v[NV];
+  const float* sb = p.summaries + bg * p.t_cap * D + lane * DL;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float s[DL];
+    if (c0 + i < N) {
+      if constexpr (DL == 4) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(sb + (int64_t)(c0 + i) * D));
+        s[0] = x.x, s[1] = x.y, s[2] = x.z, s[3] = x.w;
+      } else {
+        const float2 x = __ldg(reinterpret_cast<const float2*>(sb + (int64_t)(c0 + i) * D));
+        s[0] = x.x, s[1] = x.y;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < DL; ++e) s[e] = 0.f;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) a = fmaf(qv[h][e], s[e], a);
+      v[i * G + h] = a;
+    }
+  }
+  warp_transpose_reduce<NV>(v, lane);
+  const float coef = (p.alpha - 1.0f) * rsqrtf((float)D);
+  if constexpr (NV >= 32) {
+#pragma unroll
+    for (int j = 0; j < NV / 32; ++j) {
+      const int i = lane * (NV / 32) + j;
+      const int c = c0 + i / G, h = i % G;
+      if (c < N) p.scores[(bg * G + h) * p.t_cap + c] = coef * v[j];
+    }
+  } else {
+    constexpr int SH = NV == 16 ? 1 : (NV == 8 ? 2 : 0);
+    if ((lane & ((1 << SH) - 1)) == 0) {
+      const int i = lane >> SH;
+      const int c = c0 + i / G, h = i % G;
+      if (c < N) p.scores[(bg * G + h) * p.t_cap + c] = coef * v[0];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ entmax + compaction
+__global__ void __launch_bounds__(256) entmax_decode_kernel(DecodeParams p) {
+  extern __shared__ __align__(16) float xs[];  // [G][t_cap]
+  __shared__ float tau_s[8];
+  const int b = blockIdx.y, g = blockIdx.x;
+  const int G = p.G;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int L = clamp_len(p.seqlens, b, p.Lmax, nullptr);
+  const int N = (L - 1) / p.block;
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const float pw = 1.0f / (p.alpha - 1.0f);
+  const int kind = entmax_kind(p.alpha);
+  for (int i = threadIdx.x; i < G * N; i += blockDim.x) {
+    const int h = i / N, c = i % N;
+    xs[h * p.t_cap + c] = p.scores[(bg * G + h) * p.t_cap + c];
+  }
+  __syncthreads();
+  for (int h = warp; h < G; h += blockDim.x / 32) {
+    const float tau = N > 0 ? warp_entmax_tau(xs + h * p.t_cap, N, p.alpha, lane) : 0.f;
+    if (lane == 0) tau_s[h] = tau;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int32_t* idx = p.idx + bg * p.t_cap;
+    float* logp = p.logp + bg * p.t_cap;
+    int off = 0;
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      const int c = c0 + lane;
+      float pb = 0.f;
+      if (c < N) {
+        for (int h = 0; h < G; ++h) {
+          const float u = xs[h * p.t_cap + c] - tau_s[h];
+          if (u > 0.f) pb += pow_pw(u, pw, kind);
+        }
+        pb /= (float)G;
+      }
+      const bool sel = pb > 0.f;
+      const unsigned m = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const int o = off + __popc(m & ((1u << lane) - 1u));
+        idx[o] = c;
+        logp[o] = logf(pb);
+      }
+      off += __popc(m);
+    }
+    if (lane == 0) {
+      p.cnt[bg] = off;
+      if (p.items) {
+        const int n_it = (off + 1 + p.chunk_blocks - 1) / p.chunk_blocks;
+        const int base = atomicAdd(p.n_items, n_it);
+        p.pair_base[bg] = base;
+        for (int k = 0; k < n_it; ++k) {
+          p.items[2 * (base + k)] = (int32_t)bg;
+          p.items[2 * (base + k) + 1] = k;
+        }
+      }
+    }
+  }
+  if (p.tau || p.p_dense) {
+    for (int h = warp; h < G; h += blockDim.x / 32) {
+      const int64_t hrow = (int64_t)b * p.H + g * G + h;
+      if (p.tau && lane == 0) p.tau[hrow] = tau_s[h];
+      if (p.p_dense) {
+        for (int c = lane; c < p.t_cap; c += 32) {
+          float v = 0.f;
+          if (c < N) {
+            const float u = xs[h * p.t_cap + c] - tau_s[h];
+            if (u > 0.f) v = pow_pw(u, pw, kind);
+          }
+          p.p_dense[hrow * p.t_cap + c] = v;
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ split-KV attention
+constexpr int kStep = 64;  // tokens per pipeline step
+constexpr int kWarps = 4;  // 16 tokens per warp per step
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kWarps * 32) attend_decode_kernel(DecodeParams p) {
+  constexpr int DL = D / 32;
+  constexpr int NV = 16 * G;
+  constexpr int NVL = NV >= 32 ? NV / 32 : 1;  // values per lane after the reduce
+  constexpr int GH = G >= 2 ? G / 2 : 1;         // heads per lane parity
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  T* Ks = reinterpret_cast<T*>(smem_raw);          // [2][kStep][D]
+  T* Vs = Ks + 2 * kStep * D;                      // [2][kStep][D]
+  float* pbuf = reinterpret_cast<float*>(Vs + 2 * kStep * D);  // [kWarps][16][G]
+  float* mbuf = pbuf + kWarps * 16 * G;            // [kWarps][G]
+  float* lbuf = mbuf + kWarps * G;                 // [kWarps][G]
+  float* obuf = lbuf + kWarps * G;                 // [kWarps][G][D]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n_items = *p.n_items;
+  const float qk_scale = rsqrtf((float)D) * kLog2e;
+
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int bg = p.items[2 * item], chunk = p.items[2 * item + 1];
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int L = clamp_len(p.seqlens, b, p.Lmax, nullptr);
+    const int pos = L - 1;
+    const int t = pos / p.block;
+    const int N = t;
+    const int cnt = p.cnt[bg];
+    const int e_begin = chunk * p.chunk_blocks;
+    const int e_end = min(e_begin + p.chunk_blocks, cnt + 1);
+    const bool has_diag = e_end == cnt + 1;
+    const int spb = p.block / kStep;
+    const int n_diag = has_diag ? (pos - t * p.block) / kStep + 1 : 0;
+    const int n_sel = (has_diag ? e_end - 1 : e_end) - e_begin;
+    const int n_sub = n_sel * spb + n_diag;
+    const int32_t* idx = p.idx + (int64_t)bg * p.t_cap;
+    const float* logp = p.logp + (int64_t)bg * p.t_cap;
+    const float beta = N > 0 ? logf(1.0f / (float)N) : 0.0f;
+
+    const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
+    const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
+
+    auto sub_tok0 = [&](int s) -> int {
+      if (s < n_sel * spb) return idx[e_begin + s / spb] * p.block + (s % spb) * kStep;
+      return t * p.block + (s - n_sel * spb) * kStep;
+    };
+    auto load = [&](int s, int buf) {
+      const int tok0 = sub_tok0(s);
+      constexpr int NCH = D / 8;
+      T* kd = Ks + buf * kStep * D;
+      T* vd = Vs + buf * kStep * D;
+      for (int i = tid; i < kStep * NCH; i += kWarps * 32) {
+        const int r = i / NCH, c = i % NCH;
+        const int tok = tok0 + r;
+        const bool ok = tok < L;
+        cp_async16(kd + r * D + c * 8, kg + (int64_t)(ok ? tok : 0) * p.k.ss + c * 8, ok);
+        cp_async16(vd + r * D + c * 8, vg + (int64_t)(ok ? tok : 0) * p.v.ss + c * 8, ok);
+      }
+      cp_async_commit();
+    };
+
+    // query (pre-scaled into the log2 domain)
+    float qv[G][DL];
+    const T* q = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb;
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < DL; ++e)
+        qv[h][e] = Elt<T>::load1(q + (int64_t)(g * G + h) * p.q.sh + lane * DL + e) * qk_scale;
+
+    float m[G], o[G][DL], lown[NVL];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      m[h] = kNegInf;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) o[h][e] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) lown[j] = 0.f;
+
+    load(0, 0);
+    for (int s = 0; s < n_sub; ++s) {
+      if (s + 1 < n_sub) {
+        load(s + 1, (s + 1) & 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const int buf = s & 1;
+      const T* kb = Ks + buf * kStep * D + warp * 16 * D;
+      const T* vb = Vs + buf * kStep * D + warp * 16 * D;
+      const bool diag = s >= n_sel * spb;
+      const float bias = (diag ? beta : logp[e_begin + s / spb]) * kLog2e;
+      const int tok0 = sub_tok0(s) + warp * 16;
+
+      // logits of 16 tokens x G heads
+      float v[NV];
+#pragma unroll
+      for (int tt = 0; tt < 16; ++tt) {
+        float kf[DL];
+        if constexpr (DL == 4) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(kb + tt * D + lane * 4);
+          if constexpr (sizeof(T) == 2) {
+            uint4 w = make_uint4(raw.x, raw.y, 0u, 0u);
+            float f8[8];
+            Elt<T>::to_float(w, f8);
+            kf[0] = f8[0], kf[1] = f8[1], kf[2] = f8[2], kf[3] = f8[3];
+          }
+        } else {
+          const uint32_t raw = *reinterpret_cast<const uint32_t*>(kb + tt * D + lane * 2);
+          uint4 w = make_uint4(raw, 0u, 0u, 0u);
+          float f8[8];
+          Elt<T>::to_float(w, f8);
+          kf[0] = f8[0], kf[1] = f8[1];
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < DL; ++e) a = fmaf(qv[h][e], kf[e], a);
+          v[tt * G + h] = a;
+        }
+      }
+      warp_transpose_reduce<NV>(v, lane);
+      // lane holds token lane/2; heads (lane&1)*GH + j (G >= 2) or head 0
+      const int tok = tok0 + (lane >> 1);
+      const bool valid = tok <= pos;
+      float sl[NVL], mx[NVL];
+#pragma unroll
+      for (int j = 0; j < NVL; ++j) {
+        sl[j] = valid ? v[j] + bias : kNegInf;
+        mx[j] = sl[j];
+#pragma unroll
+        for (int off = 2; off <= 16; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], off));
+      }
+      float mu[G], sc[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float th = __shfl_sync(0xffffffffu, mx[h % GH], G >= 2 ? h / GH : 0);
+        const float mn = fmaxf(m[h], th);
+        mu[h] = mn == kNegInf ? 0.f : mn;
+        sc[h] = exp2f(m[h] - mu[h]);
+        m[h] = mn;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) o[h][e] *= sc[h];
+      }
+      float* pw = pbuf + warp * 16 * G;
+#pragma unroll
+      for (int j = 0; j < NVL; ++j) {
+        const int hd = G >= 2 ? (lane & 1) * GH + j : 0;
+        float muj = mu[j], scj = sc[j];
+        if constexpr (G >= 2) {
+          muj = (lane & 1) ? mu[GH + j] : mu[j];
+          scj = (lane & 1) ? sc[GH + j] : sc[j];
+        }
+        const float pj = exp2f(sl[j] - muj);
+        lown[j] = lown[j] * scj + pj;
+        pw[(lane >> 1) * G + hd] = pj;
+      }
+      __syncwarp();
+#pragma unroll 4
+      for (int tt = 0; tt < 16; ++tt) {
+        float vf[DL];
+        if constexpr (DL == 4) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(vb + tt * D + lane * 4);
+          uint4 w = make_uint4(raw.x, raw.y, 0u, 0u);
+          float f8[8];
+          Elt<T>::to_float(w, f8);
+          vf[0] = f8[0], vf[1] = f8[1], vf[2] = f8[2], vf[3] = f8[3];
+        } else {
+          const uint32_t raw = *reinterpret_cast<const uint32_t*>(vb + tt * D + lane * 2);
+          uint4 w = make_uint4(raw, 0u, 0u, 0u);
+          float f8[8];
+          Elt<T>::to_float(w, f8);
+          vf[0] = f8[0], vf[1] = f8[1];
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float ph = pw[tt * G + h];
+#pragma unroll
+          for (int e = 0; e < DL; ++e) o[h][e] = fmaf(ph, vf[e], o[h][e]);
+        }
+      }
+      __syncwarp();
+      __syncthreads();
+    }
+
+    // l per head: sum over the 16 lanes of the owning parity
+#pragma unroll
+    for (int j = 0; j < NVL; ++j)
+#pragma unroll
+      for (int off = 2; off <= 16; off <<= 1) lown[j] += __shfl_xor_sync(0xffffffffu, lown[j], off);
+    if (lane < 2) {
+#pragma unroll
+      for (int j = 0; j < NVL; ++j) {
+        if (G >= 2) {
+          lbuf[warp * G + lane * GH + j] = lown[j];
+        } else if (lane == 0) {
+          lbuf[warp * G] = lown[0];
+        }
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) mbuf[warp * G + h] = m[h];
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < DL; ++e) obuf[(warp * G + h) * D + lane * DL + e] = o[h][e];
+    __syncthreads();
+    const int64_t slot = (int64_t)p.pair_base[bg] + chunk;
+    for (int i = tid; i < G * D; i += kWarps * 32) {
+      const int h = i / D, e = i % D;
+      float M = kNegInf;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mbuf[w * G + h]);
+      const float Mu = M == kNegInf ? 0.f : M;
+      float acc = 0.f, lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = exp2f(mbuf[w * G + h] - Mu);
+        acc += f * obuf[(w * G + h) * D + e];
+        lsum += f * lbuf[w * G + h];
+      }
+      p.part_o[(slot * G + h) * D + e] = acc;
+      if (e == 0) {
+        p.part_ml[(slot * G + h) * 2] = M;
+        p.part_ml[(slot * G + h) * 2 + 1] = lsum;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ combine
+template <typename T, int D>
+__global__ void __launch_bounds__(256) combine_decode_kernel(DecodeParams p) {
+  const int b = blockIdx.y, g = blockIdx.x;
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const int n_it = (p.cnt[bg] + 1 + p.chunk_blocks - 1) / p.chunk_blocks;
+  const int64_t base = p.pair_base[bg];
+  T* out = static_cast<T*>(const_cast<void*>(p.out.data)) + (int64_t)b * p.out.sb;
+  for (int i = threadIdx.x; i < p.G * D; i += blockDim.x) {
+    const int h = i / D, e = i % D;
+    float M = kNegInf;
+    for (int k = 0; k < n_it; ++k) M = fmaxf(M, p.part_ml[((base + k) * p.G + h) * 2]);
+    const float Mu = M == kNegInf ? 0.f : M;
+    float acc = 0.f, lsum = 0.f;
+    for (int k = 0; k < n_it; ++k) {
+      const float f = exp2f(p.part_ml[((base + k) * p.G + h) * 2] - Mu);
+      acc += f * p.part_o[((base + k) * p.G + h) * D + e];
+      lsum += f * p.part_ml[((base + k) * p.G + h) * 2 + 1];
+    }
+    Elt<T>::store1(out + (int64_t)(g * p.G + h) * p.out.sh + e, lsum > 0.f ? acc / lsum : 0.f);
+  }
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_route_t(const DecodeParams& p, cudaStream_t stream) {
+  dim3 grid((unsigned)((p.t_cap + 63) / 64), p.Hkv, p.B);
+  score_decode_kernel<T, D, G><<<grid, 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)G * p.t_cap * sizeof(float);
+  e = cudaFuncSetAttribute(entmax_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  entmax_decode_kernel<<<dim3(p.Hkv, p.B), 256, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_attend_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+  const size_t smem = (size_t)4 * kStep * D * sizeof(T) +
+                      (size_t)(kWarps * 16 * G + 2 * kWarps * G + kWarps * G * D) * sizeof(float);
+  auto kern = attend_decode_kernel<T, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarps * 32, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  kern<<<num_sms * per_sm, kWarps * 32, smem, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  combine_decode_kernel<T, D><<<dim3(p.Hkv, p.B), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t route_d(const DecodeParams& p, cudaStream_t s) {
+  switch (p.G) {
+    case 1: return launch_route_t<T, D, 1>(p, s);
+    case 2: return launch_route_t<T, D, 2>(p, s);
+    case 4: return launch_route_t<T, D, 4>(p, s);
+    default: return launch_route_t<T, D, 8>(p, s);
+  }
+}
+template <typename T, int D>
+cudaError_t attend_d(const DecodeParams& p, int n, cudaStream_t s) {
+  switch (p.G) {
+    case 1: return launch_attend_t<T, D, 1>(p, n, s);
+    case 2: return launch_attend_t<T, D, 2>(p, n, s);
+    case 4: return launch_attend_t<T, D, 4>(p, n, s);
+    default: return launch_attend_t<T, D, 8>(p, n, s);
+  }
+}
+
+}  // namespace
+
+int64_t decode_max_items(int64_t B, int64_t Hkv, int64_t t_cap, int chunk_blocks) {
+  return B * Hkv * ((t_cap + 1 + chunk_blocks - 1) / chunk_blocks);
+}
+
+cudaError_t launch_decode_route(const DecodeParams& p, cudaStream_t stream) {
+  if (p.D == 128) {
+    if (p.dtype == 0) return route_d<float, 128>(p, stream);
+    if (p.dtype == 1) return route_d<__half, 128>(p, stream);
+    return route_d<__nv_bfloat16, 128>(p, stream);
+  }
+  if (p.dtype == 0) return route_d<float, 64>(p, stream);
+  if (p.dtype == 1) return route_d<__half, 64>(p, stream);
+  return route_d<__nv_bfloat16, 64>(p, stream);
+}
+
+cudaError_t launch_decode_attend(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+  if (p.dtype == 0) return cudaErrorInvalidValue;  // fp32 decode is not supported
+  if (p.D == 128) {
+    if (p.dtype == 1) return attend_d<__half, 128>(p, num_sms, stream);
+    return attend_d<__nv_bfloat16, 128>(p, num_sms, stream);
+  }
+  if (p.dtype == 1) return attend_d<__half, 64>(p, num_sms, stream);
+  return attend_d<__nv_bfloat16, 64>(p, num_sms, stream);
+}
+
+}  // namespace dash

@@ -1,0 +1,110 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dash {
+
+struct DeviceStatus;
+
+// A strided [B, S, H, D] view; strides in elements, D contiguous.
+struct View {
+  const void* data;
+  int64_t sb, ss, sh;
+};
+
+// ---------------------------------------------------------------- stage 0
+struct PoolParams {
+  View k;
+  int dtype;  // 0 f32, 1 f16, 2 bf16
+  int B, S, Hkv, D, block;
+  const int32_t* seqlens;  // nullable
+  const float* w_s;        // [D, D]
+  float* summaries;        // [B, Hkv, t_cap, D]
+  int64_t t_cap;
+  int64_t first_block;
+};
+cudaError_t launch_pool(const PoolParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- stage 1
+struct RouteParams {
+  View q;
+  int dtype;
+  int B, S, H, Hkv, G, D, block;
+  int causal;
+  float alpha;
+  const float* summaries;  // [B, Hkv, t_cap, D]
+  int64_t t_cap;
+  int32_t* idx;  // [B, Hkv, S, t_cap]
+  float* logp;   // [B, Hkv, S, t_cap]
+  int32_t* cnt;  // [B, Hkv, S]
+  float* tau;      // nullable [B, H, S]
+  float* p_dense;  // nullable [B, H, S, t_cap]
+};
+cudaError_t launch_route_prefill(const RouteParams& p, cudaStream_t stream);
+
+// Union of the per-row block lists over each stage-2 tile of `tile_pos`
+// consecutive positions.
+struct UnionParams {
+  int B, S, Hkv, block, tile_pos, n_tiles;
+  int64_t t_cap;
+  const int32_t* idx;
+  const int32_t* cnt;
+  int32_t* ulist;  // [B, Hkv, n_tiles, t_cap]
+  int32_t* ucnt;   // [B, Hkv, n_tiles]
+  int causal;
+  DeviceStatus* status;  // invalid list entries are skipped and reported here
+};
+cudaError_t launch_union(const UnionParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- stage 2
+struct SparseParams {
+  View q, k, v, out;
+  int dtype;
+  int B, S, H, Hkv, G, D, block;
+  int causal;
+  int64_t t_cap;
+  const int32_t* idx;
+  const float* logp;
+  const int32_t* cnt;
+  const int32_t* ulist;
+  const int32_t* ucnt;
+  int tile_pos, n_tiles;
+  DeviceStatus* status;
+};
+// rows per stage-2 tile for the tensor-core kernel
+int sparse_tile_positions(int G, int block);
+cudaError_t launch_sparse_prefill(const SparseParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode
+struct DecodeParams {
+  View q, k, v, out;
+  int dtype;
+  int B, Lmax, H, Hkv, G, D, block;
+  float alpha;
+  const int32_t* seqlens;
+  const float* summaries;
+  int64_t t_cap;
+  // workspace
+  float* scores;     // [B, Hkv, G, t_cap]
+  int32_t* idx;      // [B, Hkv, t_cap]
+  float* logp;       // [B, Hkv, t_cap]
+  int32_t* cnt;      // [B, Hkv]
+  int32_t* items;    // [max_items] packed work items
+  int32_t* n_items;  // device counter
+  int32_t* pair_base;  // [B, Hkv]
+  float* part_o;     // [max_items, G, D]
+  float* part_ml;    // [max_items, G, 2]
+  int64_t max_items;
+  int chunk_blocks;  // selected blocks per split-KV work item
+  // optional route outputs (dash_attn_route in decode mode)
+  float* tau;      // [B, H]
+  float* p_dense;  // [B, H, t_cap]
+  DeviceStatus* status;
+};
+int64_t decode_max_items(int64_t B, int64_t Hkv, int64_t t_cap, int chunk_blocks);
+cudaError_t launch_decode_route(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_decode_attend(const DecodeParams& p, int num_sms, cudaStream_t stream);
+
+}  // namespace dash

@@ -1,0 +1,291 @@
+// Stage 1 for prefill: routing scores, alpha-entmax, GQA average and the
+// compaction of each query row's support into an ascending block list.
+//
+// "Stage 1: entmax chunk routing" of the DashAttention technical summary:
+// each query scores the chunk summaries, w = alpha-entmax(gamma z) gives a
+// sparse distribution whose support size depends on the input, and under
+// GQA the probabilities of the query heads sharing a KV head are averaged
+// into one shared sparse support.  gamma = 1/sqrt(d).
+//
+// One CTA owns R rows = (R / G positions) x (G heads of one KV group); all
+// positions of a CTA lie in one block, so they share the N candidates.  The
+// CTA computes the R x N logits into shared memory chunk by chunk (fp32
+// CUDA-core GEMM, summaries staged with cp.async), solves tau for every row
+// with one warp per row, then one warp per position averages the G heads
+// and writes the list with a ballot/popc scan.
+#include "common.cuh"
+#include "internal.h"
+
+namespace dash {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ int cand_block(int ci, int t, int causal) {
+  return causal ? ci : (ci < t ? ci : ci + 1);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) route_prefill_kernel(RouteParams p, int R, int CW) {
+  extern __shared__ __align__(16) float smem[];
+  constexpr int DP = D + 4;
+  __shared__ float tau_s[64];
+
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int G = p.G;
+  const int rpos = R / G;
+  const int pos0 = blockIdx.x * rpos;
+  const int t = pos0 / p.block;
+  const int T_ = (p.S + p.block - 1) / p.block;
+  const int N = p.causal ? t : T_ - 1;
+  const int NP = (N + 3) & ~3;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float pw = 1.0f / (p.alpha - 1.0f);
+  const int kind = entmax_kind(p.alpha);
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+
+  float* Qs = smem;           // [R][DP]
+  float* Ss = Qs + R * DP;    // [CW][DP]
+  float* X = Ss + CW * DP;    // [R][NP]
+
+  if (N > 0) {
+    // ---- query rows -> fp32 shared memory
+    constexpr int EPV = Elt<T>::kPerVec;
+    constexpr int VPR = D / EPV;
+    for (int i = tid; i < R * VPR; i += kThreads) {
+      const int r = i / VPR, v = i % VPR;
+      const int pos = pos0 + r / G, head = g * G + r % G;
+      float f[EPV];
+      if (pos < p.S) {
+        const T* src = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb + (int64_t)pos * p.q.ss +
+                       (int64_t)head * p.q.sh + v * EPV;
+        Elt<T>::to_float(__ldg(reinterpret_cast<const uint4*>(src)), f);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) f[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) Qs[r * DP + v * EPV + e] = f[e];
+    }
+
+    // ---- logits x = (alpha - 1) / sqrt(d) * q . s_c
+    const float coef = (p.alpha - 1.0f) * rsqrtf((float)D);
+    const float* sbase = p.summaries + bg * p.t_cap * D;
+    const int cq = CW / 4;
+    const int rg = tid / cq, cg = tid % cq;
+    for (int ch0 = 0; ch0 < N; ch0 += CW) {
+      for (int i = tid; i < CW * (D / 4); i += kThreads) {
+        const int cand = i / (D / 4), k4 = i % (D / 4);
+        const int ci = ch0 + cand;
+        const bool ok = ci < N;
+        const float* src = sbase + (int64_t)(ok ? cand_block(ci, t, p.causal) : 0) * D + 4 * k4;
+        cp_async16(Ss + cand * DP + 4 * k4, src, ok);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncthreads();
+      if (rg < R / 4) {
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+        for (int k4 = 0; k4 < D / 4; ++k4) {
+          float4 qv[4], sv[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4*>(Qs + (4 * rg + i) * DP + 4 * k4);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sv[j] = *reinterpret_cast<const float4*>(Ss + (cg + cq * j) * DP + 4 * k4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              acc[i][j] = fmaf(qv[i].x, sv[j].x, acc[i][j]);
+              acc[i][j] = fmaf(qv[i].y, sv[j].y, acc[i][j]);
+              acc[i][j] = fmaf(qv[i].z, sv[j].z, acc[i][j]);
+              acc[i][j] = fmaf(qv[i].w, sv[j].w, acc[i][j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = ch0 + cg + cq * j;
+          if (c < NP) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) X[(4 * rg + i) * NP + c] = coef * acc[i][j];
+          }
+        }
+      }
+      __syncthreads();
+    }
+
+    // ---- tau per row (one warp per row)
+    for (int r = warp; r < R; r += kThreads / 32) {
+      const int pos = pos0 + r / G;
+      float tau = 0.f;
+      if (pos < p.S) tau = warp_entmax_tau(X + r * NP, N, p.alpha, lane);
+      if (lane == 0) tau_s[r] = tau;
+    }
+    __syncthreads();
+  }
+
+  // ---- GQA average + compaction (one warp per position)
+  for (int pp = warp; pp < rpos; pp += kThreads / 32) {
+    const int pos = pos0 + pp;
+    if (pos >= p.S) continue;
+    const int64_t row = (bg * p.S + pos);
+    int32_t* idx = p.idx + row * p.t_cap;
+    float* logp = p.logp + row * p.t_cap;
+    int off = 0;
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      const int c = c0 + lane;
+      float pb = 0.f;
+      if (c < N) {
+        for (int h = 0; h < G; ++h) {
+          const float u = X[(pp * G + h) * NP + c] - tau_s[pp * G + h];
+          if (u > 0.f) pb += pow_pw(u, pw, kind);
+        }
+        pb /= (float)G;
+      }
+      const bool sel = pb > 0.f;
+      const unsigned m = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const int o = off + __popc(m & ((1u << lane) - 1u));
+        idx[o] = cand_block(c, t, p.causal);
+        logp[o] = logf(pb);
+      }
+      off += __popc(m);
+    }
+    if (lane == 0) p.cnt[row] = off;
+  }
+
+  // ---- optional per-head outputs
+  if (p.tau || p.p_dense) {
+    for (int r = warp; r < R; r += kThreads / 32) {
+      const int pos = pos0 + r / G;
+      if (pos >= p.S) continue;
+      const int head = g * G + r % G;
+      const int64_t hrow = ((int64_t)b * p.H + head) * p.S + pos;
+      const float tau = N > 0 ? tau_s[r] : 0.f;
+      if (p.tau && lane == 0) p.tau[hrow] = tau;
+      if (p.p_dense) {
+        float* pd = p.p_dense + hrow * p.t_cap;
+        for (int cb = lane; cb < p.t_cap; cb += 32) {
+          int ci = -1;
+          if (p.causal) {
+            ci = cb < t ? cb : -1;
+          } else if (cb < T_ && cb != t) {
+            ci = cb < t ? cb : cb - 1;
+          }
+          float v = 0.f;
+          if (ci >= 0 && ci < N) {
+            const float u = X[r * NP + ci] - tau;
+            if (u > 0.f) v = pow_pw(u, pw, kind);
+          }
+          pd[cb] = v;
+        }
+      }
+    }
+  }
+}
+
+// Union of the per-row lists of `tile_pos` consecutive positions.
+__global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
+  extern __shared__ uint32_t mask[];
+  const int b = blockIdx.z, g = blockIdx.y, tile = blockIdx.x;
+  const int words = (int)((p.t_cap + 31) / 32);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int w = tid; w < words; w += kThreads) mask[w] = 0u;
+  __syncthreads();
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const int pos0 = tile * p.tile_pos;
+  const int t = pos0 / p.block;
+  const int n_blocks = (p.S + p.block - 1) / p.block;
+  for (int pp = warp; pp < p.tile_pos; pp += kThreads / 32) {
+    const int pos = pos0 + pp;
+    if (pos >= p.S) break;
+    const int64_t row = bg * p.S + pos;
+    const int n = min(max(p.cnt[row], 0), (int)p.t_cap);
+    const int32_t* idx = p.idx + row * p.t_cap;
+    for (int e = lane; e < n; e += 32) {
+      const int c = idx[e];
+      // a candidate is a block other than the own block (causal: an earlier one)
+      const bool ok = c >= 0 && c != t && (p.causal ? c < t : c < n_blocks);
+      if (ok) {
+        atomicOr(&mask[c >> 5], 1u << (c & 31));
+      } else {
+        raise_status(p.status, 1 /* DASH_ERR_INVALID_ARGUMENT */, 200);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int32_t* out = p.ulist + (bg * p.n_tiles + tile) * p.t_cap;
+    int off = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      uint32_t word = (w0 + lane < words) ? mask[w0 + lane] : 0u;
+      const int pc = __popc(word);
+      int incl = pc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int k = off + incl - pc;
+      while (word) {
+        const int bit = __ffs(word) - 1;
+        out[k++] = (w0 + lane) * 32 + bit;
+        word &= word - 1u;
+      }
+      off += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) p.ucnt[bg * p.n_tiles + tile] = off;
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_route_typed(const RouteParams& p, cudaStream_t stream) {
+  const int T_ = (p.S + p.block - 1) / p.block;
+  const int n_max = p.causal ? T_ - 1 : T_ - 1;
+  const int np = (n_max + 3) & ~3;
+  constexpr int DP = D + 4;
+  const int smem_cap = 227 * 1024 - 1024;  // leave room for the static tau array
+  int R = 64;
+  int CW = 64;
+  auto bytes = [&](int r, int cw) { return (size_t)(r * DP + cw * DP + r * np) * sizeof(float); };
+  while (R > p.G && (R > 64 || bytes(R, CW) > (size_t)smem_cap)) {
+    R /= 2;
+    CW = 128;
+  }
+  if (R < p.G || R / p.G > p.block || bytes(R, CW) > (size_t)smem_cap) return cudaErrorInvalidValue;
+  const size_t smem = bytes(R, CW);
+  auto kern = route_prefill_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int rpos = R / p.G;
+  dim3 grid((p.S + rpos - 1) / rpos, p.Hkv, p.B);
+  kern<<<grid, kThreads, smem, stream>>>(p, R, CW);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_prefill(const RouteParams& p, cudaStream_t stream) {
+  if (p.D == 128) {
+    if (p.dtype == 0) return launch_route_typed<float, 128>(p, stream);
+    if (p.dtype == 1) return launch_route_typed<__half, 128>(p, stream);
+    return launch_route_typed<__nv_bfloat16, 128>(p, stream);
+  }
+  if (p.dtype == 0) return launch_route_typed<float, 64>(p, stream);
+  if (p.dtype == 1) return launch_route_typed<__half, 64>(p, stream);
+  return launch_route_typed<__nv_bfloat16, 64>(p, stream);
+}
+
+cudaError_t launch_union(const UnionParams& p, cudaStream_t stream) {
+  const size_t smem = (size_t)((p.t_cap + 31) / 32) * sizeof(uint32_t);
+  dim3 grid(p.n_tiles, p.Hkv, p.B);
+  union_kernel<<<grid, kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace dash

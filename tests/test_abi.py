@@ -1,0 +1,143 @@
+"""The C-ABI library: it loads, exports every symbol include/dashattn.h
+declares, and rejects bad arguments on the host before touching the GPU.
+
+These run without a GPU: the argument checks return before any CUDA call,
+and the pointers handed in are never dereferenced.
+"""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_hierarchical_attention_mean_b200 as dash
+from sparse_hierarchical_attention_mean_b200 import DashTensor
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dashattn.h")
+
+FAKE = 0x100000  # 256-byte aligned, never dereferenced
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(dash_attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = dash.load()
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(dash.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", dash.library_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (dash_attn_\w+)", out))
+    assert set(names) <= exported
+    assert dash.version() == 100
+
+
+def tensor(b, s, h, d, dtype=2, data=FAKE, strides=None):
+    sb, ss, sh = strides or (s * h * d, h * d, d)
+    return DashTensor(data, dtype, 0, b, s, h, d, sb, ss, sh)
+
+
+def call_fwd(q, k, v, out, alpha=1.5, block=64, ws_bytes=1 << 40, ws=FAKE):
+    lib = dash.load()
+    st = lib.dash_attn_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), FAKE, alpha, block, 1,
+                           ctypes.byref(out), ws, ws_bytes, None)
+    return st, lib.dash_attn_last_error().decode()
+
+
+def good():
+    return tensor(1, 256, 8, 128), tensor(1, 256, 2, 128), tensor(1, 256, 2, 128), tensor(1, 256, 8, 128)
+
+
+@pytest.mark.parametrize(
+    "mutate, status, text",
+    [
+        (lambda q, k, v, o: setattr(q, "d", 96), 2, "head dim"),
+        (lambda q, k, v, o: setattr(k, "dtype", 1), 1, "dtype"),
+        (lambda q, k, v, o: setattr(q, "dtype", 7), 1, "dtype"),
+        (lambda q, k, v, o: (setattr(k, "h", 3), setattr(v, "h", 3)), 1, "multiple"),
+        (lambda q, k, v, o: (setattr(q, "h", 48), setattr(o, "h", 48), setattr(k, "h", 3), setattr(v, "h", 3)), 2,
+         "group size"),
+        (lambda q, k, v, o: setattr(q, "data", FAKE + 8), 1, "aligned"),
+        (lambda q, k, v, o: setattr(q, "data", 0), 1, "null"),
+        (lambda q, k, v, o: setattr(q, "stride_s", 8 * 128 + 4), 1, "16 bytes"),
+        (lambda q, k, v, o: setattr(k, "s", 255), 1, "equal length"),
+        (lambda q, k, v, o: setattr(o, "s", 100), 1, "shape"),
+        (lambda q, k, v, o: setattr(v, "b", 2), 1, "batch"),
+    ],
+)
+def test_fwd_rejects_bad_arguments(mutate, status, text):
+    q, k, v, o = good()
+    mutate(q, k, v, o)
+    st, msg = call_fwd(q, k, v, o)
+    assert st == status, msg
+    assert text in msg
+
+
+@pytest.mark.parametrize("alpha, block, status", [(1.0, 64, 1), (2.5, 64, 1), (float("nan"), 64, 1), (1.5, 32, 2)])
+def test_fwd_rejects_alpha_and_block(alpha, block, status):
+    st, msg = call_fwd(*good(), alpha=alpha, block=block)
+    assert st == status, msg
+
+
+def test_workspace_size_and_too_small():
+    q, k, v, o = good()
+    lib = dash.load()
+    need = lib.dash_attn_fwd_workspace_size(ctypes.byref(q), ctypes.byref(k), 64)
+    T = 4
+    # summaries + lists + counts + union lists, each 256-aligned
+    assert need >= 2 * 256 * T * 4 * 2 + 2 * T * 128 * 4
+    st, msg = call_fwd(q, k, v, o, ws_bytes=need - 1)
+    assert st == 3 and "workspace" in msg
+    st, msg = call_fwd(q, k, v, o, ws=FAKE + 16)
+    assert st == 1 and "256-byte" in msg
+    bad = tensor(1, 256, 8, 96)
+    assert lib.dash_attn_fwd_workspace_size(ctypes.byref(bad), ctypes.byref(k), 64) == 0
+
+
+def test_decode_and_route_reject_bad_arguments():
+    lib = dash.load()
+    q = tensor(4, 1, 8, 128)
+    kc = tensor(4, 4096, 2, 128)
+    o = tensor(4, 1, 8, 128)
+    ws = lib.dash_attn_decode_workspace_size(ctypes.byref(q), ctypes.byref(kc), 64, 64)
+    assert ws > 0
+    st = lib.dash_attn_decode(ctypes.byref(q), ctypes.byref(kc), ctypes.byref(kc), FAKE, FAKE, 32, 1.5, 64,
+                              ctypes.byref(o), FAKE, ws, None)
+    assert st == 1 and "t_cap" in lib.dash_attn_last_error().decode()
+    q2 = tensor(4, 2, 8, 128)
+    st = lib.dash_attn_decode(ctypes.byref(q2), ctypes.byref(kc), ctypes.byref(kc), FAKE, FAKE, 64, 1.5, 64,
+                              ctypes.byref(o), FAKE, ws, None)
+    assert st == 1
+    qf = tensor(4, 1, 8, 128, dtype=0)
+    of = tensor(4, 1, 8, 128, dtype=0)
+    kf = tensor(4, 4096, 2, 128, dtype=0)
+    st = lib.dash_attn_decode(ctypes.byref(qf), ctypes.byref(kf), ctypes.byref(kf), FAKE, FAKE, 64, 1.5, 64,
+                              ctypes.byref(of), FAKE, ws, None)
+    assert st == 2
+    st = lib.dash_attn_decode(ctypes.byref(q), ctypes.byref(kc), ctypes.byref(kc), FAKE, FAKE, 64, 1.5, 64,
+                              ctypes.byref(o), FAKE, ws - 1, None)
+    assert st == 3
+    # route: decode mode needs a workspace
+    st = lib.dash_attn_route(ctypes.byref(q), FAKE, 2, 64, FAKE, 1.5, 64, 1, FAKE, FAKE, FAKE, None, None, None, 0,
+                             None)
+    assert st == 1
+    st = lib.dash_attn_route(ctypes.byref(q), FAKE, 3, 64, None, 1.5, 64, 1, FAKE, FAKE, FAKE, None, None, None, 0,
+                             None)
+    assert st == 1
+    st = lib.dash_attn_summarize(ctypes.byref(kc), None, FAKE, 64, FAKE, 10, 0, None)
+    assert st == 1 and "t_cap" in lib.dash_attn_last_error().decode()
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+
+    x = torch.zeros(1, 64, 1, 64)
+    with pytest.raises(ValueError):
+        dash.fwd(x, x, x, torch.zeros(64, 64), 1.5, 64)

@@ -1,0 +1,203 @@
+"""GPU parity: every stage of the CUDA path against the fp64 oracle on the
+same seeded inputs, at sizes the oracle finishes in seconds that still span
+several tiles and a ragged tail, plus the edge cases (no candidates, a
+single partial block, non-causal, every group size, both head dims, the
+three alphas).  All calls go through the C ABI via the Python binding.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gen import Config, full_inputs, get_config, kv_values, make_plan
+from oracle.dash_oracle import block_summaries
+from tests._parity import (
+    OUT_TOL,
+    check_p_dense,
+    check_route_row,
+    max_abs,
+    oracle_decode_pair,
+    oracle_head,
+    to_np,
+)
+
+pytestmark = pytest.mark.gpu
+
+_BASE = get_config("prefill")
+SMALL = {
+    "pr1": get_config("pr1"),
+    "prefill_small": _BASE.with_(name="prefill_small", seq=2000),
+    "long_small": get_config("long_prefill").with_(name="long_small", seq=128 * 22 + 50),
+    "g8_small": _BASE.with_(name="g8_small", heads=16, kv_heads=2, seq=1100),
+    "g2_d64": _BASE.with_(name="g2_d64", heads=8, kv_heads=4, head_dim=64, seq=900, dtype="f16"),
+    "g1_b128": _BASE.with_(name="g1_b128", heads=4, kv_heads=4, block=128, seq=1300, alpha=2.0),
+    "noncausal": _BASE.with_(name="noncausal", seq=1000, causal=False),
+    "tiny": _BASE.with_(name="tiny", seq=40),
+    "f32_d128": _BASE.with_(name="f32_d128", heads=4, kv_heads=2, dtype="f32", seq=700, scaled=False,
+                            query_strength=11.3, key_strength=3.0),
+}
+for a in (1.25, 1.5, 2.0):
+    for s in (0.0, 4.0):
+        n = f"sweep_a{a}_s{s:g}"
+        SMALL[n] = get_config("sweep").with_(name=n, batch=2, seq=1500, alpha=a, key_strength=s)
+
+
+def _kv_subset(cfg):
+    return sorted({0, cfg.kv_heads - 1})
+
+
+@pytest.fixture(scope="module")
+def dash(cuda_lib):
+    return cuda_lib
+
+
+def _run_all(dash, cfg):
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    out = dash.fwd(q, k, v, w, cfg.alpha, cfg.block, cfg.causal)
+    summ = dash.summarize(k, w, cfg.block)
+    rt = dash.route(q, summ, cfg.alpha, cfg.block, cfg.causal, want_tau=True, want_p=True)
+    torch.cuda.synchronize()
+    return inp, out, summ, rt
+
+
+def test_generator_identical_on_gpu(dash):
+    for cfg in (SMALL["prefill_small"], SMALL["pr1"], SMALL["sweep_a1.5_s4"]):
+        gpu = full_inputs(cfg, device="cuda")
+        cpu = full_inputs(cfg, device="cpu")
+        for key in ("q", "k", "v", "w_s"):
+            assert torch.equal(gpu[key].cpu(), cpu[key]), (cfg.name, key)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_forward_parity_small(dash, name):
+    cfg = SMALL[name]
+    inp, out, summ, rt = _run_all(dash, cfg)
+    plan = inp["plan"]
+    G = cfg.group
+    tol = OUT_TOL[cfg.dtype]
+    out_np = to_np(out)
+    summ_np = summ.cpu().numpy()
+    idx, logp, cnt = rt["idx"].cpu().numpy(), rt["logp"].cpu().numpy(), rt["cnt"].cpu().numpy()
+    p_dense, tau = rt["p"].cpu().numpy(), rt["tau"].cpu().numpy()
+    rows = list(range(cfg.seq))
+    worst_out = worst_p = 0.0
+    for b in range(cfg.batch):
+        for g in _kv_subset(cfg):
+            recs, summ_o = oracle_head(cfg, plan, b, g, rows)
+            # stage 0
+            serr = np.abs(summ_np[b, g, : len(summ_o)] - summ_o).max()
+            assert serr <= 2e-5 * max(1.0, np.abs(summ_o).max()), f"{name}: summary error {serr:.3g}"
+            for pos, rec in zip(rows, recs):
+                where = f"{name} b{b} g{g} pos{pos}"
+                check_route_row(rec, idx[b, g, pos], logp[b, g, pos], cnt[b, g, pos], where)
+                e = check_p_dense(rec, p_dense[b, g * G:(g + 1) * G, pos], tau[b, g * G:(g + 1) * G, pos], where)
+                worst_p = max(worst_p, e)
+                err = max_abs(out_np[b, pos, g * G:(g + 1) * G], rec["out"])
+                worst_out = max(worst_out, err)
+                assert err <= tol, f"{where}: output error {err:.3g} > {tol}"
+    print(f"{name}: max |out err| {worst_out:.3g}, max |p err| {worst_p:.3g}")
+
+
+def test_all_selected_uniform_prior_is_full_attention(dash):
+    """Stage 2 with every candidate selected at log(1/N) equals plain causal attention."""
+    cfg = SMALL["prefill_small"].with_(heads=8, kv_heads=2, seq=777)
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    B, S, H, d = q.shape
+    Hkv, T = k.shape[2], -(-S // cfg.block)
+    pos = torch.arange(S)
+    n_cand = (pos // cfg.block).int()
+    idx = torch.arange(T, dtype=torch.int32).expand(B, Hkv, S, T).contiguous()
+    logp = torch.where(n_cand > 0, torch.log(1.0 / n_cand.clamp(min=1).double()), torch.zeros(S, dtype=torch.float64))
+    logp = logp.float()[None, None, :, None].expand(B, Hkv, S, T).contiguous()
+    cnt = n_cand[None, None].expand(B, Hkv, S).contiguous()
+    out = dash.sparse(q, k, v, idx.cuda(), logp.cuda(), cnt.cuda(), cfg.block, True)
+    qq = q.double().cpu().permute(0, 2, 1, 3)
+    kk = k.double().cpu().repeat_interleave(H // Hkv, dim=2).permute(0, 2, 1, 3)
+    vv = v.double().cpu().repeat_interleave(H // Hkv, dim=2).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=True).permute(0, 2, 1, 3)
+    assert max_abs(out.double().cpu(), ref) <= 2e-2
+
+
+def test_summarize_incremental_and_seqlens(dash):
+    cfg = SMALL["prefill_small"].with_(seq=1000)
+    inp = full_inputs(cfg, device="cuda")
+    k, w = inp["k"], inp["w_s"]
+    full = dash.summarize(k, w, cfg.block)
+    # recompute from block 7 on into a buffer holding garbage before it
+    part = torch.full_like(full, 123.0)
+    dash.summarize(k, w, cfg.block, summaries=part, first_block=7)
+    assert torch.equal(part[:, :, 7:], full[:, :, 7:])
+    assert torch.all(part[:, :, :7] == 123.0)
+    # seqlens: a shorter context pools a partial last block over its valid tokens
+    sl = torch.tensor([333], dtype=torch.int32, device="cuda")
+    s2 = dash.summarize(k, w, cfg.block, seqlens=sl)
+    kk = kv_values(cfg, inp["plan"], "k", 0, range(333), [3], as_float32=True)[:, 0].double().numpy()
+    ref = block_summaries(kk, inp["plan"].w_s.double().numpy(), cfg.block, 333)
+    got = s2[0, 3, : len(ref)].cpu().numpy()
+    assert np.abs(got - ref).max() <= 2e-5 * max(1.0, np.abs(ref).max())
+
+
+DECODE_SMALL = {
+    "decode_small": get_config("decode").with_(name="decode_small", batch=5, seq=4096, seqlen_lo=1, seqlen_hi=4096),
+    "decode_g8_d64": get_config("decode").with_(name="decode_g8_d64", batch=3, heads=16, kv_heads=2, head_dim=64,
+                                                 seq=3000, seqlen_lo=900, seqlen_hi=3000, dtype="f16", alpha=2.0),
+    "decode_b128": get_config("decode").with_(name="decode_b128", batch=3, block=128, seq=5000, seqlen_lo=100,
+                                              seqlen_hi=5000, alpha=1.25),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_SMALL))
+def test_decode_parity_small(dash, name):
+    cfg = DECODE_SMALL[name]
+    plan = make_plan(cfg)
+    if name == "decode_small":  # cover a 1-token context and an exact block boundary
+        plan.seqlens[0] = 1
+        plan.seqlens[1] = 2 * cfg.block
+        plan.seqlens[2] = 2 * cfg.block + 1
+    inp = full_inputs(cfg, device="cuda", plan=plan)
+    q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
+    summ = dash.summarize(k, w, cfg.block, seqlens=sl)
+    out = dash.decode(q, k, v, sl, summ, cfg.alpha, cfg.block)
+    rt = dash.route(q, summ, cfg.alpha, cfg.block, True, seqlens=sl, want_tau=True, want_p=True)
+    torch.cuda.synchronize()
+    G = cfg.group
+    tol = OUT_TOL[cfg.dtype]
+    out_np = to_np(out)
+    idx, logp, cnt = rt["idx"].cpu().numpy(), rt["logp"].cpu().numpy(), rt["cnt"].cpu().numpy()
+    for b in range(cfg.batch):
+        for g in range(cfg.kv_heads):
+            rec, _ = oracle_decode_pair(cfg, plan, b, g)
+            where = f"{name} b{b} g{g} L{int(plan.seqlens[b])}"
+            check_route_row(rec, idx[b, g, 0], logp[b, g, 0], cnt[b, g, 0], where)
+            check_p_dense(rec, rt["p"][b, g * G:(g + 1) * G, 0].cpu().numpy(),
+                          rt["tau"][b, g * G:(g + 1) * G, 0].cpu().numpy(), where)
+            err = max_abs(out_np[b, 0, g * G:(g + 1) * G], rec["out"])
+            assert err <= tol, f"{where}: output error {err:.3g}"
+
+
+def test_forward_is_deterministic(dash):
+    cfg = SMALL["prefill_small"]
+    inp = full_inputs(cfg, device="cuda")
+    a = dash.fwd(inp["q"], inp["k"], inp["v"], inp["w_s"], cfg.alpha, cfg.block)
+    b = dash.fwd(inp["q"], inp["k"], inp["v"], inp["w_s"], cfg.alpha, cfg.block)
+    assert torch.equal(a, b)
+
+
+def test_device_status_and_bad_seqlens(dash):
+    cfg = DECODE_SMALL["decode_small"]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
+    summ = dash.summarize(k, w, cfg.block, seqlens=sl)
+    ws = torch.empty(dash.decode_workspace_size(q, k, cfg.block, summ.shape[2]), dtype=torch.uint8, device="cuda")
+    dash.decode(q, k, v, sl, summ, cfg.alpha, cfg.block, workspace=ws)
+    assert dash.device_status(ws) == 0
+    bad = sl.clone()
+    bad[1] = cfg.seq + 5  # beyond the cache: clamped on the device and reported
+    dash.decode(q, k, v, bad, summ, cfg.alpha, cfg.block, workspace=ws)
+    assert dash.device_status(ws) == 1
+    dash.decode(q, k, v, sl, summ, cfg.alpha, cfg.block, workspace=ws)
+    assert dash.device_status(ws) == 0
