@@ -411,6 +411,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=64, help="sequences in the decode workload (64 = full)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
@@ -448,10 +450,11 @@ def main():
     dash.load()
     world, rank, _ = dist_setup(args.gpus)
     pk = peaks()
-    pre = run_prefill(dash, cfg, args.steps, warmup, world, rank, pk)
+    pre = None if args.skip_prefill else run_prefill(dash, cfg, args.steps, warmup, world, rank, pk)
     dec = None
+    dcfg = get_config("decode").with_(batch=args.decode_batch)
     if not args.skip_decode:
-        dec = run_decode(dash, get_config("decode"), max(5, args.steps), warmup, world, rank)
+        dec = run_decode(dash, dcfg, max(5, args.steps), warmup, world, rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
@@ -461,6 +464,12 @@ def main():
 
     if rank != 0:
         barrier(world)
+        finish(world)
+        return
+    if pre is None:
+        print(json.dumps({"decode_only": True, "us_per_step": None if dec is None else dec["us"]}), flush=True)
+        barrier(world)
+        finish(world)
         return
     value = pre["tokens"] * world / (pre["ms"] * 1e-3)
     peak_tf = pk["bf16_tflops"]
@@ -505,7 +514,8 @@ def main():
     if dec is not None:
         ach = dec["bytes"] / (dec["us"] * 1e-6) / 1e9
         line["decode"] = {
-            "workload": "decode: 64 seqs, 32/8 heads, d=128, bf16, cache 131072, L ~ U[65536, 131072], block 64",
+            "workload": f"decode: {dcfg.batch} seqs, 32/8 heads, d=128, bf16, cache 131072, L ~ U[65536, 131072], "
+                        "block 64",
             "us_per_step": dec["us"], "sparsity": dec["sparsity"], "summarize_ms": dec["summarize_ms"],
             "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / pk["hbm_gbs"], "traffic": None, "bytes_per_step": dec["bytes"],
@@ -514,6 +524,14 @@ def main():
         }
     print(json.dumps(line), flush=True)
     barrier(world)
+    finish(world)
+
+
+def finish(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
 
 
 if __name__ == "__main__":
