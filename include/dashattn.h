@@ -192,6 +192,32 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
                                size_t workspace_bytes, dash_stream_t stream);
 
 /*
+ * dash_attn_decode without a workspace argument.  The paper has no
+ * counterpart: this serves callers that may not allocate device memory
+ * while they run -- code inside another engine's execution hook (a serving
+ * runtime or graph-executor plugin) where allocation is forbidden or would
+ * stall the device, and programs that fix their device-memory budget at
+ * start-up.  The caller still passes inputs and outputs, exactly as for
+ * dash_attn_decode, and gets the same results.
+ *  - Scratch: one library-owned 16 MiB device array per GPU, held from the
+ *    time the library is loaded until the process exits.  Problems whose
+ *    dash_attn_decode_workspace_size() exceeds 16 MiB are refused with
+ *    DASH_ERR_UNSUPPORTED before anything is launched.
+ *  - The array is shared by all calls on a device and keeps the last call's
+ *    contents; calls whose GPU work overlaps (other streams or threads
+ *    without ordering) race and give wrong results.
+ *  - The first call on each device looks up the array's address; make that
+ *    first call before any stream capture.
+ *  - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *  - The status word it uses is the array's; dash_attn_get_device_status
+ *    cannot read it, so seqlens must be valid (1 <= seqlens[b] <= Lmax).
+ */
+dash_status_t dash_attn_decode_noalloc(const dash_tensor_t* q, const dash_tensor_t* kcache,
+                                       const dash_tensor_t* vcache, const int32_t* seqlens, const float* summaries,
+                                       int64_t t_cap, float alpha, int block, dash_tensor_t* out,
+                                       dash_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the device status word of a workspace
  * last used by dash_attn_fwd / dash_attn_decode / dash_attn_sparse /
  * dash_attn_route (each call clears it when it starts).  Returns DASH_OK,

@@ -44,6 +44,7 @@ EXPORTED = (
     "dash_attn_sparse_workspace_size",
     "dash_attn_sparse",
     "dash_attn_get_device_status",
+    "dash_attn_decode_noalloc",
 )
 
 
@@ -89,6 +90,7 @@ def _load() -> ctypes.CDLL:
         "dash_attn_sparse_workspace_size": (sz, [T, T, i32, i64]),
         "dash_attn_sparse": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, vp]),
         "dash_attn_get_device_status": (i32, [vp, vp]),
+        "dash_attn_decode_noalloc": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -278,6 +280,22 @@ def decode(q, kcache, vcache, seqlens, summaries, alpha: float, block: int, out=
     _check(_lib.dash_attn_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), seqlens.data_ptr(),
                                  summaries.data_ptr(), t_cap, alpha, block, ctypes.byref(od), ws.data_ptr(),
                                  ws.numel(), _stream(stream)))
+    return out
+
+
+def decode_noalloc(q, kcache, vcache, seqlens, summaries, alpha: float, block: int, out=None,
+                   stream=None) -> torch.Tensor:
+    """One decode step without a workspace (see dash_attn_decode_noalloc).
+
+    For callers that may not allocate device memory while they run: the
+    library keeps a fixed 16 MiB scratch array per GPU.  Only ``out`` is
+    allocated here when it is not given.  Concurrent calls on one device race.
+    """
+    out = torch.empty_like(q) if out is None else out
+    qd, kd, vd, od = _desc(q), _desc(kcache), _desc(vcache), _desc(out)
+    _check(_lib.dash_attn_decode_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), seqlens.data_ptr(),
+                                         summaries.data_ptr(), summaries.shape[2], alpha, block, ctypes.byref(od),
+                                         _stream(stream)))
     return out
 
 

@@ -194,6 +194,18 @@ dash_status_t check_fwd_shapes(const dash_tensor_t* q, const dash_tensor_t* k, c
 
 }  // namespace
 
+namespace dash {
+dash_status_t set_last_error(dash_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+}  // namespace dash
+
 extern "C" {
 
 int dash_attn_version(void) { return 100; }

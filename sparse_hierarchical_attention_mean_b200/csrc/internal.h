@@ -4,7 +4,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/dashattn.h"
+
 namespace dash {
+
+// Records the thread-local message returned by dash_attn_last_error().
+dash_status_t set_last_error(dash_status_t st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 
 struct DeviceStatus;
 
