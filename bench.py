@@ -270,7 +270,7 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk):
     cand = float(sum((p // cfg.block) for p in range(S))) * k.shape[2] * B
     sparsity = 1.0 - float(cnt.double().sum()) / cand
     achieved = flops / (seg[2] * 1e-3) / 1e12
-    traffic = profiled_traffic("sparse_prefill_mma_kernel", ["attn_prefill.cu", "common.cuh"])
+    traffic = profiled_traffic("sparse_prefill_tc_kernel", ["attn_prefill_tc.cu", "tc.cuh", "sparse_common.cuh", "common.cuh"])
 
     # end to end through the public API with host buffers
     hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
@@ -493,7 +493,7 @@ def main():
         "sparsity": pre["sparsity"],
         "stage_ms": {"pool": pre["seg_ms"][0], "route": pre["seg_ms"][1], "sparse_attention": pre["seg_ms"][2]},
         "roofline": {
-            "kernel": "sparse_prefill_mma_kernel (+ its union-list kernel)",
+            "kernel": "sparse_prefill_tc_kernel (+ its union-list kernel)",
             "bound": "tensor",
             "achieved": pre["achieved_tflops"],
             "peak": peak_tf,

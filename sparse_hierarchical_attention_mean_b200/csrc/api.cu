@@ -85,7 +85,7 @@ int num_sms() {
 
 // Workspace of dash_attn_fwd.
 struct FwdLayout {
-  size_t status, summ, idx, logp, cnt, ulist, ucnt, total;
+  size_t status, summ, idx, logp, cnt, ulist, umask, ucnt, usteps, total;
   int64_t T, n_tiles;
   int tile_pos;
 };
@@ -109,14 +109,18 @@ FwdLayout fwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, in
   off = align256(off + (size_t)B * Hkv * S * 4);
   L.ulist = off;
   off = align256(off + (size_t)B * Hkv * L.n_tiles * L.T * 4);
+  L.umask = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * L.T * 16);
   L.ucnt = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
+  L.usteps = off;
   off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
   L.total = off;
   return L;
 }
 
 struct SparseLayout {
-  size_t status, ulist, ucnt, total;
+  size_t status, ulist, umask, ucnt, usteps, total;
   int64_t n_tiles;
   int tile_pos;
 };
@@ -130,7 +134,11 @@ SparseLayout sparse_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int blo
   off = align256(off + sizeof(dash::DeviceStatus));
   L.ulist = off;
   off = align256(off + (size_t)B * Hkv * L.n_tiles * t_cap * 4);
+  L.umask = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * t_cap * 16);
   L.ucnt = off;
+  off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
+  L.usteps = off;
   off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
   L.total = off;
   return L;
@@ -331,9 +339,16 @@ size_t dash_attn_sparse_workspace_size(const dash_tensor_t* q, const dash_tensor
   return sparse_layout(q->b, q->s, q->h, k->h, block, t_cap).total;
 }
 
+struct TileLists {
+  int32_t* ulist;
+  uint4* umask;
+  int32_t* ucnt;
+  int32_t* usteps;
+};
+
 static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
                                 const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
-                                int causal, dash_tensor_t* out, int32_t* ulist, int32_t* ucnt, int tile_pos,
+                                int causal, dash_tensor_t* out, const TileLists& tl, int tile_pos,
                                 int64_t n_tiles, dash::DeviceStatus* status, cudaStream_t stream) {
   if (q->dtype != DASH_F32) {
     dash::UnionParams u{};
@@ -346,8 +361,10 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
     u.t_cap = t_cap;
     u.idx = idx;
     u.cnt = cnt;
-    u.ulist = ulist;
-    u.ucnt = ucnt;
+    u.ulist = tl.ulist;
+    u.umask = tl.umask;
+    u.ucnt = tl.ucnt;
+    u.usteps = tl.usteps;
     u.causal = causal ? 1 : 0;
     u.status = status;
     cudaError_t e = dash::launch_union(u, stream);
@@ -371,8 +388,10 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
   p.idx = idx;
   p.logp = logp;
   p.cnt = cnt;
-  p.ulist = ulist;
-  p.ucnt = ucnt;
+  p.ulist = tl.ulist;
+  p.umask = tl.umask;
+  p.ucnt = tl.ucnt;
+  p.usteps = tl.usteps;
   p.tile_pos = tile_pos;
   p.n_tiles = (int)n_tiles;
   p.status = status;
@@ -400,8 +419,10 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
-  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, out, at<int32_t>(workspace, L.ulist),
-                  at<int32_t>(workspace, L.ucnt), L.tile_pos, L.n_tiles, at<dash::DeviceStatus>(workspace, L.status), s);
+  const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
+                     at<int32_t>(workspace, L.usteps)};
+  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, out, tl, L.tile_pos, L.n_tiles,
+                  at<dash::DeviceStatus>(workspace, L.status), s);
   return st ? st : ok();
 }
 
@@ -429,8 +450,10 @@ dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   if ((st = dash_attn_route(q, summ, k->h, L.T, nullptr, alpha, block, causal, idx, logp, cnt, nullptr, nullptr,
                             nullptr, 0, stream)))
     return st;
-  st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, out, at<int32_t>(workspace, L.ulist),
-                  at<int32_t>(workspace, L.ucnt), L.tile_pos, L.n_tiles, at<dash::DeviceStatus>(workspace, L.status), s);
+  const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
+                     at<int32_t>(workspace, L.usteps)};
+  st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, out, tl, L.tile_pos, L.n_tiles,
+                  at<dash::DeviceStatus>(workspace, L.status), s);
   return st ? st : ok();
 }
 

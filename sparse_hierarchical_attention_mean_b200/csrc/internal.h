@@ -49,15 +49,17 @@ struct RouteParams {
 };
 cudaError_t launch_route_prefill(const RouteParams& p, cudaStream_t stream);
 
-// Union of the per-row block lists over each stage-2 tile of `tile_pos`
-// consecutive positions.
+// Work list of each stage-2 tile of `tile_pos` consecutive positions: the
+// union of the rows' selected blocks and the rows' own blocks, ascending.
 struct UnionParams {
   int B, S, Hkv, block, tile_pos, n_tiles;
   int64_t t_cap;
   const int32_t* idx;
   const int32_t* cnt;
   int32_t* ulist;  // [B, Hkv, n_tiles, t_cap]
+  uint4* umask;    // [B, Hkv, n_tiles, t_cap]: positions of the tile that selected the block
   int32_t* ucnt;   // [B, Hkv, n_tiles]
+  int32_t* usteps; // [B, Hkv, n_tiles]: 64-token steps of the tile
   int causal;
   DeviceStatus* status;  // invalid list entries are skipped and reported here
 };
@@ -74,13 +76,16 @@ struct SparseParams {
   const float* logp;
   const int32_t* cnt;
   const int32_t* ulist;
+  const uint4* umask;
   const int32_t* ucnt;
+  const int32_t* usteps;
   int tile_pos, n_tiles;
   DeviceStatus* status;
 };
 // rows per stage-2 tile for the tensor-core kernel
 int sparse_tile_positions(int G, int block);
 cudaError_t launch_sparse_prefill(const SparseParams& p, cudaStream_t stream);
+cudaError_t launch_sparse_prefill_tc(const SparseParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 struct DecodeParams {

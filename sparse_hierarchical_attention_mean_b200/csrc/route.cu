@@ -189,21 +189,24 @@ __global__ void __launch_bounds__(kThreads) route_prefill_kernel(RouteParams p, 
   }
 }
 
-// Union of the per-row lists of `tile_pos` consecutive positions.
+// Work list of a stage-2 tile of `tile_pos` consecutive positions: the union
+// of the rows' selected blocks and the rows' own (diagonal) blocks,
+// ascending; for each listed block, the bit mask of the tile positions that
+// selected it; and the number of 64-token steps the tile takes (the causal
+// diagonal's halves past the tile's last position are skipped).
 __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
-  extern __shared__ uint32_t mask[];
+  extern __shared__ uint4 pmask[];  // [t_cap]: bit p set if tile position p selected the block
   const int b = blockIdx.z, g = blockIdx.y, tile = blockIdx.x;
-  const int words = (int)((p.t_cap + 31) / 32);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int w = tid; w < words; w += kThreads) mask[w] = 0u;
+  for (int c = tid; c < p.t_cap; c += kThreads) pmask[c] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
   const int64_t bg = (int64_t)b * p.Hkv + g;
   const int pos0 = tile * p.tile_pos;
-  const int t = pos0 / p.block;
   const int n_blocks = (p.S + p.block - 1) / p.block;
   for (int pp = warp; pp < p.tile_pos; pp += kThreads / 32) {
     const int pos = pos0 + pp;
     if (pos >= p.S) break;
+    const int t = pos / p.block;
     const int64_t row = bg * p.S + pos;
     const int n = min(max(p.cnt[row], 0), (int)p.t_cap);
     const int32_t* idx = p.idx + row * p.t_cap;
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
       // a candidate is a block other than the own block (causal: an earlier one)
       const bool ok = c >= 0 && c != t && (p.causal ? c < t : c < n_blocks);
       if (ok) {
-        atomicOr(&mask[c >> 5], 1u << (c & 31));
+        atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (pp >> 5), 1u << (pp & 31));
       } else {
         raise_status(p.status, 1 /* DASH_ERR_INVALID_ARGUMENT */, 200);
       }
@@ -220,26 +223,36 @@ __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
   }
   __syncthreads();
   if (warp == 0) {
-    int32_t* out = p.ulist + (bg * p.n_tiles + tile) * p.t_cap;
-    int off = 0;
-    for (int w0 = 0; w0 < words; w0 += 32) {
-      uint32_t word = (w0 + lane < words) ? mask[w0 + lane] : 0u;
-      const int pc = __popc(word);
-      int incl = pc;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+    const int last = min(pos0 + p.tile_pos, p.S) - 1;
+    const int own_lo = pos0 / p.block, own_hi = last / p.block;
+    const int last_needed = p.causal ? last : p.S - 1;
+    const int64_t tix = bg * p.n_tiles + tile;
+    int32_t* out = p.ulist + tix * p.t_cap;
+    uint4* mout = p.umask + tix * p.t_cap;
+    int off = 0, steps = 0;
+    for (int c0 = 0; c0 < p.t_cap; c0 += 32) {
+      const int c = c0 + lane;
+      bool keep = false;
+      uint4 m = make_uint4(0u, 0u, 0u, 0u);
+      if (c < p.t_cap) {
+        m = pmask[c];
+        keep = (m.x | m.y | m.z | m.w) != 0u || (c >= own_lo && c <= own_hi);
       }
-      int k = off + incl - pc;
-      while (word) {
-        const int bit = __ffs(word) - 1;
-        out[k++] = (w0 + lane) * 32 + bit;
-        word &= word - 1u;
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      int st = 0;
+      if (keep) {
+        const int k = off + __popc(bal & ((1u << lane) - 1u));
+        out[k] = c;
+        mout[k] = m;
+        for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
       }
-      off += __shfl_sync(0xffffffffu, incl, 31);
+      steps += warp_sum_i(st);
+      off += __popc(bal);
     }
-    if (lane == 0) p.ucnt[bg * p.n_tiles + tile] = off;
+    if (lane == 0) {
+      p.ucnt[tix] = off;
+      p.usteps[tix] = steps;
+    }
   }
 }
 
@@ -282,7 +295,9 @@ cudaError_t launch_route_prefill(const RouteParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_union(const UnionParams& p, cudaStream_t stream) {
-  const size_t smem = (size_t)((p.t_cap + 31) / 32) * sizeof(uint32_t);
+  const size_t smem = (size_t)p.t_cap * sizeof(uint4);
+  cudaError_t e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(p.n_tiles, p.Hkv, p.B);
   union_kernel<<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();

@@ -1,0 +1,63 @@
+// Shared pieces of the stage-2 prefill kernels: the walk over a tile's work
+// list and the per-row prior bias.
+//
+// "Stage 2: prior-induced sparse softmax" of the DashAttention technical
+// summary: the logits get log g added, with g = 0 (bias -inf) on blocks the
+// routing gave no mass; the near-diagonal block has no summary and is always
+// included, here with the uniform-baseline prior log(1/N).
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dash {
+
+// Prior bias of one row for the tensor-core kernel: the tile's work list
+// carries, per block, the mask of tile positions that selected it, so a row
+// only needs its own log p_bar values in order; they are prefetched four
+// selections ahead to keep global-memory latency off the softmax path.
+struct RowPrior {
+  const float* lp;
+  int n, cur, bit, pos, t;
+  bool valid;
+  float beta;
+  float q0, q1, q2, q3;
+
+  __device__ __forceinline__ void init(const SparseParams& p, int64_t bg, int position, int pos_in_tile) {
+    pos = position;
+    bit = pos_in_tile;
+    valid = pos < p.S;
+    t = pos / p.block;
+    const int n_blocks = (p.S + p.block - 1) / p.block;
+    const int n_cand = p.causal ? t : n_blocks - 1;
+    beta = n_cand > 0 ? logf(1.0f / (float)n_cand) : 0.0f;
+    const int64_t row = bg * p.S + (valid ? pos : 0);
+    n = valid ? min(max(p.cnt[row], 0), (int)p.t_cap) : 0;
+    lp = p.logp + row * p.t_cap;
+    q0 = n > 0 ? __ldg(lp) : 0.f;
+    q1 = n > 1 ? __ldg(lp + 1) : 0.f;
+    q2 = n > 2 ? __ldg(lp + 2) : 0.f;
+    q3 = n > 3 ? __ldg(lp + 3) : 0.f;
+    cur = 4;
+  }
+  // natural-log bias of block c (-inf: masked); `mask` holds the tile
+  // positions that selected c
+  __device__ __forceinline__ float bias(int c, const uint4& mask) {
+    if (!valid) return kNegInf;
+    if (c == t) return beta;
+    const uint32_t w = bit < 32 ? mask.x : bit < 64 ? mask.y : bit < 96 ? mask.z : mask.w;
+    if (((w >> (bit & 31)) & 1u) == 0u) return kNegInf;
+    const float v = q0;
+    q0 = q1;
+    q1 = q2;
+    q2 = q3;
+    q3 = cur < n ? __ldg(lp + cur) : 0.f;
+    ++cur;
+    return v;
+  }
+  __device__ __forceinline__ bool masked(int c, int tok, int S, int causal) const {
+    return tok >= S || (causal && c == t && tok > pos);
+  }
+};
+
+}  // namespace dash
