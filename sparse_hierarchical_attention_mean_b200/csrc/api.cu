@@ -254,6 +254,76 @@ dash_status_t dash_attn_summarize(const dash_tensor_t* k, const int32_t* seqlens
   return ok();
 }
 
+}  // extern "C"
+
+namespace {
+
+struct TileLists {
+  int32_t* ulist;
+  uint4* umask;
+  int32_t* ucnt;
+  int32_t* usteps;
+};
+
+// Prefill routing.  f16/bf16 tiles whose logit row fits in TMEM run on the
+// tensor cores (and, when `tl` is given, also write the stage-2 work lists of
+// their tiles); the remaining positions, and fp32 inputs, run on the CUDA
+// cores.  Returns in *first_cuda_tile the first tile routed on the CUDA
+// cores (whose work lists still have to be built).
+dash_status_t run_route(const dash_tensor_t* q, const float* summaries, int64_t kv_heads, int64_t t_cap, float alpha,
+                        int block, int causal, int32_t* idx, float* logp, int32_t* cnt, float* tau, float* p_dense,
+                        const TileLists* tl, dash::DeviceStatus* status, cudaStream_t stream, int* first_cuda_tile) {
+  const int G = (int)(q->h / kv_heads);
+  dash::RouteParams p{};
+  p.q = view(q);
+  p.dtype = q->dtype;
+  p.B = (int)q->b;
+  p.S = (int)q->s;
+  p.H = (int)q->h;
+  p.Hkv = (int)kv_heads;
+  p.G = G;
+  p.D = (int)q->d;
+  p.block = block;
+  p.causal = causal ? 1 : 0;
+  p.alpha = alpha;
+  p.summaries = summaries;
+  p.t_cap = t_cap;
+  p.idx = idx;
+  p.logp = logp;
+  p.cnt = cnt;
+  p.tau = tau;
+  p.p_dense = p_dense;
+  p.status = status;
+  const int P = dash::sparse_tile_positions(G, block);
+  const int n_tiles = (int)((q->s + P - 1) / P);
+  const int n_blocks = (int)((q->s + block - 1) / block);
+  int split = 0;
+  if (q->dtype != DASH_F32) {
+    const int max_cols = dash::route_tc_max_cols();
+    if (causal) {
+      split = (int)(((int64_t)(max_cols + 1) * block) / P);
+      if (split > n_tiles) split = n_tiles;
+    } else {
+      split = n_blocks <= max_cols ? n_tiles : 0;
+    }
+    dash::TileOut to{};
+    if (tl) to = dash::TileOut{tl->ulist, tl->umask, tl->ucnt, tl->usteps, n_tiles};
+    cudaError_t e = dash::launch_route_prefill_tc(p, to, 0, split, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "route (tensor cores)");
+  }
+  p.pos_begin = split * P;
+  if (p.pos_begin < p.S) {
+    cudaError_t e = dash::launch_route_prefill(p, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "route");
+  }
+  if (first_cuda_tile) *first_cuda_tile = split;
+  return DASH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t dash_attn_route_workspace_size(const dash_tensor_t* q, int64_t kv_heads, int64_t t_cap, int decode) {
   if (check_tensor(q, "q") || check_group(q->h, kv_heads) || t_cap <= 0) return 0;
   if (!decode) return 0;
@@ -273,28 +343,9 @@ dash_status_t dash_attn_route(const dash_tensor_t* q, const float* summaries, in
     const int64_t T = (q->s + block - 1) / block;
     if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block)", (long long)t_cap);
     if (T > 4096) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per sequence");
-    dash::RouteParams p{};
-    p.q = view(q);
-    p.dtype = q->dtype;
-    p.B = (int)q->b;
-    p.S = (int)q->s;
-    p.H = (int)q->h;
-    p.Hkv = (int)kv_heads;
-    p.G = G;
-    p.D = (int)q->d;
-    p.block = block;
-    p.causal = causal ? 1 : 0;
-    p.alpha = alpha;
-    p.summaries = summaries;
-    p.t_cap = t_cap;
-    p.idx = idx;
-    p.logp = logp;
-    p.cnt = cnt;
-    p.tau = tau;
-    p.p_dense = p_dense;
-    cudaError_t e = dash::launch_route_prefill(p, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "route");
-    return ok();
+    st = run_route(q, summaries, kv_heads, t_cap, alpha, block, causal, idx, logp, cnt, tau, p_dense, nullptr,
+                   nullptr, (cudaStream_t)stream, nullptr);
+    return st ? st : ok();
   }
   if (q->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode-mode route needs q with s == 1");
   if (!causal) return fail(DASH_ERR_UNSUPPORTED, "decode-mode route is causal");
@@ -339,18 +390,12 @@ size_t dash_attn_sparse_workspace_size(const dash_tensor_t* q, const dash_tensor
   return sparse_layout(q->b, q->s, q->h, k->h, block, t_cap).total;
 }
 
-struct TileLists {
-  int32_t* ulist;
-  uint4* umask;
-  int32_t* ucnt;
-  int32_t* usteps;
-};
-
 static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
                                 const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
                                 int causal, dash_tensor_t* out, const TileLists& tl, int tile_pos,
-                                int64_t n_tiles, dash::DeviceStatus* status, cudaStream_t stream) {
-  if (q->dtype != DASH_F32) {
+                                int64_t n_tiles, int union_tile0, dash::DeviceStatus* status,
+                                cudaStream_t stream) {
+  if (q->dtype != DASH_F32 && union_tile0 < n_tiles) {
     dash::UnionParams u{};
     u.B = (int)q->b;
     u.S = (int)q->s;
@@ -358,6 +403,7 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
     u.block = block;
     u.tile_pos = tile_pos;
     u.n_tiles = (int)n_tiles;
+    u.tile0 = union_tile0;
     u.t_cap = t_cap;
     u.idx = idx;
     u.cnt = cnt;
@@ -421,7 +467,7 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
                      at<int32_t>(workspace, L.usteps)};
-  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, out, tl, L.tile_pos, L.n_tiles,
+  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, out, tl, L.tile_pos, L.n_tiles, 0,
                   at<dash::DeviceStatus>(workspace, L.status), s);
   return st ? st : ok();
 }
@@ -447,13 +493,15 @@ dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   int32_t* idx = at<int32_t>(workspace, L.idx);
   float* logp = at<float>(workspace, L.logp);
   int32_t* cnt = at<int32_t>(workspace, L.cnt);
-  if ((st = dash_attn_route(q, summ, k->h, L.T, nullptr, alpha, block, causal, idx, logp, cnt, nullptr, nullptr,
-                            nullptr, 0, stream)))
-    return st;
   const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
                      at<int32_t>(workspace, L.usteps)};
-  st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, out, tl, L.tile_pos, L.n_tiles,
-                  at<dash::DeviceStatus>(workspace, L.status), s);
+  dash::DeviceStatus* dst = at<dash::DeviceStatus>(workspace, L.status);
+  int first_cuda_tile = 0;
+  if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, nullptr, nullptr, &tl, dst, s,
+                      &first_cuda_tile)))
+    return st;
+  st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, out, tl, L.tile_pos, L.n_tiles, first_cuda_tile, dst,
+                  s);
   return st ? st : ok();
 }
 

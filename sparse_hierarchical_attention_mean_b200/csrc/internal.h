@@ -46,13 +46,32 @@ struct RouteParams {
   int32_t* cnt;  // [B, Hkv, S]
   float* tau;      // nullable [B, H, S]
   float* p_dense;  // nullable [B, H, S, t_cap]
+  int pos_begin;   // CUDA-core kernel: first position to route (a tile boundary)
+  DeviceStatus* status;  // nullable
 };
 cudaError_t launch_route_prefill(const RouteParams& p, cudaStream_t stream);
+
+// Stage-2 work lists written by the tensor-core routing kernel (null ulist:
+// not wanted).
+struct TileOut {
+  int32_t* ulist;
+  uint4* umask;
+  int32_t* ucnt;
+  int32_t* usteps;
+  int n_tiles;
+};
+// Tensor-core routing for f16/bf16 over tiles [tile0, tile0 + n_tiles) of
+// 128 / G positions; every tile must have at most route_tc_max_cols() logit
+// columns.
+int route_tc_max_cols();
+cudaError_t launch_route_prefill_tc(const RouteParams& p, const TileOut& to, int tile0, int n_tiles,
+                                    cudaStream_t stream);
 
 // Work list of each stage-2 tile of `tile_pos` consecutive positions: the
 // union of the rows' selected blocks and the rows' own blocks, ascending.
 struct UnionParams {
   int B, S, Hkv, block, tile_pos, n_tiles;
+  int tile0;  // first tile to build
   int64_t t_cap;
   const int32_t* idx;
   const int32_t* cnt;

@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(kThreads) route_prefill_kernel(RouteParams p, 
   const int b = blockIdx.z, g = blockIdx.y;
   const int G = p.G;
   const int rpos = R / G;
-  const int pos0 = blockIdx.x * rpos;
+  const int pos0 = p.pos_begin + blockIdx.x * rpos;
   const int t = pos0 / p.block;
   const int T_ = (p.S + p.block - 1) / p.block;
   const int N = p.causal ? t : T_ - 1;
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kThreads) route_prefill_kernel(RouteParams p, 
 // diagonal's halves past the tile's last position are skipped).
 __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
   extern __shared__ uint4 pmask[];  // [t_cap]: bit p set if tile position p selected the block
-  const int b = blockIdx.z, g = blockIdx.y, tile = blockIdx.x;
+  const int b = blockIdx.z, g = blockIdx.y, tile = p.tile0 + blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int c = tid; c < p.t_cap; c += kThreads) pmask[c] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
@@ -276,7 +276,9 @@ cudaError_t launch_route_typed(const RouteParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int rpos = R / p.G;
-  dim3 grid((p.S + rpos - 1) / rpos, p.Hkv, p.B);
+  const int n_pos = p.S - p.pos_begin;
+  if (n_pos <= 0) return cudaSuccess;
+  dim3 grid((n_pos + rpos - 1) / rpos, p.Hkv, p.B);
   kern<<<grid, kThreads, smem, stream>>>(p, R, CW);
   return cudaGetLastError();
 }
@@ -298,7 +300,8 @@ cudaError_t launch_union(const UnionParams& p, cudaStream_t stream) {
   const size_t smem = (size_t)p.t_cap * sizeof(uint4);
   cudaError_t e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_tiles, p.Hkv, p.B);
+  if (p.n_tiles - p.tile0 <= 0) return cudaSuccess;
+  dim3 grid(p.n_tiles - p.tile0, p.Hkv, p.B);
   union_kernel<<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }

@@ -1,0 +1,401 @@
+// Stage 1 for prefill on the tensor cores: routing logits (tcgen05 GEMM kept
+// in TMEM), alpha-entmax thresholds, GQA mean, per-row block lists and the
+// stage-2 work lists of each tile.
+//
+// "Stage 1: entmax chunk routing" of the DashAttention technical summary:
+// every query scores the chunk summaries, w = alpha-entmax(gamma z) gives a
+// sparse distribution whose support size depends on the input, and under
+// GQA the probabilities of the heads sharing a KV head are averaged into one
+// shared sparse support.  gamma = 1/sqrt(d).
+//
+// One CTA owns the same 128-row tile as the stage-2 kernel (128 / G
+// positions x G heads of one KV group).  Column c of the logit matrix is
+// block c; a row masks the blocks that are not its candidates (causal: c >= t;
+// otherwise its own block).
+//   Logits: A = the query rows in fp32 (bf16/f16 values are exact in tf32),
+//   B = the fp32 summaries split into a tf32 head and its exact fp32
+//   remainder (also fed as tf32), two kind::tf32 MMAs accumulated in fp32:
+//   about 21 significant bits of every summary reach the product, far below
+//   the 1e-4 selection band.  128 rows x up to 512 columns fill TMEM.
+//   Summaries stream through a double-buffered shared-memory stage that the
+//   four row warps fill (splitting and swizzling on the way); one thread
+//   issues the MMAs.
+//   Thresholds: thread r owns row r (= TMEM lane r) and runs the same Newton
+//   / exact-support solve as the CUDA-core routing kernel on its own row,
+//   reading the logits from TMEM.
+//   Output: per position, the blocks with p_bar > 0 in ascending order with
+//   log p_bar (ballot/popc per 32 columns), and per tile the union of those
+//   blocks plus the tile's own blocks, each with the mask of positions that
+//   selected it, and the tile's number of 64-token steps.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace dash {
+namespace {
+
+constexpr int kRows = 128;
+constexpr int kChunk = 64;          // candidates per B stage
+constexpr int kMaxCols = 512;       // TMEM columns
+constexpr int kWorkWarps = 12;      // loading, threshold and compaction warps
+constexpr int kMmaWarp = kWorkWarps;
+constexpr int kThreads = (kWorkWarps + 1) * 32;
+constexpr int kWork = kWorkWarps * 32;
+constexpr int kHalf = 64;           // rows whose logits sit in shared memory at once
+constexpr int kXStride = kMaxCols + 1;  // odd row stride: conflict-free column writes
+
+struct RBars {
+  uint64_t a_full;
+  uint64_t b_full[2];
+  uint64_t b_empty[2];
+  uint64_t x_ready;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+struct RLayout {
+  static constexpr int KC = D / 32;                 // 128-byte chunks of an fp32 row
+  static constexpr int kAChunk = kRows * 128;       // 16 KB
+  static constexpr int kBChunk = kChunk * 128;      // 8 KB
+  static constexpr int kBTerm = KC * kBChunk;       // one term of one stage
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + KC * kAChunk;  // [2 stages][hi, lo]
+  static constexpr int kGemmBytes = kOffB + 2 * 2 * kBTerm;
+  static constexpr int kXBytes = kHalf * kXStride * 4;  // logits of 64 rows (reuses the GEMM operands)
+  static constexpr int kOffMask = (kGemmBytes > kXBytes ? kGemmBytes : kXBytes);  // [512] uint4
+  static constexpr int kOffTau = kOffMask + kMaxCols * 16;                        // [128] fp32
+  static constexpr int kOffBar = kOffTau + kRows * 4;
+  static constexpr int kBytes = kOffBar + 128;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+// byte offset of 16-byte unit u of row r inside a 128-byte-swizzled chunk
+__device__ __forceinline__ int sw128(int r, int u) { return r * 128 + ((u ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ float4 tf32_head(float4 v) {
+  float4 h;
+  h.x = __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
+  h.y = __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
+  h.z = __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
+  h.w = __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
+  return h;
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// Instruction descriptor, kind::tf32 (A/B format 2), fp32 accumulate, K-major.
+constexpr uint32_t idesc_tf32(int m, int n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// Is logit column c a routing candidate of a row in block t?
+__device__ __forceinline__ bool is_cand(int c, int t, int n_blocks, int causal) {
+  return causal ? c < t : (c != t && c < n_blocks);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RouteParams p, TileOut to, int tile0) {
+  using L = RLayout<D>;
+  constexpr uint32_t kIdesc = idesc_tf32(kRows, kChunk);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  RBars* bars = reinterpret_cast<RBars*>(smem + L::kOffBar);
+  float* X = reinterpret_cast<float*>(smem);  // [kHalf][kXStride], after the GEMM
+  uint4* pmask = reinterpret_cast<uint4*>(smem + L::kOffMask);
+  float* tau_s = reinterpret_cast<float*>(smem + L::kOffTau);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, g = blockIdx.y, tile = tile0 + blockIdx.x;
+  const int G = p.G;
+  const int P = kRows / G;
+  const int pos0 = tile * P;
+  const int n_blocks = (p.S + p.block - 1) / p.block;
+  const int last = min(pos0 + P, p.S) - 1;
+  const int t_last = last / p.block;
+  const int n_cols = p.causal ? t_last : n_blocks;  // logit columns 0 .. n_cols-1
+  const int n_chunks = (n_cols + kChunk - 1) / kChunk;
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const float coef = (p.alpha - 1.0f) * rsqrtf((float)D);
+  const float pw = 1.0f / (p.alpha - 1.0f);
+  const int kind = entmax_kind(p.alpha);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bars->a_full, kWork);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->b_full[s], kWork);
+      tc::mbar_init(&bars->b_empty[s], 1);
+    }
+    tc::mbar_init(&bars->x_ready, 1);
+    bars->abort = 0;
+    tc::fence_barrier_init();
+  }
+  for (int c = threadIdx.x; c < kMaxCols; c += kThreads) pmask[c] = make_uint4(0u, 0u, 0u, 0u);
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(&bars->tmem_base, kMaxCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_chunks > 0) {
+      bool ok = tc::mbar_wait(&bars->a_full, 0);
+      for (int j = 0; ok && j < n_chunks; ++j) {
+        const int st = j & 1;
+        if (!tc::mbar_wait(&bars->b_full[st], (j >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint8_t* bh = smem + L::kOffB + (st * 2 + 0) * L::kBTerm;
+        const uint8_t* bl = smem + L::kOffB + (st * 2 + 1) * L::kBTerm;
+#pragma unroll
+        for (int term = 0; term < 2; ++term) {
+#pragma unroll
+          for (int kc = 0; kc < L::KC; ++kc) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = tc::smem_desc_sw128(smem + L::kOffA + kc * L::kAChunk + k * 32, 16, 1024);
+              const uint64_t bd = tc::smem_desc_sw128((term ? bl : bh) + kc * L::kBChunk + k * 32, 16, 1024);
+              mma_tf32(tmem + j * kChunk, ad, bd, kIdesc, (term | kc | k) ? 1u : 0u);
+            }
+          }
+        }
+        tc::mma_commit(&bars->b_empty[st]);
+      }
+      if (!ok) {
+        raise_status(p.status, 5 /* DASH_ERR_DEVICE_TIMEOUT */, 20);
+        atomicExch(&bars->abort, 1);
+      }
+      tc::mma_commit(&bars->x_ready);
+      tc::mbar_wait(&bars->x_ready, 0);
+    }
+  } else if (n_chunks > 0) {
+    // ------------------------------------------------------------ GEMM operands
+    bool ok = true;
+    if (threadIdx.x < kRows) {
+      // A: query row r in fp32, 128-byte swizzled
+      const int r = threadIdx.x;
+      const int pos = pos0 + r / G, head = g * G + r % G;
+      const bool valid = pos < p.S;
+      constexpr int EPV = 8;
+      const T* src = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb + (int64_t)(valid ? pos : 0) * p.q.ss +
+                     (int64_t)head * p.q.sh;
+#pragma unroll
+      for (int v = 0; v < D / EPV; ++v) {
+        float f[EPV];
+        if (valid) {
+          Elt<T>::to_float(__ldg(reinterpret_cast<const uint4*>(src + v * EPV)), f);
+        } else {
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) f[e] = 0.f;
+        }
+        const int kc = (v * EPV) / 32, u0 = ((v * EPV) % 32) / 4;
+        uint8_t* base = smem + L::kOffA + kc * L::kAChunk;
+        *reinterpret_cast<float4*>(base + sw128(r, u0)) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(base + sw128(r, u0 + 1)) = make_float4(f[4], f[5], f[6], f[7]);
+      }
+    }
+    tc::fence_proxy_async_smem();
+    tc::mbar_arrive(&bars->a_full);
+    // B: summaries of each candidate chunk, split into tf32 head + remainder
+    const float* sbase = p.summaries + bg * p.t_cap * D;
+    for (int j = 0; j < n_chunks; ++j) {
+      const int st = j & 1;
+      if (j >= 2 && !tc::mbar_wait(&bars->b_empty[st], ((j >> 1) - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      uint8_t* bh = smem + L::kOffB + (st * 2 + 0) * L::kBTerm;
+      uint8_t* bl = smem + L::kOffB + (st * 2 + 1) * L::kBTerm;
+      for (int i = threadIdx.x; i < kChunk * (D / 4); i += kWork) {
+        const int cand = i / (D / 4), k4 = i % (D / 4);
+        const int c = j * kChunk + cand;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c < n_cols) v = __ldg(reinterpret_cast<const float4*>(sbase + (int64_t)c * D) + k4);
+        const float4 h = tf32_head(v);
+        const float4 lo = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+        const int kc = k4 / 8, u = k4 % 8;
+        *reinterpret_cast<float4*>(bh + kc * L::kBChunk + sw128(cand, u)) = h;
+        *reinterpret_cast<float4*>(bl + kc * L::kBChunk + sw128(cand, u)) = lo;
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars->b_full[st]);
+    }
+    if (ok && !tc::mbar_wait(&bars->x_ready, 0)) ok = false;
+    tc::fence_after_sync();
+    if (!ok) {
+      raise_status(p.status, 5 /* DASH_ERR_DEVICE_TIMEOUT */, 21);
+      atomicExch(&bars->abort, 1);
+    }
+  }
+  __syncthreads();  // GEMM done: its shared memory now holds logits
+
+  // ---- two halves of 64 rows: TMEM -> shared, thresholds, compaction
+  const int n_wch = (n_cols + 31) / 32;  // 32-column chunks of the logit rows
+  for (int half = 0; half < 2; ++half) {
+    if (warp < kWorkWarps && n_chunks > 0 && !bars->abort) {
+      // warps whose TMEM lane quarter lies in this half copy (and scale) their rows
+      const int q4 = warp & 3;
+      if ((q4 >> 1) == half) {
+        const int r = q4 * 32 + lane;  // tile row = TMEM lane
+        const int pos = pos0 + r / G;
+        const int t = pos / p.block;
+        const bool valid = pos < p.S;
+        float* xr = X + (r - half * kHalf) * kXStride;
+        for (int ch = warp >> 2; ch < n_wch; ch += kWorkWarps / 4) {
+          uint32_t v[32];
+          tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + ch * 32, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = ch * 32 + j;
+            xr[c] = (valid && is_cand(c, t, n_blocks, p.causal)) ? coef * __uint_as_float(v[j]) : kNegInf;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (warp < kWorkWarps) {
+      // thresholds: one warp per row
+      for (int rr = warp; rr < kHalf; rr += kWorkWarps) {
+        const int r = half * kHalf + rr;
+        const int pos = pos0 + r / G;
+        const int t = pos / p.block;
+        const int n_row = pos >= p.S ? 0 : (p.causal ? t : n_blocks - 1);
+        float tau = 0.f;
+        if (n_row > 0) tau = warp_entmax_tau(X + rr * kXStride, p.causal ? t : n_blocks, p.alpha, lane);
+        if (lane == 0) tau_s[r] = tau;
+        if (p.tau && lane == 0 && pos < p.S) p.tau[((int64_t)b * p.H + g * G + r % G) * p.S + pos] = tau;
+      }
+    }
+    __syncthreads();
+    if (warp < kWorkWarps) {
+      // GQA mean and ascending lists: one warp per position of this half
+      const int pfirst = (half * kHalf) / G, pcount = kHalf / G;
+      for (int q = warp; q < pcount; q += kWorkWarps) {
+        const int tp = pfirst + q;  // tile position
+        const int pos = pos0 + tp;
+        if (pos >= p.S) continue;
+        const int t = pos / p.block;
+        const int n_row = p.causal ? t : n_blocks - 1;
+        const int ncol = p.causal ? t : n_blocks;
+        const int64_t row = bg * p.S + pos;
+        int32_t* idx = p.idx + row * p.t_cap;
+        float* logp = p.logp + row * p.t_cap;
+        int off = 0;
+        for (int c0 = 0; c0 < ncol && n_row > 0; c0 += 32) {
+          const int c = c0 + lane;
+          float pbar = 0.f;
+          if (c < ncol) {
+            for (int h = 0; h < G; ++h) {
+              const int rr = tp * G + h - half * kHalf;
+              const float u = X[rr * kXStride + c] - tau_s[tp * G + h];
+              const float ph = u > 0.f ? pow_pw(u, pw, kind) : 0.f;
+              pbar += ph;
+              if (p.p_dense) p.p_dense[(((int64_t)b * p.H + g * G + h) * p.S + pos) * p.t_cap + c] = ph;
+            }
+            pbar /= (float)G;
+          }
+          const bool sel = pbar > 0.f;
+          const unsigned m = __ballot_sync(0xffffffffu, sel);
+          if (sel) {
+            const int o = off + __popc(m & ((1u << lane) - 1u));
+            idx[o] = c;
+            logp[o] = logf(pbar);
+            atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (tp >> 5), 1u << (tp & 31));
+          }
+          off += __popc(m);
+        }
+        if (lane == 0) p.cnt[row] = off;
+        if (p.p_dense) {
+          const int from = n_row > 0 ? ncol : 0;
+          for (int h = 0; h < G; ++h) {
+            float* pd = p.p_dense + (((int64_t)b * p.H + g * G + h) * p.S + pos) * p.t_cap;
+            for (int c = from + lane; c < p.t_cap; c += 32) pd[c] = 0.f;
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- the tile's stage-2 work list
+  tc::fence_before_sync();
+  if (warp == 0 && to.ulist) {
+    const int own_lo = pos0 / p.block, own_hi = t_last;
+    const int last_needed = p.causal ? last : p.S - 1;
+    const int64_t tix = bg * to.n_tiles + tile;
+    int32_t* out = to.ulist + tix * p.t_cap;
+    uint4* mout = to.umask + tix * p.t_cap;
+    int off = 0, steps = 0;
+    const int span = max(n_cols, own_hi + 1);
+    for (int c0 = 0; c0 < span; c0 += 32) {
+      const int c = c0 + lane;
+      bool keep = false;
+      uint4 m = make_uint4(0u, 0u, 0u, 0u);
+      if (c < span) {
+        if (c < kMaxCols) m = pmask[c];
+        keep = (m.x | m.y | m.z | m.w) != 0u || (c >= own_lo && c <= own_hi);
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      int st = 0;
+      if (keep) {
+        const int k = off + __popc(bal & ((1u << lane) - 1u));
+        out[k] = c;
+        mout[k] = m;
+        for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
+      }
+      steps += warp_sum_i(st);
+      off += __popc(bal);
+    }
+    if (lane == 0) {
+      to.ucnt[tix] = off;
+      to.usteps[tix] = steps;
+    }
+  }
+  if (warp == kMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kMaxCols);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const RouteParams& p, const TileOut& to, int tile0, int n_tiles, cudaStream_t stream) {
+  using L = RLayout<D>;
+  auto kern = route_prefill_tc_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_tiles, p.Hkv, p.B);
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(p, to, tile0);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int route_tc_max_cols() { return kMaxCols; }
+
+cudaError_t launch_route_prefill_tc(const RouteParams& p, const TileOut& to, int tile0, int n_tiles,
+                                    cudaStream_t stream) {
+  if (n_tiles <= 0) return cudaSuccess;
+  if (p.D == 128) {
+    if (p.dtype == 1) return launch_t<__half, 128>(p, to, tile0, n_tiles, stream);
+    return launch_t<__nv_bfloat16, 128>(p, to, tile0, n_tiles, stream);
+  }
+  if (p.dtype == 1) return launch_t<__half, 64>(p, to, tile0, n_tiles, stream);
+  return launch_t<__nv_bfloat16, 64>(p, to, tile0, n_tiles, stream);
+}
+
+}  // namespace dash
