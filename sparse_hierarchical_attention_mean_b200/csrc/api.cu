@@ -85,8 +85,8 @@ int num_sms() {
 
 // Workspace of dash_attn_fwd.
 struct FwdLayout {
-  size_t status, summ, idx, logp, cnt, ulist, umask, ucnt, usteps, total;
-  int64_t T, n_tiles;
+  size_t status, summ, idx, logp, cnt, ulist, umask, ucnt, usteps, plist, pmask, pcnt, psteps, total;
+  int64_t T, n_tiles, n_pairs;
   int tile_pos;
 };
 
@@ -115,13 +115,22 @@ FwdLayout fwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, in
   off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
   L.usteps = off;
   off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
+  L.n_pairs = (L.n_tiles + 1) / 2;
+  L.plist = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * L.T * 4);
+  L.pmask = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * L.T * 32);
+  L.pcnt = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * 4);
+  L.psteps = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * 4);
   L.total = off;
   return L;
 }
 
 struct SparseLayout {
-  size_t status, ulist, umask, ucnt, usteps, total;
-  int64_t n_tiles;
+  size_t status, ulist, umask, ucnt, usteps, plist, pmask, pcnt, psteps, total;
+  int64_t n_tiles, n_pairs;
   int tile_pos;
 };
 
@@ -140,6 +149,15 @@ SparseLayout sparse_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int blo
   off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
   L.usteps = off;
   off = align256(off + (size_t)B * Hkv * L.n_tiles * 4);
+  L.n_pairs = (L.n_tiles + 1) / 2;
+  L.plist = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * t_cap * 4);
+  L.pmask = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * t_cap * 32);
+  L.pcnt = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * 4);
+  L.psteps = off;
+  off = align256(off + (size_t)B * Hkv * L.n_pairs * 4);
   L.total = off;
   return L;
 }
@@ -263,6 +281,11 @@ struct TileLists {
   uint4* umask;
   int32_t* ucnt;
   int32_t* usteps;
+  int32_t* plist;
+  uint4* pmask;
+  int32_t* pcnt;
+  int32_t* psteps;
+  int64_t n_pairs;
 };
 
 // Prefill routing.  f16/bf16 tiles whose logit row fits in TMEM run on the
@@ -416,6 +439,27 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
     cudaError_t e = dash::launch_union(u, stream);
     if (e != cudaSuccess) return cuda_fail(e, "union");
   }
+  if (q->dtype != DASH_F32) {
+    dash::PairParams pp{};
+    pp.B = (int)q->b;
+    pp.S = (int)q->s;
+    pp.Hkv = (int)k->h;
+    pp.block = block;
+    pp.tile_pos = tile_pos;
+    pp.n_tiles = (int)n_tiles;
+    pp.n_pairs = (int)tl.n_pairs;
+    pp.causal = causal ? 1 : 0;
+    pp.t_cap = t_cap;
+    pp.ulist = tl.ulist;
+    pp.umask = tl.umask;
+    pp.ucnt = tl.ucnt;
+    pp.plist = tl.plist;
+    pp.pmask = tl.pmask;
+    pp.pcnt = tl.pcnt;
+    pp.psteps = tl.psteps;
+    cudaError_t e = dash::launch_pairs(pp, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "pair lists");
+  }
   dash::SparseParams p{};
   p.q = view(q);
   p.k = view(k);
@@ -434,10 +478,11 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
   p.idx = idx;
   p.logp = logp;
   p.cnt = cnt;
-  p.ulist = tl.ulist;
-  p.umask = tl.umask;
-  p.ucnt = tl.ucnt;
-  p.usteps = tl.usteps;
+  p.plist = tl.plist;
+  p.pmask = tl.pmask;
+  p.pcnt = tl.pcnt;
+  p.psteps = tl.psteps;
+  p.n_pairs = (int)tl.n_pairs;
   p.tile_pos = tile_pos;
   p.n_tiles = (int)n_tiles;
   p.status = status;
@@ -466,7 +511,8 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
   cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
-                     at<int32_t>(workspace, L.usteps)};
+                     at<int32_t>(workspace, L.usteps), at<int32_t>(workspace, L.plist), at<uint4>(workspace, L.pmask),
+                     at<int32_t>(workspace, L.pcnt), at<int32_t>(workspace, L.psteps), L.n_pairs};
   st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, out, tl, L.tile_pos, L.n_tiles, 0,
                   at<dash::DeviceStatus>(workspace, L.status), s);
   return st ? st : ok();
@@ -494,7 +540,8 @@ dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   float* logp = at<float>(workspace, L.logp);
   int32_t* cnt = at<int32_t>(workspace, L.cnt);
   const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
-                     at<int32_t>(workspace, L.usteps)};
+                     at<int32_t>(workspace, L.usteps), at<int32_t>(workspace, L.plist), at<uint4>(workspace, L.pmask),
+                     at<int32_t>(workspace, L.pcnt), at<int32_t>(workspace, L.psteps), L.n_pairs};
   dash::DeviceStatus* dst = at<dash::DeviceStatus>(workspace, L.status);
   int first_cuda_tile = 0;
   if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, nullptr, nullptr, &tl, dst, s,

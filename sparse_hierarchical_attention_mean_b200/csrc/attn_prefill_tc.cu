@@ -6,22 +6,32 @@
 // included; the pages' kernel walks the active chunks of a FlashAttention
 // loop and adds the routing bias before the softmax.
 //
-// One CTA owns a tile of 128 rows = (128 / G positions) x (G heads of one KV
-// group), so each K/V block brought in serves every head of the group.  It
-// walks the tile's ascending work list (the union of its rows' selected
-// blocks plus the rows' own blocks) in 64-token steps.  Warp roles:
-//   warp 4      TMA producer: Q once, then K and V of each step into a
-//               3-stage ring (128-byte swizzle, the layout the MMA reads).
-//   warp 5      MMA issuer (one thread) and TMEM owner: S = Q K^T into one of
-//               two 64-column TMEM buffers, then O += P V into 128 TMEM
-//               columns once the softmax has written P.
-//   warps 0-3   softmax: thread r owns row r (= TMEM lane r).  It reads its
-//               64 logits from TMEM, adds its own prior bias (walking its own
-//               ascending block list), keeps the running max and sum, writes
-//               P (bf16/f16) to shared memory for the next MMA and finally
-//               normalises O.  O is rescaled in TMEM only when a row's max
-//               grows by more than 2^8, so P stays <= 256 and the result is
-//               exact (the final division uses the same reference max).
+// A tile is 128 rows = (128 / G positions) x (G heads of one KV group), so
+// each K/V block brought in serves every head of the group.  One CTA owns two
+// adjacent tiles and walks the ascending work list of the pair (the union of
+// both tiles' lists, each block with the mask of positions per tile that
+// selected it) in 64-token steps; while the softmax of one tile runs, the
+// tensor core works on the other's products.
+//
+// Tensor memory holds, per tile, the query rows (the A operand of S = Q K^T),
+// S, and O; P is written back over S (bf16/f16, two per column) and is the A
+// operand of O += P V.  Shared memory then only carries the K/V ring, so each
+// step reads 16 KB of K and 16 KB of V from it per tile.  Warp roles:
+//   warp 8      TMA producer: K and V of each step into a ring of stages
+//               (128-byte swizzle, the layout the MMA reads), publishing the
+//               step's block, first token and masks.
+//   warp 9      MMA issuer (one thread) and TMEM owner.  Per step and tile,
+//               in this order: O += P V of the previous step, then S = Q K^T
+//               of this step (in-order execution lets S overwrite P).
+//   warps 0-3   softmax of tile 0, warps 4-7 of tile 1: thread r owns row r
+//               (= TMEM lane r).  It first stores its query row into TMEM,
+//               then per step reads its 64 logits, adds the row's prior bias
+//               (log p_bar of the block if its position selected it,
+//               log(1/N) on its own block, else -inf), keeps the running max
+//               and sum, writes P into TMEM and finally normalises O.  O is
+//               rescaled in TMEM only when a row's max grows by more than 2^8,
+//               so P stays <= 256 and the result is exact (the final division
+//               uses the same reference max).
 // Every mbarrier wait is bounded; on expiry the kernel records
 // DASH_ERR_DEVICE_TIMEOUT in the workspace status word and winds down.
 #include <cuda.h>
@@ -38,48 +48,49 @@ namespace dash {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kStep = 64;      // tokens per step
-constexpr int kStages = 3;     // K/V ring depth
-constexpr int kThreads = 192;  // 4 softmax warps + producer + MMA
-constexpr int kTmemCols = 256;
-constexpr int kSCol = 0;    // two S buffers of 64 fp32 columns
-constexpr int kOCol = 128;  // O accumulator (D columns)
+constexpr int kTiles = 2;
+constexpr int kStep = 64;                   // tokens per step
+constexpr int kMaxStages = 8;               // bound of the K/V ring depth
+constexpr int kProducerWarp = 4 * kTiles;   // warp 8
+constexpr int kMmaWarp = kProducerWarp + 1; // warp 9
+constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kTmemCols = 512;
+// TMEM columns of tile t: Q at 256 t (D / 2 columns), S (and P over it) at
+// 256 t + 64, O at 256 t + 128 (D columns)
+constexpr int kTileCols = 256;
+constexpr int kSOff = 64;
+constexpr int kOOff = 128;
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
 struct Layout {
   static constexpr int KC = D / 64;               // 128-byte chunks of a row
-  static constexpr int kQChunk = kRows * 128;     // 16 KB
   static constexpr int kKVChunk = kStep * 128;    // 8 KB
   static constexpr int kKVBytes = KC * kKVChunk;  // one K (or V) stage
-  static constexpr int kPBytes = kRows * 128;     // 128 rows x 64 16-bit values
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + KC * kQChunk;
+  static constexpr int kStages = D == 128 ? 6 : 8;
+  static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffP = kOffV + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffP + 2 * kPBytes;
-  static constexpr int kBytes = kOffBar + 512;
+  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kBytes = kOffBar + 768;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-// What the producer tells the softmax warps about a step (one per ring stage).
+// What the producer tells the other roles about a step (one per ring stage).
 struct StepDesc {
   int c, tok0, first, pad;
-  uint4 mask;
+  uint4 mask[kTiles];
 };
 
 struct Bars {
-  uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t q_full;  // query rows stored into TMEM (256 arrivals)
+  uint64_t kv_full[kMaxStages];
+  uint64_t kv_empty[kMaxStages];
+  uint64_t s_full[kTiles];
+  uint64_t p_full[kTiles];
   uint64_t o_final;
   uint32_t tmem_base;
   int abort;
-  StepDesc desc[kStages];
+  StepDesc desc[kMaxStages];
 };
 
 __device__ __forceinline__ void fail_timeout(Bars* bars, DeviceStatus* st, int where) {
@@ -87,12 +98,14 @@ __device__ __forceinline__ void fail_timeout(Bars* bars, DeviceStatus* st, int w
   atomicExch(&bars->abort, 1);
 }
 
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, SparseParams p) {
+    sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                             SparseParams p) {
   using L = Layout<D>;
-  constexpr bool kBF16 = sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value;
+  constexpr int kStages = L::kStages;
+  constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescS = tc::idesc_f16(kRows, kStep, kBF16, false, false);
   constexpr uint32_t kIdescO = tc::idesc_f16(kRows, D, kBF16, false, true);
 
@@ -101,39 +114,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + L::kOffBar);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.z, g = blockIdx.y, tile = blockIdx.x;
+  const int b = blockIdx.z, g = blockIdx.y, pair = blockIdx.x;
   const int G = p.G;
-  const int P = p.tile_pos;  // 128 / G
-  const int pos0 = tile * P;
+  const int P = p.tile_pos;  // 128 / G positions per tile
+  const int pos0 = pair * kTiles * P;
   const int64_t bg = (int64_t)b * p.Hkv + g;
-  const int32_t* ulist = p.ulist + (bg * p.n_tiles + tile) * p.t_cap;
-  const int ucnt = p.ucnt[bg * p.n_tiles + tile];
-  const int n_steps = p.usteps[bg * p.n_tiles + tile];
-  const int last_pos = min(pos0 + P, p.S) - 1;
-  const int last_needed = p.causal ? last_pos : p.S - 1;
+  const int64_t pix = bg * p.n_pairs + pair;
+  const int32_t* plist = p.plist + pix * p.t_cap;
+  const uint4* pmask = p.pmask + pix * p.t_cap * kTiles;
+  const int pcnt = p.pcnt[pix];
+  const int n_steps = p.psteps[pix];
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(&bars->q_full, 1);
+    tc::mbar_init(&bars->q_full, kTiles * kRows);
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&bars->kv_full[s], 1);
       tc::mbar_init(&bars->kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->s_full[s], 1);
-      tc::mbar_init(&bars->s_free[s], 128);
-      tc::mbar_init(&bars->p_full[s], 128);
-      tc::mbar_init(&bars->pv_done[s], 1);
+    for (int t = 0; t < kTiles; ++t) {
+      tc::mbar_init(&bars->s_full[t], 1);
+      tc::mbar_init(&bars->p_full[t], kRows);
     }
     tc::mbar_init(&bars->o_final, 1);
     bars->abort = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(&bars->tmem_base, kTmemCols);
     tc::tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
-    tc::prefetch_tensormap(&tm_q);
+  if (warp == kProducerWarp && lane == 0) {
     tc::prefetch_tensormap(&tm_k);
     tc::prefetch_tensormap(&tm_v);
   }
@@ -142,30 +152,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    // The whole warp walks the work list 32 entries at a time (one coalesced
-    // load per lane); lane 0 issues the copies.
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&bars->q_full, L::KC * L::kQChunk);
-      for (int kc = 0; kc < L::KC; ++kc)
-        tc::tma_load_4d(smem + L::kOffQ + kc * L::kQChunk, &tm_q, &bars->q_full, kc * 64, g * G, pos0, b);
-    }
-    const uint4* umask = p.umask + (bg * p.n_tiles + tile) * p.t_cap;
+    // The whole warp walks the pair's work list 32 entries at a time (one
+    // coalesced load per lane); lane 0 issues the copies.
     const int spb = p.block / kStep;
+    const int last_needed = p.causal ? min(pos0 + kTiles * P, p.S) - 1 : p.S - 1;
     int i = 0;
     bool ok = true;
-    for (int u0 = 0; ok && u0 < ucnt; u0 += 32) {
-      const int my_c = u0 + lane < ucnt ? __ldg(ulist + u0 + lane) : 0;
-      const uint4 my_m = u0 + lane < ucnt ? __ldg(umask + u0 + lane) : make_uint4(0u, 0u, 0u, 0u);
-      const int nj = min(32, ucnt - u0);
+    for (int u0 = 0; ok && u0 < pcnt; u0 += 32) {
+      const bool have = u0 + lane < pcnt;
+      const int my_c = have ? __ldg(plist + u0 + lane) : 0;
+      const uint4 my_m0 = have ? __ldg(pmask + (u0 + lane) * kTiles) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 my_m1 = have ? __ldg(pmask + (u0 + lane) * kTiles + 1) : make_uint4(0u, 0u, 0u, 0u);
+      const int nj = min(32, pcnt - u0);
       for (int j = 0; ok && j < nj; ++j) {
         const int c = __shfl_sync(0xffffffffu, my_c, j);
-        uint4 m;
-        m.x = __shfl_sync(0xffffffffu, my_m.x, j);
-        m.y = __shfl_sync(0xffffffffu, my_m.y, j);
-        m.z = __shfl_sync(0xffffffffu, my_m.z, j);
-        m.w = __shfl_sync(0xffffffffu, my_m.w, j);
+        uint4 m0, m1;
+        m0.x = __shfl_sync(0xffffffffu, my_m0.x, j);
+        m0.y = __shfl_sync(0xffffffffu, my_m0.y, j);
+        m0.z = __shfl_sync(0xffffffffu, my_m0.z, j);
+        m0.w = __shfl_sync(0xffffffffu, my_m0.w, j);
+        m1.x = __shfl_sync(0xffffffffu, my_m1.x, j);
+        m1.y = __shfl_sync(0xffffffffu, my_m1.y, j);
+        m1.z = __shfl_sync(0xffffffffu, my_m1.z, j);
+        m1.w = __shfl_sync(0xffffffffu, my_m1.w, j);
         for (int h = 0; h < spb; ++h) {
           const int tok0 = c * p.block + h * kStep;
           if (tok0 > last_needed) continue;
@@ -179,7 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               d.c = c;
               d.tok0 = tok0;
               d.first = h == 0;
-              d.mask = m;
+              d.mask[0] = m0;
+              d.mask[1] = m1;
               tc::mbar_arrive_expect_tx(&bars->kv_full[st], 2 * L::kKVBytes);
               for (int kc = 0; kc < L::KC; ++kc) {
                 tc::tma_load_4d(smem + L::kOffK + st * L::kKVBytes + kc * L::kKVChunk, &tm_k, &bars->kv_full[st],
@@ -199,70 +211,100 @@ __global__ void __launch_bounds__(kThreads, 1)
       // let every issued copy land before the CTA can retire
       for (int j = (i > kStages ? i - kStages : 0); j < i; ++j)
         tc::mbar_wait(&bars->kv_full[j % kStages], (j / kStages) & 1);
-      tc::mbar_wait(&bars->q_full, 0);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = tc::mbar_wait(&bars->q_full, 0);
       if (!ok) fail_timeout(bars, p.status, 2);
-      auto issue_pv = [&](int j) -> bool {
-        const int pb = j & 1, st = j % kStages;
-        if (!tc::mbar_wait(&bars->p_full[pb], (j >> 1) & 1)) return false;
+      tc::fence_after_sync();
+      // O(t) += P(t) V of step j, A = P from TMEM (over S)
+      auto issue_pv = [&](int t, int j) -> bool {
+        if (!tc::mbar_wait(&bars->p_full[t], j & 1)) return false;
         tc::fence_after_sync();
+        const int st = j % kStages;
 #pragma unroll
         for (int k = 0; k < kStep / 16; ++k) {
-          const uint64_t ad = tc::smem_desc_sw128(smem + L::kOffP + pb * L::kPBytes + k * 32, 16, 1024);
           const uint64_t bd = tc::smem_desc_sw128(smem + L::kOffV + st * L::kKVBytes + k * 2048, L::kKVChunk, 1024);
-          tc::mma_f16_ss(tmem + kOCol, ad, bd, kIdescO, (j > 0 || k > 0) ? 1u : 0u);
+          tc::mma_f16_ts(tmem + t * kTileCols + kOOff, tmem + t * kTileCols + kSOff + k * 8, bd, kIdescO,
+                         (j > 0 || k > 0) ? 1u : 0u);
         }
-        tc::mma_commit(&bars->pv_done[pb]);
-        tc::mma_commit(&bars->kv_empty[st]);
         return true;
       };
       int i = 0;
       for (; ok && i < n_steps; ++i) {
-        const int st = i % kStages, sb = i & 1;
-        if (!tc::mbar_wait(&bars->kv_full[st], (i / kStages) & 1) ||
-            (i >= 2 && !tc::mbar_wait(&bars->s_free[sb], ((i >> 1) - 1) & 1))) {
+        const int st = i % kStages;
+        if (!tc::mbar_wait(&bars->kv_full[st], (i / kStages) & 1)) {
           fail_timeout(bars, p.status, 3);
           ok = false;
           break;
         }
         tc::fence_after_sync();
+        for (int t = 0; ok && t < kTiles; ++t) {
+          if (i >= 1 && !issue_pv(t, i - 1)) {
+            fail_timeout(bars, p.status, 4);
+            ok = false;
+            break;
+          }
+          // S(t) = Q(t) K^T, A = Q from TMEM
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t ad = tc::smem_desc_sw128(smem + L::kOffQ + (k >> 2) * L::kQChunk + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc_sw128(
-              smem + L::kOffK + st * L::kKVBytes + (k >> 2) * L::kKVChunk + (k & 3) * 32, 16, 1024);
-          tc::mma_f16_ss(tmem + kSCol + sb * kStep, ad, bd, kIdescS, k > 0 ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t bd = tc::smem_desc_sw128(
+                smem + L::kOffK + st * L::kKVBytes + (k >> 2) * L::kKVChunk + (k & 3) * 32, 16, 1024);
+            tc::mma_f16_ts(tmem + t * kTileCols + kSOff, tmem + t * kTileCols + k * 8, bd, kIdescS,
+                           k > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&bars->s_full[t]);
         }
-        tc::mma_commit(&bars->s_full[sb]);
-        if (i >= 1 && !issue_pv(i - 1)) {
-          fail_timeout(bars, p.status, 4);
-          ok = false;
-          break;
-        }
+        if (ok && i >= 1) tc::mma_commit(&bars->kv_empty[(i - 1) % kStages]);
       }
-      if (ok && i >= 1 && !issue_pv(i - 1)) fail_timeout(bars, p.status, 5);
+      if (ok && i >= 1) {
+        for (int t = 0; ok && t < kTiles; ++t)
+          if (!issue_pv(t, i - 1)) {
+            fail_timeout(bars, p.status, 5);
+            ok = false;
+          }
+      }
       // o_final arrives once every MMA issued above has completed
       tc::mma_commit(&bars->o_final);
       tc::mbar_wait(&bars->o_final, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-3)
-    const int r = threadIdx.x;
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    const int t = warp >> 2;  // tile
+    const int q4 = warp & 3;  // TMEM lane quarter
+    const int r = q4 * 32 + lane;
     RowPrior row;
-    row.init(p, bg, pos0 + r / G, r / G);
+    row.init(p, bg, pos0 + t * P + r / G, r / G);
     const int head = g * G + r % G;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + t * kTileCols;
     const float qk_scale = rsqrtf((float)D) * kLog2e;
-    uint8_t* prow = smem + L::kOffP + r * 128;
+    {
+      // the query row into TMEM: the raw 16-bit pairs are the packed columns
+      const T* src = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb +
+                     (int64_t)(row.valid ? row.pos : 0) * p.q.ss + (int64_t)head * p.q.sh;
+#pragma unroll
+      for (int cc = 0; cc < D / 64; ++cc) {
+        uint32_t w[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (row.valid) x = __ldg(reinterpret_cast<const uint4*>(src + cc * 64 + v * 8));
+          w[4 * v] = x.x;
+          w[4 * v + 1] = x.y;
+          w[4 * v + 2] = x.z;
+          w[4 * v + 3] = x.w;
+        }
+        tc::tmem_st32(tbase + cc * 32, w);
+      }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars->q_full);
+    }
     float m_used = kNegInf, lsum = 0.f, bias = kNegInf;
     bool ok = true;
-    int i = 0;
-    for (; i < n_steps; ++i) {
-      const int sb = i & 1, st = i % kStages;
+    for (int i = 0; i < n_steps; ++i) {
+      const int st = i % kStages;
       // the step's descriptor is published with its K/V copies
       if (!tc::mbar_wait(&bars->kv_full[st], (i / kStages) & 1)) {
         fail_timeout(bars, p.status, 10);
@@ -270,19 +312,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int c = bars->desc[st].c, tok0 = bars->desc[st].tok0;
-      if (bars->desc[st].first) bias = row.bias(c, bars->desc[st].mask);
-      if (!tc::mbar_wait(&bars->s_full[sb], (i >> 1) & 1)) {
+      if (bars->desc[st].first) bias = row.bias(c, bars->desc[st].mask[t]);
+      if (!tc::mbar_wait(&bars->s_full[t], i & 1)) {
         fail_timeout(bars, p.status, 6);
         ok = false;
         break;
       }
       tc::fence_after_sync();
       uint32_t sv[kStep];
-      tc::tmem_ld32(tmem + lane_base + kSCol + sb * kStep, sv);
-      tc::tmem_ld32(tmem + lane_base + kSCol + sb * kStep + 32, sv + 32);
+      tc::tmem_ld32(tbase + kSOff, sv);
+      tc::tmem_ld32(tbase + kSOff + 32, sv + 32);
       tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      tc::mbar_arrive(&bars->s_free[sb]);
 
       // valid columns of this row in this step: 0 when the row did not select
       // the block, fewer on the causal diagonal and at the ragged end
@@ -290,22 +330,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tok0 + kStep > p.S) n_valid = min(n_valid, p.S - tok0);
       if (p.causal && c == row.t) n_valid = min(n_valid, row.pos - tok0 + 1);
       const float b2 = bias * kLog2e;
-      if (n_valid == kStep) {
-#pragma unroll
-        for (int j = 0; j < kStep; ++j) sv[j] = __float_as_uint(fmaf(__uint_as_float(sv[j]), qk_scale, b2));
-      } else {
+      // The bias is constant over the step and the scale positive, so the
+      // row max of the logits is max(s) * scale + bias: take it on the raw
+      // scores (masked columns set to -inf first on the slow path).
+      if (n_valid < kStep) {
 #pragma unroll
         for (int j = 0; j < kStep; ++j)
-          sv[j] = __float_as_uint(j < n_valid ? fmaf(__uint_as_float(sv[j]), qk_scale, b2) : kNegInf);
+          if (j >= n_valid) sv[j] = __float_as_uint(kNegInf);
       }
-      // row max: a tree over 8 independent partial maxima
       float pm[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) pm[e] = __uint_as_float(sv[e]);
 #pragma unroll
       for (int j = 8; j < kStep; ++j) pm[j & 7] = fmaxf(pm[j & 7], __uint_as_float(sv[j]));
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      const float smax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      const float mx = n_valid > 0 ? fmaf(smax, qk_scale, b2) : kNegInf;
       float corr = 1.0f;
       bool resc = false;
       if (mx != kNegInf) {
@@ -317,58 +357,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           resc = true;
         }
       }
-      // P buffer sb is free once PV of step i-2 has completed
-      if (i >= 2 && !tc::mbar_wait(&bars->pv_done[sb], ((i >> 1) - 1) & 1)) {
-        fail_timeout(bars, p.status, 7);
-        ok = false;
-        break;
-      }
       if (__any_sync(0xffffffffu, resc)) {
-        // O is stable once PV of step i-1 has completed
-        if (i >= 1 && !tc::mbar_wait(&bars->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
-          fail_timeout(bars, p.status, 8);
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
+        // O is stable: the previous step's P V completed before this S
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t ov[32];
-          tc::tmem_ld32(tmem + lane_base + kOCol + cc * 32, ov);
+          const uint32_t ta = tbase + kOOff + cc * 32;
+          tc::tmem_ld32(ta, ov);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * corr);
-          tc::tmem_st32(tmem + lane_base + kOCol + cc * 32, ov);
+          tc::tmem_st32(ta, ov);
         }
-        tc::tmem_wait_st();
         lsum *= corr;
       }
-      // masked entries are -inf and give 2^-inf = 0; a row with nothing
-      // accumulated yet (m_used = -inf) writes zeros
-      const float msub = m_used == kNegInf ? 0.f : m_used;
-      uint8_t* pdst = prow + sb * L::kPBytes;
+      // p = 2^(s * scale + bias - m): one FMA and one ex2 per column; masked
+      // columns hold -inf and give 0, a row without a valid column writes zeros
+      const float off = n_valid > 0 ? b2 - m_used : kNegInf;
       float ps[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+      uint32_t pw[32];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = tc::ex2(__uint_as_float(sv[q * 8 + e]) - msub);
-          ps[e] += pv[e];
-        }
-        uint4 w;
-        w.x = pack2<T>(pv[0], pv[1]);
-        w.y = pack2<T>(pv[2], pv[3]);
-        w.z = pack2<T>(pv[4], pv[5]);
-        w.w = pack2<T>(pv[6], pv[7]);
-        *reinterpret_cast<uint4*>(pdst + ((q ^ (r & 7)) << 4)) = w;
+      for (int j = 0; j < kStep; j += 2) {
+        const float p0 = tc::ex2(fmaf(__uint_as_float(sv[j]), qk_scale, off));
+        const float p1 = tc::ex2(fmaf(__uint_as_float(sv[j + 1]), qk_scale, off));
+        ps[j & 7] += p0;
+        ps[(j + 1) & 7] += p1;
+        pw[j >> 1] = pack2<T>(p0, p1);
       }
       lsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      tc::fence_proxy_async_smem();
+      tc::tmem_st32(tbase + kSOff, pw);
+      tc::tmem_wait_st();
       tc::fence_before_sync();
-      tc::mbar_arrive(&bars->p_full[sb]);
+      tc::mbar_arrive(&bars->p_full[t]);
     }
     // ---- epilogue: O / l -> out
     if (ok && tc::mbar_wait(&bars->o_final, 0)) {
@@ -379,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t ov[32];
-        tc::tmem_ld32(tmem + lane_base + kOCol + cc * 32, ov);
+        tc::tmem_ld32(tbase + kOOff + cc * 32, ov);
         tc::tmem_wait_ld();
         if (row.valid) {
 #pragma unroll
@@ -400,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
@@ -440,21 +462,22 @@ bool make_map(CUtensorMap* map, const View& v, int dtype, int64_t B, int64_t S, 
 
 template <typename T, int D>
 cudaError_t launch_tc(const SparseParams& p, cudaStream_t stream) {
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, p.q, p.dtype, p.B, p.S, p.H, D, p.G, p.tile_pos) ||
-      !make_map(&mk, p.k, p.dtype, p.B, p.S, p.Hkv, D, 1, kStep) ||
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, p.k, p.dtype, p.B, p.S, p.Hkv, D, 1, kStep) ||
       !make_map(&mv, p.v, p.dtype, p.B, p.S, p.Hkv, D, 1, kStep))
     return cudaErrorInvalidValue;
   using L = Layout<D>;
   auto kern = sparse_prefill_tc_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_tiles, p.Hkv, p.B);
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, p);
+  dim3 grid(p.n_pairs, p.Hkv, p.B);
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(mk, mv, p);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+int sparse_tile_pair() { return kTiles; }
 
 cudaError_t launch_sparse_prefill_tc(const SparseParams& p, cudaStream_t stream) {
   if (p.D == 128) {

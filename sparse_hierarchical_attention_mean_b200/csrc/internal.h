@@ -94,15 +94,33 @@ struct SparseParams {
   const int32_t* idx;
   const float* logp;
   const int32_t* cnt;
+  const int32_t* plist;  // work lists of tile pairs (tensor-core kernel)
+  const uint4* pmask;    // [.., t_cap, 2]: per block, the selecting positions of each tile
+  const int32_t* pcnt;
+  const int32_t* psteps;
+  int tile_pos, n_tiles, n_pairs;
+  DeviceStatus* status;
+};
+// positions per stage-2 tile (tiles are 128 rows)
+int sparse_tile_positions(int G, int block);
+// tiles per CTA of the tensor-core stage-2 kernel
+int sparse_tile_pair();
+
+// Work list of each pair of adjacent tiles: the union of the two tiles'
+// lists, each block with both tiles' position masks, and the pair's number
+// of 64-token steps.
+struct PairParams {
+  int B, S, Hkv, block, tile_pos, n_tiles, n_pairs, causal;
+  int64_t t_cap;
   const int32_t* ulist;
   const uint4* umask;
   const int32_t* ucnt;
-  const int32_t* usteps;
-  int tile_pos, n_tiles;
-  DeviceStatus* status;
+  int32_t* plist;
+  uint4* pmask;
+  int32_t* pcnt;
+  int32_t* psteps;
 };
-// rows per stage-2 tile for the tensor-core kernel
-int sparse_tile_positions(int G, int block);
+cudaError_t launch_pairs(const PairParams& p, cudaStream_t stream);
 cudaError_t launch_sparse_prefill(const SparseParams& p, cudaStream_t stream);
 cudaError_t launch_sparse_prefill_tc(const SparseParams& p, cudaStream_t stream);
 

@@ -256,6 +256,61 @@ __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
   }
 }
 
+// Work list of a pair of adjacent stage-2 tiles (see internal.h).
+__global__ void __launch_bounds__(kThreads) pair_kernel(PairParams p) {
+  extern __shared__ uint4 pm2[];  // [t_cap][2] masks, then [t_cap] presence bits
+  uint32_t* pres = reinterpret_cast<uint32_t*>(pm2 + 2 * p.t_cap);
+  const int b = blockIdx.z, g = blockIdx.y, pair = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int c = tid; c < p.t_cap; c += kThreads) {
+    pm2[2 * c] = make_uint4(0u, 0u, 0u, 0u);
+    pm2[2 * c + 1] = make_uint4(0u, 0u, 0u, 0u);
+    pres[c] = 0u;
+  }
+  __syncthreads();
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  for (int t = 0; t < 2; ++t) {
+    const int tile = 2 * pair + t;
+    if (tile >= p.n_tiles) break;
+    const int64_t tix = bg * p.n_tiles + tile;
+    const int n = min(max(p.ucnt[tix], 0), (int)p.t_cap);
+    for (int e = tid; e < n; e += kThreads) {
+      const int c = p.ulist[tix * p.t_cap + e];
+      if (c < 0 || c >= p.t_cap) continue;
+      pm2[2 * c + t] = p.umask[tix * p.t_cap + e];
+      atomicOr(&pres[c], 1u << t);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int pos0 = pair * 2 * p.tile_pos;
+    const int last_needed = p.causal ? min(pos0 + 2 * p.tile_pos, p.S) - 1 : p.S - 1;
+    const int64_t pix = bg * p.n_pairs + pair;
+    int32_t* out = p.plist + pix * p.t_cap;
+    uint4* mout = p.pmask + pix * p.t_cap * 2;
+    int off = 0, steps = 0;
+    for (int c0 = 0; c0 < p.t_cap; c0 += 32) {
+      const int c = c0 + lane;
+      const bool keep = c < p.t_cap && pres[c] != 0u;
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      int st = 0;
+      if (keep) {
+        const int k = off + __popc(bal & ((1u << lane) - 1u));
+        out[k] = c;
+        mout[2 * k] = pm2[2 * c];
+        mout[2 * k + 1] = pm2[2 * c + 1];
+        for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
+      }
+      steps += warp_sum_i(st);
+      off += __popc(bal);
+    }
+    if (lane == 0) {
+      p.pcnt[pix] = off;
+      p.psteps[pix] = steps;
+    }
+  }
+}
+
 template <typename T, int D>
 cudaError_t launch_route_typed(const RouteParams& p, cudaStream_t stream) {
   const int T_ = (p.S + p.block - 1) / p.block;
@@ -303,6 +358,15 @@ cudaError_t launch_union(const UnionParams& p, cudaStream_t stream) {
   if (p.n_tiles - p.tile0 <= 0) return cudaSuccess;
   dim3 grid(p.n_tiles - p.tile0, p.Hkv, p.B);
   union_kernel<<<grid, kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pairs(const PairParams& p, cudaStream_t stream) {
+  const size_t smem = (size_t)p.t_cap * (2 * sizeof(uint4) + sizeof(uint32_t));
+  cudaError_t e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_pairs, p.Hkv, p.B);
+  pair_kernel<<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
