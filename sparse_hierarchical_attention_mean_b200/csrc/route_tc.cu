@@ -39,7 +39,7 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kChunk = 64;          // candidates per B stage
 constexpr int kMaxCols = 512;       // TMEM columns
-constexpr int kWorkWarps = 12;      // loading, threshold and compaction warps
+constexpr int kWorkWarps = 16;      // loading, threshold and compaction warps
 constexpr int kMmaWarp = kWorkWarps;
 constexpr int kThreads = (kWorkWarps + 1) * 32;
 constexpr int kWork = kWorkWarps * 32;
@@ -66,8 +66,7 @@ struct RLayout {
   static constexpr int kGemmBytes = kOffB + 2 * 2 * kBTerm;
   static constexpr int kXBytes = kHalf * kXStride * 4;  // logits of 64 rows (reuses the GEMM operands)
   static constexpr int kOffMask = (kGemmBytes > kXBytes ? kGemmBytes : kXBytes);  // [512] uint4
-  static constexpr int kOffTau = kOffMask + kMaxCols * 16;                        // [128] fp32
-  static constexpr int kOffBar = kOffTau + kRows * 4;
+  static constexpr int kOffBar = kOffMask + kMaxCols * 16;
   static constexpr int kBytes = kOffBar + 128;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -102,8 +101,107 @@ __device__ __forceinline__ bool is_cand(int c, int t, int n_blocks, int causal) 
   return causal ? c < t : (c != t && c < n_blocks);
 }
 
-template <typename T, int D>
+// alpha-entmax thresholds of RW rows that share their candidate columns,
+// solved in lockstep by one warp (their reductions interleave).  Row i's
+// logits are x[i * stride + c] for c < n, -inf on non-candidates.  Same
+// scheme as warp_entmax_tau: Newton from max - 1, where F >= 1, approaches
+// the root from below, and after every step the exact solution on the
+// current support is accepted when it is self-consistent.
+template <int RW>
+__device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride, int n, float alpha, int kind,
+                                                     int lane, float* tau) {
+  const float pw = 1.0f / (alpha - 1.0f);
+  float mx[RW];
+#pragma unroll
+  for (int i = 0; i < RW; ++i) mx[i] = kNegInf;
+  for (int c = lane; c < n; c += 32) {
+#pragma unroll
+    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], x[i * stride + c]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
+  }
+  bool done[RW];
+#pragma unroll
+  for (int i = 0; i < RW; ++i) {
+    tau[i] = mx[i] - 1.0f;
+    done[i] = mx[i] == kNegInf;
+  }
+  for (int it = 0; it < 100; ++it) {
+    float f[RW], a[RW], k[RW], umin[RW], fd[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) f[i] = a[i] = k[i] = fd[i] = 0.f, umin[i] = 3.0e38f;
+    for (int c = lane; c < n; c += 32) {
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        const float u = x[i * stride + c] - tau[i];
+        if (u > 0.f) {
+          k[i] += 1.f;
+          a[i] += u;
+          umin[i] = fminf(umin[i], u);
+          if (kind == 0) {
+            f[i] += u;
+          } else if (kind == 1) {
+            f[i] = fmaf(u, u, f[i]);
+          } else {
+            const float up = exp2f((pw - 1.0f) * log2f(u));
+            fd[i] += up;
+            f[i] = fmaf(up, u, f[i]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        f[i] += __shfl_xor_sync(0xffffffffu, f[i], o);
+        a[i] += __shfl_xor_sync(0xffffffffu, a[i], o);
+        k[i] += __shfl_xor_sync(0xffffffffu, k[i], o);
+        umin[i] = fminf(umin[i], __shfl_xor_sync(0xffffffffu, umin[i], o));
+        if (kind == 2) fd[i] += __shfl_xor_sync(0xffffffffu, fd[i], o);
+      }
+    }
+    bool all = true;
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+      if (!done[i]) {
+        if (kind == 0) {
+          const float delta = (f[i] - 1.0f) / k[i];
+          if (delta < umin[i]) {
+            tau[i] += fmaxf(delta, 0.0f);
+            done[i] = true;
+          } else {
+            tau[i] += delta;
+          }
+        } else if (kind == 1) {
+          const float disc = a[i] * a[i] - k[i] * (f[i] - 1.0f);
+          float delta = 3.0e38f;
+          if (disc >= 0.f) delta = (f[i] - 1.0f) / (a[i] + sqrtf(disc));
+          if (delta < umin[i]) {
+            tau[i] += fmaxf(delta, 0.0f);
+            done[i] = true;
+          } else {
+            tau[i] += (f[i] - 1.0f) / (2.0f * a[i]);
+          }
+        } else {
+          const float step = (f[i] - 1.0f) / (pw * fd[i]);
+          tau[i] += step;
+          if (fabsf(step) <= 1e-7f * fmaxf(1.0f, fabsf(tau[i]))) done[i] = true;
+        }
+      }
+      all = all && done[i];
+    }
+    if (all) break;
+  }
+}
+
+template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RouteParams p, TileOut to, int tile0) {
+  constexpr int RW = G > 4 ? G : 4;  // rows solved together by one warp
+  constexpr int PPT = RW / G;        // positions per warp task
   using L = RLayout<D>;
   constexpr uint32_t kIdesc = idesc_tf32(kRows, kChunk);
   extern __shared__ uint8_t smem_raw[];
@@ -111,12 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   RBars* bars = reinterpret_cast<RBars*>(smem + L::kOffBar);
   float* X = reinterpret_cast<float*>(smem);  // [kHalf][kXStride], after the GEMM
   uint4* pmask = reinterpret_cast<uint4*>(smem + L::kOffMask);
-  float* tau_s = reinterpret_cast<float*>(smem + L::kOffTau);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z, g = blockIdx.y, tile = tile0 + blockIdx.x;
-  const int G = p.G;
-  const int P = kRows / G;
+  constexpr int P = kRows / G;
   const int pos0 = tile * P;
   const int n_blocks = (p.S + p.block - 1) / p.block;
   const int last = min(pos0 + P, p.S) - 1;
@@ -269,62 +365,63 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
     }
     __syncthreads();
     if (warp < kWorkWarps) {
-      // thresholds: one warp per row
-      for (int rr = warp; rr < kHalf; rr += kWorkWarps) {
-        const int r = half * kHalf + rr;
-        const int pos = pos0 + r / G;
-        const int t = pos / p.block;
-        const int n_row = pos >= p.S ? 0 : (p.causal ? t : n_blocks - 1);
-        float tau = 0.f;
-        if (n_row > 0) tau = warp_entmax_tau(X + rr * kXStride, p.causal ? t : n_blocks, p.alpha, lane);
-        if (lane == 0) tau_s[r] = tau;
-        if (p.tau && lane == 0 && pos < p.S) p.tau[((int64_t)b * p.H + g * G + r % G) * p.S + pos] = tau;
-      }
-    }
-    __syncthreads();
-    if (warp < kWorkWarps) {
-      // GQA mean and ascending lists: one warp per position of this half
-      const int pfirst = (half * kHalf) / G, pcount = kHalf / G;
-      for (int q = warp; q < pcount; q += kWorkWarps) {
-        const int tp = pfirst + q;  // tile position
-        const int pos = pos0 + tp;
-        if (pos >= p.S) continue;
-        const int t = pos / p.block;
-        const int n_row = p.causal ? t : n_blocks - 1;
+      // one warp per task of RW rows (PPT positions x G heads): thresholds in
+      // lockstep, then the GQA mean and the ascending list of each position
+      constexpr int kTasks = kHalf / RW;
+      for (int task = warp; task < kTasks; task += kWorkWarps) {
+        const int rr0 = task * RW;                 // first row within the half
+        const int tp0 = (half * kHalf + rr0) / G;  // first tile position
+        const int pos = pos0 + tp0;
+        const int t = pos / p.block;  // the task's positions share their block
         const int ncol = p.causal ? t : n_blocks;
-        const int64_t row = bg * p.S + pos;
-        int32_t* idx = p.idx + row * p.t_cap;
-        float* logp = p.logp + row * p.t_cap;
-        int off = 0;
-        for (int c0 = 0; c0 < ncol && n_row > 0; c0 += 32) {
-          const int c = c0 + lane;
-          float pbar = 0.f;
-          if (c < ncol) {
-            for (int h = 0; h < G; ++h) {
-              const int rr = tp * G + h - half * kHalf;
-              const float u = X[rr * kXStride + c] - tau_s[tp * G + h];
-              const float ph = u > 0.f ? pow_pw(u, pw, kind) : 0.f;
-              pbar += ph;
-              if (p.p_dense) p.p_dense[(((int64_t)b * p.H + g * G + h) * p.S + pos) * p.t_cap + c] = ph;
-            }
-            pbar /= (float)G;
-          }
-          const bool sel = pbar > 0.f;
-          const unsigned m = __ballot_sync(0xffffffffu, sel);
-          if (sel) {
-            const int o = off + __popc(m & ((1u << lane) - 1u));
-            idx[o] = c;
-            logp[o] = logf(pbar);
-            atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (tp >> 5), 1u << (tp & 31));
-          }
-          off += __popc(m);
-        }
-        if (lane == 0) p.cnt[row] = off;
-        if (p.p_dense) {
-          const int from = n_row > 0 ? ncol : 0;
+        float tau[RW];
+        warp_entmax_tau_rows<RW>(X + rr0 * kXStride, kXStride, ncol, p.alpha, kind, lane, tau);
+#pragma unroll
+        for (int pp = 0; pp < PPT; ++pp) {
+          const int tp = tp0 + pp;
+          const int qpos = pos0 + tp;
+          if (qpos >= p.S) continue;
+          const int n_row = p.causal ? t : n_blocks - 1;
+#pragma unroll
           for (int h = 0; h < G; ++h) {
-            float* pd = p.p_dense + (((int64_t)b * p.H + g * G + h) * p.S + pos) * p.t_cap;
-            for (int c = from + lane; c < p.t_cap; c += 32) pd[c] = 0.f;
+            if (n_row == 0) tau[pp * G + h] = 0.f;
+            if (p.tau && lane == 0) p.tau[((int64_t)b * p.H + g * G + h) * p.S + qpos] = tau[pp * G + h];
+          }
+          const int64_t row = bg * p.S + qpos;
+          int32_t* idx = p.idx + row * p.t_cap;
+          float* logp = p.logp + row * p.t_cap;
+          int off = 0;
+          for (int c0 = 0; c0 < ncol && n_row > 0; c0 += 32) {
+            const int c = c0 + lane;
+            float pbar = 0.f;
+            if (c < ncol) {
+#pragma unroll
+              for (int h = 0; h < G; ++h) {
+                const float u = X[(rr0 + pp * G + h) * kXStride + c] - tau[pp * G + h];
+                const float ph = u > 0.f ? pow_pw(u, pw, kind) : 0.f;
+                pbar += ph;
+                if (p.p_dense) p.p_dense[(((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap + c] = ph;
+              }
+              pbar *= 1.0f / (float)G;
+            }
+            const bool sel = pbar > 0.f;
+            const unsigned m = __ballot_sync(0xffffffffu, sel);
+            if (sel) {
+              const int o = off + __popc(m & ((1u << lane) - 1u));
+              idx[o] = c;
+              logp[o] = logf(pbar);
+              atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (tp >> 5), 1u << (tp & 31));
+            }
+            off += __popc(m);
+          }
+          if (lane == 0) p.cnt[row] = off;
+          if (p.p_dense) {
+            const int from = n_row > 0 ? ncol : 0;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              float* pd = p.p_dense + (((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap;
+              for (int c = from + lane; c < p.t_cap; c += 32) pd[c] = 0.f;
+            }
           }
         }
       }
@@ -372,15 +469,25 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   }
 }
 
-template <typename T, int D>
-cudaError_t launch_t(const RouteParams& p, const TileOut& to, int tile0, int n_tiles, cudaStream_t stream) {
+template <typename T, int D, int G>
+cudaError_t launch_g(const RouteParams& p, const TileOut& to, int tile0, int n_tiles, cudaStream_t stream) {
   using L = RLayout<D>;
-  auto kern = route_prefill_tc_kernel<T, D>;
+  auto kern = route_prefill_tc_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(n_tiles, p.Hkv, p.B);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(p, to, tile0);
   return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const RouteParams& p, const TileOut& to, int tile0, int n_tiles, cudaStream_t stream) {
+  switch (p.G) {
+    case 1: return launch_g<T, D, 1>(p, to, tile0, n_tiles, stream);
+    case 2: return launch_g<T, D, 2>(p, to, tile0, n_tiles, stream);
+    case 4: return launch_g<T, D, 4>(p, to, tile0, n_tiles, stream);
+    default: return launch_g<T, D, 8>(p, to, tile0, n_tiles, stream);
+  }
 }
 
 }  // namespace
