@@ -138,7 +138,8 @@ class ClockSampler:
 # --------------------------------------------------------------------------- distributed
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU under torchrun; NCCL on GPUs, gloo for CPU-only runs."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -147,9 +148,13 @@ def dist_setup(n_gpus: int):
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -167,9 +172,20 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(cfg, rank: int) -> int:
+    """Each rank processes its own independent sequence (weak scaling)."""
+    return cfg.seed + rank
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 # --------------------------------------------------------------------------- prefill (ours)
@@ -205,7 +221,7 @@ def union_flops(cfg, idx: torch.Tensor, cnt: torch.Tensor, tile_pos: int) -> flo
 
 
 def run_prefill(dash, cfg, steps, warmup, world, rank, pk):
-    inp = full_inputs(cfg, device="cuda", seed=cfg.seed + rank)
+    inp = full_inputs(cfg, device="cuda", seed=rank_seed(cfg, rank))
     q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
     B, S, H, d = q.shape
     T = -(-S // cfg.block)
@@ -308,7 +324,7 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk):
 
 
 def run_decode(dash, cfg, steps, warmup, world, rank):
-    inp = full_inputs(cfg, device="cuda", seed=cfg.seed + rank)
+    inp = full_inputs(cfg, device="cuda", seed=rank_seed(cfg, rank))
     q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
     B, _, H, d = q.shape
     Hkv = k.shape[2]
@@ -471,7 +487,7 @@ def main():
         barrier(world)
         finish(world)
         return
-    value = pre["tokens"] * world / (pre["ms"] * 1e-3)
+    value = job_throughput(pre["tokens"], world, pre["ms"])
     peak_tf = pk["bf16_tflops"]
     line = {
         "metric": METRIC,
@@ -504,7 +520,7 @@ def main():
             "selected_flops": pre["flops"],
             "union_inflation": pre["union_flops"] / pre["flops"],
         },
-        "e2e": {"value": pre["tokens"] * world / (pre["e2e_ms"] * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(pre["tokens"], world, pre["e2e_ms"]), "unit": "tokens/s",
                 "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"]},
         "gpu_launches": 4 * args.steps,
         "clocks": pre["clocks"],
