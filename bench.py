@@ -92,18 +92,27 @@ class ClockSampler:
         self.idx = device_index
         self.proc = None
         self.path = os.path.join("/tmp", f"dash_clocks_{os.getpid()}.csv")
+        self.t_mark = None
+        self.t_end = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         time.sleep(0.3)
         return self
 
+    def mark(self):
+        """Start of the timed region (samples from here on are the ones reported)."""
+        self.t_mark = time.time()
+
     def __exit__(self, *exc):
+        self.t_end = time.time()
+        time.sleep(0.05)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -114,25 +123,34 @@ class ClockSampler:
     def summary(self) -> dict:
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, mx, reasons = [], [], set()
+        import datetime
+
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+        # samples inside the timed region; the warm-up (same work) if it was too short to catch one
+        timed = [r for r in rows if self.t_mark is not None and self.t_mark <= r[0] <= (self.t_end or 1e30)]
+        window = "timed"
+        if not timed:
+            timed = [r for r in rows if r[1] > 0.5 * max((x[1] for x in rows), default=0.0)]
+            window = "warm-up and timed (timed region shorter than the sampling interval)"
+        if not timed:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        for r in timed:
+            for n, v in zip(names, r[3]):
                 if v.lower() == "active":
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": float(np.median([r[1] for r in timed])), "sm_max_mhz": max(r[2] for r in timed),
+                "reasons": sorted(reasons), "samples": len(timed), "window": window}
 
 
 # --------------------------------------------------------------------------- distributed
@@ -232,13 +250,14 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk):
     def step():
         dash.fwd(q, k, v, w, cfg.alpha, cfg.block, True, out=out, workspace=ws)
 
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.mark()
         ev0.record(stream)
         for _ in range(steps):
             step()
@@ -288,36 +307,66 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk):
     achieved = flops / (seg[2] * 1e-3) / 1e12
     traffic = profiled_traffic("sparse_prefill_tc_kernel", ["attn_prefill_tc.cu", "tc.cuh", "sparse_common.cuh", "common.cuh"])
 
-    # end to end through the public API with host buffers
-    hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dash.fwd(dq, dk, dv, w, cfg.alpha, cfg.block, True, out=out, workspace=ws)
-        hout.copy_(out, non_blocking=True)
-
-    for _ in range(max(1, warmup)):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record(stream)
-    for _ in range(steps):
-        e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, world)
-    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
-    d2h = out.numel() * out.element_size()
+    # End to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory and reads its output back.  Copies
+    # run on their own streams, double-buffered, so step i+1's upload and
+    # step i-1's download overlap step i's kernels.
+    e2e_ms, h2d, d2h = run_e2e(dash, cfg, q, k, v, w, ws, steps, warmup, world)
+    del ws
 
     return {
         "ms": ms, "tokens": B * S, "status": status, "seg_ms": seg.tolist(), "flops": flops, "union_flops": uflops,
         "sparsity": sparsity, "achieved_tflops": achieved, "traffic": traffic, "clocks": clk.summary(),
         "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
     }
+
+
+def run_e2e(dash, cfg, q, k, v, w, ws, steps, warmup, world):
+    hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+    hout = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+    dev = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(q)) for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, comp_done, out_free = [ev() for _ in range(2)], [ev() for _ in range(2)], [ev() for _ in range(2)]
+    for e in comp_done + out_free:
+        e.record(comp)
+
+    def e2e_step(i):
+        sl = i & 1
+        dq, dk, dv, dout = dev[sl]
+        up.wait_event(comp_done[sl])  # the slot's previous step no longer reads its inputs
+        with torch.cuda.stream(up):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+        in_ready[sl].record(up)
+        comp.wait_event(in_ready[sl])
+        comp.wait_event(out_free[sl])  # the slot's previous output has been read back
+        dash.fwd(dq, dk, dv, w, cfg.alpha, cfg.block, True, out=dout, workspace=ws)
+        comp_done[sl].record(comp)
+        down.wait_event(comp_done[sl])
+        with torch.cuda.stream(down):
+            hout[sl].copy_(dout, non_blocking=True)
+        out_free[sl].record(down)
+
+    for i in range(max(1, warmup)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(up)
+    for i in range(steps):
+        e2e_step(i)
+    down.wait_stream(comp)
+    down.wait_stream(up)
+    t1.record(down)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
+    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
+    d2h = q.numel() * q.element_size()
+    return e2e_ms, h2d, d2h
 
 
 # --------------------------------------------------------------------------- decode (ours)
@@ -345,12 +394,13 @@ def run_decode(dash, cfg, steps, warmup, world, rank):
     def step():
         dash.decode(q, k, v, sl, summ, cfg.alpha, cfg.block, out=out, workspace=ws)
 
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.mark()
         e0.record(stream)
         for _ in range(steps):
             step()
@@ -413,7 +463,7 @@ def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0) -> dict
     per_row = row_t / max(n_done, 1)  # one position of one KV group (G heads)
     full_s = pool_t / cfg.kv_heads * cfg.kv_heads + per_row * cfg.seq * cfg.kv_heads
     return {"full_s": full_s, "tokens_per_s": cfg.seq / full_s, "rows": n_done, "wall_s": time.perf_counter() - t_start,
-            "sample": f"{n_done} (position, KV group) rows spread over the 32K sequence + pooling of all "
+            "sample": f"{n_done} (position, KV group) rows spread over the {cfg.seq}-token sequence + pooling of all "
                       f"{cfg.kv_heads} KV heads, extrapolated to {cfg.seq} positions x {cfg.kv_heads} groups"}
 
 
@@ -431,9 +481,13 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=64, help="sequences in the decode workload (64 = full)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--seq", type=int, default=None,
+                    help="prefill sequence length override (smaller cases for profiling; default 32768)")
     args = ap.parse_args()
     warmup = max(3, args.warmup)
     cfg = get_config("prefill")
+    if args.seq is not None:
+        cfg = cfg.with_(seq=args.seq)
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -452,7 +506,8 @@ def main():
             "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": warmup, "ms_per_step": full_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "prefill 32K GQA bf16 inputs (B=1, 32/8 heads, d=128, block 64, alpha 1.5)",
+            "config": {"workload": f"prefill GQA bf16 inputs (B=1, S={cfg.seq}, 32/8 heads, d=128, block 64, "
+                                   "alpha 1.5)",
                        "global_batch": 1, "seq_len": cfg.seq, "parallelism": "host oracle, 1 thread"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": samples["sample"] + "; each step one such sample"},
@@ -470,7 +525,7 @@ def main():
     dec = None
     dcfg = get_config("decode").with_(batch=args.decode_batch)
     if not args.skip_decode:
-        dec = run_decode(dash, dcfg, max(5, args.steps), warmup, world, rank)
+        dec = run_decode(dash, dcfg, max(20, args.steps), warmup, world, rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
@@ -502,7 +557,7 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "prefill 32K GQA: B=1, S=32768, 32 q / 8 kv heads, d=128, bf16, causal, "
+        "config": {"workload": f"prefill GQA: B=1, S={cfg.seq}, 32 q / 8 kv heads, d=128, bf16, causal, "
                                "block 64, alpha 1.5, topic-planted keys (~75% block sparsity)",
                    "global_batch": world, "seq_len": cfg.seq, "parallelism": f"dp{world} (independent sequences)",
                    "l2": "inputs larger than L2 (q 268 MB, k+v 134 MB); no flush"},

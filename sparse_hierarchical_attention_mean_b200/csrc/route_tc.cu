@@ -66,7 +66,8 @@ struct RLayout {
   static constexpr int kGemmBytes = kOffB + 2 * 2 * kBTerm;
   static constexpr int kXBytes = kHalf * kXStride * 4;  // logits of 64 rows (reuses the GEMM operands)
   static constexpr int kOffMask = (kGemmBytes > kXBytes ? kGemmBytes : kXBytes);  // [512] uint4
-  static constexpr int kOffBar = kOffMask + kMaxCols * 16;
+  static constexpr int kOffList = kOffMask + kMaxCols * 16;  // per 32-column chunk: entries, steps [2][32]
+  static constexpr int kOffBar = kOffList + 2 * 32 * 4;
   static constexpr int kBytes = kOffBar + 128;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -306,26 +307,44 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
     }
     tc::fence_proxy_async_smem();
     tc::mbar_arrive(&bars->a_full);
-    // B: summaries of each candidate chunk, split into tf32 head + remainder
+    // B: summaries of each candidate chunk, split into tf32 head + remainder.
+    // The loads of chunk j + 1 are issued before chunk j is stored, so their
+    // latency overlaps the wait for a free stage and the stores.
     const float* sbase = p.summaries + bg * p.t_cap * D;
+    constexpr int EPT = kChunk * (D / 4) / kWork;  // float4 per thread and chunk
+    static_assert(EPT * kWork == kChunk * (D / 4), "chunk not divisible among the loading threads");
+    auto load_chunk = [&](int j, float4* v) {
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        const int i = threadIdx.x + e * kWork;
+        const int cand = i / (D / 4), k4 = i % (D / 4);
+        const int c = j * kChunk + cand;
+        v[e] = c < n_cols ? __ldg(reinterpret_cast<const float4*>(sbase + (int64_t)c * D) + k4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    float4 cur[EPT], nxt[EPT];
+    load_chunk(0, cur);
     for (int j = 0; j < n_chunks; ++j) {
       const int st = j & 1;
+      if (j + 1 < n_chunks) load_chunk(j + 1, nxt);
       if (j >= 2 && !tc::mbar_wait(&bars->b_empty[st], ((j >> 1) - 1) & 1)) {
         ok = false;
         break;
       }
       uint8_t* bh = smem + L::kOffB + (st * 2 + 0) * L::kBTerm;
       uint8_t* bl = smem + L::kOffB + (st * 2 + 1) * L::kBTerm;
-      for (int i = threadIdx.x; i < kChunk * (D / 4); i += kWork) {
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        const int i = threadIdx.x + e * kWork;
         const int cand = i / (D / 4), k4 = i % (D / 4);
-        const int c = j * kChunk + cand;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c < n_cols) v = __ldg(reinterpret_cast<const float4*>(sbase + (int64_t)c * D) + k4);
+        const float4 v = cur[e];
         const float4 h = tf32_head(v);
         const float4 lo = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
         const int kc = k4 / 8, u = k4 % 8;
         *reinterpret_cast<float4*>(bh + kc * L::kBChunk + sw128(cand, u)) = h;
         *reinterpret_cast<float4*>(bl + kc * L::kBChunk + sw128(cand, u)) = lo;
+        cur[e] = nxt[e];
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bars->b_full[st]);
@@ -429,38 +448,75 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
     __syncthreads();
   }
 
-  // ---- the tile's stage-2 work list
+  // ---- the tile's stage-2 work list: the union of the positions' blocks
+  // plus the tile's own blocks, ascending; one warp per 32-column chunk
+  // counts, then every chunk writes at its prefix offset
   tc::fence_before_sync();
-  if (warp == 0 && to.ulist) {
+  if (to.ulist) {
+    int* lcnt = reinterpret_cast<int*>(smem + L::kOffList);
+    int* lsteps = lcnt + 32;
     const int own_lo = pos0 / p.block, own_hi = t_last;
     const int last_needed = p.causal ? last : p.S - 1;
-    const int64_t tix = bg * to.n_tiles + tile;
-    int32_t* out = to.ulist + tix * p.t_cap;
-    uint4* mout = to.umask + tix * p.t_cap;
-    int off = 0, steps = 0;
     const int span = max(n_cols, own_hi + 1);
-    for (int c0 = 0; c0 < span; c0 += 32) {
-      const int c = c0 + lane;
+    const int n_lch = (span + 31) / 32;
+    auto chunk = [&](int ch, uint4& m, unsigned& bal, int& st) {
+      const int c = ch * 32 + lane;
       bool keep = false;
-      uint4 m = make_uint4(0u, 0u, 0u, 0u);
+      m = make_uint4(0u, 0u, 0u, 0u);
+      st = 0;
       if (c < span) {
         if (c < kMaxCols) m = pmask[c];
         keep = (m.x | m.y | m.z | m.w) != 0u || (c >= own_lo && c <= own_hi);
+        if (keep)
+          for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
       }
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      int st = 0;
-      if (keep) {
-        const int k = off + __popc(bal & ((1u << lane) - 1u));
-        out[k] = c;
-        mout[k] = m;
-        for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
+      bal = __ballot_sync(0xffffffffu, keep);
+      return keep;
+    };
+    if (warp < kWorkWarps) {
+      for (int ch = warp; ch < n_lch; ch += kWorkWarps) {
+        uint4 m;
+        unsigned bal;
+        int st;
+        chunk(ch, m, bal, st);
+        st = warp_sum_i(st);
+        if (lane == 0) {
+          lcnt[ch] = __popc(bal);
+          lsteps[ch] = st;
+        }
       }
-      steps += warp_sum_i(st);
-      off += __popc(bal);
     }
-    if (lane == 0) {
-      to.ucnt[tix] = off;
-      to.usteps[tix] = steps;
+    __syncthreads();
+    if (warp < kWorkWarps) {
+      const int64_t tix = bg * to.n_tiles + tile;
+      int32_t* out = to.ulist + tix * p.t_cap;
+      uint4* mout = to.umask + tix * p.t_cap;
+      for (int ch = warp; ch < n_lch; ch += kWorkWarps) {
+        uint4 m;
+        unsigned bal;
+        int st;
+        const bool keep = chunk(ch, m, bal, st);
+        int off = 0;
+        for (int k = 0; k < ch; ++k) off += lcnt[k];
+        if (keep) {
+          const int k = off + __popc(bal & ((1u << lane) - 1u));
+          out[k] = ch * 32 + lane;
+          mout[k] = m;
+        }
+      }
+      if (warp == 0) {
+        int n = 0, steps = 0;
+        for (int k = lane; k < n_lch; k += 32) {
+          n += lcnt[k];
+          steps += lsteps[k];
+        }
+        n = warp_sum_i(n);
+        steps = warp_sum_i(steps);
+        if (lane == 0) {
+          to.ucnt[tix] = n;
+          to.usteps[tix] = steps;
+        }
+      }
     }
   }
   if (warp == kMmaWarp) {

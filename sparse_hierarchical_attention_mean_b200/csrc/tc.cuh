@@ -46,17 +46,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: returns false when the phase did not complete within the
-// budget (about a second of polling); the caller then records a timeout and
-// shuts down instead of hanging the GPU.
-constexpr uint32_t kWaitBudget = 1u << 22;
+// Bounded wait: returns false when the phase did not complete within about
+// a second (2^31 SM cycles); the caller then records a timeout and shuts
+// down instead of hanging the GPU.  try_wait itself suspends the thread
+// until the phase completes or a short hardware limit passes, so the loop
+// polls without sleeping: a sleep here would delay the wake-up of every
+// hand-off between the producer, MMA and softmax roles.
+constexpr long long kWaitCycles = 1ll << 31;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitBudget; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (i > 64) __nanosleep(64);
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
   }
-  return false;
+  return true;
 }
 
 // ------------------------------------------------------------------ TMA
