@@ -214,61 +214,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = tc::mbar_wait(&bars->q_full, 0);
-      if (!ok) fail_timeout(bars, p.status, 2);
+    // The whole warp runs the issue loop (descriptors stay warp-uniform);
+    // one elected lane issues each MMA and commit.
+    auto wait_all = [&](uint64_t* bar, uint32_t par) { return __all_sync(0xffffffffu, tc::mbar_wait(bar, par)); };
+    bool ok = wait_all(&bars->q_full, 0);
+    if (!ok) fail_timeout(bars, p.status, 2);
+    tc::fence_after_sync();
+    // Descriptors of stage 0; a stage or k-slice offset only moves the start
+    // address field (bytes >> 4), so the issue loops add constants.
+    const uint64_t kdesc0 = tc::smem_desc_sw128(smem + L::kOffK, 16, 1024);
+    const uint64_t vdesc0 = tc::smem_desc_sw128(smem + L::kOffV, L::kKVChunk, 1024);
+    // O(t) += P(t) V of step j, A = P from TMEM (over S)
+    auto issue_pv = [&](int t, int j) -> bool {
+      if (!wait_all(&bars->p_full[t], j & 1)) return false;
       tc::fence_after_sync();
-      // O(t) += P(t) V of step j, A = P from TMEM (over S)
-      auto issue_pv = [&](int t, int j) -> bool {
-        if (!tc::mbar_wait(&bars->p_full[t], j & 1)) return false;
-        tc::fence_after_sync();
-        const int st = j % kStages;
+      const uint64_t vd = vdesc0 + (uint64_t)(((j % kStages) * L::kKVBytes) >> 4);
+      const uint32_t d_tm = tmem + t * kTileCols + kOOff, a_tm = tmem + t * kTileCols + kSOff;
+      tc::mma_f16_ts_w(d_tm, a_tm, vd, kIdescO, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < kStep / 16; ++k) {
-          const uint64_t bd = tc::smem_desc_sw128(smem + L::kOffV + st * L::kKVBytes + k * 2048, L::kKVChunk, 1024);
-          tc::mma_f16_ts(tmem + t * kTileCols + kOOff, tmem + t * kTileCols + kSOff + k * 8, bd, kIdescO,
-                         (j > 0 || k > 0) ? 1u : 0u);
-        }
-        return true;
-      };
-      int i = 0;
-      for (; ok && i < n_steps; ++i) {
-        const int st = i % kStages;
-        if (!tc::mbar_wait(&bars->kv_full[st], (i / kStages) & 1)) {
-          fail_timeout(bars, p.status, 3);
+      for (int k = 1; k < kStep / 16; ++k) tc::mma_f16_ts_w(d_tm, a_tm + k * 8, vd + ((k * 2048) >> 4), kIdescO, 1u);
+      return true;
+    };
+    int i = 0;
+    for (; ok && i < n_steps; ++i) {
+      const int st = i % kStages;
+      if (!wait_all(&bars->kv_full[st], (i / kStages) & 1)) {
+        fail_timeout(bars, p.status, 3);
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      for (int t = 0; ok && t < kTiles; ++t) {
+        if (i >= 1 && !issue_pv(t, i - 1)) {
+          fail_timeout(bars, p.status, 4);
           ok = false;
           break;
         }
-        tc::fence_after_sync();
-        for (int t = 0; ok && t < kTiles; ++t) {
-          if (i >= 1 && !issue_pv(t, i - 1)) {
-            fail_timeout(bars, p.status, 4);
-            ok = false;
-            break;
-          }
-          // S(t) = Q(t) K^T, A = Q from TMEM
+        // S(t) = Q(t) K^T, A = Q from TMEM
+        const uint64_t kd = kdesc0 + (uint64_t)((st * L::kKVBytes) >> 4);
+        const uint32_t s_tm = tmem + t * kTileCols + kSOff, q_tm = tmem + t * kTileCols;
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t bd = tc::smem_desc_sw128(
-                smem + L::kOffK + st * L::kKVBytes + (k >> 2) * L::kKVChunk + (k & 3) * 32, 16, 1024);
-            tc::mma_f16_ts(tmem + t * kTileCols + kSOff, tmem + t * kTileCols + k * 8, bd, kIdescS,
-                           k > 0 ? 1u : 0u);
-          }
-          tc::mma_commit(&bars->s_full[t]);
-        }
-        if (ok && i >= 1) tc::mma_commit(&bars->kv_empty[(i - 1) % kStages]);
+        for (int k = 0; k < D / 16; ++k)
+          tc::mma_f16_ts_w(s_tm, q_tm + k * 8, kd + (uint64_t)((((k >> 2) * L::kKVChunk) + (k & 3) * 32) >> 4),
+                           kIdescS, k > 0 ? 1u : 0u);
+        tc::mma_commit_w(&bars->s_full[t]);
       }
-      if (ok && i >= 1) {
-        for (int t = 0; ok && t < kTiles; ++t)
-          if (!issue_pv(t, i - 1)) {
-            fail_timeout(bars, p.status, 5);
-            ok = false;
-          }
-      }
-      // o_final arrives once every MMA issued above has completed
-      tc::mma_commit(&bars->o_final);
-      tc::mbar_wait(&bars->o_final, 0);
+      if (ok && i >= 1) tc::mma_commit_w(&bars->kv_empty[(i - 1) % kStages]);
     }
+    if (ok && i >= 1) {
+      for (int t = 0; ok && t < kTiles; ++t)
+        if (!issue_pv(t, i - 1)) {
+          fail_timeout(bars, p.status, 5);
+          ok = false;
+        }
+    }
+    // o_final arrives once every MMA issued above has completed
+    tc::mma_commit_w(&bars->o_final);
+    tc::mbar_wait(&bars->o_final, 0);
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
     const int t = warp >> 2;  // tile

@@ -84,10 +84,12 @@ __device__ __forceinline__ float4 tf32_head(float4 v) {
   return h;
 }
 
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// Warp-wide: every lane executes it with the same operands, one elected
+// lane issues (see the warp-wide forms in tc.cuh).
+__device__ __forceinline__ void mma_tf32_w(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
@@ -247,36 +249,36 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
 
   if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_chunks > 0) {
-      bool ok = tc::mbar_wait(&bars->a_full, 0);
+    // whole warp (uniform descriptors), one elected lane issues
+    if (n_chunks > 0) {
+      bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->a_full, 0));
+      const uint64_t adesc0 = tc::smem_desc_sw128(smem + L::kOffA, 16, 1024);
+      const uint64_t bdesc0 = tc::smem_desc_sw128(smem + L::kOffB, 16, 1024);
       for (int j = 0; ok && j < n_chunks; ++j) {
         const int st = j & 1;
-        if (!tc::mbar_wait(&bars->b_full[st], (j >> 1) & 1)) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->b_full[st], (j >> 1) & 1))) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint8_t* bh = smem + L::kOffB + (st * 2 + 0) * L::kBTerm;
-        const uint8_t* bl = smem + L::kOffB + (st * 2 + 1) * L::kBTerm;
 #pragma unroll
         for (int term = 0; term < 2; ++term) {
+          const uint64_t bd = bdesc0 + (uint64_t)(((st * 2 + term) * L::kBTerm) >> 4);
 #pragma unroll
           for (int kc = 0; kc < L::KC; ++kc) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t ad = tc::smem_desc_sw128(smem + L::kOffA + kc * L::kAChunk + k * 32, 16, 1024);
-              const uint64_t bd = tc::smem_desc_sw128((term ? bl : bh) + kc * L::kBChunk + k * 32, 16, 1024);
-              mma_tf32(tmem + j * kChunk, ad, bd, kIdesc, (term | kc | k) ? 1u : 0u);
-            }
+            for (int k = 0; k < 4; ++k)
+              mma_tf32_w(tmem + j * kChunk, adesc0 + (uint64_t)((kc * L::kAChunk + k * 32) >> 4),
+                         bd + (uint64_t)((kc * L::kBChunk + k * 32) >> 4), kIdesc, (term | kc | k) ? 1u : 0u);
           }
         }
-        tc::mma_commit(&bars->b_empty[st]);
+        tc::mma_commit_w(&bars->b_empty[st]);
       }
       if (!ok) {
         raise_status(p.status, 5 /* DASH_ERR_DEVICE_TIMEOUT */, 20);
         atomicExch(&bars->abort, 1);
       }
-      tc::mma_commit(&bars->x_ready);
+      tc::mma_commit_w(&bars->x_ready);
       tc::mbar_wait(&bars->x_ready, 0);
     }
   } else if (n_chunks > 0) {
