@@ -28,10 +28,14 @@
 //               then per step reads its 64 logits, adds the row's prior bias
 //               (log p_bar of the block if its position selected it,
 //               log(1/N) on its own block, else -inf), keeps the running max
-//               and sum, writes P into TMEM and finally normalises O.  O is
-//               rescaled in TMEM only when a row's max grows by more than 2^8,
-//               so P stays <= 256 and the result is exact (the final division
-//               uses the same reference max).
+//               and sum, writes P into TMEM and finally normalises O.  P is
+//               taken against the row's reference max; the step's row max is
+//               only computed when the row has no reference yet or the step's
+//               sum shows a P above 2^8.  O is rescaled in TMEM only when the
+//               reference grows by more than 2^8, so P stays <= 256 and the
+//               result is exact (the final division uses the same reference).
+//               The scale-and-offset FMAs and the row sums use paired fp32
+//               instructions.
 // Every mbarrier wait is bounded; on expiry the kernel records
 // DASH_ERR_DEVICE_TIMEOUT in the workspace status word and winds down.
 #include <cuda.h>
@@ -332,36 +336,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tok0 + kStep > p.S) n_valid = min(n_valid, p.S - tok0);
       if (p.causal && c == row.t) n_valid = min(n_valid, row.pos - tok0 + 1);
       const float b2 = bias * kLog2e;
-      // The bias is constant over the step and the scale positive, so the
-      // row max of the logits is max(s) * scale + bias: take it on the raw
-      // scores (masked columns set to -inf first on the slow path).
+      // masked columns hold -inf and give p = 0
       if (n_valid < kStep) {
 #pragma unroll
         for (int j = 0; j < kStep; ++j)
           if (j >= n_valid) sv[j] = __float_as_uint(kNegInf);
       }
-      float pm[8];
+      uint32_t pw[32];
+      // p = 2^(s * scale + bias - m) for the 64 columns; returns their sum
+      auto exps = [&](float off) -> float {
+        const float2 sc2 = make_float2(qk_scale, qk_scale), off2 = make_float2(off, off);
+        float2 ps2[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) pm[e] = __uint_as_float(sv[e]);
+        for (int e = 0; e < 4; ++e) ps2[e] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int j = 8; j < kStep; ++j) pm[j & 7] = fmaxf(pm[j & 7], __uint_as_float(sv[j]));
-      const float smax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      const float mx = n_valid > 0 ? fmaf(smax, qk_scale, b2) : kNegInf;
+        for (int j = 0; j < kStep; j += 2) {
+          const float2 a = __ffma2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sc2, off2);
+          const float2 pp = make_float2(tc::ex2(a.x), tc::ex2(a.y));
+          ps2[(j >> 1) & 3] = __fadd2_rn(ps2[(j >> 1) & 3], pp);
+          pw[j >> 1] = pack2<T>(pp.x, pp.y);
+        }
+        const float2 s01 = __fadd2_rn(__fadd2_rn(ps2[0], ps2[1]), __fadd2_rn(ps2[2], ps2[3]));
+        return s01.x + s01.y;
+      };
+      // Fast path: the row's running reference max m_used is kept; valid
+      // while every p stays <= 2^8, which the step's sum bounds.  Otherwise
+      // (no reference yet, or a larger max) the row max is taken and the
+      // step recomputed; O is rescaled when the reference grows by > 2^8.
       float corr = 1.0f;
       bool resc = false;
-      if (mx != kNegInf) {
-        if (m_used == kNegInf) {
-          m_used = mx;  // nothing accumulated for this row yet
-        } else if (mx > m_used + kRescaleLog2) {
-          corr = tc::ex2(m_used - mx);
-          m_used = mx;
-          resc = true;
-        }
-      }
-      if (__any_sync(0xffffffffu, resc)) {
-        // O is stable: the previous step's P V completed before this S
+      const bool fast = m_used != kNegInf && n_valid > 0;
+      float lstep = fast ? exps(b2 - m_used) : 0.f;
+      if (!fast || !(lstep <= 256.0f)) {
+        // the bias is constant over the step and the scale positive, so the
+        // row max of the logits is max(s) * scale + bias
+        float pm[8];
 #pragma unroll
+        for (int e = 0; e < 8; ++e) pm[e] = __uint_as_float(sv[e]);
+#pragma unroll
+        for (int j = 8; j < kStep; ++j) pm[j & 7] = fmaxf(pm[j & 7], __uint_as_float(sv[j]));
+        const float smax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float mx = n_valid > 0 ? fmaf(smax, qk_scale, b2) : kNegInf;
+        if (mx != kNegInf) {
+          if (m_used == kNegInf) {
+            m_used = mx;  // nothing accumulated for this row yet
+          } else if (mx > m_used + kRescaleLog2) {
+            corr = tc::ex2(m_used - mx);
+            m_used = mx;
+            resc = true;
+          }
+        }
+        lstep = exps(n_valid > 0 ? b2 - m_used : kNegInf);
+      }
+      lsum = lsum * corr + lstep;
+      tc::tmem_st32(tbase + kSOff, pw);
+      if (__any_sync(0xffffffffu, resc)) {
+        // O rescaled to the new reference before this step's P V is issued;
+        // O is stable: the previous step's P V completed before this S
+#pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t ov[32];
           const uint32_t ta = tbase + kOOff + cc * 32;
@@ -371,25 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * corr);
           tc::tmem_st32(ta, ov);
         }
-        lsum *= corr;
       }
-      // p = 2^(s * scale + bias - m): one FMA and one ex2 per column; masked
-      // columns hold -inf and give 0, a row without a valid column writes zeros
-      const float off = n_valid > 0 ? b2 - m_used : kNegInf;
-      float ps[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
-      uint32_t pw[32];
-#pragma unroll
-      for (int j = 0; j < kStep; j += 2) {
-        const float p0 = tc::ex2(fmaf(__uint_as_float(sv[j]), qk_scale, off));
-        const float p1 = tc::ex2(fmaf(__uint_as_float(sv[j + 1]), qk_scale, off));
-        ps[j & 7] += p0;
-        ps[(j + 1) & 7] += p1;
-        pw[j >> 1] = pack2<T>(p0, p1);
-      }
-      lsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      tc::tmem_st32(tbase + kSOff, pw);
       tc::tmem_wait_st();
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->p_full[t]);

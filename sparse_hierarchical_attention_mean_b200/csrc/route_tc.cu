@@ -106,7 +106,9 @@ __device__ __forceinline__ bool is_cand(int c, int t, int n_blocks, int causal) 
 
 // alpha-entmax thresholds of RW rows that share their candidate columns,
 // solved in lockstep by one warp (their reductions interleave).  Row i's
-// logits are x[i * stride + c] for c < n, -inf on non-candidates.  Same
+// logits are x[i * stride + c] for c < n, -inf on non-candidates; columns are
+// read 64 at a time, so the rows must be readable (-inf) up to n rounded up
+// to a multiple of 64.  Same
 // scheme as warp_entmax_tau: Newton from max - 1, where F >= 1, approaches
 // the root from below, and after every step the exact solution on the
 // current support is accepted when it is self-consistent.
@@ -117,9 +119,9 @@ __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride,
   float mx[RW];
 #pragma unroll
   for (int i = 0; i < RW; ++i) mx[i] = kNegInf;
-  for (int c = lane; c < n; c += 32) {
+  for (int c = lane; c < n; c += 64) {
 #pragma unroll
-    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], x[i * stride + c]);
+    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], fmaxf(x[i * stride + c], x[i * stride + c + 32]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -136,10 +138,17 @@ __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride,
     float f[RW], a[RW], k[RW], umin[RW], fd[RW];
 #pragma unroll
     for (int i = 0; i < RW; ++i) f[i] = a[i] = k[i] = fd[i] = 0.f, umin[i] = 3.0e38f;
-    for (int c = lane; c < n; c += 32) {
+    for (int c = lane; c < n; c += 64) {
+      float xv[2 * RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
-        const float u = x[i * stride + c] - tau[i];
+        xv[2 * i] = x[i * stride + c];
+        xv[2 * i + 1] = x[i * stride + c + 32];
+      }
+#pragma unroll
+      for (int e = 0; e < 2 * RW; ++e) {
+        const int i = e >> 1;
+        const float u = xv[e] - tau[i];
         if (u > 0.f) {
           k[i] += 1.f;
           a[i] += u;
@@ -361,7 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   __syncthreads();  // GEMM done: its shared memory now holds logits
 
   // ---- two halves of 64 rows: TMEM -> shared, thresholds, compaction
-  const int n_wch = (n_cols + 31) / 32;  // 32-column chunks of the logit rows
+  // 32-column chunks of the logit rows, an even number: the threshold passes
+  // read columns in pairs of chunks (the extra columns hold -inf)
+  const int n_wch = ((n_cols + 63) / 64) * 2;
   for (int half = 0; half < 2; ++half) {
     if (warp < kWorkWarps && n_chunks > 0 && !bars->abort) {
       // warps whose TMEM lane quarter lies in this half copy (and scale) their rows
