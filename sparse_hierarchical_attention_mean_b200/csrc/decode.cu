@@ -16,12 +16,16 @@
 //                    items (chunks of selected blocks) appended with one
 //                    atomic per (b, g).
 //  attend_decode     persistent CTAs over the work items: K/V rows of the
-//                    selected blocks stream through a cp.async double
-//                    buffer; each warp owns 16 tokens of a 64-token step,
-//                    computes the G x 16 logits with a reduce-scatter, keeps
-//                    an online softmax per head and accumulates P V; the 4
-//                    warps merge into one (m, l, o) partial per item.
+//                    selected blocks stream through a cp.async ring; each
+//                    warp owns 16 tokens of a 64-token step, keeps an online
+//                    softmax per head and accumulates P V; the 4 warps merge
+//                    into one (m, l, o) partial per item.  f16/bf16 take both
+//                    products on the tensor cores with warp-level MMAs
+//                    (attend_decode_mma_kernel); fp32 computes them with a
+//                    reduce-scatter on the CUDA cores.
 //  combine_decode    log-sum-exp merge of the partials of each (b, g).
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -413,6 +417,251 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_kernel(DecodeParams
   }
 }
 
+// ------------------------------------------------------------------ split-KV attention, f16/bf16
+// The same work items and partials as attend_decode_kernel, with the two
+// per-warp products on the tensor cores through warp-level mma (m16n8k16,
+// fp32 accumulate): a KV head has only G <= 8 query rows, far below the
+// 64-row minimum of the 5th-generation MMA, and the kernel is HBM-bound, so
+// the MMAs only serve to take the dot products off the issue slots.
+//   S^T (16 x 8 tokens) = Qpad (16 x D) K^T: rows are the G heads (zero
+//   padding above G), B fragments come from the K rows by ldmatrix;
+//   O (16 x D) += P (16 x 16 tokens) V: P is the S accumulator re-packed in
+//   registers (the accumulator layout of two 8-token tiles is the A layout of
+//   one 16-token tile), V fragments by ldmatrix.trans.
+// K/V stream through a kDStages-deep cp.async ring; each row of 16-byte
+// chunks is stored XOR-swizzled by (token & 7) so the ldmatrix row reads are
+// free of bank conflicts.  Each warp owns 16 tokens of every 64-token step and
+// keeps its own online softmax; O is rescaled only when a head's reference
+// max grows by more than 2^8 (P <= 256, exact after the final division).
+constexpr int kDStages = 3;
+
+template <typename T>
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  if constexpr (std::is_same<T, __half>::value) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodeParams p) {
+  static_assert(G <= 8, "heads of a group must fit the 8 live MMA rows");
+  constexpr int NCH = D / 8;       // 16-byte chunks per row
+  constexpr int NT = D / 8;        // 8-wide d tiles of O
+  constexpr int KS = D / 16;       // k steps of S
+  constexpr int kStageElems = kStep * D;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  T* Ks = reinterpret_cast<T*>(smem_raw);               // [kDStages][kStep][D] swizzled
+  T* Vs = Ks + kDStages * kStageElems;                  // [kDStages][kStep][D] swizzled
+  float* mbuf = reinterpret_cast<float*>(Vs + kDStages * kStageElems);  // [kWarps][G]
+  float* lbuf = mbuf + kWarps * G;                      // [kWarps][G]
+  float* obuf = lbuf + kWarps * G;                      // [kWarps][G][D]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;  // fragment row group / thread in group
+  const int n_items = *p.n_items;
+  const float qk_scale = rsqrtf((float)D) * kLog2e;
+  const uint32_t ks_base = smem_u32(Ks), vs_base = smem_u32(Vs);
+
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int bg = p.items[2 * item], chunk = p.items[2 * item + 1];
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int L = clamp_len(p.seqlens, b, p.Lmax, nullptr);
+    const int pos = L - 1;
+    const int t = pos / p.block;
+    const int N = t;
+    const int cnt = p.cnt[bg];
+    const int e_begin = chunk * p.chunk_blocks;
+    const int e_end = min(e_begin + p.chunk_blocks, cnt + 1);
+    const bool has_diag = e_end == cnt + 1;
+    const int spb = p.block / kStep;
+    const int n_diag = has_diag ? (pos - t * p.block) / kStep + 1 : 0;
+    const int n_sel = (has_diag ? e_end - 1 : e_end) - e_begin;
+    const int n_sub = n_sel * spb + n_diag;
+    const int32_t* idx = p.idx + (int64_t)bg * p.t_cap;
+    const float* logp = p.logp + (int64_t)bg * p.t_cap;
+    const float beta = N > 0 ? logf(1.0f / (float)N) : 0.0f;
+    const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
+    const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
+
+    auto sub_tok0 = [&](int s) -> int {
+      if (s < n_sel * spb) return idx[e_begin + s / spb] * p.block + (s % spb) * kStep;
+      return t * p.block + (s - n_sel * spb) * kStep;
+    };
+    auto load = [&](int s) {
+      if (s < n_sub) {
+        const int tok0 = sub_tok0(s);
+        T* kd = Ks + (s % kDStages) * kStageElems;
+        T* vd = Vs + (s % kDStages) * kStageElems;
+        for (int i = tid; i < kStep * NCH; i += kWarps * 32) {
+          const int r = i / NCH, c = i % NCH;
+          const int tok = tok0 + r;
+          const bool ok = tok < L;  // rows past the context are zero-filled
+          const int pc = c ^ (r & 7);
+          cp_async16(kd + r * D + pc * 8, kg + (int64_t)(ok ? tok : 0) * p.k.ss + c * 8, ok);
+          cp_async16(vd + r * D + pc * 8, vg + (int64_t)(ok ? tok : 0) * p.v.ss + c * 8, ok);
+        }
+      }
+      cp_async_commit();
+    };
+
+    // query A fragments: rows = heads (row gq < G), 16 d per k step
+    uint32_t qa[KS][2];
+    {
+      const T* q = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb + (int64_t)(g * G + (gq < G ? gq : 0)) * p.q.sh;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        qa[kk][0] = gq < G ? *reinterpret_cast<const uint32_t*>(q + kk * 16 + 2 * tq) : 0u;
+        qa[kk][1] = gq < G ? *reinterpret_cast<const uint32_t*>(q + kk * 16 + 8 + 2 * tq) : 0u;
+      }
+    }
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_used = kNegInf, lpart = 0.f;
+
+#pragma unroll
+    for (int s = 0; s < kDStages - 1; ++s) load(s);
+    for (int s = 0; s < n_sub; ++s) {
+      load(s + kDStages - 1);
+      cp_async_wait<kDStages - 1>();
+      __syncthreads();
+      const int st = s % kDStages;
+      const uint32_t kst = ks_base + (uint32_t)(st * kStageElems * sizeof(T));
+      const uint32_t vst = vs_base + (uint32_t)(st * kStageElems * sizeof(T));
+      const bool diag = s >= n_sel * spb;
+      const float bias = (diag ? beta : logp[e_begin + s / spb]) * kLog2e;
+      const int tok0 = sub_tok0(s) + warp * 16;
+
+      // S^T = Q K^T for this warp's 16 tokens (two 8-token tiles)
+      float sacc[2][4];
+#pragma unroll
+      for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+      {
+        const int m = lane >> 3, rr = lane & 7;
+        const int tok = warp * 16 + (m >> 1) * 8 + rr;  // row within the stage
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const int c = 2 * kk + (m & 1);
+          uint32_t bf[4];
+          ldsm_x4(kst + (uint32_t)((tok * D + ((c ^ (tok & 7)) * 8)) * sizeof(T)), bf);
+          const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
+          mma16816<T>(sacc[0], a, bf[0], bf[1]);
+          mma16816<T>(sacc[1], a, bf[2], bf[3]);
+        }
+      }
+      // logits (log2 domain) of head gq for tokens 2tq, 2tq+1, 8+2tq, 9+2tq
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tk = tok0 + (e >> 1) * 8 + 2 * tq + (e & 1);
+        x[e] = tk <= pos ? fmaf(sacc[e >> 1][e & 1], qk_scale, bias) : kNegInf;
+      }
+      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      float corr = 1.0f;
+      bool resc = false;
+      if (mx != kNegInf) {
+        if (m_used == kNegInf) {
+          m_used = mx;
+        } else if (mx > m_used + 8.0f) {
+          corr = exp2f(m_used - mx);
+          m_used = mx;
+          resc = true;
+        }
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          o[n][0] *= corr;
+          o[n][1] *= corr;
+        }
+        lpart *= corr;
+      }
+      float pe[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pe[e] = m_used == kNegInf ? 0.f : exp2f(x[e] - m_used);
+      lpart += (pe[0] + pe[1]) + (pe[2] + pe[3]);
+      const uint32_t pa[4] = {pack2<T>(pe[0], pe[1]), 0u, pack2<T>(pe[2], pe[3]), 0u};
+
+      // O += P V: B fragments of two 8-wide d tiles per ldmatrix
+      {
+        const int m = lane >> 3, rr = lane & 7;
+        const int tok = warp * 16 + (m & 1) * 8 + rr;
+#pragma unroll
+        for (int j = 0; j < NT / 2; ++j) {
+          const int c = 2 * j + (m >> 1);
+          uint32_t bf[4];
+          ldsm_x4_t(vst + (uint32_t)((tok * D + ((c ^ (tok & 7)) * 8)) * sizeof(T)), bf);
+          mma16816<T>(o[2 * j], pa, bf[0], bf[1]);
+          mma16816<T>(o[2 * j + 1], pa, bf[2], bf[3]);
+        }
+      }
+      __syncthreads();  // the stage is free for the load issued next iteration
+    }
+    cp_async_wait<0>();
+
+    // merge the 4 warps: rows gq < G hold head gq; lanes of a row group split d
+    float l = lpart;
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if (gq < G) {
+      if (tq == 0) {
+        mbuf[warp * G + gq] = m_used;
+        lbuf[warp * G + gq] = l;
+      }
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        obuf[(warp * G + gq) * D + n * 8 + 2 * tq] = o[n][0];
+        obuf[(warp * G + gq) * D + n * 8 + 2 * tq + 1] = o[n][1];
+      }
+    }
+    __syncthreads();
+    const int64_t slot = (int64_t)p.pair_base[bg] + chunk;
+    for (int i = tid; i < G * D; i += kWarps * 32) {
+      const int h = i / D, e = i % D;
+      float M = kNegInf;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mbuf[w * G + h]);
+      const float Mu = M == kNegInf ? 0.f : M;
+      float acc = 0.f, lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = exp2f(mbuf[w * G + h] - Mu);
+        acc += f * obuf[(w * G + h) * D + e];
+        lsum += f * lbuf[w * G + h];
+      }
+      p.part_o[(slot * G + h) * D + e] = acc;
+      if (e == 0) {
+        p.part_ml[(slot * G + h) * 2] = M;
+        p.part_ml[(slot * G + h) * 2 + 1] = lsum;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // ------------------------------------------------------------------ combine
 template <typename T, int D>
 __global__ void __launch_bounds__(256) combine_decode_kernel(DecodeParams p) {
@@ -451,9 +700,12 @@ cudaError_t launch_route_t(const DecodeParams& p, cudaStream_t stream) {
 
 template <typename T, int D, int G>
 cudaError_t launch_attend_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
-  const size_t smem = (size_t)4 * kStep * D * sizeof(T) +
-                      (size_t)(kWarps * 16 * G + 2 * kWarps * G + kWarps * G * D) * sizeof(float);
-  auto kern = attend_decode_kernel<T, D, G>;
+  constexpr bool kMma = !std::is_same<T, float>::value;
+  const size_t smem = kMma ? (size_t)2 * kDStages * kStep * D * sizeof(T) +
+                                 (size_t)(2 * kWarps * G + kWarps * G * D) * sizeof(float)
+                           : (size_t)4 * kStep * D * sizeof(T) +
+                                 (size_t)(kWarps * 16 * G + 2 * kWarps * G + kWarps * G * D) * sizeof(float);
+  auto kern = kMma ? attend_decode_mma_kernel<T, D, G> : attend_decode_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
