@@ -7,9 +7,9 @@
 // by the fixed projection W_s (row vector times matrix).
 //
 // HBM-bound: every key is read once with 16-byte vector loads; the mean and
-// the projection are fp32.  One CTA pools `bpc` consecutive blocks of one
-// (batch, KV head) and projects them together so each W_s column is read
-// once per CTA.
+// the projection are fp32.  One CTA pools up to 32 consecutive blocks of one
+// (batch, KV head) and projects them together so each W_s row is read once
+// per CTA.
 #include "common.cuh"
 #include "internal.h"
 
@@ -17,16 +17,25 @@ namespace dash {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarpsP = kThreads / 32;
 constexpr int kMaxBpc = 32;
 
+// One CTA: up to kMaxBpc consecutive blocks of one (batch, KV head).
+//   Pooling: each warp takes whole blocks (w, w + 8, ...); a lane owns one
+//   16-byte column vector of a row group and sums its rows in registers with
+//   eight loads in flight, then the lanes holding the same columns combine by
+//   shuffles.  No barrier per block.
+//   Projection: means[nb][D] x W_s[D][D] with a 4 x 4 (blocks x columns)
+//   register tile per thread; W_s rows are read as float4 through L1.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
-  constexpr int EPV = Elt<T>::kPerVec;
-  constexpr int VPR = D / EPV;        // 16-byte vectors per key row
-  constexpr int RP = kThreads / VPR;  // key rows per pass
-  constexpr int NG = kThreads / D;    // thread groups in the projection
-  __shared__ float red[RP][D];
-  __shared__ float means[kMaxBpc][D];
+  constexpr int EPV = Elt<T>::kPerVec;     // elements per 16-byte vector
+  constexpr int VPR = D / EPV;             // vectors per key row (8, 16 or 32)
+  constexpr int RPL = 32 / VPR;            // rows per warp-wide load
+  constexpr int CG = D / 4;                // 4-column groups of the projection
+  constexpr int BG = kThreads / CG;        // block groups
+  constexpr int BPT = kMaxBpc / BG;        // blocks per thread in the projection
+  __shared__ __align__(16) float means[kMaxBpc][D];
 
   const int b = blockIdx.z, g = blockIdx.y;
   int n_tok = p.S;
@@ -35,55 +44,68 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
   const int64_t c_begin = p.first_block + (int64_t)blockIdx.x * bpc;
   if (c_begin >= nblk) return;
   const int nb = (int)(nblk - c_begin < bpc ? nblk - c_begin : bpc);
-  const int tid = threadIdx.x;
-  const int vrow = tid / VPR, vcol = tid % VPR;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int vcol = lane % VPR, vrow = lane / VPR;
   const T* kbase = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh + vcol * EPV;
 
-  for (int i = 0; i < nb; ++i) {
+  for (int i = warp; i < nb; i += kWarpsP) {
     const int64_t lo = (c_begin + i) * p.block;
     const int64_t hi = lo + p.block < n_tok ? lo + p.block : (int64_t)n_tok;
     float acc[EPV];
 #pragma unroll
     for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
-#pragma unroll 8
-    for (int64_t j = lo + vrow; j < hi; j += RP) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(kbase + j * p.k.ss));
-      float f[EPV];
-      Elt<T>::to_float(v, f);
+    for (int64_t j0 = lo; j0 < hi; j0 += 8 * RPL) {
+      uint4 v[8];
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) acc[e] += f[e];
+      for (int u = 0; u < 8; ++u) {
+        const int64_t j = j0 + u * RPL + vrow;
+        v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kbase + j * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float f[EPV];
+        Elt<T>::to_float(v[u], f);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) acc[e] += f[e];
+      }
     }
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) red[vrow][vcol * EPV + e] = acc[e];
-    __syncthreads();
-    if (tid < D) {
-      float s = 0.f;
+    for (int off = VPR; off < 32; off <<= 1)
 #pragma unroll
-      for (int r = 0; r < RP; ++r) s += red[r][tid];
-      means[i][tid] = s / (float)(hi - lo);
+      for (int e = 0; e < EPV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    if (vrow == 0) {
+      const float inv = 1.0f / (float)(hi - lo);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) means[i][vcol * EPV + e] = acc[e] * inv;
     }
-    __syncthreads();
   }
+  __syncthreads();
 
   // s[i][col] = sum_k mean[i][k] * W_s[k][col]
-  const int col = tid % D, grp = tid / D;
-  constexpr int PER = kMaxBpc / NG;
-  float acc[PER];
+  const int cg = tid % CG, bgp = tid / CG;
+  float acc[BPT][4];
 #pragma unroll
-  for (int m = 0; m < PER; ++m) acc[m] = 0.f;
+  for (int m = 0; m < BPT; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+  const float4* w4 = reinterpret_cast<const float4*>(p.w_s) + cg;
+#pragma unroll 4
   for (int k = 0; k < D; ++k) {
-    const float w = __ldg(p.w_s + k * D + col);
+    const float4 w = __ldg(w4 + k * (D / 4));
 #pragma unroll
-    for (int m = 0; m < PER; ++m) {
-      const int i = grp + NG * m;
-      if (i < nb) acc[m] += means[i][k] * w;
+    for (int m = 0; m < BPT; ++m) {
+      const float mk = means[bgp * BPT + m][k];
+      acc[m][0] = fmaf(mk, w.x, acc[m][0]);
+      acc[m][1] = fmaf(mk, w.y, acc[m][1]);
+      acc[m][2] = fmaf(mk, w.z, acc[m][2]);
+      acc[m][3] = fmaf(mk, w.w, acc[m][3]);
     }
   }
   float* out = p.summaries + ((int64_t)b * p.Hkv + g) * p.t_cap * D;
 #pragma unroll
-  for (int m = 0; m < PER; ++m) {
-    const int i = grp + NG * m;
-    if (i < nb) out[(c_begin + i) * D + col] = acc[m];
+  for (int m = 0; m < BPT; ++m) {
+    const int i = bgp * BPT + m;
+    if (i < nb)
+      *reinterpret_cast<float4*>(out + (c_begin + i) * D + cg * 4) =
+          make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
   }
 }
 
@@ -93,8 +115,9 @@ cudaError_t launch_typed(const PoolParams& p, cudaStream_t stream) {
   const int64_t span = max_blk - p.first_block;
   if (span <= 0) return cudaSuccess;
   const int64_t total = span * p.B * p.Hkv;
-  int bpc = 4;
-  while (bpc < kMaxBpc && total / (bpc * 2) >= 148 * 16) bpc *= 2;
+  // as many blocks per CTA as keep about four CTAs per SM busy
+  int bpc = kMaxBpc;
+  while (bpc > kWarpsP && total / bpc < 148 * 4) bpc /= 2;
   dim3 grid((unsigned)((span + bpc - 1) / bpc), p.Hkv, p.B);
   pool_kernel<T, D><<<grid, kThreads, 0, stream>>>(p, bpc);
   return cudaGetLastError();
