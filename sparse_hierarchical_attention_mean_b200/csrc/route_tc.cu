@@ -104,65 +104,49 @@ __device__ __forceinline__ bool is_cand(int c, int t, int n_blocks, int causal) 
   return causal ? c < t : (c != t && c < n_blocks);
 }
 
-// alpha-entmax thresholds of RW rows that share their candidate columns,
-// solved in lockstep by one warp (their reductions interleave).  Row i's
-// logits are x[i * stride + c] for c < n, -inf on non-candidates; columns are
-// read 64 at a time, so the rows must be readable (-inf) up to n rounded up
-// to a multiple of 64.  Same
-// scheme as warp_entmax_tau: Newton from max - 1, where F >= 1, approaches
-// the root from below, and after every step the exact solution on the
-// current support is accepted when it is self-consistent.
-template <int RW>
-__device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride, int n, float alpha, int kind,
-                                                     int lane, float* tau) {
-  const float pw = 1.0f / (alpha - 1.0f);
-  float mx[RW];
-#pragma unroll
-  for (int i = 0; i < RW; ++i) mx[i] = kNegInf;
-  for (int c = lane; c < n; c += 64) {
-#pragma unroll
-    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], fmaxf(x[i * stride + c], x[i * stride + c + 32]));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
-  }
-  bool done[RW];
-#pragma unroll
-  for (int i = 0; i < RW; ++i) {
-    tau[i] = mx[i] - 1.0f;
-    done[i] = mx[i] == kNegInf;
-  }
+// Newton passes from below with the exact check on the current support, for
+// RW rows in lockstep.  COLS = 1: each lane holds one value per row in v[i]
+// (32 values per row); COLS = 2: row i's values are x[i * stride + c], read 64
+// columns per iteration for c < n (readable, -inf, up to n rounded up to 64).
+// tau[i] must be a lower bound of the root (F >= 1); rows with done[i] set are
+// left alone.
+template <int RW, int COLS>
+__device__ __forceinline__ void entmax_newton_rows(const float* x, int stride, int n, float pw, int kind, int lane,
+                                                   float* tau, bool* done) {
   for (int it = 0; it < 100; ++it) {
     float f[RW], a[RW], k[RW], umin[RW], fd[RW];
 #pragma unroll
     for (int i = 0; i < RW; ++i) f[i] = a[i] = k[i] = fd[i] = 0.f, umin[i] = 3.0e38f;
-    for (int c = lane; c < n; c += 64) {
-      float xv[2 * RW];
-#pragma unroll
-      for (int i = 0; i < RW; ++i) {
-        xv[2 * i] = x[i * stride + c];
-        xv[2 * i + 1] = x[i * stride + c + 32];
-      }
-#pragma unroll
-      for (int e = 0; e < 2 * RW; ++e) {
-        const int i = e >> 1;
-        const float u = xv[e] - tau[i];
-        if (u > 0.f) {
-          k[i] += 1.f;
-          a[i] += u;
-          umin[i] = fminf(umin[i], u);
-          if (kind == 0) {
-            f[i] += u;
-          } else if (kind == 1) {
-            f[i] = fmaf(u, u, f[i]);
-          } else {
-            const float up = exp2f((pw - 1.0f) * log2f(u));
-            fd[i] += up;
-            f[i] = fmaf(up, u, f[i]);
-          }
+    auto add = [&](int i, float xv) {
+      const float u = xv - tau[i];
+      if (u > 0.f) {
+        k[i] += 1.f;
+        a[i] += u;
+        umin[i] = fminf(umin[i], u);
+        if (kind == 0) {
+          f[i] += u;
+        } else if (kind == 1) {
+          f[i] = fmaf(u, u, f[i]);
+        } else {
+          const float up = exp2f((pw - 1.0f) * log2f(u));
+          fd[i] += up;
+          f[i] = fmaf(up, u, f[i]);
         }
+      }
+    };
+    if constexpr (COLS == 1) {
+#pragma unroll
+      for (int i = 0; i < RW; ++i) add(i, x[i]);
+    } else {
+      for (int c = lane; c < n; c += 64) {
+        float xv[2 * RW];
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+          xv[2 * i] = x[i * stride + c];
+          xv[2 * i + 1] = x[i * stride + c + 32];
+        }
+#pragma unroll
+        for (int e = 0; e < 2 * RW; ++e) add(e >> 1, xv[e]);
       }
     }
 #pragma unroll
@@ -210,6 +194,48 @@ __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride,
   }
 }
 
+// alpha-entmax thresholds of RW rows that share their candidate columns,
+// solved in lockstep by one warp (their reductions interleave).  Row i's
+// logits are x[i * stride + c] for c < n, -inf on non-candidates; columns are
+// read 64 at a time, so the rows must be readable (-inf) up to n rounded up
+// to a multiple of 64.  Same
+// scheme as warp_entmax_tau: Newton from max - 1, where F >= 1, approaches
+// the root from below, and after every step the exact solution on the
+// current support is accepted when it is self-consistent.
+template <int RW>
+__device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride, int n, float alpha, int kind,
+                                                     int lane, float* tau) {
+  const float pw = 1.0f / (alpha - 1.0f);
+  float mx[RW];
+#pragma unroll
+  for (int i = 0; i < RW; ++i) mx[i] = kNegInf;
+  for (int c = lane; c < n; c += 64) {
+#pragma unroll
+    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], fmaxf(x[i * stride + c], x[i * stride + c + 32]));
+  }
+  // The lane maxima are a subset of the row, and the threshold of any subset
+  // is a lower bound on the row's (F over the row >= F over the subset): solve
+  // the 32 lane maxima first, in registers, and start the passes over the row
+  // from there instead of from max - 1.
+  float lmx[RW];
+#pragma unroll
+  for (int i = 0; i < RW; ++i) lmx[i] = mx[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
+  }
+  bool done[RW];
+#pragma unroll
+  for (int i = 0; i < RW; ++i) {
+    tau[i] = mx[i] - 1.0f;
+    done[i] = mx[i] == kNegInf;
+  }
+  entmax_newton_rows<RW, 1>(lmx, 0, 32, pw, kind, lane, tau, done);
+#pragma unroll
+  for (int i = 0; i < RW; ++i) done[i] = mx[i] == kNegInf;
+  entmax_newton_rows<RW, 2>(x, stride, n, pw, kind, lane, tau, done);
+}
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RouteParams p, TileOut to, int tile0) {
   constexpr int RW = G > 4 ? G : 4;  // rows solved together by one warp
@@ -407,7 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
         const int t = pos / p.block;  // the task's positions share their block
         const int ncol = p.causal ? t : n_blocks;
         float tau[RW];
-        warp_entmax_tau_rows<RW>(X + rr0 * kXStride, kXStride, ncol, p.alpha, kind, lane, tau);
+        // thresholds four rows at a time (register budget)
+#pragma unroll
+        for (int r4 = 0; r4 < RW; r4 += 4)
+          warp_entmax_tau_rows<4>(X + (rr0 + r4) * kXStride, kXStride, ncol, p.alpha, kind, lane, tau + r4);
 #pragma unroll
         for (int pp = 0; pp < PPT; ++pp) {
           const int tp = tp0 + pp;
