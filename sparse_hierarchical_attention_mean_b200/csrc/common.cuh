@@ -166,18 +166,17 @@ __device__ __forceinline__ int entmax_kind(float alpha) {
   return alpha == 2.0f ? 0 : (alpha == 1.5f ? 1 : 2);
 }
 
-__device__ inline float warp_entmax_tau(const float* x, int n, float alpha, int lane) {
-  const float pw = 1.0f / (alpha - 1.0f);
-  const int kind = entmax_kind(alpha);
-  float mx = kNegInf;
-  for (int c = lane; c < n; c += 32) mx = fmaxf(mx, x[c]);
-  mx = warp_max(mx);
-  float tau = mx - 1.0f;
+// Newton passes from below with the exact check on the current support (see
+// warp_entmax_tau).  SUBSET: each lane contributes the single value v;
+// otherwise the row is x[c] for c < n, strided over the lanes.  tau must be a
+// lower bound of the root (F(tau) >= 1).
+template <bool SUBSET>
+__device__ inline float entmax_newton(const float* x, float v, int n, float tau, float pw, int kind, int lane) {
   for (int it = 0; it < 100; ++it) {
     float f = 0.f, fd = 0.f, a = 0.f, umin = 3.0e38f;
     int k = 0;
-    for (int c = lane; c < n; c += 32) {
-      const float u = x[c] - tau;
+    for (int c = SUBSET ? 0 : lane; c < (SUBSET ? 1 : n); c += 32) {
+      const float u = (SUBSET ? v : x[c]) - tau;
       if (u > 0.f) {
         ++k;
         a += u;
@@ -218,6 +217,27 @@ __device__ inline float warp_entmax_tau(const float* x, int n, float alpha, int 
     }
   }
   return tau;
+}
+
+// alpha-entmax threshold of one row x[0..n) by one warp.  F(tau) =
+// sum_c [x_c - tau]_+^(1/(alpha-1)) is convex and decreasing, F(max - 1) >= 1,
+// so Newton from below approaches the root monotonically; after every step
+// the exact solution on the current support (linear for sparsemax, quadratic
+// for alpha = 1.5) is accepted when it is self-consistent.  The start is the
+// threshold of the 32 lane maxima, solved first in registers: they are a
+// subset of the row and F over a subset is below F over the row, so that
+// threshold is a lower bound too, and usually one pass over the row from
+// there finds the exact support.
+__device__ inline float warp_entmax_tau(const float* x, int n, float alpha, int lane) {
+  const float pw = 1.0f / (alpha - 1.0f);
+  const int kind = entmax_kind(alpha);
+  float lm = kNegInf;
+  for (int c = lane; c < n; c += 32) lm = fmaxf(lm, x[c]);
+  const float mx = warp_max(lm);
+  float tau = mx - 1.0f;
+  if (mx == kNegInf) return tau;
+  tau = entmax_newton<true>(nullptr, lm, 1, tau, pw, kind, lane);
+  return entmax_newton<false>(x, 0.f, n, tau, pw, kind, lane);
 }
 
 // Status word kept in the first bytes of every workspace.
