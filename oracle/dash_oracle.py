@@ -21,7 +21,9 @@ the pages leave open (all fixed here and in the CUDA path alike):
 * gamma, the routing temperature in "w = alpha-entmax(gamma z)", is
   1/sqrt(d).
 * The summary of block c is the mean of its keys times W_s, taken as a row
-  vector times the matrix: s_c = mean_j(k_j) @ W_s.
+  vector times the matrix: s_c = mean_j(k_j) @ W_s.  The learned-query form
+  (block_summaries_sdpa) weights the keys by softmax(q_bar . k_j / sqrt(d))
+  over the block, with one q_bar per KV head; q_bar = 0 is the mean.
 * Causal: the candidates of a query at position pos are the complete blocks
   before its own block t = pos // B (N = t of them); the own block is the
   always-included "diagonal" block, masked to tokens <= pos.  Non-causal:
@@ -69,6 +71,36 @@ def block_summaries(k: np.ndarray, w_s: np.ndarray, block: int, n_tokens: int) -
         lo, hi = c * block, min(n_tokens, (c + 1) * block)
         mean = k[lo:hi].sum(axis=0) / (hi - lo)
         out[c] = mean @ w_s
+    return out
+
+
+def block_summaries_sdpa(k: np.ndarray, w_s: np.ndarray, qbar: np.ndarray, block: int, n_tokens: int) -> np.ndarray:
+    """Stage 0 with the learned summary query ("Stage 0: local chunk summary").
+
+    The pages' summariser: a learned query vector q_bar attends to the keys of
+    each chunk through local scaled dot-product attention, and the keys are
+    what it averages (the summary lives in key space, so stage 1 can score
+    queries against it).  For block c with valid tokens j:
+
+        a_j = q_bar . k_j / sqrt(d),   w = softmax(a) over the block,
+        s_c = (sum_j w_j k_j) @ W_s.
+
+    q_bar = 0 gives uniform weights, i.e. block_summaries (the pages' zero
+    initialisation).  k: [L, d] keys of one (batch, KV head); qbar: [d], the
+    query of that KV head.  Returns [ceil(n_tokens / block), d].
+    """
+    k = np.asarray(k, dtype=np.float64)
+    w_s = np.asarray(w_s, dtype=np.float64)
+    qbar = np.asarray(qbar, dtype=np.float64)
+    d = k.shape[1]
+    n_blocks = -(-n_tokens // block)
+    out = np.zeros((n_blocks, d))
+    for c in range(n_blocks):
+        lo, hi = c * block, min(n_tokens, (c + 1) * block)
+        a = k[lo:hi] @ qbar / math.sqrt(d)
+        w = np.exp(a - a.max())
+        w /= w.sum()
+        out[c] = (w @ k[lo:hi]) @ w_s
     return out
 
 

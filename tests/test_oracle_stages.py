@@ -16,8 +16,11 @@ import torch
 import torch.nn.functional as F
 from scipy.optimize import minimize
 
+from scipy.special import expit
+
 from oracle.dash_oracle import (
     block_summaries,
+    block_summaries_sdpa,
     decode_pair,
     diagonal_bias,
     forward,
@@ -54,6 +57,61 @@ def test_block_mean_matches_numpy_and_orientation():
     # a partial trailing block is averaged over its valid tokens only
     s3 = block_summaries(k, np.eye(d), B, 600)
     np.testing.assert_allclose(s3[-1], k[576:600].mean(axis=0), atol=1e-14)
+
+
+def test_sdpa_summary_hand_example():
+    # d = 2, W_s = I, one block of two orthogonal keys; q_bar chosen so the
+    # scaled scores are (ln 3, 0): weights 3/4 and 1/4
+    k = np.array([[1.0, 0.0], [0.0, 1.0]])
+    qbar = np.array([math.sqrt(2.0) * math.log(3.0), 0.0])
+    s = block_summaries_sdpa(k, np.eye(2), qbar, block=2, n_tokens=2)
+    np.testing.assert_allclose(s, [[0.75, 0.25]], atol=1e-15)
+
+
+def test_sdpa_summary_zero_query_is_mean_pooling():
+    # the pages' zero initialisation behaves as uniform mean pooling
+    rng = np.random.default_rng(3)
+    L, d, B = 700, 32, 64
+    k = rng.normal(size=(L, d))
+    w = np.eye(d) + 0.1 * rng.normal(size=(d, d))
+    np.testing.assert_allclose(block_summaries_sdpa(k, w, np.zeros(d), B, L), block_summaries(k, w, B, L),
+                               atol=1e-13)
+
+
+def test_sdpa_summary_two_token_logistic_form():
+    # two tokens: s = sigmoid(a) k1 + sigmoid(-a) k2 with a = q_bar.(k1 - k2)/sqrt(d)
+    rng = np.random.default_rng(4)
+    d = 8
+    for _ in range(20):
+        k = rng.normal(size=(2, d))
+        qbar = 3.0 * rng.normal(size=d)
+        a = qbar @ (k[0] - k[1]) / math.sqrt(d)
+        ref = expit(a) * k[0] + expit(-a) * k[1]
+        np.testing.assert_allclose(block_summaries_sdpa(k, np.eye(d), qbar, 2, 2)[0], ref, atol=1e-13)
+
+
+def test_sdpa_summary_invariances_and_limits():
+    rng = np.random.default_rng(5)
+    d, B = 16, 8
+    w = rng.normal(size=(d, d))
+    # identical keys: the summary is that key whatever the query
+    k = np.tile(rng.normal(size=(1, d)), (B, 1))
+    np.testing.assert_allclose(block_summaries_sdpa(k, w, 50.0 * rng.normal(size=d), B, B)[0], k[0] @ w,
+                               atol=1e-12)
+    # permuting the tokens of a block changes nothing
+    k = rng.normal(size=(B, d))
+    qbar = rng.normal(size=d)
+    s = block_summaries_sdpa(k, w, qbar, B, B)
+    np.testing.assert_allclose(block_summaries_sdpa(k[rng.permutation(B)], w, qbar, B, B), s, atol=1e-13)
+    # a query aligned ever more strongly with one key selects that key
+    m = 5
+    far = block_summaries_sdpa(k, w, 1e4 * k[m], B, B)[0]
+    np.testing.assert_allclose(far, k[m] @ w, atol=1e-9)
+    # a partial trailing block weights only its valid tokens
+    k = rng.normal(size=(3 * B, d))
+    s = block_summaries_sdpa(k, np.eye(d), qbar, B, 2 * B + 3)
+    np.testing.assert_allclose(s[-1], block_summaries_sdpa(k[2 * B:2 * B + 3], np.eye(d), qbar, B, 3)[0],
+                               atol=1e-14)
 
 
 # --------------------------------------------------------------------------
