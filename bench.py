@@ -402,6 +402,18 @@ def run_decode(dash, cfg, steps, warmup, world, rank):
     e1.record(stream)
     torch.cuda.synchronize()
     summarize_ms = e0.elapsed_time(e1)
+    # the same cache with learned summary queries (seeded q_bar per KV head)
+    qbar = torch.from_numpy(np.random.default_rng(11).normal(size=(Hkv, d)) * 3.0).float().cuda()
+    summ_q = torch.zeros_like(summ)
+    dash.summarize(k, w, cfg.block, seqlens=sl, summaries=summ_q, qbar=qbar)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    dash.summarize(k, w, cfg.block, seqlens=sl, summaries=summ_q, qbar=qbar)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    summarize_sdpa_ms = e0.elapsed_time(e1)
+    del summ_q
+    pool_bytes = float(sl.double().sum()) * Hkv * d * k.element_size() + float(summ.numel()) * 4
     out = torch.empty_like(q)
     ws = torch.empty(dash.decode_workspace_size(q, k, cfg.block, T), dtype=torch.uint8, device="cuda")
 
@@ -436,7 +448,8 @@ def run_decode(dash, cfg, steps, warmup, world, rank):
     total = bytes_summ + bytes_kv + bytes_q
     sparsity = 1.0 - float(cnt.sum()) / float(n_cand.sum() * Hkv)
     return {"us": us, "bytes": total, "bytes_summaries": bytes_summ, "sparsity": sparsity,
-            "summarize_ms": summarize_ms, "status": status, "clocks": clk.summary()}
+            "summarize_ms": summarize_ms, "summarize_sdpa_ms": summarize_sdpa_ms, "pool_bytes": pool_bytes,
+            "status": status, "clocks": clk.summary()}
 
 
 # --------------------------------------------------------------------------- oracle timing
@@ -552,7 +565,8 @@ def main():
         finish(world)
         return
     if pre is None:
-        print(json.dumps({"decode_only": True, "us_per_step": None if dec is None else dec["us"]}), flush=True)
+        print(json.dumps({"decode_only": True, "us_per_step": None if dec is None else dec["us"],
+                          "decode": None if dec is None else decode_object(dec, dcfg, pk)}), flush=True)
         barrier(world)
         finish(world)
         return
@@ -598,19 +612,28 @@ def main():
         "cpu_baseline": cpu,
     }
     if dec is not None:
-        ach = dec["bytes"] / (dec["us"] * 1e-6) / 1e9
-        line["decode"] = {
-            "workload": f"decode: {dcfg.batch} seqs, 32/8 heads, d=128, bf16, cache 131072, L ~ U[65536, 131072], "
-                        "block 64",
-            "us_per_step": dec["us"], "sparsity": dec["sparsity"], "summarize_ms": dec["summarize_ms"],
-            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": ach / pk["hbm_gbs"], "traffic": None, "bytes_per_step": dec["bytes"],
-                         "peak_source": f"{pk['source']} HBM copy"},
-            "clocks": dec["clocks"], "device_status": dec["status"], "gpu_launches_per_step": 4,
-        }
+        line["decode"] = decode_object(dec, dcfg, pk)
     print(json.dumps(line), flush=True)
     barrier(world)
     finish(world)
+
+
+def decode_object(dec, dcfg, pk):
+    ach = dec["bytes"] / (dec["us"] * 1e-6) / 1e9
+    return {
+        "workload": f"decode: {dcfg.batch} seqs, 32/8 heads, d=128, bf16, cache 131072, L ~ U[65536, 131072], "
+                    "block 64",
+        "us_per_step": dec["us"], "sparsity": dec["sparsity"],
+        "summary_cache": {"bytes": dec["pool_bytes"], "mean_ms": dec["summarize_ms"],
+                          "mean_gbs": dec["pool_bytes"] / (dec["summarize_ms"] * 1e-3) / 1e9,
+                          "learned_query_ms": dec["summarize_sdpa_ms"],
+                          "learned_query_gbs": dec["pool_bytes"] / (dec["summarize_sdpa_ms"] * 1e-3) / 1e9,
+                          "peak_gbs": pk["hbm_gbs"]},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": ach / pk["hbm_gbs"], "traffic": None, "bytes_per_step": dec["bytes"],
+                     "peak_source": f"{pk['source']} HBM copy"},
+        "clocks": dec["clocks"], "device_status": dec["status"], "gpu_launches_per_step": 4,
+    }
 
 
 def finish(world):

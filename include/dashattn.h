@@ -125,6 +125,21 @@ dash_status_t dash_attn_summarize(const dash_tensor_t* k, const int32_t* seqlens
                                   dash_stream_t stream);
 
 /*
+ * Stage 0 with the learned summary query ("Stage 0: local chunk summary":
+ * a learned query vector attends to the keys of each chunk through local
+ * scaled dot-product attention; initialised at zero it is uniform mean
+ * pooling).  Same as dash_attn_summarize, with the mean replaced by
+ *   sum_j softmax_j(qbar[g] . k[b, j, g, :] / sqrt(d)) k[b, j, g, :]
+ * over the block's valid tokens, then @ w_s.
+ *   qbar  device fp32 [Hkv, d], one query per KV head, 16-byte aligned, or
+ *         NULL (then identical to dash_attn_summarize).
+ * Errors and the other arguments as for dash_attn_summarize.
+ */
+dash_status_t dash_attn_summarize_sdpa(const dash_tensor_t* k, const int32_t* seqlens, const float* w_s,
+                                       const float* qbar, int block, float* summaries, int64_t t_cap,
+                                       int64_t first_block, dash_stream_t stream);
+
+/*
  * Bytes of workspace dash_attn_decode needs for q [B, 1, H, d] against a KV
  * cache [B, Lmax, Hkv, d] with summaries of capacity t_cap blocks.
  */

@@ -37,6 +37,7 @@ EXPORTED = (
     "dash_attn_fwd_workspace_size",
     "dash_attn_fwd",
     "dash_attn_summarize",
+    "dash_attn_summarize_sdpa",
     "dash_attn_decode_workspace_size",
     "dash_attn_decode",
     "dash_attn_route_workspace_size",
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "dash_attn_fwd_workspace_size": (sz, [T, T, i32]),
         "dash_attn_fwd": (i32, [T, T, T, vp, f32, i32, i32, T, vp, sz, vp]),
         "dash_attn_summarize": (i32, [T, vp, vp, i32, vp, i64, i64, vp]),
+        "dash_attn_summarize_sdpa": (i32, [T, vp, vp, vp, i32, vp, i64, i64, vp]),
         "dash_attn_decode_workspace_size": (sz, [T, T, i32, i64]),
         "dash_attn_decode": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp, sz, vp]),
         "dash_attn_route_workspace_size": (sz, [T, i64, i64, i32]),
@@ -168,15 +170,25 @@ def n_blocks(seq: int, block: int) -> int:
 
 
 def summarize(k: torch.Tensor, w_s: torch.Tensor, block: int, seqlens: torch.Tensor | None = None,
-              summaries: torch.Tensor | None = None, first_block: int = 0, stream=None) -> torch.Tensor:
-    """Block summaries [B, Hkv, t_cap, d] fp32 (see dash_attn_summarize)."""
+              summaries: torch.Tensor | None = None, first_block: int = 0, stream=None,
+              qbar: torch.Tensor | None = None) -> torch.Tensor:
+    """Block summaries [B, Hkv, t_cap, d] fp32 (see dash_attn_summarize).
+
+    qbar: optional fp32 [Hkv, d] learned summary queries (dash_attn_summarize_sdpa).
+    """
     B, S, Hkv, d = k.shape
     if summaries is None:
         summaries = torch.zeros((B, Hkv, n_blocks(S, block), d), dtype=torch.float32, device=k.device)
     assert summaries.is_contiguous() and summaries.dtype == torch.float32
     kd = _desc(k)
-    _check(_lib.dash_attn_summarize(ctypes.byref(kd), _ptr(seqlens), w_s.data_ptr(), block,
-                                    summaries.data_ptr(), summaries.shape[2], first_block, _stream(stream)))
+    if qbar is None:
+        _check(_lib.dash_attn_summarize(ctypes.byref(kd), _ptr(seqlens), w_s.data_ptr(), block,
+                                        summaries.data_ptr(), summaries.shape[2], first_block, _stream(stream)))
+    else:
+        assert qbar.is_contiguous() and qbar.dtype == torch.float32 and tuple(qbar.shape) == (Hkv, d)
+        _check(_lib.dash_attn_summarize_sdpa(ctypes.byref(kd), _ptr(seqlens), w_s.data_ptr(), qbar.data_ptr(),
+                                             block, summaries.data_ptr(), summaries.shape[2], first_block,
+                                             _stream(stream)))
     return summaries
 
 

@@ -246,11 +246,19 @@ size_t dash_attn_fwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t*
 
 dash_status_t dash_attn_summarize(const dash_tensor_t* k, const int32_t* seqlens, const float* w_s, int block,
                                   float* summaries, int64_t t_cap, int64_t first_block, dash_stream_t stream) {
+  return dash_attn_summarize_sdpa(k, seqlens, w_s, nullptr, block, summaries, t_cap, first_block, stream);
+}
+
+dash_status_t dash_attn_summarize_sdpa(const dash_tensor_t* k, const int32_t* seqlens, const float* w_s,
+                                       const float* qbar, int block, float* summaries, int64_t t_cap,
+                                       int64_t first_block, dash_stream_t stream) {
   dash_status_t st;
   if ((st = check_tensor(k, "k"))) return st;
   if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
   if (!w_s || !summaries) return fail(DASH_ERR_INVALID_ARGUMENT, "null w_s or summaries");
   if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(w_s) % 16 || reinterpret_cast<uintptr_t>(qbar) % 16)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "w_s or qbar not 16-byte aligned");
   const int64_t T = (k->s + block - 1) / block;
   if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block) = %lld", (long long)t_cap, (long long)T);
   if (first_block < 0) return fail(DASH_ERR_INVALID_ARGUMENT, "first_block < 0");
@@ -264,6 +272,7 @@ dash_status_t dash_attn_summarize(const dash_tensor_t* k, const int32_t* seqlens
   p.block = block;
   p.seqlens = seqlens;
   p.w_s = w_s;
+  p.qbar = qbar;
   p.summaries = summaries;
   p.t_cap = t_cap;
   p.first_block = first_block;

@@ -26,6 +26,7 @@ struct PoolParams {
   int B, S, Hkv, D, block;
   const int32_t* seqlens;  // nullable
   const float* w_s;        // [D, D]
+  const float* qbar;       // [Hkv, D] learned summary queries, or null (mean pooling)
   float* summaries;        // [B, Hkv, t_cap, D]
   int64_t t_cap;
   int64_t first_block;

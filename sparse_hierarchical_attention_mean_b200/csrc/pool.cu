@@ -6,6 +6,10 @@
 // which is uniform mean pooling; here the summary is the block mean followed
 // by the fixed projection W_s (row vector times matrix).
 //
+// With a learned summary query q_bar (one per KV head) the block's keys are
+// weighted by softmax_j(q_bar . k_j / sqrt(d)) instead of uniformly; q_bar = 0
+// is the mean (the pages' zero initialisation).
+//
 // HBM-bound: every key is read once with 16-byte vector loads; the mean and
 // the projection are fp32.  One CTA pools up to 32 consecutive blocks of one
 // (batch, KV head) and projects them together so each W_s row is read once
@@ -27,7 +31,7 @@ constexpr int kMaxBpc = 32;
 //   shuffles.  No barrier per block.
 //   Projection: means[nb][D] x W_s[D][D] with a 4 x 4 (blocks x columns)
 //   register tile per thread; W_s rows are read as float4 through L1.
-template <typename T, int D>
+template <typename T, int D, bool SDPA>
 __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
   constexpr int EPV = Elt<T>::kPerVec;     // elements per 16-byte vector
   constexpr int VPR = D / EPV;             // vectors per key row (8, 16 or 32)
@@ -48,35 +52,118 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
   const int vcol = lane % VPR, vrow = lane / VPR;
   const T* kbase = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh + vcol * EPV;
 
-  for (int i = warp; i < nb; i += kWarpsP) {
-    const int64_t lo = (c_begin + i) * p.block;
-    const int64_t hi = lo + p.block < n_tok ? lo + p.block : (int64_t)n_tok;
-    float acc[EPV];
+  if constexpr (!SDPA) {
+    for (int i = warp; i < nb; i += kWarpsP) {
+      const int64_t lo = (c_begin + i) * p.block;
+      const int64_t hi = lo + p.block < n_tok ? lo + p.block : (int64_t)n_tok;
+      float acc[EPV];
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
-    for (int64_t j0 = lo; j0 < hi; j0 += 8 * RPL) {
-      uint4 v[8];
+      for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
+      for (int64_t j0 = lo; j0 < hi; j0 += 8 * RPL) {
+        uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t j = j0 + u * RPL + vrow;
-        v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kbase + j * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < 8; ++u) {
+          const int64_t j = j0 + u * RPL + vrow;
+          v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kbase + j * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float f[EPV];
+          Elt<T>::to_float(v[u], f);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) acc[e] += f[e];
+        }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float f[EPV];
-        Elt<T>::to_float(v[u], f);
+      for (int off = VPR; off < 32; off <<= 1)
 #pragma unroll
-        for (int e = 0; e < EPV; ++e) acc[e] += f[e];
+        for (int e = 0; e < EPV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+      if (vrow == 0) {
+        const float inv = 1.0f / (float)(hi - lo);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) means[i][vcol * EPV + e] = acc[e] * inv;
       }
     }
+  } else {
+    // learned summary query: weights softmax_j(q_bar . k_j / sqrt(D)) over the
+    // block.  Each lane keeps an online softmax (reference max, denominator,
+    // weighted key sum) over its rows; the row score is the sum of the
+    // partial dot products of the VPR lanes holding the row; the lanes of
+    // the block merge at the end.  Scores are in the log2 domain.
+    float qv[EPV];
+    {
+      const float sc = rsqrtf((float)D) * kLog2e;
+      const float* qb = p.qbar + (int64_t)g * D + vcol * EPV;
 #pragma unroll
-    for (int off = VPR; off < 32; off <<= 1)
+      for (int e = 0; e < EPV; ++e) qv[e] = __ldg(qb + e) * sc;
+    }
+    for (int i = warp; i < nb; i += kWarpsP) {
+      const int64_t lo = (c_begin + i) * p.block;
+      const int64_t hi = lo + p.block < n_tok ? lo + p.block : (int64_t)n_tok;
+      float acc[EPV], m = kNegInf, den = 0.f;
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
-    if (vrow == 0) {
-      const float inv = 1.0f / (float)(hi - lo);
+      for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
+      for (int64_t j0 = lo; j0 < hi; j0 += 8 * RPL) {
+        uint4 v[8];
 #pragma unroll
-      for (int e = 0; e < EPV; ++e) means[i][vcol * EPV + e] = acc[e] * inv;
+        for (int u = 0; u < 8; ++u) {
+          const int64_t j = j0 + u * RPL + vrow;
+          v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kbase + j * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float f[EPV];
+          Elt<T>::to_float(v[u], f);
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) d = fmaf(qv[e], f[e], d);
+          a[u] = d;
+        }
+#pragma unroll
+        for (int off = 1; off < VPR; off <<= 1)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a[u] += __shfl_xor_sync(0xffffffffu, a[u], off);
+        float mr = m;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u * RPL + vrow >= hi) a[u] = kNegInf;
+          mr = fmaxf(mr, a[u]);
+        }
+        const float ms = mr == kNegInf ? 0.f : mr;
+        const float corr = exp2f(m - ms);
+        den *= corr;
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) acc[e] *= corr;
+        m = mr;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float w = exp2f(a[u] - ms);
+          float f[EPV];
+          Elt<T>::to_float(v[u], f);
+          den += w;
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+        }
+      }
+      // merge the lanes that hold the same columns (different rows)
+#pragma unroll
+      for (int off = VPR; off < 32; off <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+        const float dn = __shfl_xor_sync(0xffffffffu, den, off);
+        const float mm = fmaxf(m, mo);
+        const float ms = mm == kNegInf ? 0.f : mm;
+        const float c0 = exp2f(m - ms), c1 = exp2f(mo - ms);
+        den = den * c0 + dn * c1;
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) acc[e] = acc[e] * c0 + __shfl_xor_sync(0xffffffffu, acc[e], off) * c1;
+        m = mm;
+      }
+      if (vrow == 0) {
+        const float inv = 1.0f / den;
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) means[i][vcol * EPV + e] = acc[e] * inv;
+      }
     }
   }
   __syncthreads();
@@ -119,7 +206,10 @@ cudaError_t launch_typed(const PoolParams& p, cudaStream_t stream) {
   int bpc = kMaxBpc;
   while (bpc > kWarpsP && total / bpc < 148 * 4) bpc /= 2;
   dim3 grid((unsigned)((span + bpc - 1) / bpc), p.Hkv, p.B);
-  pool_kernel<T, D><<<grid, kThreads, 0, stream>>>(p, bpc);
+  if (p.qbar)
+    pool_kernel<T, D, true><<<grid, kThreads, 0, stream>>>(p, bpc);
+  else
+    pool_kernel<T, D, false><<<grid, kThreads, 0, stream>>>(p, bpc);
   return cudaGetLastError();
 }
 

@@ -133,6 +133,11 @@ def test_decode_and_route_reject_bad_arguments():
     assert st == 1
     st = lib.dash_attn_summarize(ctypes.byref(kc), None, FAKE, 64, FAKE, 10, 0, None)
     assert st == 1 and "t_cap" in lib.dash_attn_last_error().decode()
+    # learned summary queries: misaligned qbar, and the same checks as summarize
+    st = lib.dash_attn_summarize_sdpa(ctypes.byref(kc), None, FAKE, FAKE + 4, 64, FAKE, 64, 0, None)
+    assert st == 1 and "aligned" in lib.dash_attn_last_error().decode()
+    st = lib.dash_attn_summarize_sdpa(ctypes.byref(kc), None, FAKE, FAKE, 96, FAKE, 64, 0, None)
+    assert st == 2
 
 
 def test_binding_refuses_host_tensors():

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from gen import Config, full_inputs, get_config, kv_values, make_plan
-from oracle.dash_oracle import block_summaries
+from oracle.dash_oracle import block_summaries, block_summaries_sdpa
 from tests._parity import (
     OUT_TOL,
     check_p_dense,
@@ -139,6 +139,31 @@ def test_summarize_incremental_and_seqlens(dash):
     ref = block_summaries(kk, inp["plan"].w_s.double().numpy(), cfg.block, 333)
     got = s2[0, 3, : len(ref)].cpu().numpy()
     assert np.abs(got - ref).max() <= 2e-5 * max(1.0, np.abs(ref).max())
+
+
+@pytest.mark.parametrize("name,scale", [("prefill_small", 0.0), ("prefill_small", 3.0), ("prefill_small", 30.0),
+                                        ("g2_d64", 3.0), ("g1_b128", 10.0), ("f32_d128", 3.0)])
+def test_summarize_sdpa(dash, name, scale):
+    """Stage 0 with learned summary queries against the oracle; a trailing partial block and seqlens."""
+    cfg = SMALL[name]
+    inp = full_inputs(cfg, device="cuda")
+    k, w, plan = inp["k"], inp["w_s"], inp["plan"]
+    d, Hkv = cfg.head_dim, cfg.kv_heads
+    qbar = torch.from_numpy(np.random.default_rng(11).normal(size=(Hkv, d)) * scale).float()
+    sl = torch.tensor([cfg.seq - 37] * cfg.batch, dtype=torch.int32, device="cuda")
+    got = dash.summarize(k, w, cfg.block, qbar=qbar.cuda())
+    got_sl = dash.summarize(k, w, cfg.block, seqlens=sl, qbar=qbar.cuda())
+    torch.cuda.synchronize()
+    if scale == 0.0:
+        mean = dash.summarize(k, w, cfg.block)
+        assert torch.allclose(got, mean, rtol=1e-6, atol=1e-6)
+    for b in range(cfg.batch):
+        for g in _kv_subset(cfg):
+            kk = kv_values(cfg, plan, "k", b, range(cfg.seq), [g], as_float32=True)[:, 0].double().numpy()
+            for n_tok, out in ((cfg.seq, got), (cfg.seq - 37, got_sl)):
+                ref = block_summaries_sdpa(kk, plan.w_s.double().numpy(), qbar[g].double().numpy(), cfg.block, n_tok)
+                err = np.abs(out[b, g, : len(ref)].cpu().numpy() - ref).max()
+                assert err <= 2e-5 * max(1.0, np.abs(ref).max()), f"{name} scale {scale} b{b} g{g}: {err:.3g}"
 
 
 DECODE_SMALL = {
