@@ -278,11 +278,17 @@ def candidate_blocks(pos: int, block: int, n_tokens: int, causal: bool) -> tuple
 
 
 def forward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: np.ndarray,
-                pos: int, n_tokens: int, block: int, alpha: float, causal: bool = True) -> dict:
+                pos: int, n_tokens: int, block: int, alpha: float, causal: bool = True,
+                sigma: float = 1.0) -> dict:
     """Stages 1 and 2 for one query position of one KV group.
 
     q_group: [G, d]; k, v: [L, d] of the KV head; summaries: all block
     summaries of that head (stage 0); n_tokens: valid context length.
+    sigma: strength of the prior ("Stage 2: prior-induced sparse softmax"
+    names a strength that balances the prior against the uniform baseline):
+    the bias is sigma * log p_bar on the selected blocks and sigma * log(1/N)
+    on the diagonal block, so a uniform prior still gives full attention for
+    every sigma, and sigma = 0 is plain softmax over the selected tokens.
     Returns the route dict of :func:`route_row` (with ``idx`` as block ids)
     plus ``beta`` and ``out`` [G, d].
     """
@@ -294,16 +300,29 @@ def forward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: np
     for c, lp in zip(sel, r["logp"]):
         span = np.arange(c * block, min(n_tokens, (c + 1) * block))
         tok.append(span)
-        bias.append(np.full(len(span), lp))
+        bias.append(np.full(len(span), sigma * lp))
     last = pos if causal else min(n_tokens, (t + 1) * block) - 1
     span = np.arange(t * block, last + 1)
     tok.append(span)
-    bias.append(np.full(len(span), beta))
+    bias.append(np.full(len(span), sigma * beta))
     tok = np.concatenate(tok)
     bias = np.concatenate(bias)
     out = np.stack([prior_softmax_attend(q_group[h], k[tok], v[tok], bias) for h in range(len(q_group))])
     r.update({"blocks": np.array(sel, dtype=np.int64), "cand": cand, "beta": beta, "out": out})
     return r
+
+
+def lists_to_mask(idx: np.ndarray, cnt: np.ndarray, n_words: int) -> np.ndarray:
+    """Bit-packed active-block mask (the pages' kernel walks such a mask of the
+    active chunks): word w of a row has bit b set iff block 32 w + b is among
+    the row's cnt selected blocks.  idx [..., t_cap], cnt [...] -> [..., n_words] uint32."""
+    idx = np.asarray(idx)
+    cnt = np.asarray(cnt)
+    out = np.zeros(cnt.shape + (n_words,), dtype=np.uint32)
+    for pos in np.ndindex(cnt.shape):
+        for c in idx[pos][: int(cnt[pos])]:
+            out[pos + (int(c) // 32,)] |= np.uint32(1 << (int(c) % 32))
+    return out
 
 
 def forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, alpha: float, block: int,

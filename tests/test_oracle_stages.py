@@ -25,6 +25,7 @@ from oracle.dash_oracle import (
     diagonal_bias,
     forward,
     forward_row,
+    lists_to_mask,
     prior_softmax_attend,
     route_row,
 )
@@ -195,6 +196,65 @@ def test_zero_w_s_is_full_attention(causal):
     for (pos, g), r in res["routes"].items():
         assert len(r["blocks"]) == len(r["cand"])
         assert r["beta"] == diagonal_bias(len(r["cand"]))
+
+
+@pytest.mark.parametrize("sigma", [0.0, 0.3, 2.5])
+def test_uniform_prior_is_full_attention_for_any_sigma(sigma):
+    """Tempering scales every bias by sigma; with a uniform prior all biases are
+    equal, so the forward is plain causal attention whatever sigma is."""
+    rng = np.random.default_rng(8)
+    S, G, d, B = 150, 2, 16, 16
+    q, k, v = rng.normal(size=(S, G, d)), rng.normal(size=(S, 1, d)), rng.normal(size=(S, 1, d))
+    summ = np.zeros((-(-S // B), d))  # zero summaries: every candidate uniform
+    ref = _sdpa(q, k, v, True)
+    for pos in (0, 17, 64, 149):
+        r = forward_row(q[pos], k[:, 0], v[:, 0], summ, pos, S, B, 1.5, True, sigma=sigma)
+        np.testing.assert_allclose(r["out"], ref[pos], atol=1e-12)
+
+
+def test_sigma_zero_is_softmax_over_the_selected_tokens():
+    """sigma = 0 drops the prior: masked scaled dot-product attention (torch, fp64)
+    over the tokens of the selected blocks and the causal diagonal block."""
+    rng = np.random.default_rng(9)
+    S, G, d, B = 300, 3, 16, 16
+    q, k, v = rng.normal(size=(S, G, d)), rng.normal(size=(S, d)), rng.normal(size=(S, d))
+    for b in range(4):  # plant a few strong blocks so the selection is sparse
+        k[b * 3 * B:(b * 3 + 1) * B] += 3.0 * q[299, 0] / np.linalg.norm(q[299, 0])
+    summ = block_summaries(k, np.eye(d), B, S)
+    sparse = []
+    for pos in (100, 255, 299):
+        r = forward_row(q[pos], k, v, summ, pos, S, B, 1.5, True, sigma=0.0)
+        t = pos // B
+        allowed = np.zeros(S, dtype=bool)
+        for c in r["blocks"]:
+            allowed[c * B:(c + 1) * B] = True
+        allowed[t * B:pos + 1] = True
+        sparse.append(bool(allowed.sum() < pos + 1))
+        qq = torch.from_numpy(q[pos])[:, None, :]
+        kk = torch.from_numpy(k)[None].expand(G, S, d)
+        vv = torch.from_numpy(v)[None].expand(G, S, d)
+        ref = F.scaled_dot_product_attention(qq, kk, vv, attn_mask=torch.from_numpy(allowed)[None, None, :])
+        np.testing.assert_allclose(r["out"], ref[:, 0].numpy(), atol=1e-12)
+    assert any(sparse)  # the selection skipped blocks for some row
+
+
+def test_lists_to_mask():
+    idx = np.array([[[0, 5, 31, 32, 70, -1], [3, -1, -1, -1, -1, -1]]])
+    cnt = np.array([[5, 1]])
+    m = lists_to_mask(idx, cnt, 3)
+    assert m.shape == (1, 2, 3) and m.dtype == np.uint32
+    assert m[0, 0].tolist() == [(1 << 0) | (1 << 5) | (1 << 31), 1 << 0, 1 << 6]
+    assert m[0, 1].tolist() == [1 << 3, 0, 0]
+    # round trip against the set of listed blocks
+    rng = np.random.default_rng(2)
+    idx = np.sort(rng.choice(100, size=(4, 40), replace=True), axis=1)
+    idx = np.stack([np.unique(r)[:30] if len(np.unique(r)) >= 30 else np.pad(np.unique(r), (0, 30 - len(np.unique(r))))
+                    for r in idx])
+    cnt = np.array([len(set(r.tolist())) if len(set(r.tolist())) < 30 else 30 for r in idx])
+    m = lists_to_mask(idx, cnt, 4)
+    for r in range(4):
+        bits = np.unpackbits(m[r].view(np.uint8), bitorder="little")
+        assert set(np.nonzero(bits)[0].tolist()) == set(idx[r][: cnt[r]].tolist())
 
 
 def test_first_block_rows_attend_within_the_block():
