@@ -140,6 +140,43 @@ dash_status_t dash_attn_summarize_sdpa(const dash_tensor_t* k, const int32_t* se
                                        int64_t first_block, dash_stream_t stream);
 
 /*
+ * Options of the variants the pages name beside the path the spec fixes.
+ * Pass NULL for the defaults (sigma = 1, mean pooling).
+ *   sigma  strength of the prior ("Stage 2: prior-induced sparse softmax"
+ *          names a strength that balances the prior against the uniform
+ *          baseline): the stage-2 bias is sigma * log p_bar on a selected
+ *          block and sigma * log(1/N) on the diagonal block, so a uniform
+ *          prior is full attention for every sigma and sigma = 0 is plain
+ *          softmax over the selected tokens.  Finite, >= 0.
+ *   qbar   learned summary queries, device fp32 [Hkv, d], 16-byte aligned,
+ *          or NULL: stage 0 as dash_attn_summarize_sdpa.  Only the prefill
+ *          forward computes summaries; the other calls reject a non-NULL qbar.
+ */
+typedef struct {
+  float sigma;
+  const float* qbar;
+} dash_options_t;
+
+/* dash_attn_fwd with options (opts may be NULL). */
+dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                               const float* w_s, float alpha, int block, int causal, dash_tensor_t* out,
+                               void* workspace, size_t workspace_bytes, const dash_options_t* opts,
+                               dash_stream_t stream);
+
+/*
+ * Bit-packed active-block masks from routing lists (the pages' kernel walks
+ * a mask of the active chunks; the lists of dash_attn_route carry the same
+ * sets plus log p_bar): for each of `rows` rows (e.g. B * Hkv * S of the
+ * route layout), word w of mask[row] has bit b set iff block 32 w + b is
+ * among idx[row, 0 .. cnt[row]).
+ *   idx      device int32 [rows, t_cap]; cnt device int32 [rows].
+ *   mask     device uint32 [rows, n_words], fully written.
+ *   n_words  words per row, n_words * 32 >= t_cap, at most 128.
+ */
+dash_status_t dash_attn_lists_to_mask(const int32_t* idx, const int32_t* cnt, int64_t rows, int64_t t_cap,
+                                      uint32_t* mask, int64_t n_words, dash_stream_t stream);
+
+/*
  * Bytes of workspace dash_attn_decode needs for q [B, 1, H, d] against a KV
  * cache [B, Lmax, Hkv, d] with summaries of capacity t_cap blocks.
  */
@@ -162,6 +199,12 @@ dash_status_t dash_attn_decode(const dash_tensor_t* q, const dash_tensor_t* kcac
                                const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha,
                                int block, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
                                dash_stream_t stream);
+
+/* dash_attn_decode with options (opts may be NULL; opts->qbar must be NULL). */
+dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,
+                                  const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha,
+                                  int block, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                                  const dash_options_t* opts, dash_stream_t stream);
 
 /*
  * Stage 1 alone ("Stage 1: entmax chunk routing", including GQA handling),
@@ -205,6 +248,12 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
                                const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap,
                                int block, int causal, dash_tensor_t* out, void* workspace,
                                size_t workspace_bytes, dash_stream_t stream);
+
+/* dash_attn_sparse with options (opts may be NULL; opts->qbar must be NULL). */
+dash_status_t dash_attn_sparse_ex(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                                  const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                                  int causal, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                                  const dash_options_t* opts, dash_stream_t stream);
 
 /*
  * dash_attn_decode without a workspace argument.  The paper has no

@@ -38,6 +38,10 @@ EXPORTED = (
     "dash_attn_fwd",
     "dash_attn_summarize",
     "dash_attn_summarize_sdpa",
+    "dash_attn_fwd_ex",
+    "dash_attn_sparse_ex",
+    "dash_attn_decode_ex",
+    "dash_attn_lists_to_mask",
     "dash_attn_decode_workspace_size",
     "dash_attn_decode",
     "dash_attn_route_workspace_size",
@@ -53,6 +57,10 @@ class DashError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{_STATUS.get(status, status)}: {message}")
         self.status = status
+
+
+class DashOptions(ctypes.Structure):
+    _fields_ = [("sigma", ctypes.c_float), ("qbar", ctypes.c_void_p)]
 
 
 class DashTensor(ctypes.Structure):
@@ -77,6 +85,7 @@ def _load() -> ctypes.CDLL:
         )
     lib = ctypes.CDLL(_LIB_PATH)
     T = ctypes.POINTER(DashTensor)
+    O = ctypes.POINTER(DashOptions)
     vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
     sig = {
         "dash_attn_version": (i32, []),
@@ -91,6 +100,10 @@ def _load() -> ctypes.CDLL:
         "dash_attn_route": (i32, [T, vp, i64, i64, vp, f32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
         "dash_attn_sparse_workspace_size": (sz, [T, T, i32, i64]),
         "dash_attn_sparse": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, vp]),
+        "dash_attn_fwd_ex": (i32, [T, T, T, vp, f32, i32, i32, T, vp, sz, O, vp]),
+        "dash_attn_sparse_ex": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, O, vp]),
+        "dash_attn_decode_ex": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
+        "dash_attn_lists_to_mask": (i32, [vp, vp, i64, i64, vp, i64, vp]),
         "dash_attn_get_device_status": (i32, [vp, vp]),
         "dash_attn_decode_noalloc": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp]),
     }
@@ -154,6 +167,15 @@ def _ptr(t: torch.Tensor | None):
 def _stream(stream=None):
     s = torch.cuda.current_stream() if stream is None else stream
     return s.cuda_stream
+
+
+def _options(sigma: float, qbar: torch.Tensor | None):
+    """None for the defaults (sigma 1, mean pooling), else a pointer to DashOptions."""
+    if sigma == 1.0 and qbar is None:
+        return None
+    if qbar is not None:
+        assert qbar.is_cuda and qbar.is_contiguous() and qbar.dtype == torch.float32
+    return ctypes.byref(DashOptions(float(sigma), None if qbar is None else qbar.data_ptr()))
 
 
 def _workspace(nbytes: int, device, given: torch.Tensor | None) -> torch.Tensor:
@@ -237,16 +259,32 @@ def sparse_workspace_size(q: torch.Tensor, k: torch.Tensor, block: int, t_cap: i
 
 
 def sparse(q, k, v, idx, logp, cnt, block: int, causal: bool = True, out=None, workspace=None,
-           stream=None) -> torch.Tensor:
-    """Stage 2 alone on caller-given routing (layout of :func:`route`)."""
+           stream=None, sigma: float = 1.0) -> torch.Tensor:
+    """Stage 2 alone on caller-given routing (layout of :func:`route`); sigma: prior strength."""
     out = torch.empty_like(q) if out is None else out
     t_cap = idx.shape[-1]
     ws = _workspace(sparse_workspace_size(q, k, block, t_cap), q.device, workspace)
     qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
-    _check(_lib.dash_attn_sparse(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), idx.data_ptr(),
-                                 logp.data_ptr(), cnt.data_ptr(), t_cap, block, 1 if causal else 0,
-                                 ctypes.byref(od), ws.data_ptr(), ws.numel(), _stream(stream)))
+    opts = _options(sigma, None)
+    args = (ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), idx.data_ptr(), logp.data_ptr(), cnt.data_ptr(),
+            t_cap, block, 1 if causal else 0, ctypes.byref(od), ws.data_ptr(), ws.numel())
+    if opts is None:
+        _check(_lib.dash_attn_sparse(*args, _stream(stream)))
+    else:
+        _check(_lib.dash_attn_sparse_ex(*args, opts, _stream(stream)))
     return out
+
+
+def lists_to_mask(idx: torch.Tensor, cnt: torch.Tensor, n_words: int | None = None, stream=None) -> torch.Tensor:
+    """Bit-packed active-block masks [..., n_words] (int32 bit patterns) from lists idx [..., t_cap], cnt [...]."""
+    t_cap = idx.shape[-1]
+    n_words = -(-t_cap // 32) if n_words is None else n_words
+    rows = cnt.numel()
+    mask = torch.empty(tuple(cnt.shape) + (n_words,), dtype=torch.int32, device=idx.device)
+    assert idx.is_contiguous() and cnt.is_contiguous() and idx.dtype == torch.int32 and cnt.dtype == torch.int32
+    _check(_lib.dash_attn_lists_to_mask(idx.data_ptr(), cnt.data_ptr(), rows, t_cap, mask.data_ptr(), n_words,
+                                        _stream(stream)))
+    return mask
 
 
 # ------------------------------------------------------------------ full forward
@@ -261,13 +299,18 @@ def fwd_workspace_size(q: torch.Tensor, k: torch.Tensor, block: int) -> int:
 
 
 def fwd(q, k, v, w_s, alpha: float, block: int, causal: bool = True, out=None, workspace=None,
-        stream=None) -> torch.Tensor:
-    """Full prefill forward (stages 0-2); see dash_attn_fwd."""
+        stream=None, sigma: float = 1.0, qbar: torch.Tensor | None = None) -> torch.Tensor:
+    """Full prefill forward (stages 0-2); see dash_attn_fwd (and dash_attn_fwd_ex for sigma / qbar)."""
     out = torch.empty_like(q) if out is None else out
     ws = _workspace(fwd_workspace_size(q, k, block), q.device, workspace)
     qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
-    _check(_lib.dash_attn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), w_s.data_ptr(), alpha, block,
-                              1 if causal else 0, ctypes.byref(od), ws.data_ptr(), ws.numel(), _stream(stream)))
+    opts = _options(sigma, qbar)
+    args = (ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), w_s.data_ptr(), alpha, block, 1 if causal else 0,
+            ctypes.byref(od), ws.data_ptr(), ws.numel())
+    if opts is None:
+        _check(_lib.dash_attn_fwd(*args, _stream(stream)))
+    else:
+        _check(_lib.dash_attn_fwd_ex(*args, opts, _stream(stream)))
     return out
 
 
@@ -283,15 +326,19 @@ def decode_workspace_size(q: torch.Tensor, kcache: torch.Tensor, block: int, t_c
 
 
 def decode(q, kcache, vcache, seqlens, summaries, alpha: float, block: int, out=None, workspace=None,
-           stream=None) -> torch.Tensor:
-    """One decode step for q [B, 1, H, d] (see dash_attn_decode)."""
+           stream=None, sigma: float = 1.0) -> torch.Tensor:
+    """One decode step for q [B, 1, H, d] (see dash_attn_decode); sigma: prior strength."""
     out = torch.empty_like(q) if out is None else out
     t_cap = summaries.shape[2]
     ws = _workspace(decode_workspace_size(q, kcache, block, t_cap), q.device, workspace)
     qd, kd, vd, od = _desc(q), _desc(kcache), _desc(vcache), _desc(out)
-    _check(_lib.dash_attn_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), seqlens.data_ptr(),
-                                 summaries.data_ptr(), t_cap, alpha, block, ctypes.byref(od), ws.data_ptr(),
-                                 ws.numel(), _stream(stream)))
+    opts = _options(sigma, None)
+    args = (ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), seqlens.data_ptr(), summaries.data_ptr(), t_cap,
+            alpha, block, ctypes.byref(od), ws.data_ptr(), ws.numel())
+    if opts is None:
+        _check(_lib.dash_attn_decode(*args, _stream(stream)))
+    else:
+        _check(_lib.dash_attn_decode_ex(*args, opts, _stream(stream)))
     return out
 
 

@@ -391,6 +391,7 @@ dash_status_t dash_attn_route(const dash_tensor_t* q, const float* summaries, in
   cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   dash::DecodeParams p{};
+  p.sigma = 1.0f;
   p.q = view(q);
   p.dtype = q->dtype;
   p.B = (int)q->b;
@@ -424,7 +425,7 @@ size_t dash_attn_sparse_workspace_size(const dash_tensor_t* q, const dash_tensor
 
 static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
                                 const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
-                                int causal, dash_tensor_t* out, const TileLists& tl, int tile_pos,
+                                int causal, float sigma, dash_tensor_t* out, const TileLists& tl, int tile_pos,
                                 int64_t n_tiles, int union_tile0, dash::DeviceStatus* status,
                                 cudaStream_t stream) {
   if (q->dtype != DASH_F32 && union_tile0 < n_tiles) {
@@ -494,9 +495,22 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
   p.n_pairs = (int)tl.n_pairs;
   p.tile_pos = tile_pos;
   p.n_tiles = (int)n_tiles;
+  p.sigma = sigma;
   p.status = status;
   cudaError_t e = dash::launch_sparse_prefill(p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
+  return DASH_OK;
+}
+
+static dash_status_t read_options(const dash_options_t* opts, bool qbar_allowed, float* sigma, const float** qbar) {
+  *sigma = 1.0f;
+  *qbar = nullptr;
+  if (!opts) return DASH_OK;
+  if (!(opts->sigma >= 0.0f) || opts->sigma > 3.0e38f)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "sigma must be finite and >= 0");
+  if (opts->qbar && !qbar_allowed) return fail(DASH_ERR_INVALID_ARGUMENT, "qbar is not used here; pass NULL");
+  *sigma = opts->sigma;
+  *qbar = opts->qbar;
   return DASH_OK;
 }
 
@@ -504,7 +518,18 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
                                const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
                                int causal, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
                                dash_stream_t stream) {
+  return dash_attn_sparse_ex(q, k, v, idx, logp, cnt, t_cap, block, causal, out, workspace, workspace_bytes, nullptr,
+                             stream);
+}
+
+dash_status_t dash_attn_sparse_ex(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                                  const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                                  int causal, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                                  const dash_options_t* opts, dash_stream_t stream) {
   dash_status_t st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
   if ((st = check_fwd_shapes(q, k, v, out))) return st;
   if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
   if (k->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "prefill needs k and q of equal length");
@@ -522,7 +547,7 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
   const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
                      at<int32_t>(workspace, L.usteps), at<int32_t>(workspace, L.plist), at<uint4>(workspace, L.pmask),
                      at<int32_t>(workspace, L.pcnt), at<int32_t>(workspace, L.psteps), L.n_pairs};
-  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, out, tl, L.tile_pos, L.n_tiles, 0,
+  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, sigma, out, tl, L.tile_pos, L.n_tiles, 0,
                   at<dash::DeviceStatus>(workspace, L.status), s);
   return st ? st : ok();
 }
@@ -530,7 +555,17 @@ dash_status_t dash_attn_sparse(const dash_tensor_t* q, const dash_tensor_t* k, c
 dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v, const float* w_s,
                             float alpha, int block, int causal, dash_tensor_t* out, void* workspace,
                             size_t workspace_bytes, dash_stream_t stream) {
+  return dash_attn_fwd_ex(q, k, v, w_s, alpha, block, causal, out, workspace, workspace_bytes, nullptr, stream);
+}
+
+dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                               const float* w_s, float alpha, int block, int causal, dash_tensor_t* out,
+                               void* workspace, size_t workspace_bytes, const dash_options_t* opts,
+                               dash_stream_t stream) {
   dash_status_t st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, true, &sigma, &qbar))) return st;
   if ((st = check_fwd_shapes(q, k, v, out)) || (st = check_common(alpha, block))) return st;
   if (k->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "prefill needs k and q of equal length");
   if (!w_s) return fail(DASH_ERR_INVALID_ARGUMENT, "null w_s");
@@ -544,7 +579,7 @@ dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   float* summ = at<float>(workspace, L.summ);
-  if ((st = dash_attn_summarize(k, nullptr, w_s, block, summ, L.T, 0, stream))) return st;
+  if ((st = dash_attn_summarize_sdpa(k, nullptr, w_s, qbar, block, summ, L.T, 0, stream))) return st;
   int32_t* idx = at<int32_t>(workspace, L.idx);
   float* logp = at<float>(workspace, L.logp);
   int32_t* cnt = at<int32_t>(workspace, L.cnt);
@@ -556,8 +591,8 @@ dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, nullptr, nullptr, &tl, dst, s,
                       &first_cuda_tile)))
     return st;
-  st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, out, tl, L.tile_pos, L.n_tiles, first_cuda_tile, dst,
-                  s);
+  st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, sigma, out, tl, L.tile_pos, L.n_tiles, first_cuda_tile,
+                  dst, s);
   return st ? st : ok();
 }
 
@@ -571,7 +606,18 @@ size_t dash_attn_decode_workspace_size(const dash_tensor_t* q, const dash_tensor
 dash_status_t dash_attn_decode(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,
                                const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha, int block,
                                dash_tensor_t* out, void* workspace, size_t workspace_bytes, dash_stream_t stream) {
+  return dash_attn_decode_ex(q, kcache, vcache, seqlens, summaries, t_cap, alpha, block, out, workspace,
+                             workspace_bytes, nullptr, stream);
+}
+
+dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,
+                                  const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha,
+                                  int block, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                                  const dash_options_t* opts, dash_stream_t stream) {
   dash_status_t st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
   if ((st = check_tensor(q, "q")) || (st = check_tensor(kcache, "kcache")) || (st = check_tensor(vcache, "vcache")) ||
       (st = check_tensor(out, "out")) || (st = check_common(alpha, block)) || (st = check_group(q->h, kcache->h)))
     return st;
@@ -625,11 +671,23 @@ dash_status_t dash_attn_decode(const dash_tensor_t* q, const dash_tensor_t* kcac
   p.part_ml = at<float>(workspace, L.part_ml);
   p.max_items = L.max_items;
   p.chunk_blocks = L.chunk;
+  p.sigma = sigma;
   p.status = at<dash::DeviceStatus>(workspace, L.status);
   e = dash::launch_decode_route(p, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode route");
   e = dash::launch_decode_attend(p, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "decode attend");
+  return ok();
+}
+
+dash_status_t dash_attn_lists_to_mask(const int32_t* idx, const int32_t* cnt, int64_t rows, int64_t t_cap,
+                                      uint32_t* mask, int64_t n_words, dash_stream_t stream) {
+  if (rows < 0 || t_cap <= 0) return fail(DASH_ERR_INVALID_ARGUMENT, "rows < 0 or t_cap <= 0");
+  if (rows > 0 && (!idx || !cnt || !mask)) return fail(DASH_ERR_INVALID_ARGUMENT, "null idx, cnt or mask");
+  if (n_words * 32 < t_cap) return fail(DASH_ERR_INVALID_ARGUMENT, "n_words * 32 < t_cap");
+  if (n_words > 128) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per row");
+  cudaError_t e = dash::launch_lists_to_mask(idx, cnt, rows, t_cap, mask, (int)n_words, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "lists to mask");
   return ok();
 }
 

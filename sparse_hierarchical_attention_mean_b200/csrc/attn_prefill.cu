@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(256) sparse_simt_kernel(SparseParams p) {
     o[e] = 0.f;
   }
   float m = kNegInf, l = 0.f;
-  const float beta = N > 0 ? logf(1.0f / (float)N) : 0.0f;
+  const float beta = N > 0 ? p.sigma * logf(1.0f / (float)N) : 0.0f;
   for (int it = 0; it <= n; ++it) {
     const bool diag = it == n;
     const int c = diag ? t : idx[it];
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) sparse_simt_kernel(SparseParams p) {
       raise_status(p.status, 1 /* DASH_ERR_INVALID_ARGUMENT */, 201);
       continue;
     }
-    const float bias = diag ? beta : logp[it];
+    const float bias = diag ? beta : p.sigma * logp[it];
     const int lo = c * p.block;
     int hi = min(lo + p.block, p.S);
     if (diag && p.causal) hi = pos + 1;

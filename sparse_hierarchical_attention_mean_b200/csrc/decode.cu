@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_kernel(DecodeParams
     const int n_sub = n_sel * spb + n_diag;
     const int32_t* idx = p.idx + (int64_t)bg * p.t_cap;
     const float* logp = p.logp + (int64_t)bg * p.t_cap;
-    const float beta = N > 0 ? logf(1.0f / (float)N) : 0.0f;
+    const float beta = N > 0 ? p.sigma * logf(1.0f / (float)N) : 0.0f;
 
     const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
     const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_kernel(DecodeParams
       const T* kb = Ks + buf * kStep * D + warp * 16 * D;
       const T* vb = Vs + buf * kStep * D + warp * 16 * D;
       const bool diag = s >= n_sel * spb;
-      const float bias = (diag ? beta : logp[e_begin + s / spb]) * kLog2e;
+      const float bias = (diag ? beta : p.sigma * logp[e_begin + s / spb]) * kLog2e;
       const int tok0 = sub_tok0(s) + warp * 16;
 
       // logits of 16 tokens x G heads
@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
     const int n_sub = n_sel * spb + n_diag;
     const int32_t* idx = p.idx + (int64_t)bg * p.t_cap;
     const float* logp = p.logp + (int64_t)bg * p.t_cap;
-    const float beta = N > 0 ? logf(1.0f / (float)N) : 0.0f;
+    const float beta = N > 0 ? p.sigma * logf(1.0f / (float)N) : 0.0f;
     const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
     const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
 
@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
       const uint32_t kst = ks_base + (uint32_t)(st * kStageElems * sizeof(T));
       const uint32_t vst = vs_base + (uint32_t)(st * kStageElems * sizeof(T));
       const bool diag = s >= n_sel * spb;
-      const float bias = (diag ? beta : logp[e_begin + s / spb]) * kLog2e;
+      const float bias = (diag ? beta : p.sigma * logp[e_begin + s / spb]) * kLog2e;
       const int tok0 = sub_tok0(s) + warp * 16;
 
       // S^T = Q K^T for this warp's 16 tokens (two 8-token tiles)

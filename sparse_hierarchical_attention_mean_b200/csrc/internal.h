@@ -100,6 +100,7 @@ struct SparseParams {
   const int32_t* pcnt;
   const int32_t* psteps;
   int tile_pos, n_tiles, n_pairs;
+  float sigma;  // prior strength: bias sigma * log p_bar (diagonal: sigma * log(1/N))
   DeviceStatus* status;
 };
 // positions per stage-2 tile (tiles are 128 rows)
@@ -146,6 +147,7 @@ struct DecodeParams {
   float* part_ml;    // [max_items, G, 2]
   int64_t max_items;
   int chunk_blocks;  // selected blocks per split-KV work item
+  float sigma;       // prior strength (as in SparseParams)
   // optional route outputs (dash_attn_route in decode mode)
   float* tau;      // [B, H]
   float* p_dense;  // [B, H, t_cap]
@@ -153,6 +155,9 @@ struct DecodeParams {
 };
 int64_t decode_max_items(int64_t B, int64_t Hkv, int64_t t_cap, int chunk_blocks);
 cudaError_t launch_decode_route(const DecodeParams& p, cudaStream_t stream);
+// bit-packed active-block masks from ascending lists: rows x n_words uint32
+cudaError_t launch_lists_to_mask(const int32_t* idx, const int32_t* cnt, int64_t rows, int64_t t_cap,
+                                 uint32_t* mask, int n_words, cudaStream_t stream);
 cudaError_t launch_decode_attend(const DecodeParams& p, int num_sms, cudaStream_t stream);
 
 }  // namespace dash

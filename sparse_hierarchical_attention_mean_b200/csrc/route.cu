@@ -370,4 +370,41 @@ cudaError_t launch_pairs(const PairParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Bit-packed active-block masks (the pages' kernel walks a mask of the active
+// chunks): one warp per row sets the bits of its listed blocks in a
+// shared-memory copy of the row's words, then writes the words out.
+namespace {
+constexpr int kMaskWarps = 8;
+constexpr int kMaskMaxWords = 128;  // t_cap <= 4096
+
+__global__ void __launch_bounds__(kMaskWarps * 32)
+    mask_kernel(const int32_t* idx, const int32_t* cnt, int64_t rows, int64_t t_cap, uint32_t* mask, int n_words) {
+  __shared__ uint32_t words[kMaskWarps][kMaskMaxWords];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t r = (int64_t)blockIdx.x * kMaskWarps + warp; r < rows; r += (int64_t)gridDim.x * kMaskWarps) {
+    for (int w = lane; w < n_words; w += 32) words[warp][w] = 0u;
+    __syncwarp();
+    const int n = min(max(cnt[r], 0), (int)t_cap);
+    const int32_t* li = idx + r * t_cap;
+    for (int i = lane; i < n; i += 32) {
+      const int c = li[i];
+      if (c >= 0 && c < n_words * 32) atomicOr(&words[warp][c >> 5], 1u << (c & 31));
+    }
+    __syncwarp();
+    for (int w = lane; w < n_words; w += 32) mask[r * n_words + w] = words[warp][w];
+    __syncwarp();
+  }
+}
+}  // namespace
+
+cudaError_t launch_lists_to_mask(const int32_t* idx, const int32_t* cnt, int64_t rows, int64_t t_cap,
+                                 uint32_t* mask, int n_words, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  if (n_words > kMaskMaxWords) return cudaErrorInvalidValue;
+  const int64_t want = (rows + kMaskWarps - 1) / kMaskWarps;
+  const unsigned grid = (unsigned)(want < 148 * 16 ? want : 148 * 16);
+  mask_kernel<<<grid, kMaskWarps * 32, 0, stream>>>(idx, cnt, rows, t_cap, mask, n_words);
+  return cudaGetLastError();
+}
+
 }  // namespace dash

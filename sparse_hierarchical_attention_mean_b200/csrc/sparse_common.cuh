@@ -12,15 +12,16 @@
 
 namespace dash {
 
-// Prior bias of one row for the tensor-core kernel: the tile's work list
-// carries, per block, the mask of tile positions that selected it, so a row
-// only needs its own log p_bar values in order; they are prefetched four
+// Prior bias of one row for the tensor-core kernel (sigma * log p_bar; the
+// diagonal block sigma * log(1/N)): the tile's work list carries, per block,
+// the mask of tile positions that selected it, so a row only needs its own
+// log p_bar values in order; they are prefetched four
 // selections ahead to keep global-memory latency off the softmax path.
 struct RowPrior {
   const float* lp;
   int n, cur, bit, pos, t;
   bool valid;
-  float beta;
+  float beta, sigma;
   float q0, q1, q2, q3;
 
   __device__ __forceinline__ void init(const SparseParams& p, int64_t bg, int position, int pos_in_tile) {
@@ -30,7 +31,8 @@ struct RowPrior {
     t = pos / p.block;
     const int n_blocks = (p.S + p.block - 1) / p.block;
     const int n_cand = p.causal ? t : n_blocks - 1;
-    beta = n_cand > 0 ? logf(1.0f / (float)n_cand) : 0.0f;
+    sigma = p.sigma;
+    beta = n_cand > 0 ? sigma * logf(1.0f / (float)n_cand) : 0.0f;
     const int64_t row = bg * p.S + (valid ? pos : 0);
     n = valid ? min(max(p.cnt[row], 0), (int)p.t_cap) : 0;
     lp = p.logp + row * p.t_cap;
@@ -47,7 +49,7 @@ struct RowPrior {
     if (c == t) return beta;
     const uint32_t w = bit < 32 ? mask.x : bit < 64 ? mask.y : bit < 96 ? mask.z : mask.w;
     if (((w >> (bit & 31)) & 1u) == 0u) return kNegInf;
-    const float v = q0;
+    const float v = sigma * q0;
     q0 = q1;
     q1 = q2;
     q2 = q3;

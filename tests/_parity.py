@@ -15,30 +15,36 @@ import numpy as np
 import torch
 
 from gen import kv_values, q_values
-from oracle.dash_oracle import block_summaries, candidate_blocks, forward_row
+from oracle.dash_oracle import block_summaries, block_summaries_sdpa, candidate_blocks, forward_row
 
 BAND = 1e-4
 P_TOL = 1e-5
 OUT_TOL = {"f32": 1e-4, "f16": 2e-2, "bf16": 2e-2}
 
 
-def oracle_head(cfg, plan, b, g, rows, n_tokens=None):
-    """Oracle records for query positions ``rows`` of (batch b, KV group g)."""
+def oracle_head(cfg, plan, b, g, rows, n_tokens=None, sigma=1.0, qbar=None):
+    """Oracle records for query positions ``rows`` of (batch b, KV group g).
+
+    sigma: prior strength; qbar: learned summary query of this KV head [d] (None: mean pooling).
+    """
     G, d = cfg.group, cfg.head_dim
     n_tokens = cfg.seq if n_tokens is None else n_tokens
     k = kv_values(cfg, plan, "k", b, range(n_tokens), [g], as_float32=True)[:, 0].double().numpy()
     v = kv_values(cfg, plan, "v", b, range(n_tokens), [g], as_float32=True)[:, 0].double().numpy()
     q = q_values(cfg, plan, b, rows, range(g * G, (g + 1) * G), as_float32=True).double().numpy()
     w = plan.w_s.double().numpy()
-    summ = block_summaries(k, w, cfg.block, n_tokens)
+    if qbar is None:
+        summ = block_summaries(k, w, cfg.block, n_tokens)
+    else:
+        summ = block_summaries_sdpa(k, w, np.asarray(qbar, dtype=np.float64), cfg.block, n_tokens)
     recs = []
     for ri, pos in enumerate(rows):
-        r = forward_row(q[ri], k, v, summ, pos, n_tokens, cfg.block, cfg.alpha, cfg.causal)
+        r = forward_row(q[ri], k, v, summ, pos, n_tokens, cfg.block, cfg.alpha, cfg.causal, sigma=sigma)
         recs.append(r)
     return recs, summ
 
 
-def oracle_decode_pair(cfg, plan, b, g):
+def oracle_decode_pair(cfg, plan, b, g, sigma=1.0):
     G = cfg.group
     L = int(plan.seqlens[b])
     k = kv_values(cfg, plan, "k", b, range(L), [g], as_float32=True)[:, 0].double().numpy()
@@ -46,7 +52,7 @@ def oracle_decode_pair(cfg, plan, b, g):
     q = q_values(cfg, plan, b, [0], range(g * G, (g + 1) * G), as_float32=True)[0].double().numpy()
     n_complete = (L - 1) // cfg.block
     summ = block_summaries(k[: n_complete * cfg.block], plan.w_s.double().numpy(), cfg.block, n_complete * cfg.block)
-    rec = forward_row(q, k, v, summ, L - 1, L, cfg.block, cfg.alpha, True)
+    rec = forward_row(q, k, v, summ, L - 1, L, cfg.block, cfg.alpha, True, sigma=sigma)
     return rec, summ
 
 

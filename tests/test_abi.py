@@ -138,6 +138,18 @@ def test_decode_and_route_reject_bad_arguments():
     assert st == 1 and "aligned" in lib.dash_attn_last_error().decode()
     st = lib.dash_attn_summarize_sdpa(ctypes.byref(kc), None, FAKE, FAKE, 96, FAKE, 64, 0, None)
     assert st == 2
+    # options: negative sigma; a learned query where no summaries are computed
+    bad = dash.DashOptions(-1.0, None)
+    st = lib.dash_attn_decode_ex(ctypes.byref(q), ctypes.byref(kc), ctypes.byref(kc), FAKE, FAKE, 64, 1.5, 64,
+                                 ctypes.byref(o), FAKE, ws, ctypes.byref(bad), None)
+    assert st == 1 and "sigma" in lib.dash_attn_last_error().decode()
+    withq = dash.DashOptions(1.0, FAKE)
+    st = lib.dash_attn_decode_ex(ctypes.byref(q), ctypes.byref(kc), ctypes.byref(kc), FAKE, FAKE, 64, 1.5, 64,
+                                 ctypes.byref(o), FAKE, ws, ctypes.byref(withq), None)
+    assert st == 1 and "qbar" in lib.dash_attn_last_error().decode()
+    # masks: too few words for the list capacity
+    st = lib.dash_attn_lists_to_mask(FAKE, FAKE, 10, 100, FAKE, 3, None)
+    assert st == 1 and "n_words" in lib.dash_attn_last_error().decode()
 
 
 def test_binding_refuses_host_tensors():

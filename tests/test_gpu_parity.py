@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from gen import Config, full_inputs, get_config, kv_values, make_plan
-from oracle.dash_oracle import block_summaries, block_summaries_sdpa
+from oracle.dash_oracle import block_summaries, block_summaries_sdpa, lists_to_mask
 from tests._parity import (
     OUT_TOL,
     check_p_dense,
@@ -164,6 +164,59 @@ def test_summarize_sdpa(dash, name, scale):
                 ref = block_summaries_sdpa(kk, plan.w_s.double().numpy(), qbar[g].double().numpy(), cfg.block, n_tok)
                 err = np.abs(out[b, g, : len(ref)].cpu().numpy() - ref).max()
                 assert err <= 2e-5 * max(1.0, np.abs(ref).max()), f"{name} scale {scale} b{b} g{g}: {err:.3g}"
+
+
+@pytest.mark.parametrize("name,sigma,qscale", [("prefill_small", 0.0, None), ("prefill_small", 0.5, None),
+                                               ("prefill_small", 2.0, 3.0), ("g1_b128", 0.5, 10.0),
+                                               ("f32_d128", 0.5, 3.0)])
+def test_forward_options(dash, name, sigma, qscale):
+    """dash_attn_fwd_ex: prior strength sigma and learned summary queries, against the oracle."""
+    cfg = SMALL[name]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w, plan = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["plan"]
+    qbar = None
+    if qscale is not None:
+        qbar = torch.from_numpy(np.random.default_rng(12).normal(size=(cfg.kv_heads, cfg.head_dim)) * qscale).float()
+    out = dash.fwd(q, k, v, w, cfg.alpha, cfg.block, cfg.causal, sigma=sigma,
+                   qbar=None if qbar is None else qbar.cuda())
+    torch.cuda.synchronize()
+    G, tol = cfg.group, OUT_TOL[cfg.dtype]
+    out_np = to_np(out)
+    rows = list(range(cfg.seq))
+    for g in _kv_subset(cfg):
+        recs, _ = oracle_head(cfg, plan, 0, g, rows, sigma=sigma,
+                              qbar=None if qbar is None else qbar[g].double().numpy())
+        for pos, rec in zip(rows, recs):
+            err = max_abs(out_np[0, pos, g * G:(g + 1) * G], rec["out"])
+            assert err <= tol, f"{name} sigma {sigma} g{g} pos{pos}: output error {err:.3g}"
+
+
+def test_decode_sigma(dash):
+    cfg = get_config("decode").with_(name="decode_sigma", batch=3, seq=3000, seqlen_lo=200, seqlen_hi=3000)
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
+    summ = dash.summarize(k, w, cfg.block, seqlens=sl)
+    out = dash.decode(q, k, v, sl, summ, cfg.alpha, cfg.block, sigma=0.5)
+    torch.cuda.synchronize()
+    G, out_np = cfg.group, to_np(out)
+    for b in range(cfg.batch):
+        for g in range(cfg.kv_heads):
+            rec, _ = oracle_decode_pair(cfg, inp["plan"], b, g, sigma=0.5)
+            err = max_abs(out_np[b, 0, g * G:(g + 1) * G], rec["out"])
+            assert err <= OUT_TOL[cfg.dtype], f"b{b} g{g}: {err:.3g}"
+
+
+def test_lists_to_mask_bit_exact(dash):
+    cfg = SMALL["prefill_small"]
+    inp = full_inputs(cfg, device="cuda")
+    summ = dash.summarize(inp["k"], inp["w_s"], cfg.block)
+    rt = dash.route(inp["q"], summ, cfg.alpha, cfg.block, True)
+    for n_words in (None, 5):
+        m = dash.lists_to_mask(rt["idx"], rt["cnt"], n_words)
+        torch.cuda.synchronize()
+        nw = m.shape[-1]
+        ref = lists_to_mask(rt["idx"].cpu().numpy(), rt["cnt"].cpu().numpy(), nw)
+        assert np.array_equal(m.cpu().numpy().view(np.uint32), ref)
 
 
 DECODE_SMALL = {
