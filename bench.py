@@ -455,12 +455,13 @@ def run_decode(dash, cfg, steps, warmup, world, rank):
 # --------------------------------------------------------------------------- oracle timing
 
 
-def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0) -> dict:
+def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0, groups=None) -> dict:
     """Times the oracle on a bounded sample of the prefill workload on this host.
 
-    For each KV group: pooling of the whole sequence once, then the routing and
-    sparse attention of ``n_rows`` evenly spread query positions.  Returns the
-    extrapolated full-sequence time and tokens/s.
+    For each sampled KV group (default: all): pooling of the whole sequence
+    once, then the routing and sparse attention of ``n_rows`` evenly spread
+    query positions.  Returns the full-sequence time (all KV groups and
+    positions) extrapolated from the sample, and tokens/s.
     """
     from threadpoolctl import threadpool_limits
 
@@ -472,8 +473,9 @@ def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0) -> dict
     pool_t = row_t = 0.0
     n_done = 0
     t_start = time.perf_counter()
+    groups = list(range(cfg.kv_heads)) if groups is None else list(groups)
     with threadpool_limits(1):
-        for g in range(cfg.kv_heads):
+        for g in groups:
             k = kv_values(cfg, plan, "k", 0, range(cfg.seq), [g], as_float32=True)[:, 0].double().numpy()
             v = kv_values(cfg, plan, "v", 0, range(cfg.seq), [g], as_float32=True)[:, 0].double().numpy()
             q = q_values(cfg, plan, 0, rows, range(g * G, (g + 1) * G), as_float32=True).double().numpy()
@@ -488,10 +490,11 @@ def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0) -> dict
                     break
             row_t += time.perf_counter() - t1
     per_row = row_t / max(n_done, 1)  # one position of one KV group (G heads)
-    full_s = pool_t / cfg.kv_heads * cfg.kv_heads + per_row * cfg.seq * cfg.kv_heads
+    full_s = pool_t / len(groups) * cfg.kv_heads + per_row * cfg.seq * cfg.kv_heads
     return {"full_s": full_s, "tokens_per_s": cfg.seq / full_s, "rows": n_done, "wall_s": time.perf_counter() - t_start,
-            "sample": f"{n_done} (position, KV group) rows spread over the {cfg.seq}-token sequence + pooling of all "
-                      f"{cfg.kv_heads} KV heads, extrapolated to {cfg.seq} positions x {cfg.kv_heads} groups"}
+            "sample": f"{n_done} (position, KV group) rows spread over the {cfg.seq}-token sequence + pooling of "
+                      f"{len(groups)} of {cfg.kv_heads} KV heads, extrapolated to {cfg.seq} positions x "
+                      f"{cfg.kv_heads} groups"}
 
 
 # --------------------------------------------------------------------------- main
@@ -523,7 +526,8 @@ def main():
         per_step = []
         samples = None
         for i in range(warmup + args.steps):
-            r = oracle_sample_time(cfg, n_rows=3, budget_s=30.0, seed=cfg.seed)
+            # each step: one KV group (rotating), its pooling and 3 rows
+            r = oracle_sample_time(cfg, n_rows=3, budget_s=30.0, seed=cfg.seed, groups=[i % cfg.kv_heads])
             if i >= warmup:
                 per_step.append(r["full_s"])
                 samples = r
