@@ -596,7 +596,8 @@ def main():
         "sparsity": pre["sparsity"],
         "stage_ms": {"pool": pre["seg_ms"][0], "route": pre["seg_ms"][1], "sparse_attention": pre["seg_ms"][2]},
         "roofline": {
-            "kernel": "sparse_prefill_tc_kernel (+ its pair-list kernel), timed alone back to back",
+            "kernel": "sparse_prefill_tc_kernel, timed through the stage-2 entry point (with its union- and "
+                      "pair-list kernels, ~4%) launched back to back",
             "ms_per_launch": pre["sparse_ms"],
             "bound": "tensor",
             "achieved": pre["achieved_tflops"],
