@@ -44,7 +44,8 @@ constexpr int kMmaWarp = kWorkWarps;
 constexpr int kThreads = (kWorkWarps + 1) * 32;
 constexpr int kWork = kWorkWarps * 32;
 constexpr int kHalf = 64;           // rows whose logits sit in shared memory at once
-constexpr int kXStride = kMaxCols + 1;  // odd row stride: conflict-free column writes
+constexpr int kXStride = kMaxCols + 4;  // row stride: 16-byte row starts, conflict-free 16-byte writes
+constexpr int kSeed = 32;               // seed values per row: the top two of each 32-column chunk
 
 struct RBars {
   uint64_t a_full;
@@ -67,7 +68,8 @@ struct RLayout {
   static constexpr int kXBytes = kHalf * kXStride * 4;  // logits of 64 rows (reuses the GEMM operands)
   static constexpr int kOffMask = (kGemmBytes > kXBytes ? kGemmBytes : kXBytes);  // [512] uint4
   static constexpr int kOffList = kOffMask + kMaxCols * 16;  // per 32-column chunk: entries, steps [2][32]
-  static constexpr int kOffBar = kOffList + 2 * 32 * 4;
+  static constexpr int kOffSeed = kOffList + 2 * 32 * 4;  // [kHalf][kSeed] fp32
+  static constexpr int kOffBar = kOffSeed + kHalf * kSeed * 4;
   static constexpr int kBytes = kOffBar + 128;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -195,31 +197,21 @@ __device__ __forceinline__ void entmax_newton_rows(const float* x, int stride, i
 }
 
 // alpha-entmax thresholds of RW rows that share their candidate columns,
-// solved in lockstep by one warp (their reductions interleave).  Row i's
-// logits are x[i * stride + c] for c < n, -inf on non-candidates; columns are
-// read 64 at a time, so the rows must be readable (-inf) up to n rounded up
-// to a multiple of 64.  Same
-// scheme as warp_entmax_tau: Newton from max - 1, where F >= 1, approaches
-// the root from below, and after every step the exact solution on the
-// current support is accepted when it is self-consistent.
+// solved in lockstep by one warp.  Row i's logits are x[i * stride + c] for
+// c < n, -inf on non-candidates, readable up to n rounded up to 64.  seed[i *
+// kSeed + l] are kSeed values of row i (the top two of each 32-column chunk,
+// -inf where a chunk has fewer): their maximum is the row's, and their
+// threshold, solved first in registers, is a lower bound on the row's (F
+// over the row >= F over any subset), so the passes over the row start there
+// instead of at max - 1 and usually find the exact support at once.
 template <int RW>
-__device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride, int n, float alpha, int kind,
-                                                     int lane, float* tau) {
+__device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride, int n, const float* seed,
+                                                     float alpha, int kind, int lane, float* tau) {
+  static_assert(kSeed == 32, "one seed value per lane");
   const float pw = 1.0f / (alpha - 1.0f);
-  float mx[RW];
+  float sv[RW], mx[RW];
 #pragma unroll
-  for (int i = 0; i < RW; ++i) mx[i] = kNegInf;
-  for (int c = lane; c < n; c += 64) {
-#pragma unroll
-    for (int i = 0; i < RW; ++i) mx[i] = fmaxf(mx[i], fmaxf(x[i * stride + c], x[i * stride + c + 32]));
-  }
-  // The lane maxima are a subset of the row, and the threshold of any subset
-  // is a lower bound on the row's (F over the row >= F over the subset): solve
-  // the 32 lane maxima first, in registers, and start the passes over the row
-  // from there instead of from max - 1.
-  float lmx[RW];
-#pragma unroll
-  for (int i = 0; i < RW; ++i) lmx[i] = mx[i];
+  for (int i = 0; i < RW; ++i) sv[i] = mx[i] = seed[i * kSeed + lane];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
@@ -231,11 +223,12 @@ __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride,
     tau[i] = mx[i] - 1.0f;
     done[i] = mx[i] == kNegInf;
   }
-  entmax_newton_rows<RW, 1>(lmx, 0, 32, pw, kind, lane, tau, done);
+  entmax_newton_rows<RW, 1>(sv, 0, 32, pw, kind, lane, tau, done);
 #pragma unroll
   for (int i = 0; i < RW; ++i) done[i] = mx[i] == kNegInf;
   entmax_newton_rows<RW, 2>(x, stride, n, pw, kind, lane, tau, done);
 }
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RouteParams p, TileOut to, int tile0) {
   constexpr int RW = G > 4 ? G : 4;  // rows solved together by one warp
@@ -246,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   RBars* bars = reinterpret_cast<RBars*>(smem + L::kOffBar);
   float* X = reinterpret_cast<float*>(smem);  // [kHalf][kXStride], after the GEMM
+  float* seed = reinterpret_cast<float*>(smem + L::kOffSeed);  // [kHalf][kSeed]
   uint4* pmask = reinterpret_cast<uint4*>(smem + L::kOffMask);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -409,16 +403,28 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
         const int t = pos / p.block;
         const bool valid = pos < p.S;
         float* xr = X + (r - half * kHalf) * kXStride;
+        float* sr = seed + (r - half * kHalf) * kSeed;
         for (int ch = warp >> 2; ch < n_wch; ch += kWorkWarps / 4) {
           uint32_t v[32];
           tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + ch * 32, v);
           tc::tmem_wait_ld();
+          float m1 = kNegInf, m2 = kNegInf;  // top two of the chunk
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int c = ch * 32 + j;
-            xr[c] = (valid && is_cand(c, t, n_blocks, p.causal)) ? coef * __uint_as_float(v[j]) : kNegInf;
+          for (int j = 0; j < 32; j += 4) {
+            float y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = ch * 32 + j + e;
+              y[e] = (valid && is_cand(c, t, n_blocks, p.causal)) ? coef * __uint_as_float(v[j + e]) : kNegInf;
+              m2 = fmaxf(m2, fminf(m1, y[e]));
+              m1 = fmaxf(m1, y[e]);
+            }
+            *reinterpret_cast<float4*>(xr + ch * 32 + j) = make_float4(y[0], y[1], y[2], y[3]);
           }
+          sr[2 * ch] = m1;
+          sr[2 * ch + 1] = m2;
         }
+        for (int e = 2 * n_wch + (warp >> 2); e < kSeed; e += kWorkWarps / 4) sr[e] = kNegInf;
       }
     }
     __syncthreads();
@@ -435,8 +441,15 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
         float tau[RW];
         // thresholds four rows at a time (register budget)
 #pragma unroll
-        for (int r4 = 0; r4 < RW; r4 += 4)
-          warp_entmax_tau_rows<4>(X + (rr0 + r4) * kXStride, kXStride, ncol, p.alpha, kind, lane, tau + r4);
+        for (int r4 = 0; r4 < RW; r4 += 4) {
+          if (ncol > 0) {
+            warp_entmax_tau_rows<4>(X + (rr0 + r4) * kXStride, kXStride, ncol, seed + (rr0 + r4) * kSeed, p.alpha,
+                                    kind, lane, tau + r4);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tau[r4 + i] = 0.f;  // no candidates (nothing was copied)
+          }
+        }
 #pragma unroll
         for (int pp = 0; pp < PPT; ++pp) {
           const int tp = tp0 + pp;
