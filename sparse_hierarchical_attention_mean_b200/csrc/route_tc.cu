@@ -43,8 +43,8 @@ constexpr int kWorkWarps = 16;      // loading, threshold and compaction warps
 constexpr int kMmaWarp = kWorkWarps;
 constexpr int kThreads = (kWorkWarps + 1) * 32;
 constexpr int kWork = kWorkWarps * 32;
-constexpr int kHalf = 64;           // rows whose logits sit in shared memory at once
-constexpr int kXStride = kMaxCols + 4;  // row stride: 16-byte row starts, conflict-free 16-byte writes
+constexpr int kHalf = 64;           // rows whose logits sit in shared memory at once (512 columns)
+constexpr int kXStride = kMaxCols + 4;  // widest row stride: 16-byte row starts, conflict-free 16-byte writes
 constexpr int kSeed = 32;               // seed values per row: the top two of each 32-column chunk
 
 struct RBars {
@@ -65,11 +65,12 @@ struct RLayout {
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + KC * kAChunk;  // [2 stages][hi, lo]
   static constexpr int kGemmBytes = kOffB + 2 * 2 * kBTerm;
-  static constexpr int kXBytes = kHalf * kXStride * 4;  // logits of 64 rows (reuses the GEMM operands)
-  static constexpr int kOffMask = (kGemmBytes > kXBytes ? kGemmBytes : kXBytes);  // [512] uint4
+  // logits of 64 wide or 128 narrow rows, over the GEMM operands (no longer needed then)
+  static constexpr int kXBytes = (kGemmBytes > kHalf * kXStride * 4 ? kGemmBytes : kHalf * kXStride * 4);
+  static constexpr int kOffMask = kXBytes;  // [512] uint4
   static constexpr int kOffList = kOffMask + kMaxCols * 16;  // per 32-column chunk: entries, steps [2][32]
-  static constexpr int kOffSeed = kOffList + 2 * 32 * 4;  // [kHalf][kSeed] fp32
-  static constexpr int kOffBar = kOffSeed + kHalf * kSeed * 4;
+  static constexpr int kOffSeed = kOffList + 2 * 32 * 4;  // [kRows][kSeed] fp32
+  static constexpr int kOffBar = kOffSeed + kRows * kSeed * 4;
   static constexpr int kBytes = kOffBar + 128;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -238,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   RBars* bars = reinterpret_cast<RBars*>(smem + L::kOffBar);
-  float* X = reinterpret_cast<float*>(smem);  // [kHalf][kXStride], after the GEMM
-  float* seed = reinterpret_cast<float*>(smem + L::kOffSeed);  // [kHalf][kSeed]
+  float* X = reinterpret_cast<float*>(smem);  // [round rows][xstride], after the GEMM
+  float* seed = reinterpret_cast<float*>(smem + L::kOffSeed);  // [round rows][kSeed]
   uint4* pmask = reinterpret_cast<uint4*>(smem + L::kOffMask);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -389,21 +390,25 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   }
   __syncthreads();  // GEMM done: its shared memory now holds logits
 
-  // ---- two halves of 64 rows: TMEM -> shared, thresholds, compaction
+  // ---- rounds of rows: TMEM -> shared, thresholds, compaction.  All 128
+  // rows in one round when their logits fit the buffer (up to 256 columns),
+  // else two rounds of 64.
   // 32-column chunks of the logit rows, an even number: the threshold passes
   // read columns in pairs of chunks (the extra columns hold -inf)
   const int n_wch = ((n_cols + 63) / 64) * 2;
-  for (int half = 0; half < 2; ++half) {
+  const int xstride = n_wch * 32 + 4;
+  const int round_rows = kRows * xstride * 4 <= L::kXBytes ? kRows : kHalf;
+  for (int half = 0; half * round_rows < kRows; ++half) {
     if (warp < kWorkWarps && n_chunks > 0 && !bars->abort) {
-      // warps whose TMEM lane quarter lies in this half copy (and scale) their rows
+      // warps whose TMEM lane quarter lies in this round copy (and scale) their rows
       const int q4 = warp & 3;
-      if ((q4 >> 1) == half) {
+      if (q4 * 32 >= half * round_rows && q4 * 32 < (half + 1) * round_rows) {
         const int r = q4 * 32 + lane;  // tile row = TMEM lane
         const int pos = pos0 + r / G;
         const int t = pos / p.block;
         const bool valid = pos < p.S;
-        float* xr = X + (r - half * kHalf) * kXStride;
-        float* sr = seed + (r - half * kHalf) * kSeed;
+        float* xr = X + (r - half * round_rows) * xstride;
+        float* sr = seed + (r - half * round_rows) * kSeed;
         for (int ch = warp >> 2; ch < n_wch; ch += kWorkWarps / 4) {
           uint32_t v[32];
           tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + ch * 32, v);
@@ -431,10 +436,10 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
     if (warp < kWorkWarps) {
       // one warp per task of RW rows (PPT positions x G heads): thresholds in
       // lockstep, then the GQA mean and the ascending list of each position
-      constexpr int kTasks = kHalf / RW;
-      for (int task = warp; task < kTasks; task += kWorkWarps) {
-        const int rr0 = task * RW;                 // first row within the half
-        const int tp0 = (half * kHalf + rr0) / G;  // first tile position
+      const int n_tasks = round_rows / RW;
+      for (int task = warp; task < n_tasks; task += kWorkWarps) {
+        const int rr0 = task * RW;                       // first row within the round
+        const int tp0 = (half * round_rows + rr0) / G;  // first tile position
         const int pos = pos0 + tp0;
         const int t = pos / p.block;  // the task's positions share their block
         const int ncol = p.causal ? t : n_blocks;
@@ -443,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
 #pragma unroll
         for (int r4 = 0; r4 < RW; r4 += 4) {
           if (ncol > 0) {
-            warp_entmax_tau_rows<4>(X + (rr0 + r4) * kXStride, kXStride, ncol, seed + (rr0 + r4) * kSeed, p.alpha,
+            warp_entmax_tau_rows<4>(X + (rr0 + r4) * xstride, xstride, ncol, seed + (rr0 + r4) * kSeed, p.alpha,
                                     kind, lane, tau + r4);
           } else {
 #pragma unroll
@@ -471,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
             if (c < ncol) {
 #pragma unroll
               for (int h = 0; h < G; ++h) {
-                const float u = X[(rr0 + pp * G + h) * kXStride + c] - tau[pp * G + h];
+                const float u = X[(rr0 + pp * G + h) * xstride + c] - tau[pp * G + h];
                 const float ph = u > 0.f ? pow_pw(u, pw, kind) : 0.f;
                 pbar += ph;
                 if (p.p_dense) p.p_dense[(((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap + c] = ph;
