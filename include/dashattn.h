@@ -164,6 +164,43 @@ dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, c
                                dash_stream_t stream);
 
 /*
+ * Context-parallel decode: one sequence's context split over R ranks (one
+ * process per GPU), each holding the cache tokens [tok_lo, tok_lo + n) of
+ * every sequence (tok_lo and n multiples of the block) and the summaries of
+ * the blocks in that range.  The result equals dash_attn_decode on the whole
+ * cache.  One step, on every rank:
+ *   1. dash_attn_cp_scores: the routing logits of this rank's candidate
+ *      blocks into a zero-filled score buffer [B, Hkv, G, t_cap] fp32;
+ *   2. a sum all-reduce of that buffer over the ranks (the ranges are
+ *      disjoint, so the sum is the whole score vector);
+ *   3. dash_attn_cp_lists: alpha-entmax, GQA mean and ascending lists, the
+ *      same on every rank;
+ *   4. dash_attn_cp_attend: stage 2 over this rank's selected blocks and, if
+ *      it holds it, the diagonal block -> partials [B, H, d + 2] fp32 (o
+ *      relative to its reference max m, m in log2 units, l);
+ *   5. an all-gather of the partials ([R, B, H, d + 2]) and dash_attn_cp_merge.
+ * q is [B, 1, H, d] (f16/bf16), seqlens device int32 [B] with
+ * 1 <= seqlens[b] <= lmax, t_cap >= ceil(lmax / block), at most 4096.
+ *   summaries  this rank's summaries, block c at index c - block_lo of a
+ *              [B, Hkv, summ_cap, d] fp32 buffer (dash_attn_summarize on the
+ *              shard); block_lo <= c < block_hi are scored.
+ */
+dash_status_t dash_attn_cp_scores(const dash_tensor_t* q, int64_t kv_heads, const float* summaries, int64_t summ_cap,
+                                  int64_t block_lo, int64_t block_hi, const int32_t* seqlens, int64_t lmax, float alpha,
+                                  int block, float* scores, int64_t t_cap, dash_stream_t stream);
+dash_status_t dash_attn_cp_lists(const dash_tensor_t* q, int64_t kv_heads, const float* scores, const int32_t* seqlens,
+                                 int64_t lmax, float alpha, int block, int32_t* idx, float* logp, int32_t* cnt,
+                                 int64_t t_cap, dash_stream_t stream);
+/*   kshard, vshard  [B, n, Hkv, d]: cache tokens tok_lo .. tok_lo + n - 1.
+ *   opts            NULL or sigma only (opts->qbar must be NULL). */
+dash_status_t dash_attn_cp_attend(const dash_tensor_t* q, const dash_tensor_t* kshard, const dash_tensor_t* vshard,
+                                  int64_t tok_lo, const int32_t* seqlens, int64_t lmax, const int32_t* idx,
+                                  const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                                  const dash_options_t* opts, float* part, dash_stream_t stream);
+/*   parts  device fp32 [n_parts, B, H, d + 2]; out [B, 1, H, d] (f16/bf16). */
+dash_status_t dash_attn_cp_merge(const float* parts, int64_t n_parts, dash_tensor_t* out, dash_stream_t stream);
+
+/*
  * Bit-packed active-block masks from routing lists (the pages' kernel walks
  * a mask of the active chunks; the lists of dash_attn_route carry the same
  * sets plus log p_bar): for each of `rows` rows (e.g. B * Hkv * S of the

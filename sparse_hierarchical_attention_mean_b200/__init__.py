@@ -42,6 +42,10 @@ EXPORTED = (
     "dash_attn_sparse_ex",
     "dash_attn_decode_ex",
     "dash_attn_lists_to_mask",
+    "dash_attn_cp_scores",
+    "dash_attn_cp_lists",
+    "dash_attn_cp_attend",
+    "dash_attn_cp_merge",
     "dash_attn_decode_workspace_size",
     "dash_attn_decode",
     "dash_attn_route_workspace_size",
@@ -104,6 +108,10 @@ def _load() -> ctypes.CDLL:
         "dash_attn_sparse_ex": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, O, vp]),
         "dash_attn_decode_ex": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
         "dash_attn_lists_to_mask": (i32, [vp, vp, i64, i64, vp, i64, vp]),
+        "dash_attn_cp_scores": (i32, [T, i64, vp, i64, i64, i64, vp, i64, f32, i32, vp, i64, vp]),
+        "dash_attn_cp_lists": (i32, [T, i64, vp, vp, i64, f32, i32, vp, vp, vp, i64, vp]),
+        "dash_attn_cp_attend": (i32, [T, T, T, i64, vp, i64, vp, vp, vp, i64, i32, O, vp, vp]),
+        "dash_attn_cp_merge": (i32, [vp, i64, T, vp]),
         "dash_attn_get_device_status": (i32, [vp, vp]),
         "dash_attn_decode_noalloc": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp]),
     }
@@ -362,3 +370,51 @@ def device_status(workspace: torch.Tensor, stream=None) -> int:
     """Status word of the last call that used ``workspace`` (synchronises)."""
     return _lib.dash_attn_get_device_status(workspace.data_ptr(), _stream(stream))
 
+
+
+# ------------------------------------------------------------------ context-parallel decode
+
+
+def cp_scores(q, summaries, block_lo: int, block_hi: int, seqlens, lmax: int, alpha: float, block: int,
+              scores: torch.Tensor, stream=None) -> torch.Tensor:
+    """This rank's routing logits into ``scores`` [B, Hkv, G, t_cap] (see dash_attn_cp_scores)."""
+    B, Hkv, summ_cap, d = summaries.shape
+    qd = _desc(q)
+    _check(_lib.dash_attn_cp_scores(ctypes.byref(qd), Hkv, summaries.data_ptr(), summ_cap, block_lo, block_hi,
+                                    seqlens.data_ptr(), lmax, alpha, block, scores.data_ptr(), scores.shape[3],
+                                    _stream(stream)))
+    return scores
+
+
+def cp_lists(q, kv_heads: int, scores, seqlens, lmax: int, alpha: float, block: int, stream=None) -> dict:
+    """alpha-entmax, GQA mean and ascending lists from whole score vectors (see dash_attn_cp_lists)."""
+    B, Hkv, G, t_cap = scores.shape
+    dev = q.device
+    idx = torch.full((B, Hkv, t_cap), -1, dtype=torch.int32, device=dev)
+    logp = torch.zeros((B, Hkv, t_cap), dtype=torch.float32, device=dev)
+    cnt = torch.zeros((B, Hkv), dtype=torch.int32, device=dev)
+    qd = _desc(q)
+    _check(_lib.dash_attn_cp_lists(ctypes.byref(qd), kv_heads, scores.data_ptr(), seqlens.data_ptr(), lmax, alpha,
+                                   block, idx.data_ptr(), logp.data_ptr(), cnt.data_ptr(), t_cap, _stream(stream)))
+    return {"idx": idx, "logp": logp, "cnt": cnt}
+
+
+def cp_attend(q, kshard, vshard, tok_lo: int, seqlens, lmax: int, lists: dict, block: int, sigma: float = 1.0,
+              part=None, stream=None) -> torch.Tensor:
+    """Partials [B, H, d + 2] of this rank's tokens (see dash_attn_cp_attend)."""
+    B, _, H, d = q.shape
+    part = torch.empty((B, H, d + 2), dtype=torch.float32, device=q.device) if part is None else part
+    qd, kd, vd = _desc(q), _desc(kshard), _desc(vshard)
+    t_cap = lists["idx"].shape[-1]
+    _check(_lib.dash_attn_cp_attend(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), tok_lo, seqlens.data_ptr(),
+                                    lmax, lists["idx"].data_ptr(), lists["logp"].data_ptr(), lists["cnt"].data_ptr(),
+                                    t_cap, block, _options(sigma, None), part.data_ptr(), _stream(stream)))
+    return part
+
+
+def cp_merge(parts: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Merge partials [R, B, H, d + 2] into out [B, 1, H, d] (see dash_attn_cp_merge)."""
+    assert parts.is_contiguous() and parts.dtype == torch.float32
+    od = _desc(out)
+    _check(_lib.dash_attn_cp_merge(parts.data_ptr(), parts.shape[0], ctypes.byref(od), _stream(stream)))
+    return out

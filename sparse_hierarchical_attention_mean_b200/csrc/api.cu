@@ -392,6 +392,9 @@ dash_status_t dash_attn_route(const dash_tensor_t* q, const float* summaries, in
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   dash::DecodeParams p{};
   p.sigma = 1.0f;
+  p.c_lo = 0;
+  p.c_hi = (int)t_cap;
+  p.summ_cap = t_cap;
   p.q = view(q);
   p.dtype = q->dtype;
   p.B = (int)q->b;
@@ -672,11 +675,133 @@ dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* k
   p.max_items = L.max_items;
   p.chunk_blocks = L.chunk;
   p.sigma = sigma;
+  p.c_lo = 0;
+  p.c_hi = (int)t_cap;
+  p.summ_cap = t_cap;
   p.status = at<dash::DeviceStatus>(workspace, L.status);
   e = dash::launch_decode_route(p, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode route");
   e = dash::launch_decode_attend(p, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "decode attend");
+  return ok();
+}
+
+// ------------------------------------------------------------------ context-parallel decode
+
+static dash_status_t cp_common(const dash_tensor_t* q, int64_t kv_heads, const int32_t* seqlens, int64_t lmax,
+                               int block, int64_t t_cap) {
+  dash_status_t st;
+  if ((st = check_tensor(q, "q")) || (st = check_group(q->h, kv_heads))) return st;
+  if (q->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode takes one query token (s == 1)");
+  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "context-parallel decode supports f16 and bf16");
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  if (!seqlens || lmax < 1) return fail(DASH_ERR_INVALID_ARGUMENT, "null seqlens or lmax < 1");
+  if (t_cap < (lmax + block - 1) / block) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap < ceil(lmax / block)");
+  if (t_cap > 4096) return fail(DASH_ERR_UNSUPPORTED, "t_cap above 4096");
+  return DASH_OK;
+}
+
+static dash::DecodeParams cp_params(const dash_tensor_t* q, int64_t kv_heads, const int32_t* seqlens, int64_t lmax,
+                                    int block, int64_t t_cap) {
+  dash::DecodeParams p{};
+  p.q = view(q);
+  p.dtype = q->dtype;
+  p.B = (int)q->b;
+  p.Lmax = (int)lmax;
+  p.H = (int)q->h;
+  p.Hkv = (int)kv_heads;
+  p.G = (int)(q->h / kv_heads);
+  p.D = (int)q->d;
+  p.block = block;
+  p.seqlens = seqlens;
+  p.t_cap = t_cap;
+  p.sigma = 1.0f;
+  p.c_lo = 0;
+  p.c_hi = (int)t_cap;
+  p.summ_cap = t_cap;
+  return p;
+}
+
+dash_status_t dash_attn_cp_scores(const dash_tensor_t* q, int64_t kv_heads, const float* summaries, int64_t summ_cap,
+                                  int64_t block_lo, int64_t block_hi, const int32_t* seqlens, int64_t lmax, float alpha,
+                                  int block, float* scores, int64_t t_cap, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = cp_common(q, kv_heads, seqlens, lmax, block, t_cap)) || (st = check_common(alpha, block))) return st;
+  if (!summaries || !scores) return fail(DASH_ERR_INVALID_ARGUMENT, "null summaries or scores");
+  if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
+  if (block_lo < 0 || block_hi < block_lo || block_hi - block_lo > summ_cap || block_hi > t_cap)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "bad block range [%lld, %lld) for summ_cap %lld",
+                (long long)block_lo, (long long)block_hi, (long long)summ_cap);
+  dash::DecodeParams p = cp_params(q, kv_heads, seqlens, lmax, block, t_cap);
+  p.alpha = alpha;
+  p.summaries = summaries;
+  p.summ_cap = summ_cap;
+  p.c_lo = (int)block_lo;
+  p.c_hi = (int)block_hi;
+  p.scores = scores;
+  cudaError_t e = dash::launch_cp_scores(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "context-parallel scores");
+  return ok();
+}
+
+dash_status_t dash_attn_cp_lists(const dash_tensor_t* q, int64_t kv_heads, const float* scores, const int32_t* seqlens,
+                                 int64_t lmax, float alpha, int block, int32_t* idx, float* logp, int32_t* cnt,
+                                 int64_t t_cap, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = cp_common(q, kv_heads, seqlens, lmax, block, t_cap)) || (st = check_common(alpha, block))) return st;
+  if (!scores || !idx || !logp || !cnt) return fail(DASH_ERR_INVALID_ARGUMENT, "null scores or lists");
+  dash::DecodeParams p = cp_params(q, kv_heads, seqlens, lmax, block, t_cap);
+  p.alpha = alpha;
+  p.scores = const_cast<float*>(scores);
+  p.idx = idx;
+  p.logp = logp;
+  p.cnt = cnt;
+  cudaError_t e = dash::launch_cp_lists(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "context-parallel lists");
+  return ok();
+}
+
+dash_status_t dash_attn_cp_attend(const dash_tensor_t* q, const dash_tensor_t* kshard, const dash_tensor_t* vshard,
+                                  int64_t tok_lo, const int32_t* seqlens, int64_t lmax, const int32_t* idx,
+                                  const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                                  const dash_options_t* opts, float* part, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_tensor(kshard, "kshard")) || (st = check_tensor(vshard, "vshard"))) return st;
+  if ((st = cp_common(q, kshard->h, seqlens, lmax, block, t_cap))) return st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
+  if (q->dtype != kshard->dtype || q->dtype != vshard->dtype) return fail(DASH_ERR_INVALID_ARGUMENT, "dtype mismatch");
+  if (kshard->b != q->b || vshard->b != q->b || kshard->d != q->d || vshard->d != q->d || vshard->h != kshard->h ||
+      vshard->s != kshard->s)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "shard shapes do not match q");
+  if (tok_lo < 0 || tok_lo % block || kshard->s % block)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "shard start and length must be multiples of the block");
+  if (!idx || !logp || !cnt || !part) return fail(DASH_ERR_INVALID_ARGUMENT, "null lists or partials");
+  dash::DecodeParams p = cp_params(q, kshard->h, seqlens, lmax, block, t_cap);
+  p.k = view(kshard);
+  p.v = view(vshard);
+  p.sigma = sigma;
+  p.idx = const_cast<int32_t*>(idx);
+  p.logp = const_cast<float*>(logp);
+  p.cnt = const_cast<int32_t*>(cnt);
+  p.tok_lo = (int)tok_lo;
+  p.tok_n = (int)kshard->s;
+  p.part = part;
+  cudaError_t e = dash::launch_cp_attend(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "context-parallel attention");
+  return ok();
+}
+
+dash_status_t dash_attn_cp_merge(const float* parts, int64_t n_parts, dash_tensor_t* out, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_tensor(out, "out"))) return st;
+  if (out->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "out must be [B, 1, H, d]");
+  if (out->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "context-parallel decode supports f16 and bf16");
+  if (!parts || n_parts < 1) return fail(DASH_ERR_INVALID_ARGUMENT, "null parts or n_parts < 1");
+  cudaError_t e = dash::launch_cp_merge(parts, (int)n_parts, (int)out->b, (int)out->h, (int)out->d, view(out),
+                                        out->dtype, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "context-parallel merge");
   return ok();
 }
 

@@ -49,9 +49,9 @@ __global__ void __launch_bounds__(256) score_decode_kernel(DecodeParams p) {
   const int b = blockIdx.z, g = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int L = clamp_len(p.seqlens, b, p.Lmax, p.status);
-  const int N = (L - 1) / p.block;
+  const int N = min((L - 1) / p.block, p.c_hi);  // scored here: candidates c_lo <= c < N
   const int c0 = blockIdx.x * 64 + warp * 8;
-  if (c0 >= N) return;
+  if (c0 >= N || c0 + 8 <= p.c_lo) return;
   const int64_t bg = (int64_t)b * p.Hkv + g;
   float qv[G][DL];
   const T* q = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb;
@@ -60,16 +60,17 @@ __global__ void __launch_bounds__(256) score_decode_kernel(DecodeParams p) {
 #pragma unroll
     for (int e = 0; e < DL; ++e) qv[h][e] = Elt<T>::load1(q + (int64_t)(g * G + h) * p.q.sh + lane * DL + e);
   float v[NV];
-  const float* sb = p.summaries + bg * p.t_cap * D + lane * DL;
+  const float* sb = p.summaries + bg * p.summ_cap * D + lane * DL;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float s[DL];
-    if (c0 + i < N) {
+    if (c0 + i < N && c0 + i >= p.c_lo) {
+      const int64_t si = c0 + i - p.c_lo;
       if constexpr (DL == 4) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(sb + (int64_t)(c0 + i) * D));
+        const float4 x = __ldg(reinterpret_cast<const float4*>(sb + si * D));
         s[0] = x.x, s[1] = x.y, s[2] = x.z, s[3] = x.w;
       } else {
-        const float2 x = __ldg(reinterpret_cast<const float2*>(sb + (int64_t)(c0 + i) * D));
+        const float2 x = __ldg(reinterpret_cast<const float2*>(sb + si * D));
         s[0] = x.x, s[1] = x.y;
       }
     } else {
@@ -91,14 +92,14 @@ __global__ void __launch_bounds__(256) score_decode_kernel(DecodeParams p) {
     for (int j = 0; j < NV / 32; ++j) {
       const int i = lane * (NV / 32) + j;
       const int c = c0 + i / G, h = i % G;
-      if (c < N) p.scores[(bg * G + h) * p.t_cap + c] = coef * v[j];
+      if (c < N && c >= p.c_lo) p.scores[(bg * G + h) * p.t_cap + c] = coef * v[j];
     }
   } else {
     constexpr int SH = NV == 16 ? 1 : (NV == 8 ? 2 : 0);
     if ((lane & ((1 << SH) - 1)) == 0) {
       const int i = lane >> SH;
       const int c = c0 + i / G, h = i % G;
-      if (c < N) p.scores[(bg * G + h) * p.t_cap + c] = coef * v[0];
+      if (c < N && c >= p.c_lo) p.scores[(bg * G + h) * p.t_cap + c] = coef * v[0];
     }
   }
 }
@@ -662,6 +663,238 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
   }
 }
 
+// ------------------------------------------------------------------ context-parallel shard attention
+// One CTA per (KV head, sequence) over this shard's part of the selected
+// blocks (a contiguous range of the ascending list) and, when the shard
+// holds it, the diagonal block; 16-token units go round-robin to the 4
+// warps, each keeping an online softmax per head (logits by a warp
+// reduce-scatter, P broadcast through shared memory).  The 4 warps merge into
+// one partial per head: o relative to the reference max m (log2 units) and l.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(128) attend_shard_kernel(DecodeParams p) {
+  constexpr int DL = D / 32;
+  constexpr int NV = 16 * G;
+  constexpr int NVL = NV >= 32 ? NV / 32 : 1;
+  constexpr int GH = G >= 2 ? G / 2 : 1;
+  constexpr int W = 4;
+  __shared__ float pbuf[W][16 * G];
+  __shared__ float mbuf[W][G], lbuf[W][G];
+  __shared__ float obuf[W][G][D];
+  __shared__ int erange[2];
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const int L = clamp_len(p.seqlens, b, p.Lmax, nullptr);
+  const int pos = L - 1, t = pos / p.block, N = t;
+  const float beta = N > 0 ? p.sigma * logf(1.0f / (float)N) : 0.0f;
+  const int c_lo = p.tok_lo / p.block, c_hi = (p.tok_lo + p.tok_n) / p.block;
+  const int cnt = min(max(p.cnt[bg], 0), (int)p.t_cap);
+  const int32_t* idx = p.idx + bg * p.t_cap;
+  const float* logp = p.logp + bg * p.t_cap;
+  if (warp == 0) {
+    int nlo = 0, nhi = 0;
+    for (int e = lane; e < cnt; e += 32) {
+      const int c = idx[e];
+      nlo += c < c_lo ? 1 : 0;
+      nhi += c < c_hi ? 1 : 0;
+    }
+    nlo = warp_sum_i(nlo);
+    nhi = warp_sum_i(nhi);
+    if (lane == 0) {
+      erange[0] = nlo;
+      erange[1] = nhi;
+    }
+  }
+  __syncthreads();
+  const int e_lo = erange[0], n_sel = erange[1] - erange[0];
+  const bool diag = t >= c_lo && t < c_hi;
+  const int upb = p.block / 16;  // 16-token units per block
+  const int n_units = n_sel * upb + (diag ? (pos - t * p.block) / 16 + 1 : 0);
+  const float qk_scale = rsqrtf((float)D) * kLog2e;
+  const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
+  const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
+
+  float qv[G][DL];
+  {
+    const T* q = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb;
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < DL; ++e)
+        qv[h][e] = Elt<T>::load1(q + (int64_t)(g * G + h) * p.q.sh + lane * DL + e) * qk_scale;
+  }
+  auto load_row = [&](const T* base, int64_t ss, int tok, float* f) {  // this lane's DL values of a cache row
+    const T* src = base + (int64_t)(tok - p.tok_lo) * ss + lane * DL;
+    float f8[8];
+    if constexpr (DL == 4) {
+      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src));
+      Elt<T>::to_float(make_uint4(raw.x, raw.y, 0u, 0u), f8);
+    } else {
+      const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(src));
+      Elt<T>::to_float(make_uint4(raw, 0u, 0u, 0u), f8);
+    }
+#pragma unroll
+    for (int e = 0; e < DL; ++e) f[e] = f8[e];
+  };
+
+  float m[G], o[G][DL], lown[NVL];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m[h] = kNegInf;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) o[h][e] = 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < NVL; ++j) lown[j] = 0.f;
+
+  for (int u = warp; u < n_units; u += W) {
+    int tok0;
+    float bias;
+    if (u < n_sel * upb) {
+      const int e = e_lo + u / upb;
+      tok0 = idx[e] * p.block + (u % upb) * 16;
+      bias = p.sigma * logp[e] * kLog2e;
+    } else {
+      tok0 = t * p.block + (u - n_sel * upb) * 16;
+      bias = beta * kLog2e;
+    }
+    float v[NV];
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) {
+      float kf[DL];
+      if (tok0 + tt <= pos) {
+        load_row(kg, p.k.ss, tok0 + tt, kf);
+      } else {
+#pragma unroll
+        for (int e = 0; e < DL; ++e) kf[e] = 0.f;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) a = fmaf(qv[h][e], kf[e], a);
+        v[tt * G + h] = a;
+      }
+    }
+    warp_transpose_reduce<NV>(v, lane);
+    // lane holds token lane/2; heads (lane&1)*GH + j (G >= 2) or head 0
+    const bool valid = tok0 + (lane >> 1) <= pos;
+    float sl[NVL], mx[NVL];
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+      sl[j] = valid ? v[j] + bias : kNegInf;
+      mx[j] = sl[j];
+#pragma unroll
+      for (int off = 2; off <= 16; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], off));
+    }
+    float mu[G], sc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float th = __shfl_sync(0xffffffffu, mx[h % GH], G >= 2 ? h / GH : 0);
+      const float mn = fmaxf(m[h], th);
+      mu[h] = mn == kNegInf ? 0.f : mn;
+      sc[h] = exp2f(m[h] - mu[h]);
+      m[h] = mn;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) o[h][e] *= sc[h];
+    }
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+      const int hd = G >= 2 ? (lane & 1) * GH + j : 0;
+      float muj = mu[j], scj = sc[j];
+      if constexpr (G >= 2) {
+        muj = (lane & 1) ? mu[GH + j] : mu[j];
+        scj = (lane & 1) ? sc[GH + j] : sc[j];
+      }
+      const float pj = exp2f(sl[j] - muj);
+      lown[j] = lown[j] * scj + pj;
+      pbuf[warp][(lane >> 1) * G + hd] = pj;
+    }
+    __syncwarp();
+#pragma unroll 4
+    for (int tt = 0; tt < 16; ++tt) {
+      if (tok0 + tt > pos) break;
+      float vf[DL];
+      load_row(vg, p.v.ss, tok0 + tt, vf);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float ph = pbuf[warp][tt * G + h];
+#pragma unroll
+        for (int e = 0; e < DL; ++e) o[h][e] = fmaf(ph, vf[e], o[h][e]);
+      }
+    }
+    __syncwarp();
+  }
+
+  // merge the warps: l per head over the 16 lanes of its parity
+#pragma unroll
+  for (int j = 0; j < NVL; ++j)
+#pragma unroll
+    for (int off = 2; off <= 16; off <<= 1) lown[j] += __shfl_xor_sync(0xffffffffu, lown[j], off);
+  if (lane < 2) {
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+      if (G >= 2) {
+        lbuf[warp][lane * GH + j] = lown[j];
+      } else if (lane == 0) {
+        lbuf[warp][0] = lown[0];
+      }
+    }
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) mbuf[warp][h] = m[h];
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < DL; ++e) obuf[warp][h][lane * DL + e] = o[h][e];
+  __syncthreads();
+  for (int i = tid; i < G * D; i += W * 32) {
+    const int h = i / D, e = i % D;
+    float M = kNegInf;
+#pragma unroll
+    for (int w = 0; w < W; ++w) M = fmaxf(M, mbuf[w][h]);
+    const float Mu = M == kNegInf ? 0.f : M;
+    float acc = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const float f = exp2f(mbuf[w][h] - Mu);
+      acc += f * obuf[w][h][e];
+      lsum += f * lbuf[w][h];
+    }
+    float* part = p.part + ((int64_t)b * p.H + g * G + h) * (D + 2);
+    part[e] = acc;
+    if (e == 0) {
+      part[D] = M;
+      part[D + 1] = lsum;
+    }
+  }
+}
+
+// Log-sum-exp merge of the shards' partials into the output.
+template <typename T>
+__global__ void __launch_bounds__(128) cp_merge_kernel(const float* parts, int n_parts, int B, int H, int D,
+                                                       View out) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int64_t stride = (int64_t)B * H * (D + 2);
+  const float* p0 = parts + ((int64_t)b * H + h) * (D + 2);
+  float M = kNegInf;
+  for (int r = 0; r < n_parts; ++r) M = fmaxf(M, p0[r * stride + D]);
+  const float Mu = M == kNegInf ? 0.f : M;
+  T* dst = static_cast<T*>(const_cast<void*>(out.data)) + (int64_t)b * out.sb + (int64_t)h * out.sh;
+  for (int e = threadIdx.x; e < D; e += blockDim.x) {
+    float acc = 0.f, lsum = 0.f;
+    for (int r = 0; r < n_parts; ++r) {
+      const float* pr = p0 + r * stride;
+      const float f = exp2f(pr[D] - Mu);
+      acc += f * pr[e];
+      lsum += f * pr[D + 1];
+    }
+    Elt<T>::store1(dst + e, lsum > 0.f ? acc / lsum : 0.f);
+  }
+}
+
 // ------------------------------------------------------------------ combine
 template <typename T, int D>
 __global__ void __launch_bounds__(256) combine_decode_kernel(DecodeParams p) {
@@ -763,6 +996,59 @@ cudaError_t launch_decode_attend(const DecodeParams& p, int num_sms, cudaStream_
   }
   if (p.dtype == 1) return attend_d<__half, 64>(p, num_sms, stream);
   return attend_d<__nv_bfloat16, 64>(p, num_sms, stream);
+}
+
+namespace {
+template <typename T, int D>
+cudaError_t cp_scores_d(const DecodeParams& p, cudaStream_t s) {
+  dim3 grid((unsigned)((p.t_cap + 63) / 64), p.Hkv, p.B);
+  switch (p.G) {
+    case 1: score_decode_kernel<T, D, 1><<<grid, 256, 0, s>>>(p); break;
+    case 2: score_decode_kernel<T, D, 2><<<grid, 256, 0, s>>>(p); break;
+    case 4: score_decode_kernel<T, D, 4><<<grid, 256, 0, s>>>(p); break;
+    default: score_decode_kernel<T, D, 8><<<grid, 256, 0, s>>>(p); break;
+  }
+  return cudaGetLastError();
+}
+template <typename T, int D>
+cudaError_t cp_attend_d(const DecodeParams& p, cudaStream_t s) {
+  dim3 grid(p.Hkv, p.B);
+  switch (p.G) {
+    case 1: attend_shard_kernel<T, D, 1><<<grid, 128, 0, s>>>(p); break;
+    case 2: attend_shard_kernel<T, D, 2><<<grid, 128, 0, s>>>(p); break;
+    case 4: attend_shard_kernel<T, D, 4><<<grid, 128, 0, s>>>(p); break;
+    default: attend_shard_kernel<T, D, 8><<<grid, 128, 0, s>>>(p); break;
+  }
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_cp_scores(const DecodeParams& p, cudaStream_t stream) {
+  if (p.D == 128) return p.dtype == 1 ? cp_scores_d<__half, 128>(p, stream) : cp_scores_d<__nv_bfloat16, 128>(p, stream);
+  return p.dtype == 1 ? cp_scores_d<__half, 64>(p, stream) : cp_scores_d<__nv_bfloat16, 64>(p, stream);
+}
+
+cudaError_t launch_cp_lists(const DecodeParams& p, cudaStream_t stream) {
+  const size_t smem = (size_t)p.G * p.t_cap * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(entmax_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  entmax_decode_kernel<<<dim3(p.Hkv, p.B), 256, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cp_attend(const DecodeParams& p, cudaStream_t stream) {
+  if (p.D == 128) return p.dtype == 1 ? cp_attend_d<__half, 128>(p, stream) : cp_attend_d<__nv_bfloat16, 128>(p, stream);
+  return p.dtype == 1 ? cp_attend_d<__half, 64>(p, stream) : cp_attend_d<__nv_bfloat16, 64>(p, stream);
+}
+
+cudaError_t launch_cp_merge(const float* parts, int n_parts, int B, int H, int D, const View& out, int dtype,
+                            cudaStream_t stream) {
+  dim3 grid(H, B);
+  if (dtype == 1)
+    cp_merge_kernel<__half><<<grid, 128, 0, stream>>>(parts, n_parts, B, H, D, out);
+  else
+    cp_merge_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(parts, n_parts, B, H, D, out);
+  return cudaGetLastError();
 }
 
 }  // namespace dash

@@ -148,6 +148,15 @@ struct DecodeParams {
   int64_t max_items;
   int chunk_blocks;  // selected blocks per split-KV work item
   float sigma;       // prior strength (as in SparseParams)
+  // context parallelism: this shard scores blocks [c_lo, c_hi) whose summaries
+  // sit at index c - c_lo of `summaries` (capacity summ_cap blocks); the
+  // whole-context decode uses c_lo = 0, c_hi = t_cap, summ_cap = t_cap
+  int c_lo, c_hi;
+  int64_t summ_cap;
+  // shard attention: cache tokens [tok_lo, tok_lo + k.s) of every sequence,
+  // partials [B, H, D + 2] (o relative to m, m in log2 units, l)
+  int tok_lo, tok_n;
+  float* part;
   // optional route outputs (dash_attn_route in decode mode)
   float* tau;      // [B, H]
   float* p_dense;  // [B, H, t_cap]
@@ -159,5 +168,12 @@ cudaError_t launch_decode_route(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_lists_to_mask(const int32_t* idx, const int32_t* cnt, int64_t rows, int64_t t_cap,
                                  uint32_t* mask, int n_words, cudaStream_t stream);
 cudaError_t launch_decode_attend(const DecodeParams& p, int num_sms, cudaStream_t stream);
+// context parallelism: shard scores (score kernel only), lists from a score
+// buffer (entmax kernel without work items), shard attention, partial merge
+cudaError_t launch_cp_scores(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_cp_lists(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_cp_attend(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_cp_merge(const float* parts, int n_parts, int B, int H, int D, const View& out, int dtype,
+                            cudaStream_t stream);
 
 }  // namespace dash

@@ -1,0 +1,72 @@
+"""Context-parallel decode on one GPU: R ranks emulated one after the other
+(the score all-reduce is a sum of the ranks' buffers, the all-gather a stack
+of their partials).  Checked against the whole-cache decode (identical
+lists; outputs within the decode tolerance of each other) and the oracle."""
+
+import pytest
+import torch
+
+from gen import full_inputs, get_config
+from tests._parity import OUT_TOL, max_abs, oracle_decode_pair, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dash(cuda_lib):
+    return cuda_lib
+
+
+CASES = {
+    "bf16_g4_r2": (get_config("decode").with_(name="cp_a", batch=3, seq=4096, seqlen_lo=200, seqlen_hi=4096), 2, 1.0),
+    "bf16_g4_r4_sigma": (get_config("decode").with_(name="cp_b", batch=3, seq=4096, seqlen_lo=1, seqlen_hi=4096), 4,
+                         0.5),
+    "f16_g8_d64_b128_r2": (get_config("decode").with_(name="cp_c", batch=2, heads=16, kv_heads=2, head_dim=64,
+                                                      dtype="f16", block=128, seq=3072, seqlen_lo=500,
+                                                      seqlen_hi=3072), 2, 1.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_context_parallel_decode(dash, name):
+    cfg, R, sigma = CASES[name]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
+    B, lmax, Hkv, d = k.shape
+    H, G, blk = q.shape[2], cfg.group, cfg.block
+    t_cap = -(-lmax // blk)
+    # whole cache
+    summ = dash.summarize(k, w, blk, seqlens=sl)
+    ref = dash.decode(q, k, v, sl, summ, cfg.alpha, blk, sigma=sigma)
+    rt = dash.route(q, summ, cfg.alpha, blk, True, seqlens=sl)
+    # shards: block-aligned token ranges
+    bounds = [((lmax // blk) * r // R) * blk for r in range(R)] + [lmax]
+    scores = torch.zeros((B, Hkv, G, t_cap), dtype=torch.float32, device="cuda")
+    shards = []
+    for r in range(R):
+        lo, hi = bounds[r], bounds[r + 1]
+        ks, vs = k[:, lo:hi].contiguous(), v[:, lo:hi].contiguous()
+        sl_r = (sl - lo).clamp(0, hi - lo).to(torch.int32)
+        summ_r = dash.summarize(ks, w, blk, seqlens=sl_r)
+        part_scores = torch.zeros_like(scores)
+        dash.cp_scores(q, summ_r, lo // blk, hi // blk, sl, lmax, cfg.alpha, blk, part_scores)
+        scores += part_scores
+        shards.append((lo, ks, vs))
+    lists = dash.cp_lists(q, Hkv, scores, sl, lmax, cfg.alpha, blk)
+    parts = torch.stack([dash.cp_attend(q, ks, vs, lo, sl, lmax, lists, blk, sigma=sigma) for lo, ks, vs in shards])
+    out = dash.cp_merge(parts.contiguous(), torch.empty_like(q))
+    torch.cuda.synchronize()
+    # the routing is the whole cache's, bit for bit
+    assert torch.equal(lists["cnt"], rt["cnt"][:, :, 0])
+    for b in range(B):
+        for g in range(Hkv):
+            n = int(lists["cnt"][b, g])
+            assert torch.equal(lists["idx"][b, g, :n], rt["idx"][b, g, 0, :n])
+            assert torch.equal(lists["logp"][b, g, :n], rt["logp"][b, g, 0, :n])
+    tol = OUT_TOL[cfg.dtype]
+    assert max_abs(to_np(out), to_np(ref)) <= tol
+    for b in range(B):
+        for g in sorted({0, Hkv - 1}):
+            rec, _ = oracle_decode_pair(cfg, inp["plan"], b, g, sigma=sigma)
+            err = max_abs(to_np(out)[b, 0, g * G:(g + 1) * G], rec["out"])
+            assert err <= tol, f"{name} b{b} g{g}: {err:.3g}"
