@@ -164,6 +164,27 @@ dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, c
                                dash_stream_t stream);
 
 /*
+ * Paged KV cache (the layout of serving engines): the cache is a pool of
+ * pages of `block` tokens, k_pages / v_pages [n_pages, block, Hkv, d]
+ * (dash_tensor_t with b = n_pages, s = block), and block c of sequence b
+ * lives in page block_table[b * max_blocks + c] (device int32
+ * [batch, max_blocks]; entries past a sequence's blocks are not read).  The
+ * context bound is lmax = max_blocks * block.  Results are those of
+ * dash_attn_summarize_sdpa / dash_attn_decode_ex on the same cache laid out
+ * densely.  The decode workspace is dash_attn_decode_workspace_size of a
+ * dense cache with the same B, Hkv and d.
+ */
+dash_status_t dash_attn_summarize_paged(const dash_tensor_t* k_pages, const int32_t* block_table, int64_t max_blocks,
+                                        int64_t batch, const int32_t* seqlens, const float* w_s, const float* qbar,
+                                        int block, float* summaries, int64_t t_cap, int64_t first_block,
+                                        dash_stream_t stream);
+dash_status_t dash_attn_decode_paged(const dash_tensor_t* q, const dash_tensor_t* k_pages, const dash_tensor_t* v_pages,
+                                     const int32_t* block_table, int64_t max_blocks, const int32_t* seqlens,
+                                     const float* summaries, int64_t t_cap, float alpha, int block, dash_tensor_t* out,
+                                     void* workspace, size_t workspace_bytes, const dash_options_t* opts,
+                                     dash_stream_t stream);
+
+/*
  * Context-parallel decode: one sequence's context split over R ranks (one
  * process per GPU), each holding the cache tokens [tok_lo, tok_lo + n) of
  * every sequence (tok_lo and n multiples of the block) and the summaries of

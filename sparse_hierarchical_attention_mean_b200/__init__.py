@@ -46,6 +46,8 @@ EXPORTED = (
     "dash_attn_cp_lists",
     "dash_attn_cp_attend",
     "dash_attn_cp_merge",
+    "dash_attn_summarize_paged",
+    "dash_attn_decode_paged",
     "dash_attn_decode_workspace_size",
     "dash_attn_decode",
     "dash_attn_route_workspace_size",
@@ -112,6 +114,8 @@ def _load() -> ctypes.CDLL:
         "dash_attn_cp_lists": (i32, [T, i64, vp, vp, i64, f32, i32, vp, vp, vp, i64, vp]),
         "dash_attn_cp_attend": (i32, [T, T, T, i64, vp, i64, vp, vp, vp, i64, i32, O, vp, vp]),
         "dash_attn_cp_merge": (i32, [vp, i64, T, vp]),
+        "dash_attn_summarize_paged": (i32, [T, vp, i64, i64, vp, vp, vp, i32, vp, i64, i64, vp]),
+        "dash_attn_decode_paged": (i32, [T, T, T, vp, i64, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
         "dash_attn_get_device_status": (i32, [vp, vp]),
         "dash_attn_decode_noalloc": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp]),
     }
@@ -417,4 +421,41 @@ def cp_merge(parts: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tenso
     assert parts.is_contiguous() and parts.dtype == torch.float32
     od = _desc(out)
     _check(_lib.dash_attn_cp_merge(parts.data_ptr(), parts.shape[0], ctypes.byref(od), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ paged KV cache
+
+
+def summarize_paged(k_pages, block_table, seqlens, w_s, block: int, summaries=None, t_cap: int | None = None,
+                    first_block: int = 0, qbar=None, stream=None) -> torch.Tensor:
+    """Summaries [B, Hkv, t_cap, d] from a paged cache (see dash_attn_summarize_paged)."""
+    n_pages, page, Hkv, d = k_pages.shape
+    B, max_blocks = block_table.shape
+    t_cap = max_blocks if t_cap is None else t_cap
+    if summaries is None:
+        summaries = torch.zeros((B, Hkv, t_cap, d), dtype=torch.float32, device=k_pages.device)
+    kd = _desc(k_pages)
+    _check(_lib.dash_attn_summarize_paged(ctypes.byref(kd), block_table.data_ptr(), max_blocks, B, seqlens.data_ptr(),
+                                          w_s.data_ptr(), _ptr(qbar), block, summaries.data_ptr(), summaries.shape[2],
+                                          first_block, _stream(stream)))
+    return summaries
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, summaries, alpha: float, block: int, out=None,
+                 workspace=None, sigma: float = 1.0, stream=None) -> torch.Tensor:
+    """One decode step against a paged cache (see dash_attn_decode_paged)."""
+    out = torch.empty_like(q) if out is None else out
+    B, max_blocks = block_table.shape
+    t_cap = summaries.shape[2]
+    qd, kd, vd, od = _desc(q), _desc(k_pages), _desc(v_pages), _desc(out)
+    # the workspace is that of a dense cache of the same B, Hkv, d (only the shape enters the size query)
+    dk = DashTensor(k_pages.data_ptr(), kd.dtype, 0, B, max_blocks * block, kd.h, kd.d,
+                    kd.h * kd.d * max_blocks * block, kd.h * kd.d, kd.d)
+    nbytes = _lib.dash_attn_decode_workspace_size(ctypes.byref(qd), ctypes.byref(dk), block, t_cap)
+    ws = _workspace(nbytes, q.device, workspace)
+    _check(_lib.dash_attn_decode_paged(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), block_table.data_ptr(),
+                                       max_blocks, seqlens.data_ptr(), summaries.data_ptr(), t_cap, alpha, block,
+                                       ctypes.byref(od), ws.data_ptr(), ws.numel(), _options(sigma, None),
+                                       _stream(stream)))
     return out

@@ -613,31 +613,14 @@ dash_status_t dash_attn_decode(const dash_tensor_t* q, const dash_tensor_t* kcac
                              workspace_bytes, nullptr, stream);
 }
 
-dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,
-                                  const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha,
-                                  int block, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
-                                  const dash_options_t* opts, dash_stream_t stream) {
-  dash_status_t st;
-  float sigma;
-  const float* qbar;
-  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
-  if ((st = check_tensor(q, "q")) || (st = check_tensor(kcache, "kcache")) || (st = check_tensor(vcache, "vcache")) ||
-      (st = check_tensor(out, "out")) || (st = check_common(alpha, block)) || (st = check_group(q->h, kcache->h)))
-    return st;
-  if (q->s != 1 || out->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode takes one query token (s == 1)");
-  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "decode supports f16 and bf16");
-  if (q->dtype != kcache->dtype || q->dtype != vcache->dtype || q->dtype != out->dtype)
-    return fail(DASH_ERR_INVALID_ARGUMENT, "q, caches and out must share one dtype");
-  if (kcache->b != q->b || vcache->b != q->b || out->b != q->b) return fail(DASH_ERR_INVALID_ARGUMENT, "batch mismatch");
-  if (kcache->d != q->d || vcache->d != q->d || out->d != q->d) return fail(DASH_ERR_INVALID_ARGUMENT, "head dim mismatch");
-  if (vcache->h != kcache->h || vcache->s != kcache->s) return fail(DASH_ERR_INVALID_ARGUMENT, "kcache and vcache differ");
-  if (out->h != q->h) return fail(DASH_ERR_INVALID_ARGUMENT, "out must have q's shape");
-  if (!seqlens || !summaries) return fail(DASH_ERR_INVALID_ARGUMENT, "null seqlens or summaries");
-  if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
-  const int64_t T = (kcache->s + block - 1) / block;
-  if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(Lmax / block)", (long long)t_cap);
-  if (t_cap > 4096) return fail(DASH_ERR_UNSUPPORTED, "t_cap above 4096");
-  const DecodeLayout L = decode_layout(q->b, q->h, kcache->h, q->d, block, t_cap);
+// The decode step once its arguments are checked: dense cache (table null;
+// k/v views of [B, Lmax, Hkv, d]) or paged (k/v views of [pages, block, Hkv,
+// d], sb = page stride).
+static dash_status_t run_decode_step(const dash_tensor_t* q, dash::View kv, dash::View vv, int64_t Hkv, int64_t lmax,
+                                     const int32_t* table, int64_t max_blocks, const int32_t* seqlens,
+                                     const float* summaries, int64_t t_cap, float alpha, int block, dash_tensor_t* out,
+                                     void* workspace, size_t workspace_bytes, float sigma, dash_stream_t stream) {
+  const DecodeLayout L = decode_layout(q->b, q->h, Hkv, q->d, block, t_cap);
   if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
     return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
   if (workspace_bytes < L.total)
@@ -648,15 +631,17 @@ dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* k
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   dash::DecodeParams p{};
   p.q = view(q);
-  p.k = view(kcache);
-  p.v = view(vcache);
+  p.k = kv;
+  p.v = vv;
+  p.block_table = table;
+  p.max_blocks = (int)max_blocks;
   p.out = view(out);
   p.dtype = q->dtype;
   p.B = (int)q->b;
-  p.Lmax = (int)kcache->s;
+  p.Lmax = (int)lmax;
   p.H = (int)q->h;
-  p.Hkv = (int)kcache->h;
-  p.G = (int)(q->h / kcache->h);
+  p.Hkv = (int)Hkv;
+  p.G = (int)(q->h / Hkv);
   p.D = (int)q->d;
   p.block = block;
   p.alpha = alpha;
@@ -684,6 +669,110 @@ dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* k
   e = dash::launch_decode_attend(p, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "decode attend");
   return ok();
+}
+
+dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,
+                                  const int32_t* seqlens, const float* summaries, int64_t t_cap, float alpha,
+                                  int block, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                                  const dash_options_t* opts, dash_stream_t stream) {
+  dash_status_t st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
+  if ((st = check_tensor(q, "q")) || (st = check_tensor(kcache, "kcache")) || (st = check_tensor(vcache, "vcache")) ||
+      (st = check_tensor(out, "out")) || (st = check_common(alpha, block)) || (st = check_group(q->h, kcache->h)))
+    return st;
+  if (q->s != 1 || out->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode takes one query token (s == 1)");
+  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "decode supports f16 and bf16");
+  if (q->dtype != kcache->dtype || q->dtype != vcache->dtype || q->dtype != out->dtype)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "q, caches and out must share one dtype");
+  if (kcache->b != q->b || vcache->b != q->b || out->b != q->b) return fail(DASH_ERR_INVALID_ARGUMENT, "batch mismatch");
+  if (kcache->d != q->d || vcache->d != q->d || out->d != q->d) return fail(DASH_ERR_INVALID_ARGUMENT, "head dim mismatch");
+  if (vcache->h != kcache->h || vcache->s != kcache->s) return fail(DASH_ERR_INVALID_ARGUMENT, "kcache and vcache differ");
+  if (out->h != q->h) return fail(DASH_ERR_INVALID_ARGUMENT, "out must have q's shape");
+  if (!seqlens || !summaries) return fail(DASH_ERR_INVALID_ARGUMENT, "null seqlens or summaries");
+  if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
+  const int64_t T = (kcache->s + block - 1) / block;
+  if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(Lmax / block)", (long long)t_cap);
+  if (t_cap > 4096) return fail(DASH_ERR_UNSUPPORTED, "t_cap above 4096");
+  return run_decode_step(q, view(kcache), view(vcache), kcache->h, kcache->s, nullptr, 0, seqlens, summaries, t_cap,
+                         alpha, block, out, workspace, workspace_bytes, sigma, stream);
+}
+
+// ------------------------------------------------------------------ paged KV cache
+
+static dash_status_t check_pages(const dash_tensor_t* pages, const char* name, int block, const int32_t* table,
+                                 int64_t max_blocks) {
+  dash_status_t st;
+  if ((st = check_tensor(pages, name))) return st;
+  if (pages->s != block) return fail(DASH_ERR_INVALID_ARGUMENT, "%s: page size %lld != block %d", name,
+                                     (long long)pages->s, block);
+  if (!table || max_blocks < 1) return fail(DASH_ERR_INVALID_ARGUMENT, "null block table or max_blocks < 1");
+  return DASH_OK;
+}
+
+dash_status_t dash_attn_summarize_paged(const dash_tensor_t* k_pages, const int32_t* block_table, int64_t max_blocks,
+                                        int64_t batch, const int32_t* seqlens, const float* w_s, const float* qbar,
+                                        int block, float* summaries, int64_t t_cap, int64_t first_block,
+                                        dash_stream_t stream) {
+  dash_status_t st;
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  if ((st = check_pages(k_pages, "k_pages", block, block_table, max_blocks))) return st;
+  if (batch < 1 || !seqlens) return fail(DASH_ERR_INVALID_ARGUMENT, "batch < 1 or null seqlens");
+  if (!w_s || !summaries) return fail(DASH_ERR_INVALID_ARGUMENT, "null w_s or summaries");
+  if (reinterpret_cast<uintptr_t>(summaries) % 16 || reinterpret_cast<uintptr_t>(w_s) % 16 ||
+      reinterpret_cast<uintptr_t>(qbar) % 16)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "summaries, w_s or qbar not 16-byte aligned");
+  if (t_cap < max_blocks) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap < max_blocks");
+  if (first_block < 0) return fail(DASH_ERR_INVALID_ARGUMENT, "first_block < 0");
+  dash::PoolParams p{};
+  p.k = view(k_pages);
+  p.dtype = k_pages->dtype;
+  p.B = (int)batch;
+  p.S = (int)(max_blocks * block);
+  p.Hkv = (int)k_pages->h;
+  p.D = (int)k_pages->d;
+  p.block = block;
+  p.seqlens = seqlens;
+  p.w_s = w_s;
+  p.qbar = qbar;
+  p.block_table = block_table;
+  p.max_blocks = (int)max_blocks;
+  p.summaries = summaries;
+  p.t_cap = t_cap;
+  p.first_block = first_block;
+  cudaError_t e = dash::launch_pool(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "summarize (paged)");
+  return ok();
+}
+
+dash_status_t dash_attn_decode_paged(const dash_tensor_t* q, const dash_tensor_t* k_pages, const dash_tensor_t* v_pages,
+                                     const int32_t* block_table, int64_t max_blocks, const int32_t* seqlens,
+                                     const float* summaries, int64_t t_cap, float alpha, int block, dash_tensor_t* out,
+                                     void* workspace, size_t workspace_bytes, const dash_options_t* opts,
+                                     dash_stream_t stream) {
+  dash_status_t st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
+  if ((st = check_tensor(q, "q")) || (st = check_tensor(out, "out")) || (st = check_common(alpha, block))) return st;
+  if ((st = check_pages(k_pages, "k_pages", block, block_table, max_blocks)) ||
+      (st = check_pages(v_pages, "v_pages", block, block_table, max_blocks)) || (st = check_group(q->h, k_pages->h)))
+    return st;
+  if (q->s != 1 || out->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode takes one query token (s == 1)");
+  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "decode supports f16 and bf16");
+  if (q->dtype != k_pages->dtype || q->dtype != v_pages->dtype || q->dtype != out->dtype)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "q, pages and out must share one dtype");
+  if (k_pages->d != q->d || v_pages->d != q->d || out->d != q->d || v_pages->h != k_pages->h ||
+      v_pages->b != k_pages->b)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "page shapes do not match q");
+  if (out->b != q->b || out->h != q->h) return fail(DASH_ERR_INVALID_ARGUMENT, "out must have q's shape");
+  if (!seqlens || !summaries) return fail(DASH_ERR_INVALID_ARGUMENT, "null seqlens or summaries");
+  if (reinterpret_cast<uintptr_t>(summaries) % 16) return fail(DASH_ERR_INVALID_ARGUMENT, "summaries not 16-byte aligned");
+  if (t_cap < max_blocks) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap < max_blocks");
+  if (t_cap > 4096) return fail(DASH_ERR_UNSUPPORTED, "t_cap above 4096");
+  return run_decode_step(q, view(k_pages), view(v_pages), k_pages->h, max_blocks * block, block_table, max_blocks,
+                         seqlens, summaries, t_cap, alpha, block, out, workspace, workspace_bytes, sigma, stream);
 }
 
 // ------------------------------------------------------------------ context-parallel decode

@@ -502,8 +502,8 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
     const int32_t* idx = p.idx + (int64_t)bg * p.t_cap;
     const float* logp = p.logp + (int64_t)bg * p.t_cap;
     const float beta = N > 0 ? p.sigma * logf(1.0f / (float)N) : 0.0f;
-    const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
-    const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
+    const T* kg = static_cast<const T*>(p.k.data) + (int64_t)g * p.k.sh;
+    const T* vg = static_cast<const T*>(p.v.data) + (int64_t)g * p.v.sh;
 
     auto sub_tok0 = [&](int s) -> int {
       if (s < n_sel * spb) return idx[e_begin + s / spb] * p.block + (s % spb) * kStep;
@@ -512,15 +512,26 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
     auto load = [&](int s) {
       if (s < n_sub) {
         const int tok0 = sub_tok0(s);
+        // first row of the step: a step never crosses a block, so a paged
+        // cache needs one page lookup per step
+        int64_t kr0, vr0;
+        if (p.block_table) {
+          const int64_t page = p.block_table[(int64_t)b * p.max_blocks + tok0 / p.block];
+          kr0 = page * p.k.sb + (int64_t)(tok0 % p.block) * p.k.ss;
+          vr0 = page * p.v.sb + (int64_t)(tok0 % p.block) * p.v.ss;
+        } else {
+          kr0 = (int64_t)b * p.k.sb + (int64_t)tok0 * p.k.ss;
+          vr0 = (int64_t)b * p.v.sb + (int64_t)tok0 * p.v.ss;
+        }
         T* kd = Ks + (s % kDStages) * kStageElems;
         T* vd = Vs + (s % kDStages) * kStageElems;
         for (int i = tid; i < kStep * NCH; i += kWarps * 32) {
           const int r = i / NCH, c = i % NCH;
-          const int tok = tok0 + r;
-          const bool ok = tok < L;  // rows past the context are zero-filled
+          const bool ok = tok0 + r < L;  // rows past the context are zero-filled
           const int pc = c ^ (r & 7);
-          cp_async16(kd + r * D + pc * 8, kg + (int64_t)(ok ? tok : 0) * p.k.ss + c * 8, ok);
-          cp_async16(vd + r * D + pc * 8, vg + (int64_t)(ok ? tok : 0) * p.v.ss + c * 8, ok);
+          const int rr = ok ? r : 0;
+          cp_async16(kd + r * D + pc * 8, kg + kr0 + (int64_t)rr * p.k.ss + c * 8, ok);
+          cp_async16(vd + r * D + pc * 8, vg + vr0 + (int64_t)rr * p.v.ss + c * 8, ok);
         }
       }
       cp_async_commit();

@@ -27,6 +27,8 @@ struct PoolParams {
   const int32_t* seqlens;  // nullable
   const float* w_s;        // [D, D]
   const float* qbar;       // [Hkv, D] learned summary queries, or null (mean pooling)
+  const int32_t* block_table;  // paged cache: block c of sequence b is page block_table[b * max_blocks + c]
+  int max_blocks;              //   (k.sb = page stride, k.ss = row stride); null for a dense cache
   float* summaries;        // [B, Hkv, t_cap, D]
   int64_t t_cap;
   int64_t first_block;
@@ -157,6 +159,10 @@ struct DecodeParams {
   // partials [B, H, D + 2] (o relative to m, m in log2 units, l)
   int tok_lo, tok_n;
   float* part;
+  // paged cache (split-KV decode): block c of sequence b is page
+  // block_table[b * max_blocks + c] of k / v (sb = page stride); null: dense
+  const int32_t* block_table;
+  int max_blocks;
   // optional route outputs (dash_attn_route in decode mode)
   float* tau;      // [B, H]
   float* p_dense;  // [B, H, t_cap]

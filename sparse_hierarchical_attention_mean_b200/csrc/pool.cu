@@ -50,12 +50,18 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
   const int nb = (int)(nblk - c_begin < bpc ? nblk - c_begin : bpc);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int vcol = lane % VPR, vrow = lane / VPR;
-  const T* kbase = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh + vcol * EPV;
+  const T* kbase = static_cast<const T*>(p.k.data) + (int64_t)g * p.k.sh + vcol * EPV;
+  // rows of block c: row j (absolute token) at block_base(c) + (j - c * block) * ss
+  auto block_base = [&](int64_t c) -> const T* {
+    if (p.block_table) return kbase + (int64_t)p.block_table[(int64_t)b * p.max_blocks + c] * p.k.sb;
+    return kbase + (int64_t)b * p.k.sb + c * p.block * p.k.ss;
+  };
 
   if constexpr (!SDPA) {
     for (int i = warp; i < nb; i += kWarpsP) {
       const int64_t lo = (c_begin + i) * p.block;
       const int64_t hi = lo + p.block < n_tok ? lo + p.block : (int64_t)n_tok;
+      const T* kb = block_base(c_begin + i);
       float acc[EPV];
 #pragma unroll
       for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
@@ -64,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int64_t j = j0 + u * RPL + vrow;
-          v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kbase + j * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
+          v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kb + (j - lo) * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -100,6 +106,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
     for (int i = warp; i < nb; i += kWarpsP) {
       const int64_t lo = (c_begin + i) * p.block;
       const int64_t hi = lo + p.block < n_tok ? lo + p.block : (int64_t)n_tok;
+      const T* kb = block_base(c_begin + i);
       float acc[EPV], m = kNegInf, den = 0.f;
 #pragma unroll
       for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
@@ -108,7 +115,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int64_t j = j0 + u * RPL + vrow;
-          v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kbase + j * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
+          v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kb + (j - lo) * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
         }
         float a[8];
 #pragma unroll

@@ -70,3 +70,32 @@ def test_context_parallel_decode(dash, name):
             rec, _ = oracle_decode_pair(cfg, inp["plan"], b, g, sigma=sigma)
             err = max_abs(to_np(out)[b, 0, g * G:(g + 1) * G], rec["out"])
             assert err <= tol, f"{name} b{b} g{g}: {err:.3g}"
+
+
+@pytest.mark.parametrize("block,dtype,qscale", [(64, "bf16", None), (128, "f16", 3.0)])
+def test_paged_cache_matches_dense(dash, block, dtype, qscale):
+    """A paged cache (pages of one block, shuffled, through a block table) gives the
+    dense cache's summaries and decode output bit for bit."""
+    cfg = get_config("decode").with_(name="paged", batch=3, seq=4096, seqlen_lo=100, seqlen_hi=4096, block=block,
+                                     dtype=dtype)
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
+    B, lmax, Hkv, d = k.shape
+    nb = lmax // block
+    qbar = None
+    if qscale is not None:
+        qbar = (torch.randn((Hkv, d), generator=torch.Generator().manual_seed(5)) * qscale).float().cuda()
+    # pages: every (sequence, block) in a shuffled pool, plus unused pages
+    perm = torch.randperm(B * nb + 7, generator=torch.Generator().manual_seed(3))
+    table = perm[: B * nb].view(B, nb).to(torch.int32).cuda()
+    kp = torch.zeros((B * nb + 7, block, Hkv, d), dtype=k.dtype, device="cuda")
+    vp = torch.zeros_like(kp)
+    kp[table.view(-1).long()] = k.view(B, nb, block, Hkv, d).reshape(B * nb, block, Hkv, d)
+    vp[table.view(-1).long()] = v.view(B, nb, block, Hkv, d).reshape(B * nb, block, Hkv, d)
+    summ = dash.summarize(k, w, block, seqlens=sl, qbar=qbar)
+    summ_p = dash.summarize_paged(kp, table, sl, w, block, qbar=qbar)
+    ref = dash.decode(q, k, v, sl, summ, cfg.alpha, block)
+    out = dash.decode_paged(q, kp, vp, table, sl, summ_p, cfg.alpha, block)
+    torch.cuda.synchronize()
+    assert torch.equal(summ_p, summ)
+    assert torch.equal(out, ref)
