@@ -15,15 +15,15 @@
 //                    mean, ballot/popc compaction, and the split-KV work
 //                    items (chunks of selected blocks) appended with one
 //                    atomic per (b, g).
-//  attend_decode     persistent CTAs over the work items: K/V rows of the
-//                    selected blocks stream through a cp.async ring; each
-//                    warp owns 16 tokens of a 64-token step, keeps an online
-//                    softmax per head and accumulates P V; the 4 warps merge
-//                    into one (m, l, o) partial per item.  f16/bf16 take both
-//                    products on the tensor cores with warp-level MMAs
-//                    (attend_decode_mma_kernel); fp32 computes them with a
-//                    reduce-scatter on the CUDA cores.
+//  attend_decode_mma persistent CTAs over the work items: K/V rows of the
+//                    selected blocks (dense or paged cache) stream through a
+//                    cp.async ring; each warp owns 16 tokens of a 64-token
+//                    step, takes both products on the tensor cores with
+//                    warp-level MMAs, keeps an online softmax per head; the
+//                    4 warps merge into one (m, l, o) partial per item.
 //  combine_decode    log-sum-exp merge of the partials of each (b, g).
+//  attend_shard, cp_merge  context parallelism: stage 2 over one rank's
+//                    tokens into per-head partials, and their merge.
 #include <type_traits>
 
 #include "common.cuh"
@@ -184,244 +184,9 @@ __global__ void __launch_bounds__(256) entmax_decode_kernel(DecodeParams p) {
 constexpr int kStep = 64;  // tokens per pipeline step
 constexpr int kWarps = 4;  // 16 tokens per warp per step
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kWarps * 32) attend_decode_kernel(DecodeParams p) {
-  constexpr int DL = D / 32;
-  constexpr int NV = 16 * G;
-  constexpr int NVL = NV >= 32 ? NV / 32 : 1;  // values per lane after the reduce
-  constexpr int GH = G >= 2 ? G / 2 : 1;         // heads per lane parity
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  T* Ks = reinterpret_cast<T*>(smem_raw);          // [2][kStep][D]
-  T* Vs = Ks + 2 * kStep * D;                      // [2][kStep][D]
-  float* pbuf = reinterpret_cast<float*>(Vs + 2 * kStep * D);  // [kWarps][16][G]
-  float* mbuf = pbuf + kWarps * 16 * G;            // [kWarps][G]
-  float* lbuf = mbuf + kWarps * G;                 // [kWarps][G]
-  float* obuf = lbuf + kWarps * G;                 // [kWarps][G][D]
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n_items = *p.n_items;
-  const float qk_scale = rsqrtf((float)D) * kLog2e;
-
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int bg = p.items[2 * item], chunk = p.items[2 * item + 1];
-    const int b = bg / p.Hkv, g = bg % p.Hkv;
-    const int L = clamp_len(p.seqlens, b, p.Lmax, nullptr);
-    const int pos = L - 1;
-    const int t = pos / p.block;
-    const int N = t;
-    const int cnt = p.cnt[bg];
-    const int e_begin = chunk * p.chunk_blocks;
-    const int e_end = min(e_begin + p.chunk_blocks, cnt + 1);
-    const bool has_diag = e_end == cnt + 1;
-    const int spb = p.block / kStep;
-    const int n_diag = has_diag ? (pos - t * p.block) / kStep + 1 : 0;
-    const int n_sel = (has_diag ? e_end - 1 : e_end) - e_begin;
-    const int n_sub = n_sel * spb + n_diag;
-    const int32_t* idx = p.idx + (int64_t)bg * p.t_cap;
-    const float* logp = p.logp + (int64_t)bg * p.t_cap;
-    const float beta = N > 0 ? p.sigma * logf(1.0f / (float)N) : 0.0f;
-
-    const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
-    const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
-
-    auto sub_tok0 = [&](int s) -> int {
-      if (s < n_sel * spb) return idx[e_begin + s / spb] * p.block + (s % spb) * kStep;
-      return t * p.block + (s - n_sel * spb) * kStep;
-    };
-    auto load = [&](int s, int buf) {
-      const int tok0 = sub_tok0(s);
-      constexpr int NCH = D / 8;
-      T* kd = Ks + buf * kStep * D;
-      T* vd = Vs + buf * kStep * D;
-      for (int i = tid; i < kStep * NCH; i += kWarps * 32) {
-        const int r = i / NCH, c = i % NCH;
-        const int tok = tok0 + r;
-        const bool ok = tok < L;
-        cp_async16(kd + r * D + c * 8, kg + (int64_t)(ok ? tok : 0) * p.k.ss + c * 8, ok);
-        cp_async16(vd + r * D + c * 8, vg + (int64_t)(ok ? tok : 0) * p.v.ss + c * 8, ok);
-      }
-      cp_async_commit();
-    };
-
-    // query (pre-scaled into the log2 domain)
-    float qv[G][DL];
-    const T* q = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb;
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < DL; ++e)
-        qv[h][e] = Elt<T>::load1(q + (int64_t)(g * G + h) * p.q.sh + lane * DL + e) * qk_scale;
-
-    float m[G], o[G][DL], lown[NVL];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m[h] = kNegInf;
-#pragma unroll
-      for (int e = 0; e < DL; ++e) o[h][e] = 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < NVL; ++j) lown[j] = 0.f;
-
-    load(0, 0);
-    for (int s = 0; s < n_sub; ++s) {
-      if (s + 1 < n_sub) {
-        load(s + 1, (s + 1) & 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncthreads();
-      const int buf = s & 1;
-      const T* kb = Ks + buf * kStep * D + warp * 16 * D;
-      const T* vb = Vs + buf * kStep * D + warp * 16 * D;
-      const bool diag = s >= n_sel * spb;
-      const float bias = (diag ? beta : p.sigma * logp[e_begin + s / spb]) * kLog2e;
-      const int tok0 = sub_tok0(s) + warp * 16;
-
-      // logits of 16 tokens x G heads
-      float v[NV];
-#pragma unroll
-      for (int tt = 0; tt < 16; ++tt) {
-        float kf[DL];
-        if constexpr (DL == 4) {
-          const uint2 raw = *reinterpret_cast<const uint2*>(kb + tt * D + lane * 4);
-          if constexpr (sizeof(T) == 2) {
-            uint4 w = make_uint4(raw.x, raw.y, 0u, 0u);
-            float f8[8];
-            Elt<T>::to_float(w, f8);
-            kf[0] = f8[0], kf[1] = f8[1], kf[2] = f8[2], kf[3] = f8[3];
-          }
-        } else {
-          const uint32_t raw = *reinterpret_cast<const uint32_t*>(kb + tt * D + lane * 2);
-          uint4 w = make_uint4(raw, 0u, 0u, 0u);
-          float f8[8];
-          Elt<T>::to_float(w, f8);
-          kf[0] = f8[0], kf[1] = f8[1];
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < DL; ++e) a = fmaf(qv[h][e], kf[e], a);
-          v[tt * G + h] = a;
-        }
-      }
-      warp_transpose_reduce<NV>(v, lane);
-      // lane holds token lane/2; heads (lane&1)*GH + j (G >= 2) or head 0
-      const int tok = tok0 + (lane >> 1);
-      const bool valid = tok <= pos;
-      float sl[NVL], mx[NVL];
-#pragma unroll
-      for (int j = 0; j < NVL; ++j) {
-        sl[j] = valid ? v[j] + bias : kNegInf;
-        mx[j] = sl[j];
-#pragma unroll
-        for (int off = 2; off <= 16; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], off));
-      }
-      float mu[G], sc[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float th = __shfl_sync(0xffffffffu, mx[h % GH], G >= 2 ? h / GH : 0);
-        const float mn = fmaxf(m[h], th);
-        mu[h] = mn == kNegInf ? 0.f : mn;
-        sc[h] = exp2f(m[h] - mu[h]);
-        m[h] = mn;
-#pragma unroll
-        for (int e = 0; e < DL; ++e) o[h][e] *= sc[h];
-      }
-      float* pw = pbuf + warp * 16 * G;
-#pragma unroll
-      for (int j = 0; j < NVL; ++j) {
-        const int hd = G >= 2 ? (lane & 1) * GH + j : 0;
-        float muj = mu[j], scj = sc[j];
-        if constexpr (G >= 2) {
-          muj = (lane & 1) ? mu[GH + j] : mu[j];
-          scj = (lane & 1) ? sc[GH + j] : sc[j];
-        }
-        const float pj = exp2f(sl[j] - muj);
-        lown[j] = lown[j] * scj + pj;
-        pw[(lane >> 1) * G + hd] = pj;
-      }
-      __syncwarp();
-#pragma unroll 4
-      for (int tt = 0; tt < 16; ++tt) {
-        float vf[DL];
-        if constexpr (DL == 4) {
-          const uint2 raw = *reinterpret_cast<const uint2*>(vb + tt * D + lane * 4);
-          uint4 w = make_uint4(raw.x, raw.y, 0u, 0u);
-          float f8[8];
-          Elt<T>::to_float(w, f8);
-          vf[0] = f8[0], vf[1] = f8[1], vf[2] = f8[2], vf[3] = f8[3];
-        } else {
-          const uint32_t raw = *reinterpret_cast<const uint32_t*>(vb + tt * D + lane * 2);
-          uint4 w = make_uint4(raw, 0u, 0u, 0u);
-          float f8[8];
-          Elt<T>::to_float(w, f8);
-          vf[0] = f8[0], vf[1] = f8[1];
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float ph = pw[tt * G + h];
-#pragma unroll
-          for (int e = 0; e < DL; ++e) o[h][e] = fmaf(ph, vf[e], o[h][e]);
-        }
-      }
-      __syncwarp();
-      __syncthreads();
-    }
-
-    // l per head: sum over the 16 lanes of the owning parity
-#pragma unroll
-    for (int j = 0; j < NVL; ++j)
-#pragma unroll
-      for (int off = 2; off <= 16; off <<= 1) lown[j] += __shfl_xor_sync(0xffffffffu, lown[j], off);
-    if (lane < 2) {
-#pragma unroll
-      for (int j = 0; j < NVL; ++j) {
-        if (G >= 2) {
-          lbuf[warp * G + lane * GH + j] = lown[j];
-        } else if (lane == 0) {
-          lbuf[warp * G] = lown[0];
-        }
-      }
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) mbuf[warp * G + h] = m[h];
-    }
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < DL; ++e) obuf[(warp * G + h) * D + lane * DL + e] = o[h][e];
-    __syncthreads();
-    const int64_t slot = (int64_t)p.pair_base[bg] + chunk;
-    for (int i = tid; i < G * D; i += kWarps * 32) {
-      const int h = i / D, e = i % D;
-      float M = kNegInf;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mbuf[w * G + h]);
-      const float Mu = M == kNegInf ? 0.f : M;
-      float acc = 0.f, lsum = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float f = exp2f(mbuf[w * G + h] - Mu);
-        acc += f * obuf[(w * G + h) * D + e];
-        lsum += f * lbuf[w * G + h];
-      }
-      p.part_o[(slot * G + h) * D + e] = acc;
-      if (e == 0) {
-        p.part_ml[(slot * G + h) * 2] = M;
-        p.part_ml[(slot * G + h) * 2 + 1] = lsum;
-      }
-    }
-    __syncthreads();
-  }
-}
-
-// ------------------------------------------------------------------ split-KV attention, f16/bf16
-// The same work items and partials as attend_decode_kernel, with the two
-// per-warp products on the tensor cores through warp-level mma (m16n8k16,
-// fp32 accumulate): a KV head has only G <= 8 query rows, far below the
+// Split-KV attention over the work items (chunks of selected blocks of one
+// (sequence, KV head)), one partial per item.  The two per-warp products run
+// on the tensor cores through warp-level mma (m16n8k16, fp32 accumulate): a KV head has only G <= 8 query rows, far below the
 // 64-row minimum of the 5th-generation MMA, and the kernel is HBM-bound, so
 // the MMAs only serve to take the dot products off the issue slots.
 //   S^T (16 x 8 tokens) = Qpad (16 x D) K^T: rows are the G heads (zero
@@ -944,12 +709,9 @@ cudaError_t launch_route_t(const DecodeParams& p, cudaStream_t stream) {
 
 template <typename T, int D, int G>
 cudaError_t launch_attend_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
-  constexpr bool kMma = !std::is_same<T, float>::value;
-  const size_t smem = kMma ? (size_t)2 * kDStages * kStep * D * sizeof(T) +
-                                 (size_t)(2 * kWarps * G + kWarps * G * D) * sizeof(float)
-                           : (size_t)4 * kStep * D * sizeof(T) +
-                                 (size_t)(kWarps * 16 * G + 2 * kWarps * G + kWarps * G * D) * sizeof(float);
-  auto kern = kMma ? attend_decode_mma_kernel<T, D, G> : attend_decode_kernel<T, D, G>;
+  const size_t smem =
+      (size_t)2 * kDStages * kStep * D * sizeof(T) + (size_t)(2 * kWarps * G + kWarps * G * D) * sizeof(float);
+  auto kern = attend_decode_mma_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;

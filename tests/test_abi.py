@@ -152,6 +152,35 @@ def test_decode_and_route_reject_bad_arguments():
     assert st == 1 and "n_words" in lib.dash_attn_last_error().decode()
 
 
+def test_paged_and_context_parallel_reject_bad_arguments():
+    lib = dash.load()
+    q = tensor(4, 1, 8, 128)
+    o = tensor(4, 1, 8, 128)
+    pages = tensor(100, 64, 2, 128)
+    # page size must equal the block; a block table is required
+    st = lib.dash_attn_decode_paged(ctypes.byref(q), ctypes.byref(pages), ctypes.byref(pages), FAKE, 16, FAKE, FAKE, 64,
+                                    1.5, 128, ctypes.byref(o), FAKE, 1 << 30, None, None)
+    assert st == 1 and "page size" in lib.dash_attn_last_error().decode()
+    st = lib.dash_attn_decode_paged(ctypes.byref(q), ctypes.byref(pages), ctypes.byref(pages), None, 16, FAKE, FAKE, 64,
+                                    1.5, 64, ctypes.byref(o), FAKE, 1 << 30, None, None)
+    assert st == 1 and "block table" in lib.dash_attn_last_error().decode()
+    st = lib.dash_attn_decode_paged(ctypes.byref(q), ctypes.byref(pages), ctypes.byref(pages), FAKE, 16, FAKE, FAKE, 8,
+                                    1.5, 64, ctypes.byref(o), FAKE, 1 << 30, None, None)
+    assert st == 1 and "t_cap" in lib.dash_attn_last_error().decode()
+    st = lib.dash_attn_summarize_paged(ctypes.byref(pages), FAKE, 16, 4, FAKE, FAKE, None, 64, FAKE, 8, 0, None)
+    assert st == 1 and "t_cap" in lib.dash_attn_last_error().decode()
+    # context parallelism: shard ranges must be block-aligned, the block range must fit
+    shard = tensor(4, 100, 2, 128)
+    st = lib.dash_attn_cp_attend(ctypes.byref(q), ctypes.byref(shard), ctypes.byref(shard), 64, FAKE, 4096, FAKE, FAKE,
+                                 FAKE, 64, 64, None, FAKE, None)
+    assert st == 1 and "multiples of the block" in lib.dash_attn_last_error().decode()
+    st = lib.dash_attn_cp_scores(ctypes.byref(q), 2, FAKE, 8, 10, 30, FAKE, 4096, 1.5, 64, FAKE, 64, None)
+    assert st == 1 and "block range" in lib.dash_attn_last_error().decode()
+    qf = tensor(4, 1, 8, 128, dtype=0)
+    st = lib.dash_attn_cp_lists(ctypes.byref(qf), 2, FAKE, FAKE, 4096, 1.5, 64, FAKE, FAKE, FAKE, 64, None)
+    assert st == 2
+
+
 def test_binding_refuses_host_tensors():
     import torch
 
