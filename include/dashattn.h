@@ -280,8 +280,11 @@ dash_status_t dash_attn_decode_ex(const dash_tensor_t* q, const dash_tensor_t* k
  *              head on the (alpha - 1) * z scale (0 when N = 0).
  *   p_dense    optional device fp32 [B, H, Sq, t_cap]: per-head entmax
  *              weight of every block (0 for non-candidates).
- *   workspace  decode mode only: dash_attn_route_workspace_size() bytes,
- *              256-byte aligned (the per-head logits); NULL in prefill mode.
+ *   workspace  decode mode: dash_attn_route_workspace_size(..., 1) bytes,
+ *              256-byte aligned (the per-head logits).  Prefill mode: NULL,
+ *              or dash_attn_route_workspace_size(..., 0) bytes, 256-byte
+ *              aligned, where the f16/bf16 path keeps the summaries split
+ *              for the tensor cores (same results, faster).
  */
 size_t dash_attn_route_workspace_size(const dash_tensor_t* q, int64_t kv_heads, int64_t t_cap, int decode);
 

@@ -255,6 +255,8 @@ def route(q: torch.Tensor, summaries: torch.Tensor, alpha: float, block: int, ca
     ws = None
     if seqlens is not None:
         ws = _workspace(route_workspace_size(q, Hkv, t_cap, True), dev, workspace)
+    elif q.dtype != torch.float32:
+        ws = _workspace(route_workspace_size(q, Hkv, t_cap, False), dev, workspace)  # split summaries
     qd = _desc(q)
     _check(_lib.dash_attn_route(ctypes.byref(qd), summaries.data_ptr(), Hkv, t_cap, _ptr(seqlens), alpha, block,
                                 1 if causal else 0, idx.data_ptr(), logp.data_ptr(), cnt.data_ptr(), _ptr(tau),

@@ -85,7 +85,7 @@ int num_sms() {
 
 // Workspace of dash_attn_fwd.
 struct FwdLayout {
-  size_t status, summ, idx, logp, cnt, ulist, umask, ucnt, usteps, plist, pmask, pcnt, psteps, total;
+  size_t status, summ, split, idx, logp, cnt, ulist, umask, ucnt, usteps, plist, pmask, pcnt, psteps, total;
   int64_t T, n_tiles, n_pairs;
   int tile_pos;
 };
@@ -101,6 +101,8 @@ FwdLayout fwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, in
   off = align256(off + sizeof(dash::DeviceStatus));
   L.summ = off;
   off = align256(off + (size_t)B * Hkv * L.T * D * 4);
+  L.split = off;  // summaries split for the tensor-core routing kernel
+  off = align256(off + dash::route_split_bytes(B, Hkv, L.T, (int)D));
   L.idx = off;
   off = align256(off + (size_t)B * Hkv * S * L.T * 4);
   L.logp = off;
@@ -304,7 +306,8 @@ struct TileLists {
 // cores (whose work lists still have to be built).
 dash_status_t run_route(const dash_tensor_t* q, const float* summaries, int64_t kv_heads, int64_t t_cap, float alpha,
                         int block, int causal, int32_t* idx, float* logp, int32_t* cnt, float* tau, float* p_dense,
-                        const TileLists* tl, dash::DeviceStatus* status, cudaStream_t stream, int* first_cuda_tile) {
+                        const TileLists* tl, dash::DeviceStatus* status, cudaStream_t stream, int* first_cuda_tile,
+                        float* split_buf = nullptr) {
   const int G = (int)(q->h / kv_heads);
   dash::RouteParams p{};
   p.q = view(q);
@@ -340,7 +343,13 @@ dash_status_t run_route(const dash_tensor_t* q, const float* summaries, int64_t 
     }
     dash::TileOut to{};
     if (tl) to = dash::TileOut{tl->ulist, tl->umask, tl->ucnt, tl->usteps, n_tiles};
+    if (split_buf && split > 0) {
+      cudaError_t e = dash::launch_route_split(p, split_buf, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "route (split summaries)");
+      p.summ_split = split_buf;
+    }
     cudaError_t e = dash::launch_route_prefill_tc(p, to, 0, split, stream);
+    p.summ_split = nullptr;
     if (e != cudaSuccess) return cuda_fail(e, "route (tensor cores)");
   }
   p.pos_begin = split * P;
@@ -358,7 +367,7 @@ extern "C" {
 
 size_t dash_attn_route_workspace_size(const dash_tensor_t* q, int64_t kv_heads, int64_t t_cap, int decode) {
   if (check_tensor(q, "q") || check_group(q->h, kv_heads) || t_cap <= 0) return 0;
-  if (!decode) return 0;
+  if (!decode) return dash::route_split_bytes(q->b, kv_heads, t_cap, (int)q->d);  // optional in prefill mode
   return decode_layout(q->b, q->h, kv_heads, q->d, 64, t_cap).idx;  // status + per-head logits
 }
 
@@ -375,8 +384,13 @@ dash_status_t dash_attn_route(const dash_tensor_t* q, const float* summaries, in
     const int64_t T = (q->s + block - 1) / block;
     if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block)", (long long)t_cap);
     if (T > 4096) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per sequence");
+    // a workspace, when given, holds the split summaries of the tensor-core kernel
+    float* split = nullptr;
+    if (workspace && reinterpret_cast<uintptr_t>(workspace) % 256 == 0 &&
+        workspace_bytes >= dash::route_split_bytes(q->b, kv_heads, t_cap, (int)q->d))
+      split = static_cast<float*>(workspace);
     st = run_route(q, summaries, kv_heads, t_cap, alpha, block, causal, idx, logp, cnt, tau, p_dense, nullptr,
-                   nullptr, (cudaStream_t)stream, nullptr);
+                   nullptr, (cudaStream_t)stream, nullptr, split);
     return st ? st : ok();
   }
   if (q->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode-mode route needs q with s == 1");
@@ -592,7 +606,7 @@ dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, c
   dash::DeviceStatus* dst = at<dash::DeviceStatus>(workspace, L.status);
   int first_cuda_tile = 0;
   if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, nullptr, nullptr, &tl, dst, s,
-                      &first_cuda_tile)))
+                      &first_cuda_tile, at<float>(workspace, L.split))))
     return st;
   st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, sigma, out, tl, L.tile_pos, L.n_tiles, first_cuda_tile,
                   dst, s);

@@ -51,8 +51,15 @@ struct RouteParams {
   float* p_dense;  // nullable [B, H, S, t_cap]
   int pos_begin;   // CUDA-core kernel: first position to route (a tile boundary)
   DeviceStatus* status;  // nullable
+  // tensor-core kernel: the summaries already split into tf32 head and
+  // remainder in the kernel's shared-memory operand layout (route_split_bytes),
+  // streamed by bulk copies; null: the kernel splits them itself
+  const float* summ_split;
 };
 cudaError_t launch_route_prefill(const RouteParams& p, cudaStream_t stream);
+// bytes of the split summaries of [B, Hkv, t_cap, D]; launch_route_split writes them
+size_t route_split_bytes(int64_t B, int64_t Hkv, int64_t t_cap, int D);
+cudaError_t launch_route_split(const RouteParams& p, float* split, cudaStream_t stream);
 
 // Stage-2 work lists written by the tensor-core routing kernel (null ulist:
 // not wanted).

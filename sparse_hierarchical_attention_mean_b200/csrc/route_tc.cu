@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars->a_full, kWork);
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->b_full[s], kWork);
+      tc::mbar_init(&bars->b_full[s], p.summ_split ? 1 : kWork);
       tc::mbar_init(&bars->b_empty[s], 1);
     }
     tc::mbar_init(&bars->x_ready, 1);
@@ -339,47 +339,65 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
     }
     tc::fence_proxy_async_smem();
     tc::mbar_arrive(&bars->a_full);
-    // B: summaries of each candidate chunk, split into tf32 head + remainder.
-    // The loads of chunk j + 1 are issued before chunk j is stored, so their
-    // latency overlaps the wait for a free stage and the stores.
-    const float* sbase = p.summaries + bg * p.t_cap * D;
-    constexpr int EPT = kChunk * (D / 4) / kWork;  // float4 per thread and chunk
-    static_assert(EPT * kWork == kChunk * (D / 4), "chunk not divisible among the loading threads");
-    auto load_chunk = [&](int j, float4* v) {
-#pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        const int i = threadIdx.x + e * kWork;
-        const int cand = i / (D / 4), k4 = i % (D / 4);
-        const int c = j * kChunk + cand;
-        v[e] = c < n_cols ? __ldg(reinterpret_cast<const float4*>(sbase + (int64_t)c * D) + k4)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p.summ_split) {
+      // B: the pre-split chunks, two bulk copies per stage by one thread
+      if (warp == kWorkWarps - 1 && lane == 0) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.summ_split) +
+                             bg * (int64_t)((p.t_cap + kChunk - 1) / kChunk) * 2 * L::kBTerm;
+        for (int j = 0; j < n_chunks; ++j) {
+          const int st = j & 1;
+          if (j >= 2 && !tc::mbar_wait(&bars->b_empty[st], ((j >> 1) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&bars->b_full[st], 2 * L::kBTerm);
+          tc::bulk_load(smem + L::kOffB + (st * 2) * L::kBTerm, src + (int64_t)j * 2 * L::kBTerm, 2 * L::kBTerm,
+                        &bars->b_full[st]);
+        }
       }
-    };
-    float4 cur[EPT], nxt[EPT];
-    load_chunk(0, cur);
-    for (int j = 0; j < n_chunks; ++j) {
-      const int st = j & 1;
-      if (j + 1 < n_chunks) load_chunk(j + 1, nxt);
-      if (j >= 2 && !tc::mbar_wait(&bars->b_empty[st], ((j >> 1) - 1) & 1)) {
-        ok = false;
-        break;
+    } else {
+      // B: summaries of each candidate chunk, split into tf32 head + remainder.
+      // The loads of chunk j + 1 are issued before chunk j is stored, so their
+      // latency overlaps the wait for a free stage and the stores.
+      const float* sbase = p.summaries + bg * p.t_cap * D;
+      constexpr int EPT = kChunk * (D / 4) / kWork;  // float4 per thread and chunk
+      static_assert(EPT * kWork == kChunk * (D / 4), "chunk not divisible among the loading threads");
+      auto load_chunk = [&](int j, float4* v) {
+  #pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          const int i = threadIdx.x + e * kWork;
+          const int cand = i / (D / 4), k4 = i % (D / 4);
+          const int c = j * kChunk + cand;
+          v[e] = c < n_cols ? __ldg(reinterpret_cast<const float4*>(sbase + (int64_t)c * D) + k4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      };
+      float4 cur[EPT], nxt[EPT];
+      load_chunk(0, cur);
+      for (int j = 0; j < n_chunks; ++j) {
+        const int st = j & 1;
+        if (j + 1 < n_chunks) load_chunk(j + 1, nxt);
+        if (j >= 2 && !tc::mbar_wait(&bars->b_empty[st], ((j >> 1) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        uint8_t* bh = smem + L::kOffB + (st * 2 + 0) * L::kBTerm;
+        uint8_t* bl = smem + L::kOffB + (st * 2 + 1) * L::kBTerm;
+  #pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          const int i = threadIdx.x + e * kWork;
+          const int cand = i / (D / 4), k4 = i % (D / 4);
+          const float4 v = cur[e];
+          const float4 h = tf32_head(v);
+          const float4 lo = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+          const int kc = k4 / 8, u = k4 % 8;
+          *reinterpret_cast<float4*>(bh + kc * L::kBChunk + sw128(cand, u)) = h;
+          *reinterpret_cast<float4*>(bl + kc * L::kBChunk + sw128(cand, u)) = lo;
+          cur[e] = nxt[e];
+        }
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&bars->b_full[st]);
       }
-      uint8_t* bh = smem + L::kOffB + (st * 2 + 0) * L::kBTerm;
-      uint8_t* bl = smem + L::kOffB + (st * 2 + 1) * L::kBTerm;
-#pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        const int i = threadIdx.x + e * kWork;
-        const int cand = i / (D / 4), k4 = i % (D / 4);
-        const float4 v = cur[e];
-        const float4 h = tf32_head(v);
-        const float4 lo = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
-        const int kc = k4 / 8, u = k4 % 8;
-        *reinterpret_cast<float4*>(bh + kc * L::kBChunk + sw128(cand, u)) = h;
-        *reinterpret_cast<float4*>(bl + kc * L::kBChunk + sw128(cand, u)) = lo;
-        cur[e] = nxt[e];
-      }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bars->b_full[st]);
     }
     if (ok && !tc::mbar_wait(&bars->x_ready, 0)) ok = false;
     tc::fence_after_sync();
@@ -606,9 +624,47 @@ cudaError_t launch_t(const RouteParams& p, const TileOut& to, int tile0, int n_t
   }
 }
 
+// The summaries of one (batch, KV head) chunk of 64 candidates, split into
+// the tf32 head and its remainder and laid out exactly as the routing
+// kernel's B stage (128-byte swizzled K-major chunks, head then remainder),
+// zero past t_cap.
+template <int D>
+__global__ void __launch_bounds__(256) route_split_kernel(const float* summaries, int64_t t_cap, float* split) {
+  using L = RLayout<D>;
+  const int j = blockIdx.x;
+  const int64_t bg = (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
+  const int64_t n_ch = (t_cap + kChunk - 1) / kChunk;
+  uint8_t* dst = reinterpret_cast<uint8_t*>(split) + (bg * n_ch + j) * 2 * L::kBTerm;
+  const float* sbase = summaries + bg * t_cap * D;
+  for (int i = threadIdx.x; i < kChunk * (D / 4); i += blockDim.x) {
+    const int cand = i / (D / 4), k4 = i % (D / 4);
+    const int64_t c = (int64_t)j * kChunk + cand;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c < t_cap) v = __ldg(reinterpret_cast<const float4*>(sbase + c * D) + k4);
+    const float4 h = tf32_head(v);
+    const int kc = k4 / 8, u = k4 % 8;
+    *reinterpret_cast<float4*>(dst + kc * L::kBChunk + sw128(cand, u)) = h;
+    *reinterpret_cast<float4*>(dst + L::kBTerm + kc * L::kBChunk + sw128(cand, u)) =
+        make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+  }
+}
+
 }  // namespace
 
 int route_tc_max_cols() { return kMaxCols; }
+
+size_t route_split_bytes(int64_t B, int64_t Hkv, int64_t t_cap, int D) {
+  return (size_t)(B * Hkv) * (size_t)((t_cap + kChunk - 1) / kChunk) * 2 * (size_t)(D / 32) * kChunk * 128;
+}
+
+cudaError_t launch_route_split(const RouteParams& p, float* split, cudaStream_t stream) {
+  dim3 grid((unsigned)((p.t_cap + kChunk - 1) / kChunk), p.Hkv, p.B);
+  if (p.D == 128)
+    route_split_kernel<128><<<grid, 256, 0, stream>>>(p.summaries, p.t_cap, split);
+  else
+    route_split_kernel<64><<<grid, 256, 0, stream>>>(p.summaries, p.t_cap, split);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_route_prefill_tc(const RouteParams& p, const TileOut& to, int tile0, int n_tiles,
                                     cudaStream_t stream) {

@@ -74,6 +74,16 @@ __device__ __forceinline__ void tma_load_4d(void* smem, const CUtensorMap* map, 
       : "memory");
 }
 
+// Contiguous bulk copy global -> shared (16-byte aligned, size a multiple of
+// 16), completion counted on `bar` in bytes.  No cluster multicast.
+__device__ __forceinline__ void bulk_load(void* smem, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(smem)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
