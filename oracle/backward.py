@@ -1,0 +1,165 @@
+"""Plain fp64 CPU oracle of the DashAttention backward pass.
+
+TEST INFRASTRUCTURE ONLY, like ``oracle.dash_oracle`` (whose forward it
+differentiates): only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import it.
+
+Source.  The page "DashAttention: Differentiable and Adaptive Sparse
+Hierarchical Attention" (gist.science explainer of arXiv 2605.18753),
+sections "Stage 1: entmax chunk routing" (the router is differentiable, so
+the loss reaches the summaries and the queries through the routing
+probabilities) and "Stage 2: prior-induced sparse softmax" (the prior enters
+the logits as log p_bar, so its gradient is the softmax gradient summed over
+the tokens of the block).  The alpha-entmax Jacobian follows Peters, Niculae
+& Martins (2019), "Sparse Sequence-to-Sequence Models", section 3: with
+u_c = p_c^(2 - alpha) on the support (0 elsewhere),
+dp/dz = diag(u) - u u^T / sum(u).
+
+The loss is L = sum(dout * out) for the forward of ``oracle.dash_oracle``
+(mean-pooled summaries, prior strength sigma); every gradient below is the
+exact derivative of that forward, taken step by step in reverse order:
+
+  stage 2   l_j = q . k_j / sqrt(d) + bias_j,  o = softmax(l) V
+            dP_j = dout . v_j,  D = dout . o,  dS_j = P_j (dP_j - D)
+            dq += dS K / sqrt(d),  dk_j += dS_j q / sqrt(d),  dv_j += P_j dout
+            d log p_bar_c = sigma * sum_{j in c} dS_j   (summed over the heads)
+  GQA mean  dp_{h,c} = d log p_bar_c / (G p_bar_c)
+  entmax    dz_h = u_h * (dp_h - <u_h, dp_h> / sum(u_h))
+  scores    z_{h,c} = gamma q_h . s_c:  dq_h += gamma dz_h S,  ds_c += gamma dz_{h,c} q_h
+  stage 0   s_c = kbar_c W_s:  dkbar_c = ds_c W_s^T,  dW_s += kbar_c^T ds_c,
+            dk_j += dkbar_c / |c|  for j in c
+
+The diagonal block's bias sigma * log(1/N) is a constant and carries no
+gradient.  Blocks outside the support carry none either: their probability is
+exactly 0 on a neighbourhood of the input (the support is locally constant
+away from ties at the threshold).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from .dash_oracle import block_summaries, forward, forward_row
+
+
+def entmax_vjp(p: np.ndarray, g: np.ndarray, alpha: float) -> np.ndarray:
+    """dL/dz of p = alpha-entmax(z) given g = dL/dp (Peters et al. 2019, section 3).
+
+    On the support u_c = p_c^(2 - alpha) (u_c = 1 for alpha = 2, sparsemax);
+    off the support u_c = 0.  The Jacobian diag(u) - u u^T / sum(u) is
+    symmetric, so the vector-Jacobian product is u * (g - <u, g> / sum(u)).
+    """
+    p = np.asarray(p, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    u = np.where(p > 0.0, np.power(np.where(p > 0.0, p, 1.0), 2.0 - alpha), 0.0)
+    su = u.sum()
+    if su == 0.0:
+        return np.zeros_like(p)
+    return u * (g - (u * g).sum() / su)
+
+
+def _attended(r: dict, pos: int, n_tokens: int, block: int, causal: bool, sigma: float):
+    """Token ids, biases and owning list entry (-1: diagonal) of one row, as in forward_row."""
+    tok, bias, owner = [], [], []
+    for e, (c, lp) in enumerate(zip(r["blocks"], r["logp"])):
+        span = np.arange(c * block, min(n_tokens, (c + 1) * block))
+        tok.append(span)
+        bias.append(np.full(len(span), sigma * lp))
+        owner.append(np.full(len(span), e))
+    t = pos // block
+    last = pos if causal else min(n_tokens, (t + 1) * block) - 1
+    span = np.arange(t * block, last + 1)
+    tok.append(span)
+    bias.append(np.full(len(span), sigma * r["beta"]))
+    owner.append(np.full(len(span), -1))
+    return np.concatenate(tok), np.concatenate(bias), np.concatenate(owner)
+
+
+def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout: np.ndarray, alpha: float,
+             block: int, causal: bool = True, sigma: float = 1.0) -> dict:
+    """Gradients of L = sum(dout * out) for one batch element of the prefill forward.
+
+    q, dout: [S, H, d]; k, v: [S, Hkv, d]; w_s: [d, d].  Inputs are promoted
+    to fp64.  Returns dq, dk, dv (shapes of q, k, v) and dw_s [d, d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    w_s = np.asarray(w_s, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    S, H, d = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    scale = 1.0 / math.sqrt(d)
+    gamma = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dw_s = np.zeros_like(w_s)
+    n_blocks = -(-S // block)
+    for g in range(Hkv):
+        kg, vg = k[:, g], v[:, g]
+        summ = block_summaries(kg, w_s, block, S)
+        ds = np.zeros((n_blocks, d))
+        for pos in range(S):
+            qg = q[pos, g * G:(g + 1) * G]
+            r = forward_row(qg, kg, vg, summ, pos, S, block, alpha, causal, sigma)
+            tok, bias, owner = _attended(r, pos, S, block, causal, sigma)
+            dlogp = np.zeros(len(r["blocks"]))
+            for h in range(G):
+                hh = g * G + h
+                logits = kg[tok] @ qg[h] * scale + bias
+                w = np.exp(logits - logits.max())
+                P = w / w.sum()
+                o = P @ vg[tok]
+                dP = vg[tok] @ dout[pos, hh]
+                dS = P * (dP - dout[pos, hh] @ o)
+                dq[pos, hh] += scale * (dS @ kg[tok])
+                dk[tok, g] += scale * np.outer(dS, qg[h])
+                dv[tok, g] += np.outer(P, dout[pos, hh])
+                for e in range(len(dlogp)):
+                    dlogp[e] += sigma * dS[owner == e].sum()
+            if len(r["blocks"]) == 0:
+                continue
+            # through the GQA mean: p_bar = mean_h p_h, and log
+            cand = np.asarray(r["cand"], dtype=np.int64)
+            gp = np.zeros(len(cand))
+            gp[r["idx"]] = dlogp / (G * r["pbar"][r["idx"]])
+            for h in range(G):
+                dz = entmax_vjp(r["p"][h], gp, alpha)
+                dq[pos, g * G + h] += gamma * (dz @ summ[cand])
+                ds[cand] += gamma * np.outer(dz, qg[h])
+        # stage 0: s_c = kbar_c W_s over the c's valid tokens
+        for c in range(n_blocks):
+            lo, hi = c * block, min(S, (c + 1) * block)
+            kbar = kg[lo:hi].sum(axis=0) / (hi - lo)
+            dw_s += np.outer(kbar, ds[c])
+            dk[lo:hi, g] += (w_s @ ds[c]) / (hi - lo)
+    return {"dq": dq, "dk": dk, "dv": dv, "dw_s": dw_s}
+
+
+def loss(q, k, v, w_s, dout, alpha, block, causal=True, sigma=1.0) -> float:
+    """L = sum(dout * out) of the forward oracle (the function the gradients differentiate)."""
+    out = _forward_sigma(q, k, v, w_s, alpha, block, causal, sigma)
+    return float((np.asarray(dout, dtype=np.float64) * out).sum())
+
+
+def _forward_sigma(q, k, v, w_s, alpha, block, causal, sigma) -> np.ndarray:
+    """Whole-sequence forward with prior strength sigma, [S, H, d]."""
+    if sigma == 1.0:
+        return forward(q, k, v, w_s, alpha, block, causal)["out"]
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    S, H, d = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    out = np.zeros((S, H, d))
+    for g in range(Hkv):
+        summ = block_summaries(k[:, g], w_s, block, S)
+        for pos in range(S):
+            r = forward_row(q[pos, g * G:(g + 1) * G], k[:, g], v[:, g], summ, pos, S, block, alpha, causal, sigma)
+            out[pos, g * G:(g + 1) * G] = r["out"]
+    return out
