@@ -238,7 +238,7 @@ def union_flops(cfg, idx: torch.Tensor, cnt: torch.Tensor, tile_pos: int) -> flo
     return 4.0 * cfg.head_dim * rows * per_bg
 
 
-def run_prefill(dash, cfg, steps, warmup, world, rank, pk):
+def run_prefill(dash, cfg, steps, warmup, world, rank, pk, do_backward=True):
     inp = full_inputs(cfg, device="cuda", seed=rank_seed(cfg, rank))
     q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
     B, S, H, d = q.shape
@@ -326,13 +326,48 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk):
     # step i-1's download overlap step i's kernels.
     e2e_ms, h2d, d2h = run_e2e(dash, cfg, q, k, v, w, ws, steps, warmup, world)
     del ws
+    bwd = run_backward(dash, cfg, q, k, v, w, out, min(steps, 5), warmup, flops) if do_backward else None
 
     return {
         "ms": ms, "tokens": B * S, "status": status, "seg_ms": seg.tolist(), "sparse_ms": sparse_ms, "flops": flops,
         "union_flops": uflops,
         "sparsity": sparsity, "achieved_tflops": achieved, "traffic": traffic, "clocks": clk.summary(),
-        "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+        "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "backward": bwd,
     }
+
+
+def run_backward(dash, cfg, q, k, v, w, out, steps, warmup, fwd_flops):
+    """The backward pass (dash_attn_bwd) on the same inputs, timed with CUDA events.
+
+    Algorithmic work: 2.5x the forward's selected FLOPs (the scores S = QK^T
+    recomputed, dP = dout V^T, and the three gradient products dV = P^T dout,
+    dK = dS^T Q, dQ = dS K, against the forward's two products).
+    """
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    dout = torch.randn(q.shape, generator=gen, device="cuda", dtype=torch.float32).to(q.dtype)
+    ws = torch.empty(dash.bwd_workspace_size(q, k, cfg.block), dtype=torch.uint8, device="cuda")
+    grads = {"dq": torch.empty(q.shape, dtype=torch.float32, device="cuda"),
+             "dk": torch.empty(k.shape, dtype=torch.float32, device="cuda"),
+             "dv": torch.empty(v.shape, dtype=torch.float32, device="cuda"),
+             "dw_s": torch.empty((q.shape[-1], q.shape[-1]), dtype=torch.float32, device="cuda")}
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dash.bwd(q, k, v, w, out, dout, cfg.alpha, cfg.block, True, grads=grads, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    status = dash.device_status(ws)
+    del ws
+    return {"ms": ms, "flops": 2.5 * fwd_flops, "steps": steps, "status": status}
 
 
 def run_e2e(dash, cfg, q, k, v, w, ws, steps, warmup, world):
@@ -510,6 +545,7 @@ def main():
     ap.add_argument("--skip-prefill", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=64, help="sequences in the decode workload (64 = full)")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--seq", type=int, default=None,
                     help="prefill sequence length override (smaller cases for profiling; default 32768)")
@@ -552,7 +588,8 @@ def main():
     dash.load()
     world, rank, _ = dist_setup(args.gpus)
     pk = peaks()
-    pre = None if args.skip_prefill else run_prefill(dash, cfg, args.steps, warmup, world, rank, pk)
+    pre = None if args.skip_prefill else run_prefill(dash, cfg, args.steps, warmup, world, rank, pk,
+                                                         not args.skip_backward)
     dec = None
     dcfg = get_config("decode").with_(batch=args.decode_batch)
     if not args.skip_decode:
@@ -618,6 +655,18 @@ def main():
     }
     if dec is not None:
         line["decode"] = decode_object(dec, dcfg, pk)
+    if pre["backward"] is not None:
+        bw = pre["backward"]
+        ach = bw["flops"] / (bw["ms"] * 1e-3) / 1e12
+        line["backward"] = {
+            "workload": "gradients of the prefill workload above (dq, dk, dv fp32 and dW_s), dout ~ N(0, 1)",
+            "ms": bw["ms"], "steps": bw["steps"], "device_status": bw["status"],
+            "roofline": {"kernels": "the whole backward call: pooling, routing, bwd_row, bwd_route, bwd_key, "
+                                    "bwd_ws (warp-level MMAs)",
+                         "bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
+                         "traffic": None, "algorithmic_flops": bw["flops"],
+                         "peak_source": f"{pk['source']} bf16 (burst)"},
+        }
     print(json.dumps(line), flush=True)
     barrier(world)
     finish(world)

@@ -1,6 +1,6 @@
 /*
- * dashattn.h -- C ABI of libdashattn, the B200 (sm_100a) forward of
- * DashAttention sparse hierarchical attention.
+ * dashattn.h -- C ABI of libdashattn, the B200 (sm_100a) forward and
+ * backward of DashAttention sparse hierarchical attention.
  *
  * Source of the method: "DashAttention: Differentiable and Adaptive Sparse
  * Hierarchical Attention" (gist.science explainer of arXiv 2605.18753),
@@ -162,6 +162,43 @@ dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, c
                                const float* w_s, float alpha, int block, int causal, dash_tensor_t* out,
                                void* workspace, size_t workspace_bytes, const dash_options_t* opts,
                                dash_stream_t stream);
+
+/*
+ * Backward pass of the prefill forward (dash_attn_fwd_ex with the same
+ * arguments): the gradients of sum(dout * out) with respect to q, k, v and
+ * W_s.  "Stage 1: entmax chunk routing" of the cited technical summary makes
+ * the router differentiable, so the loss reaches W_s and q through the
+ * prior log p_bar: per query row and KV group,
+ *   stage 2   dS_j = P_j (dout . v_j - dout . out); dq, dk, dv as in softmax
+ *             attention; d log p_bar_c = sigma * sum_{j in c, heads} dS_j
+ *   routing   dp_h = d log p_bar / (G p_bar);  dz_h = u (dp_h - <u, dp_h> / sum u)
+ *             with u = p_h^(2 - alpha) on the support (the alpha-entmax
+ *             Jacobian, Peters, Niculae & Martins 2019, section 3)
+ *   scores    dq_h += dz_h S / sqrt(d);  ds_c += dz_{h,c} q_h / sqrt(d)
+ *   stage 0   dW_s = sum_c kbar_c^T ds_c;  dk_j += ds_c W_s^T / |c| for j in c.
+ * The diagonal block's prior is a constant.  Stage 0 is mean pooling
+ * (opts->qbar must be NULL); opts->sigma is the forward's prior strength.
+ *   q, k, v, w_s, alpha, block, causal  as for dash_attn_fwd; dtype f16 or bf16
+ *             (DASH_F32 inputs return DASH_ERR_UNSUPPORTED).
+ *   out       the forward's output [B, S, H, d], dtype of q.
+ *   dout      dL/dout [B, S, H, d], dtype of q.
+ *   dq        fp32 [B, S, H, d]; dk, dv fp32 [B, S, Hkv, d]; every element
+ *             is overwritten.
+ *   dw_s      device fp32 [d, d], overwritten.
+ *   workspace at least dash_attn_bwd_workspace_size() bytes, 256-byte
+ *             aligned: summaries, routing lists and thresholds (recomputed
+ *             here), row statistics, per-head routing gradients
+ *             [B, Hkv, S, T, G] fp32, block means and summary gradients.
+ * Arithmetic: the three attention products of each tile run as bf16/f16
+ * tensor-core MMAs with fp32 accumulation (P and dS are rounded to the input
+ * type as MMA operands); the routing gradient is fp32.
+ */
+size_t dash_attn_bwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t* k, int block);
+dash_status_t dash_attn_bwd(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                            const float* w_s, const dash_tensor_t* out, const dash_tensor_t* dout, float alpha,
+                            int block, int causal, const dash_options_t* opts, dash_tensor_t* dq, dash_tensor_t* dk,
+                            dash_tensor_t* dv, float* dw_s, void* workspace, size_t workspace_bytes,
+                            dash_stream_t stream);
 
 /*
  * Paged KV cache (the layout of serving engines): the cache is a pool of

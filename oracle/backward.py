@@ -77,6 +77,52 @@ def _attended(r: dict, pos: int, n_tokens: int, block: int, causal: bool, sigma:
     return np.concatenate(tok), np.concatenate(bias), np.concatenate(owner)
 
 
+def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: np.ndarray, dout_group: np.ndarray,
+                 pos: int, n_tokens: int, block: int, alpha: float, causal: bool = True, sigma: float = 1.0) -> dict:
+    """The contribution of one query position of one KV group to the gradients.
+
+    q_group, dout_group: [G, d]; k, v: [L, d] of the KV head; summaries: all
+    block summaries of that head.  Returns dq [G, d] (complete: a row's query
+    gradient has no other source), the attended token ids ``tok`` with their
+    dk / dv contributions [len(tok), d], and the candidate ids ``cand`` with
+    their summary gradients ds [len(cand), d].
+    """
+    q_group = np.asarray(q_group, dtype=np.float64)
+    dout_group = np.asarray(dout_group, dtype=np.float64)
+    G, d = q_group.shape
+    scale = 1.0 / math.sqrt(d)
+    gamma = 1.0 / math.sqrt(d)
+    r = forward_row(q_group, k, v, summaries, pos, n_tokens, block, alpha, causal, sigma)
+    tok, bias, owner = _attended(r, pos, n_tokens, block, causal, sigma)
+    dq = np.zeros((G, d))
+    dk_tok = np.zeros((len(tok), d))
+    dv_tok = np.zeros((len(tok), d))
+    dlogp = np.zeros(len(r["blocks"]))
+    for h in range(G):
+        logits = k[tok] @ q_group[h] * scale + bias
+        w = np.exp(logits - logits.max())
+        P = w / w.sum()
+        o = P @ v[tok]
+        dP = v[tok] @ dout_group[h]
+        dS = P * (dP - dout_group[h] @ o)
+        dq[h] += scale * (dS @ k[tok])
+        dk_tok += scale * np.outer(dS, q_group[h])
+        dv_tok += np.outer(P, dout_group[h])
+        for e in range(len(dlogp)):
+            dlogp[e] += sigma * dS[owner == e].sum()
+    cand = np.asarray(r["cand"], dtype=np.int64)
+    ds = np.zeros((len(cand), d))
+    if len(r["blocks"]):
+        # through the GQA mean p_bar = mean_h p_h and the log
+        gp = np.zeros(len(cand))
+        gp[r["idx"]] = dlogp / (G * r["pbar"][r["idx"]])
+        for h in range(G):
+            dz = entmax_vjp(r["p"][h], gp, alpha)
+            dq[h] += gamma * (dz @ summaries[cand])
+            ds += gamma * np.outer(dz, q_group[h])
+    return {"dq": dq, "tok": tok, "dk_tok": dk_tok, "dv_tok": dv_tok, "cand": cand, "ds": ds}
+
+
 def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout: np.ndarray, alpha: float,
              block: int, causal: bool = True, sigma: float = 1.0) -> dict:
     """Gradients of L = sum(dout * out) for one batch element of the prefill forward.
@@ -92,8 +138,6 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
     S, H, d = q.shape
     Hkv = k.shape[1]
     G = H // Hkv
-    scale = 1.0 / math.sqrt(d)
-    gamma = 1.0 / math.sqrt(d)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
@@ -104,33 +148,12 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
         summ = block_summaries(kg, w_s, block, S)
         ds = np.zeros((n_blocks, d))
         for pos in range(S):
-            qg = q[pos, g * G:(g + 1) * G]
-            r = forward_row(qg, kg, vg, summ, pos, S, block, alpha, causal, sigma)
-            tok, bias, owner = _attended(r, pos, S, block, causal, sigma)
-            dlogp = np.zeros(len(r["blocks"]))
-            for h in range(G):
-                hh = g * G + h
-                logits = kg[tok] @ qg[h] * scale + bias
-                w = np.exp(logits - logits.max())
-                P = w / w.sum()
-                o = P @ vg[tok]
-                dP = vg[tok] @ dout[pos, hh]
-                dS = P * (dP - dout[pos, hh] @ o)
-                dq[pos, hh] += scale * (dS @ kg[tok])
-                dk[tok, g] += scale * np.outer(dS, qg[h])
-                dv[tok, g] += np.outer(P, dout[pos, hh])
-                for e in range(len(dlogp)):
-                    dlogp[e] += sigma * dS[owner == e].sum()
-            if len(r["blocks"]) == 0:
-                continue
-            # through the GQA mean: p_bar = mean_h p_h, and log
-            cand = np.asarray(r["cand"], dtype=np.int64)
-            gp = np.zeros(len(cand))
-            gp[r["idx"]] = dlogp / (G * r["pbar"][r["idx"]])
-            for h in range(G):
-                dz = entmax_vjp(r["p"][h], gp, alpha)
-                dq[pos, g * G + h] += gamma * (dz @ summ[cand])
-                ds[cand] += gamma * np.outer(dz, qg[h])
+            hs = slice(g * G, (g + 1) * G)
+            rb = backward_row(q[pos, hs], kg, vg, summ, dout[pos, hs], pos, S, block, alpha, causal, sigma)
+            dq[pos, hs] = rb["dq"]
+            dk[rb["tok"], g] += rb["dk_tok"]
+            dv[rb["tok"], g] += rb["dv_tok"]
+            ds[rb["cand"]] += rb["ds"]
         # stage 0: s_c = kbar_c W_s over the c's valid tokens
         for c in range(n_blocks):
             lo, hi = c * block, min(S, (c + 1) * block)

@@ -1,4 +1,4 @@
-"""Python binding of libdashattn (the DashAttention forward for B200).
+"""Python binding of libdashattn (the DashAttention forward and backward for B200).
 
 Argument marshalling only: every step of the computation runs in the CUDA
 kernels behind the C ABI declared in ``include/dashattn.h``.  PyTorch is used
@@ -56,6 +56,8 @@ EXPORTED = (
     "dash_attn_sparse",
     "dash_attn_get_device_status",
     "dash_attn_decode_noalloc",
+    "dash_attn_bwd_workspace_size",
+    "dash_attn_bwd",
 )
 
 
@@ -118,6 +120,8 @@ def _load() -> ctypes.CDLL:
         "dash_attn_decode_paged": (i32, [T, T, T, vp, i64, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
         "dash_attn_get_device_status": (i32, [vp, vp]),
         "dash_attn_decode_noalloc": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp]),
+        "dash_attn_bwd_workspace_size": (sz, [T, T, i32]),
+        "dash_attn_bwd": (i32, [T, T, T, vp, T, T, f32, i32, i32, O, T, T, T, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -326,6 +330,62 @@ def fwd(q, k, v, w_s, alpha: float, block: int, causal: bool = True, out=None, w
     else:
         _check(_lib.dash_attn_fwd_ex(*args, opts, _stream(stream)))
     return out
+
+
+# ------------------------------------------------------------------ backward
+
+
+def bwd_workspace_size(q: torch.Tensor, k: torch.Tensor, block: int) -> int:
+    qd, kd = _desc(q), _desc(k)
+    n = _lib.dash_attn_bwd_workspace_size(ctypes.byref(qd), ctypes.byref(kd), block)
+    if n == 0:
+        raise DashError(1, "arguments rejected by dash_attn_bwd_workspace_size")
+    return n
+
+
+def bwd(q, k, v, w_s, out, dout, alpha: float, block: int, causal: bool = True, sigma: float = 1.0,
+        grads=None, workspace=None, stream=None) -> dict:
+    """Gradients of sum(dout * out) (see dash_attn_bwd): dq, dk, dv fp32 and dw_s [d, d] fp32.
+
+    grads: optional dict of preallocated fp32 dq / dk / dv / dw_s.
+    """
+    d = q.shape[-1]
+    g = grads or {}
+    dq = g.get("dq", torch.empty(q.shape, dtype=torch.float32, device=q.device))
+    dk = g.get("dk", torch.empty(k.shape, dtype=torch.float32, device=q.device))
+    dv = g.get("dv", torch.empty(v.shape, dtype=torch.float32, device=q.device))
+    dw_s = g.get("dw_s", torch.empty((d, d), dtype=torch.float32, device=q.device))
+    ws = _workspace(bwd_workspace_size(q, k, block), q.device, workspace)
+    descs = [_desc(t) for t in (q, k, v, out, dout, dq, dk, dv)]
+    qd, kd, vd, od, dod, dqd, dkd, dvd = descs
+    opts = ctypes.byref(DashOptions(float(sigma), None))
+    _check(_lib.dash_attn_bwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), w_s.data_ptr(), ctypes.byref(od),
+                              ctypes.byref(dod), alpha, block, 1 if causal else 0, opts, ctypes.byref(dqd),
+                              ctypes.byref(dkd), ctypes.byref(dvd), dw_s.data_ptr(), ws.data_ptr(), ws.numel(),
+                              _stream(stream)))
+    return {"dq": dq, "dk": dk, "dv": dv, "dw_s": dw_s}
+
+
+class _DashAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, w_s, alpha, block, causal, sigma):
+        out = fwd(q, k, v, w_s, alpha, block, causal, sigma=sigma)
+        ctx.save_for_backward(q, k, v, w_s, out)
+        ctx.args = (alpha, block, causal, sigma)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, w_s, out = ctx.saved_tensors
+        alpha, block, causal, sigma = ctx.args
+        g = bwd(q, k, v, w_s, out, dout.contiguous(), alpha, block, causal, sigma)
+        return (g["dq"].to(q.dtype), g["dk"].to(k.dtype), g["dv"].to(v.dtype), g["dw_s"].to(w_s.dtype),
+                None, None, None, None)
+
+
+def attention(q, k, v, w_s, alpha: float, block: int, causal: bool = True, sigma: float = 1.0) -> torch.Tensor:
+    """Differentiable DashAttention prefill (f16/bf16): forward by dash_attn_fwd_ex, gradients by dash_attn_bwd."""
+    return _DashAttention.apply(q, k, v, w_s, alpha, block, causal, sigma)
 
 
 # ------------------------------------------------------------------ decode

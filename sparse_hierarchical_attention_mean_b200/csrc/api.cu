@@ -200,6 +200,39 @@ DecodeLayout decode_layout(int64_t B, int64_t H, int64_t Hkv, int64_t D, int blo
   return L;
 }
 
+// Workspace of dash_attn_bwd.
+struct BwdLayout {
+  size_t status, summ, split, idx, logp, cnt, tau, lse, dd, dz, umask, kbar, ds, total;
+  int64_t T, n_words;
+};
+
+BwdLayout bwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, int block) {
+  BwdLayout L{};
+  const int64_t G = H / Hkv;
+  L.T = (S + block - 1) / block;
+  L.n_words = (L.T + 31) / 32;
+  size_t off = 0;
+  auto take = [&](size_t& field, size_t bytes) {
+    field = off;
+    off = align256(off + bytes);
+  };
+  take(L.status, sizeof(dash::DeviceStatus));
+  take(L.summ, (size_t)B * Hkv * L.T * D * 4);
+  take(L.split, dash::route_split_bytes(B, Hkv, L.T, (int)D));
+  take(L.idx, (size_t)B * Hkv * S * L.T * 4);
+  take(L.logp, (size_t)B * Hkv * S * L.T * 4);
+  take(L.cnt, (size_t)B * Hkv * S * 4);
+  take(L.tau, (size_t)B * H * S * 4);
+  take(L.lse, (size_t)B * H * S * 4);
+  take(L.dd, (size_t)B * H * S * 4);
+  take(L.dz, (size_t)B * Hkv * S * L.T * G * 4);
+  take(L.umask, (size_t)B * Hkv * L.T * L.n_words * 4);
+  take(L.kbar, (size_t)B * Hkv * L.T * D * 4);
+  take(L.ds, (size_t)B * Hkv * L.T * D * 4);
+  L.total = off;
+  return L;
+}
+
 template <typename P>
 P* at(void* base, size_t off) {
   return reinterpret_cast<P*>(static_cast<char*>(base) + off);
@@ -611,6 +644,101 @@ dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, c
   st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, sigma, out, tl, L.tile_pos, L.n_tiles, first_cuda_tile,
                   dst, s);
   return st ? st : ok();
+}
+
+size_t dash_attn_bwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t* k, int block) {
+  if (check_tensor(q, "q") || check_tensor(k, "k") || (block != 64 && block != 128) || check_group(q->h, k->h))
+    return 0;
+  return bwd_layout(q->b, q->s, q->h, k->h, q->d, block).total;
+}
+
+static dash_status_t check_grad(const dash_tensor_t* g, const dash_tensor_t* like, const char* name) {
+  dash_status_t st;
+  if ((st = check_tensor(g, name))) return st;
+  if (g->dtype != DASH_F32) return fail(DASH_ERR_INVALID_ARGUMENT, "%s must be fp32", name);
+  if (g->b != like->b || g->s != like->s || g->h != like->h || g->d != like->d)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "%s must have the shape of its input", name);
+  return DASH_OK;
+}
+
+dash_status_t dash_attn_bwd(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                            const float* w_s, const dash_tensor_t* out, const dash_tensor_t* dout, float alpha,
+                            int block, int causal, const dash_options_t* opts, dash_tensor_t* dq, dash_tensor_t* dk,
+                            dash_tensor_t* dv, float* dw_s, void* workspace, size_t workspace_bytes,
+                            dash_stream_t stream) {
+  dash_status_t st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
+  if ((st = check_fwd_shapes(q, k, v, out)) || (st = check_common(alpha, block))) return st;
+  if ((st = check_tensor(dout, "dout"))) return st;
+  if (dout->dtype != q->dtype || dout->b != q->b || dout->s != q->s || dout->h != q->h || dout->d != q->d)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "dout must have q's shape and dtype");
+  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "the backward pass takes f16 or bf16 inputs");
+  if (k->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "prefill needs k and q of equal length");
+  if ((st = check_grad(dq, q, "dq")) || (st = check_grad(dk, k, "dk")) || (st = check_grad(dv, v, "dv"))) return st;
+  if (!w_s || !dw_s) return fail(DASH_ERR_INVALID_ARGUMENT, "null w_s or dw_s");
+  if (reinterpret_cast<uintptr_t>(w_s) % 16 || reinterpret_cast<uintptr_t>(dw_s) % 16)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "w_s and dw_s must be 16-byte aligned");
+  const BwdLayout L = bwd_layout(q->b, q->s, q->h, k->h, q->d, block);
+  if (L.T > 4096) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per sequence");
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < L.total)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  float* summ = at<float>(workspace, L.summ);
+  if ((st = dash_attn_summarize_sdpa(k, nullptr, w_s, nullptr, block, summ, L.T, 0, stream))) return st;
+  dash::DeviceStatus* dst = at<dash::DeviceStatus>(workspace, L.status);
+  int32_t* idx = at<int32_t>(workspace, L.idx);
+  float* logp = at<float>(workspace, L.logp);
+  int32_t* cnt = at<int32_t>(workspace, L.cnt);
+  float* tau = at<float>(workspace, L.tau);
+  if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, tau, nullptr, nullptr, dst, s, nullptr,
+                      at<float>(workspace, L.split))))
+    return st;
+  dash::BwdParams p{};
+  p.idx = idx;
+  p.logp = logp;
+  p.cnt = cnt;
+  p.tau = tau;
+  p.q = view(q);
+  p.k = view(k);
+  p.v = view(v);
+  p.o = view(out);
+  p.dout = view(dout);
+  p.dq = view(dq);
+  p.dk = view(dk);
+  p.dv = view(dv);
+  p.dtype = q->dtype;
+  p.B = (int)q->b;
+  p.S = (int)q->s;
+  p.H = (int)q->h;
+  p.Hkv = (int)k->h;
+  p.G = (int)(q->h / k->h);
+  p.D = (int)q->d;
+  p.block = block;
+  p.causal = causal ? 1 : 0;
+  p.alpha = alpha;
+  p.sigma = sigma;
+  p.w_s = w_s;
+  p.summaries = summ;
+  p.t_cap = L.T;
+  p.n_qblocks = (int)L.T;
+  p.n_words = (int)L.n_words;
+  p.lse = at<float>(workspace, L.lse);
+  p.dd = at<float>(workspace, L.dd);
+  p.dz = at<float>(workspace, L.dz);
+  p.umask = at<uint32_t>(workspace, L.umask);
+  p.kbar = at<float>(workspace, L.kbar);
+  p.ds = at<float>(workspace, L.ds);
+  p.dw_s = dw_s;
+  p.status = dst;
+  e = dash::launch_bwd(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "backward");
+  return ok();
 }
 
 size_t dash_attn_decode_workspace_size(const dash_tensor_t* q, const dash_tensor_t* kcache, int block, int64_t t_cap) {

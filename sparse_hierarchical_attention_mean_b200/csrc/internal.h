@@ -189,4 +189,39 @@ cudaError_t launch_cp_attend(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_cp_merge(const float* parts, int n_parts, int B, int H, int D, const View& out, int dtype,
                             cudaStream_t stream);
 
+// ---------------------------------------------------------------- backward
+// Gradients of sum(dout * out) for the prefill forward (f16/bf16 inputs,
+// fp32 gradients).  The summaries, lists and thresholds are the forward's,
+// recomputed by the caller before the four kernels run in order:
+//   row    (query block, head): LSE, dq of stage 2, d log p_bar per head
+//   route  (row, KV head): entmax vector-Jacobian product, dq of stage 1
+//   key    (key block, KV head): dk, dv of stage 2, the summary gradient and
+//          its stage-0 projection into dk
+//   ws     dW_s = sum over blocks of kbar^T ds
+struct BwdParams {
+  View q, k, v, o, dout;  // [B, S, H or Hkv, D], dtype
+  View dq, dk, dv;        // fp32, same shapes
+  int dtype;
+  int B, S, H, Hkv, G, D, block, causal;
+  float alpha, sigma;
+  const float* w_s;        // [D, D]
+  const float* summaries;  // [B, Hkv, t_cap, D]
+  int64_t t_cap;           // ceil(S / block)
+  int n_qblocks;           // ceil(S / block)
+  int n_words;             // ceil(t_cap / 32)
+  const int32_t* idx;      // [B, Hkv, S, t_cap]
+  const float* logp;       // [B, Hkv, S, t_cap]
+  const int32_t* cnt;      // [B, Hkv, S]
+  const float* tau;        // [B, H, S]
+  float* lse;              // [B, H, S] log-sum-exp of the logits, log2 units
+  float* dd;               // [B, H, S] dout . out
+  float* dz;               // [B, Hkv, S, t_cap, G]: d log p_bar per head, then dL/dz
+  uint32_t* umask;         // [B, Hkv, n_qblocks, n_words]: blocks some row of the query block selected
+  float* kbar;             // [B, Hkv, t_cap, D] block means
+  float* ds;               // [B, Hkv, t_cap, D] dL/d(summary)
+  float* dw_s;             // [D, D]
+  DeviceStatus* status;
+};
+cudaError_t launch_bwd(const BwdParams& p, cudaStream_t stream);
+
 }  // namespace dash

@@ -187,3 +187,54 @@ def test_binding_refuses_host_tensors():
     x = torch.zeros(1, 64, 1, 64)
     with pytest.raises(ValueError):
         dash.fwd(x, x, x, torch.zeros(64, 64), 1.5, 64)
+
+
+def call_bwd(q, k, v, o, do, dq, dk, dv, ws_bytes=1 << 42, opts=None, dw_s=FAKE):
+    lib = dash.load()
+    st = lib.dash_attn_bwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), FAKE, ctypes.byref(o), ctypes.byref(do),
+                           1.5, 64, 1, opts, ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), dw_s, FAKE,
+                           ws_bytes, None)
+    return st, lib.dash_attn_last_error().decode()
+
+
+def good_bwd():
+    q, k, v, o = good()
+    return q, k, v, o, tensor(1, 256, 8, 128), tensor(1, 256, 8, 128, dtype=0), tensor(1, 256, 2, 128, dtype=0), \
+        tensor(1, 256, 2, 128, dtype=0)
+
+
+@pytest.mark.parametrize(
+    "mutate, status, text",
+    [
+        (lambda a: [setattr(t, "dtype", 0) for t in a[:5]], 2, "f16 or bf16"),
+        (lambda a: setattr(a[5], "dtype", 2), 1, "fp32"),
+        (lambda a: setattr(a[6], "h", 8), 1, "shape of its input"),
+        (lambda a: setattr(a[4], "s", 128), 1, "dout"),
+        (lambda a: setattr(a[4], "dtype", 1), 1, "dout"),
+        (lambda a: setattr(a[7], "data", FAKE + 4), 1, "aligned"),
+    ],
+)
+def test_bwd_rejects_bad_arguments(mutate, status, text):
+    args = list(good_bwd())
+    mutate(args)
+    st, msg = call_bwd(*args)
+    assert st == status, msg
+    assert text in msg
+
+
+def test_bwd_workspace_options_and_outputs():
+    lib = dash.load()
+    q, k, v, o, do, dq, dk, dv = good_bwd()
+    need = lib.dash_attn_bwd_workspace_size(ctypes.byref(q), ctypes.byref(k), 64)
+    # at least the per-head routing gradients [B, Hkv, S, T, G] fp32
+    assert need >= 1 * 2 * 256 * 4 * 4 * 4
+    st, msg = call_bwd(q, k, v, o, do, dq, dk, dv, ws_bytes=need - 1)
+    assert st == 3 and "workspace" in msg
+    st, msg = call_bwd(q, k, v, o, do, dq, dk, dv, dw_s=None)
+    assert st == 1 and "dw_s" in msg
+    opts = dash.DashOptions(1.0, FAKE)
+    st, msg = call_bwd(q, k, v, o, do, dq, dk, dv, opts=ctypes.byref(opts))
+    assert st == 1 and "qbar" in msg
+    opts = dash.DashOptions(-1.0, None)
+    st, msg = call_bwd(q, k, v, o, do, dq, dk, dv, opts=ctypes.byref(opts))
+    assert st == 1 and "sigma" in msg

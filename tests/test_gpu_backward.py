@@ -1,0 +1,132 @@
+"""GPU parity of the backward pass (dash_attn_bwd) against the fp64 oracle.
+
+Small cases run the whole oracle backward and compare every gradient; they
+span several query and key blocks with a ragged tail, every group size, both
+head dims and block sizes, the three alphas, sigma != 1, non-causal routing,
+a batch of two and a single partial block.  At the full prefill size the
+query gradients of sampled rows are compared with the oracle row by row, and
+dk / dv with two identities that hold at any size: the loss does not change
+when every key of a KV head moves by one vector (softmax and entmax are
+shift invariant), so sum_j dk_j = 0; each softmax row sums to one, so
+sum_j dv_j = sum of dout over the rows and the group's heads.
+
+Tolerance (bf16 and f16 alike, written per gradient tensor): the inputs are
+the same rounded values on both sides, and the kernel rounds P and dS to the
+input type once each as tensor-core operands (relative 2^-8 for bf16), with
+fp32 accumulation.  Errors of that kind are unbiased, so a gradient's
+normwise relative error stays at a few units of 2^-8: the bound is 2e-2,
+and 5e-2 of the largest reference magnitude element by element.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gen import full_inputs, get_config
+from oracle.backward import backward, backward_row
+from oracle.dash_oracle import block_summaries
+
+pytestmark = pytest.mark.gpu
+
+NORM_TOL = 2e-2
+ELEM_TOL = 5e-2
+
+_BASE = get_config("prefill")
+CASES = {
+    "b64_g4": (_BASE.with_(name="b64_g4", heads=8, kv_heads=2, seq=700), 1.0),
+    "b128_g8_d64_f16_noncausal": (_BASE.with_(name="b128_g8", heads=8, kv_heads=1, head_dim=64, dtype="f16",
+                                              block=128, seq=420, causal=False), 0.7),
+    "g1_alpha2": (_BASE.with_(name="g1_a2", heads=2, kv_heads=2, seq=333, alpha=2.0), 1.0),
+    "g2_alpha125_b128": (_BASE.with_(name="g2_a125", heads=4, kv_heads=2, block=128, seq=600, alpha=1.25), 1.3),
+    "batch2_f16_d64": (get_config("sweep").with_(name="sweep_b2", batch=2, heads=4, kv_heads=4, seq=300), 1.0),
+    "single_partial_block": (_BASE.with_(name="tiny", heads=4, kv_heads=1, seq=40), 1.0),
+    "full_heads_1k": (_BASE.with_(name="full_heads_1k", seq=1024), 1.0),
+}
+
+
+def _dout(q, seed=1234):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return torch.randn(q.shape, generator=g, dtype=torch.float32).to(q.dtype).to(q.device)
+
+
+def _np(t):
+    return t.detach().double().cpu().numpy()
+
+
+def _close(name, got, ref):
+    err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    elem = np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    assert err <= NORM_TOL and elem <= ELEM_TOL, f"{name}: normwise {err:.3g}, elementwise {elem:.3g}"
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_backward_matches_oracle(cuda_lib, case):
+    dash = cuda_lib
+    cfg, sigma = CASES[case]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w_s = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    out = dash.fwd(q, k, v, w_s, cfg.alpha, cfg.block, cfg.causal, sigma=sigma)
+    dout = _dout(q)
+    g = dash.bwd(q, k, v, w_s, out, dout, cfg.alpha, cfg.block, cfg.causal, sigma=sigma)
+    torch.cuda.synchronize()
+    dw_ref = np.zeros((cfg.head_dim, cfg.head_dim))
+    for b in range(cfg.batch):
+        ref = backward(_np(q[b]), _np(k[b]), _np(v[b]), _np(w_s), _np(dout[b]), cfg.alpha, cfg.block, cfg.causal,
+                       sigma)
+        for name in ("dq", "dk", "dv"):
+            _close(f"{case} b{b} {name}", _np(g[name][b]), ref[name])
+        dw_ref += ref["dw_s"]
+    if cfg.seq > cfg.block:
+        _close(f"{case} dw_s", _np(g["dw_s"]), dw_ref)
+    else:
+        assert torch.all(g["dw_s"] == 0)
+
+
+def test_backward_autograd_wrapper(cuda_lib):
+    # torch.autograd through the library: the wrapper returns the same gradients
+    dash = cuda_lib
+    cfg = _BASE.with_(name="ag", heads=4, kv_heads=2, seq=200)
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v = (inp[n].clone().requires_grad_(True) for n in ("q", "k", "v"))
+    w_s = inp["w_s"].clone().requires_grad_(True)
+    out = dash.attention(q, k, v, w_s, cfg.alpha, cfg.block, True)
+    dout = _dout(out)
+    out.backward(dout)
+    g = dash.bwd(inp["q"], inp["k"], inp["v"], inp["w_s"], out.detach(), dout, cfg.alpha, cfg.block, True)
+    torch.cuda.synchronize()
+    assert torch.equal(q.grad, g["dq"].to(q.dtype))
+    assert torch.equal(k.grad, g["dk"].to(k.dtype))
+    assert torch.equal(v.grad, g["dv"].to(v.dtype))
+    assert torch.equal(w_s.grad, g["dw_s"])
+
+
+def test_backward_full_prefill(cuda_lib):
+    # the full prefill workload: sampled rows' dq against the oracle, and the
+    # two identities for dk and dv over every KV head
+    dash = cuda_lib
+    cfg = get_config("prefill")
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w_s = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    out = dash.fwd(q, k, v, w_s, cfg.alpha, cfg.block, True)
+    dout = _dout(q, seed=99)
+    g = dash.bwd(q, k, v, w_s, out, dout, cfg.alpha, cfg.block, True)
+    torch.cuda.synchronize()
+    for name in ("dq", "dk", "dv", "dw_s"):
+        assert torch.isfinite(g[name]).all(), name
+    G = cfg.group
+    for kv in range(cfg.kv_heads):
+        dk = g["dk"][0, :, kv].double()
+        assert (dk.sum(0).abs() <= 1e-3 * dk.abs().sum(0) + 1e-6).all(), f"sum dk, KV head {kv}"
+        dv_sum = g["dv"][0, :, kv].double().sum(0)
+        do = dout[0, :, kv * G:(kv + 1) * G].double()
+        assert ((dv_sum - do.sum((0, 1))).abs() <= 1e-3 * do.abs().sum((0, 1))).all(), f"sum dv, KV head {kv}"
+    w = _np(w_s)
+    for kv in (0, cfg.kv_heads - 1):
+        kg, vg = _np(k[0, :, kv]), _np(v[0, :, kv])
+        summ = block_summaries(kg, w, cfg.block, cfg.seq)
+        for pos in (0, 63, 64, 1000, 16385, cfg.seq - 1):
+            hs = slice(kv * G, (kv + 1) * G)
+            rb = backward_row(_np(q[0, pos, hs]), kg, vg, summ, _np(dout[0, pos, hs]), pos, cfg.seq, cfg.block,
+                              cfg.alpha, True)
+            _close(f"dq row {pos} KV head {kv}", _np(g["dq"][0, pos, hs]), rb["dq"])

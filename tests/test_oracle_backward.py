@@ -147,3 +147,19 @@ def test_backward_single_block_is_local_attention():
     out.transpose(0, 1).backward(torch.tensor(dout))
     np.testing.assert_allclose(g["dq"], tq.grad.numpy(), atol=1e-12)
     np.testing.assert_allclose(g["dk"], tk.grad.numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_shift_and_normalisation_identities(causal):
+    # shifting every key of a KV head by one vector moves each row's logits
+    # and each row's block scores by a constant, which neither softmax nor
+    # entmax sees: sum_j dk_j = 0.  Each softmax row sums to one:
+    # sum_j dv_j = sum over the rows and the group's heads of dout.
+    S, H, Hkv, d = 40, 4, 2, 8
+    q, k, v, w_s, dout = _tiny(21, S=S, H=H, Hkv=Hkv, d=d)
+    g = backward(q, k, v, w_s, dout, 1.5, 8, causal, sigma=0.8)
+    G = H // Hkv
+    for kv in range(Hkv):
+        np.testing.assert_allclose(g["dk"][:, kv].sum(axis=0), 0.0, atol=1e-11)
+        np.testing.assert_allclose(g["dv"][:, kv].sum(axis=0), dout[:, kv * G:(kv + 1) * G].sum(axis=(0, 1)),
+                                   atol=1e-11)
