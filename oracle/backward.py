@@ -86,6 +86,12 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
     gradient has no other source), the attended token ids ``tok`` with their
     dk / dv contributions [len(tok), d], and the candidate ids ``cand`` with
     their summary gradients ds [len(cand), d].
+
+    Also returns, for error bounds of reduced-precision implementations, the
+    magnitudes the gradients are sums of (elementwise absolute values, not
+    derivatives): dq_abs [G, d], dk_abs_tok and dv_abs_tok.  A product whose
+    operand dS (or P) carries a relative rounding error u is off by at most
+    u times these; dq and dk also count the term through D = dout . out.
     """
     q_group = np.asarray(q_group, dtype=np.float64)
     dout_group = np.asarray(dout_group, dtype=np.float64)
@@ -97,7 +103,11 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
     dq = np.zeros((G, d))
     dk_tok = np.zeros((len(tok), d))
     dv_tok = np.zeros((len(tok), d))
+    dq_abs = np.zeros((G, d))
+    dk_abs = np.zeros((len(tok), d))
+    dv_abs = np.zeros((len(tok), d))
     dlogp = np.zeros(len(r["blocks"]))
+    dlogp_abs = np.zeros(len(r["blocks"]))
     for h in range(G):
         logits = k[tok] @ q_group[h] * scale + bias
         w = np.exp(logits - logits.max())
@@ -108,19 +118,33 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
         dq[h] += scale * (dS @ k[tok])
         dk_tok += scale * np.outer(dS, q_group[h])
         dv_tok += np.outer(P, dout_group[h])
+        mag = np.abs(dS) + P * (np.abs(dout_group[h]) @ np.abs(o))
+        dq_abs[h] += scale * (mag @ np.abs(k[tok]))
+        dk_abs += scale * np.outer(mag, np.abs(q_group[h]))
+        dv_abs += np.outer(P, np.abs(dout_group[h]))
         for e in range(len(dlogp)):
             dlogp[e] += sigma * dS[owner == e].sum()
+            dlogp_abs[e] += sigma * mag[owner == e].sum()
     cand = np.asarray(r["cand"], dtype=np.int64)
     ds = np.zeros((len(cand), d))
+    ds_abs = np.zeros((len(cand), d))
     if len(r["blocks"]):
         # through the GQA mean p_bar = mean_h p_h and the log
         gp = np.zeros(len(cand))
         gp[r["idx"]] = dlogp / (G * r["pbar"][r["idx"]])
+        gp_abs = np.zeros(len(cand))
+        gp_abs[r["idx"]] = dlogp_abs / (G * r["pbar"][r["idx"]])
         for h in range(G):
             dz = entmax_vjp(r["p"][h], gp, alpha)
             dq[h] += gamma * (dz @ summaries[cand])
             ds += gamma * np.outer(dz, q_group[h])
-    return {"dq": dq, "tok": tok, "dk_tok": dk_tok, "dv_tok": dv_tok, "cand": cand, "ds": ds}
+            # magnitudes through u * (g - <u, g> / sum(u))
+            u = np.where(r["p"][h] > 0.0, np.power(np.where(r["p"][h] > 0.0, r["p"][h], 1.0), 2.0 - alpha), 0.0)
+            dz_abs = u * (gp_abs + (u @ gp_abs) / max(u.sum(), 1e-300))
+            dq_abs[h] += gamma * (dz_abs @ np.abs(summaries[cand]))
+            ds_abs += gamma * np.outer(dz_abs, np.abs(q_group[h]))
+    return {"dq": dq, "tok": tok, "dk_tok": dk_tok, "dv_tok": dv_tok, "cand": cand, "ds": ds,
+            "dq_abs": dq_abs, "dk_abs_tok": dk_abs, "dv_abs_tok": dv_abs, "ds_abs": ds_abs}
 
 
 def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout: np.ndarray, alpha: float,
@@ -142,11 +166,13 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     dw_s = np.zeros_like(w_s)
+    mags = {"dq_abs": np.zeros_like(q), "dk_abs": np.zeros_like(k), "dv_abs": np.zeros_like(v)}
     n_blocks = -(-S // block)
     for g in range(Hkv):
         kg, vg = k[:, g], v[:, g]
         summ = block_summaries(kg, w_s, block, S)
         ds = np.zeros((n_blocks, d))
+        ds_abs = np.zeros((n_blocks, d))
         for pos in range(S):
             hs = slice(g * G, (g + 1) * G)
             rb = backward_row(q[pos, hs], kg, vg, summ, dout[pos, hs], pos, S, block, alpha, causal, sigma)
@@ -154,13 +180,18 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
             dk[rb["tok"], g] += rb["dk_tok"]
             dv[rb["tok"], g] += rb["dv_tok"]
             ds[rb["cand"]] += rb["ds"]
+            ds_abs[rb["cand"]] += rb["ds_abs"]
+            mags["dq_abs"][pos, hs] = rb["dq_abs"]
+            mags["dk_abs"][rb["tok"], g] += rb["dk_abs_tok"]
+            mags["dv_abs"][rb["tok"], g] += rb["dv_abs_tok"]
         # stage 0: s_c = kbar_c W_s over the c's valid tokens
         for c in range(n_blocks):
             lo, hi = c * block, min(S, (c + 1) * block)
             kbar = kg[lo:hi].sum(axis=0) / (hi - lo)
             dw_s += np.outer(kbar, ds[c])
             dk[lo:hi, g] += (w_s @ ds[c]) / (hi - lo)
-    return {"dq": dq, "dk": dk, "dv": dv, "dw_s": dw_s}
+            mags["dk_abs"][lo:hi, g] += (np.abs(w_s) @ ds_abs[c]) / (hi - lo)
+    return {"dq": dq, "dk": dk, "dv": dv, "dw_s": dw_s, **mags}
 
 
 def loss(q, k, v, w_s, dout, alpha, block, causal=True, sigma=1.0) -> float:

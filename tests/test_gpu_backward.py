@@ -10,12 +10,18 @@ when every key of a KV head moves by one vector (softmax and entmax are
 shift invariant), so sum_j dk_j = 0; each softmax row sums to one, so
 sum_j dv_j = sum of dout over the rows and the group's heads.
 
-Tolerance (bf16 and f16 alike, written per gradient tensor): the inputs are
-the same rounded values on both sides, and the kernel rounds P and dS to the
-input type once each as tensor-core operands (relative 2^-8 for bf16), with
-fp32 accumulation.  Errors of that kind are unbiased, so a gradient's
-normwise relative error stays at a few units of 2^-8: the bound is 2e-2,
-and 5e-2 of the largest reference magnitude element by element.
+Tolerance, derived from the arithmetic: both sides read the same rounded
+inputs; the kernel rounds P and dS once each to the input type as
+tensor-core operands (unit roundoff u = 2^-8 for bf16, 2^-11 for f16), takes
+D = dout . out from the stored (rounded) forward output, and accumulates in
+fp32.  Each gradient element is a sum of such products, so its error is at
+most about u times the sum of the magnitudes of its terms, which the oracle
+returns alongside the gradients (dq_abs, dk_abs, dv_abs).  The bound is
+2 u times that magnitude (plus 1e-6 of its largest value) element by element.
+It is not a fixed fraction of the gradient: where dS nearly cancels against
+key components shared by a block (sum_j dS_j = 0 exactly), |dq| is much
+smaller than the sum it comes from.  dW_s comes out of the fp32 routing
+gradient and is held to 2e-2 normwise.
 """
 
 import numpy as np
@@ -29,7 +35,7 @@ from oracle.dash_oracle import block_summaries
 pytestmark = pytest.mark.gpu
 
 NORM_TOL = 2e-2
-ELEM_TOL = 5e-2
+UNIT_ROUNDOFF = {torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}
 
 _BASE = get_config("prefill")
 CASES = {
@@ -55,9 +61,17 @@ def _np(t):
 
 def _close(name, got, ref):
     err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
-    elem = np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30)
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
-    assert err <= NORM_TOL and elem <= ELEM_TOL, f"{name}: normwise {err:.3g}, elementwise {elem:.3g}"
+    assert err <= NORM_TOL, f"{name}: normwise {err:.3g}"
+
+
+def _within(name, got, ref, mag, u):
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    bound = 2.0 * u * mag + 1e-6 * mag.max()
+    excess = np.abs(got - ref) / bound
+    worst = np.unravel_index(np.argmax(excess), excess.shape)
+    assert excess.max() <= 1.0, (f"{name}: error {abs(got - ref)[worst]:.3g} at {worst} above the bound "
+                                 f"{bound[worst]:.3g} (magnitude {mag[worst]:.3g})")
 
 
 @pytest.mark.parametrize("case", list(CASES))
@@ -75,7 +89,7 @@ def test_backward_matches_oracle(cuda_lib, case):
         ref = backward(_np(q[b]), _np(k[b]), _np(v[b]), _np(w_s), _np(dout[b]), cfg.alpha, cfg.block, cfg.causal,
                        sigma)
         for name in ("dq", "dk", "dv"):
-            _close(f"{case} b{b} {name}", _np(g[name][b]), ref[name])
+            _within(f"{case} b{b} {name}", _np(g[name][b]), ref[name], ref[name + "_abs"], UNIT_ROUNDOFF[q.dtype])
         dw_ref += ref["dw_s"]
     if cfg.seq > cfg.block:
         _close(f"{case} dw_s", _np(g["dw_s"]), dw_ref)
@@ -129,4 +143,5 @@ def test_backward_full_prefill(cuda_lib):
             hs = slice(kv * G, (kv + 1) * G)
             rb = backward_row(_np(q[0, pos, hs]), kg, vg, summ, _np(dout[0, pos, hs]), pos, cfg.seq, cfg.block,
                               cfg.alpha, True)
-            _close(f"dq row {pos} KV head {kv}", _np(g["dq"][0, pos, hs]), rb["dq"])
+            _within(f"dq row {pos} KV head {kv}", _np(g["dq"][0, pos, hs]), rb["dq"], rb["dq_abs"],
+                    UNIT_ROUNDOFF[q.dtype])

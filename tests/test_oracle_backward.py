@@ -163,3 +163,14 @@ def test_backward_shift_and_normalisation_identities(causal):
         np.testing.assert_allclose(g["dk"][:, kv].sum(axis=0), 0.0, atol=1e-11)
         np.testing.assert_allclose(g["dv"][:, kv].sum(axis=0), dout[:, kv * G:(kv + 1) * G].sum(axis=(0, 1)),
                                    atol=1e-11)
+
+
+def test_backward_magnitudes_bound_the_gradients():
+    # the magnitude sums returned for error bounds dominate the gradients
+    # element by element (triangle inequality), and are zero only where the
+    # gradient has no terms
+    q, k, v, w_s, dout = _tiny(13, S=40, H=4, Hkv=2, d=8)
+    g = backward(q, k, v, w_s, dout, 1.5, 8, True, sigma=0.9)
+    for name in ("dq", "dk", "dv"):
+        assert np.all(g[name + "_abs"] >= np.abs(g[name]) - 1e-12), name
+        assert g[name + "_abs"].min() >= 0.0
