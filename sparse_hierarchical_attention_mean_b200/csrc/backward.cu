@@ -132,9 +132,9 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   T* Qs = reinterpret_cast<T*>(smem);  // [BLK][D]
   T* dOs = Qs + BLK * D;               // [BLK][D]
-  T* Ks = dOs + BLK * D;               // [64][D]
-  T* Vs = Ks + kKeyChunk * D;          // [64][D]
-  float* Dsm = reinterpret_cast<float*>(Vs + kKeyChunk * D);  // [BLK] dout . out
+  T* Ks = dOs + BLK * D;               // [2][64][D] (double buffer)
+  T* Vs = Ks + 2 * kKeyChunk * D;      // [2][64][D]
+  float* Dsm = reinterpret_cast<float*>(Vs + 2 * kKeyChunk * D);  // [BLK] dout . out
   uint32_t* um = reinterpret_cast<uint32_t*>(Dsm + BLK);      // [n_words] union bitmap
   int32_t* ulist = reinterpret_cast<int32_t*>(um + p.n_words);  // [t_cap + 1] union, then the diagonal
   __shared__ int nu_s;
@@ -258,8 +258,36 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
       }
   };
 
-  // pass 1: log-sum-exp of every row
+  // chunks with keys to process (the others are past the sequence end or,
+  // on the causal diagonal, past every row of the block)
+  auto chunk_ok = [&](int ch) -> bool {
+    const int bi = ch / SPB, sub = ch - bi * SPB;
+    const int key0 = ulist[bi] * BLK + sub * kKeyChunk;
+    return !(key0 >= S || (bi == nu && p.causal && key0 > row0 + nrows - 1));
+  };
+  auto next_ok = [&](int ch) -> int {
+    while (ch < nchunks && !chunk_ok(ch)) ++ch;
+    return ch;
+  };
+  // K (and V) rows of chunk ch into buffer buf
+  auto issue = [&](int ch, int buf, bool with_v) {
+    if (ch < nchunks) {
+      const int bi = ch / SPB, sub = ch - bi * SPB;
+      const int key0 = ulist[bi] * BLK + sub * kKeyChunk;
+      const int nk = min(kKeyChunk, S - key0);
+      load_rows<T, D>(Ks + buf * kKeyChunk * D, kg + (int64_t)key0 * p.k.ss, p.k.ss, nk, kKeyChunk, tid, NTH);
+      if (with_v)
+        load_rows<T, D>(Vs + buf * kKeyChunk * D, vg + (int64_t)key0 * p.v.ss, p.v.ss, nk, kKeyChunk, tid, NTH);
+    }
+    cp_async_commit();
+  };
+  constexpr uint32_t kBufBytes = kKeyChunk * D * sizeof(T);
+
+  // pass 1: log-sum-exp of every row.  The next chunk's K streams in while
+  // this one is reduced.
   float m_a = kNegInf, m_b = kNegInf, l_a = 0.f, l_b = 0.f;
+  int buf = 0;
+  issue(next_ok(0), 0, false);
   for (int ch = 0; ch < nchunks; ++ch) {
     const int bi = ch / SPB, sub = ch - bi * SPB;
     const int c = ulist[bi];
@@ -268,14 +296,13 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
     float ba, bb;
     int ea, eb;
     row_bias(c, diag, sub, ba, bb, ea, eb);
-    if (key0 >= S || (diag && p.causal && key0 > row0 + nrows - 1)) continue;
-    __syncthreads();  // the previous chunk's readers are done with Ks
-    load_rows<T, D>(Ks, kg + (int64_t)key0 * p.k.ss, p.k.ss, min(kKeyChunk, S - key0), kKeyChunk, tid, NTH);
-    cp_async_commit();
-    cp_async_wait<0>();
+    if (!chunk_ok(ch)) continue;
+    __syncthreads();  // the other buffer's readers are done
+    issue(next_ok(ch + 1), buf ^ 1, false);
+    cp_async_wait<1>();
     __syncthreads();
     float s[8][4];
-    tile_abt<T, D, 4>(qs_b, warp * 16, ks_b, lane, s);
+    tile_abt<T, D, 4>(qs_b, warp * 16, ks_b + buf * kBufBytes, lane, s);
     logits(s, key0, diag, ba, bb);
     float mx_a = kNegInf, mx_b = kNegInf;
 #pragma unroll
@@ -299,7 +326,9 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
     if (m_b != kNegInf)
 #pragma unroll
       for (int n = 0; n < 8; ++n) l_b += exp2f(s[n][2] - m_b) + exp2f(s[n][3] - m_b);
+    buf ^= 1;
   }
+  cp_async_wait<0>();
   l_a = quad_sum(l_a);
   l_b = quad_sum(l_b);
   // every valid row attends at least its own token, so m and l are finite
@@ -311,7 +340,7 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
   }
   const float d_a = Dsm[ra], d_b = Dsm[rb];
 
-  // pass 2: dS, dq and d log p_bar
+  // pass 2: dS, dq and d log p_bar, with the same prefetch of K and V
   float dq[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
@@ -319,6 +348,9 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
   cur_a = cur_b = 0;
   float* dz_a = p.dz + (rowbase + (va ? pa : row0)) * tc * p.G + hh;
   float* dz_b = p.dz + (rowbase + (vb ? pb : row0)) * tc * p.G + hh;
+  __syncthreads();  // pass 1's readers are done with both buffers
+  buf = 0;
+  issue(next_ok(0), 0, true);
   for (int ch = 0; ch < nchunks; ++ch) {
     const int bi = ch / SPB, sub = ch - bi * SPB;
     const int c = ulist[bi];
@@ -327,17 +359,15 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
     float ba, bb;
     int ea, eb;
     row_bias(c, diag, sub, ba, bb, ea, eb);
-    if (!(key0 >= S || (diag && p.causal && key0 > row0 + nrows - 1))) {
+    if (chunk_ok(ch)) {
       __syncthreads();
-      const int nk = min(kKeyChunk, S - key0);
-      load_rows<T, D>(Ks, kg + (int64_t)key0 * p.k.ss, p.k.ss, nk, kKeyChunk, tid, NTH);
-      load_rows<T, D>(Vs, vg + (int64_t)key0 * p.v.ss, p.v.ss, nk, kKeyChunk, tid, NTH);
-      cp_async_commit();
-      cp_async_wait<0>();
+      issue(next_ok(ch + 1), buf ^ 1, true);
+      cp_async_wait<1>();
       __syncthreads();
+      const uint32_t kb = ks_b + buf * kBufBytes, vb_ = vs_b + buf * kBufBytes;
       float s[8][4], dp[8][4];
-      tile_abt<T, D, 4>(qs_b, warp * 16, ks_b, lane, s);
-      tile_abt<T, D, 4>(do_b, warp * 16, vs_b, lane, dp);
+      tile_abt<T, D, 4>(qs_b, warp * 16, kb, lane, s);
+      tile_abt<T, D, 4>(do_b, warp * 16, vb_, lane, dp);
       logits(s, key0, diag, ba, bb);
 #pragma unroll
       for (int n = 0; n < 8; ++n)
@@ -349,7 +379,8 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
           if (e < 2) dl_a += dsv;
           else dl_b += dsv;
         }
-      tile_xb<T, D, 4>(s, ks_b, lane, dq);
+      tile_xb<T, D, 4>(s, kb, lane, dq);
+      buf ^= 1;
     }
     if (!diag && sub == SPB - 1) {
       dl_a = quad_sum(dl_a);
@@ -361,6 +392,7 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
     }
     if (sub == SPB - 1) dl_a = dl_b = 0.f;
   }
+  cp_async_wait<0>();
 
   const float qsc = rsqrtf((float)D);
   float* dqg = static_cast<float*>(const_cast<void*>(p.dq.data)) + (int64_t)b * p.dq.sb + (int64_t)h * p.dq.sh;
@@ -476,23 +508,29 @@ __global__ void __launch_bounds__(128) bwd_route_kernel(BwdParams p) {
 }
 
 // ------------------------------------------------------------------ bwd_key
+// 4-byte cp.async (zero fill when !valid; `gmem` must still be a readable address)
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+
 template <typename T, int D, int BLK>
-__global__ void __launch_bounds__(2 * BLK) bwd_key_kernel(BwdParams p) {
+__global__ void __launch_bounds__(2 * BLK, BLK == 64 ? 3 : 1) bwd_key_kernel(BwdParams p) {
   constexpr int NW = BLK / 16, NTH = NW * 32;
   constexpr int NT = D / 8;
   constexpr int NRC = BLK / kRowChunk;
+  constexpr int RC = kRowChunk;
   extern __shared__ __align__(128) uint8_t smem[];
   T* Ks = reinterpret_cast<T*>(smem);  // [BLK][D]
   T* Vs = Ks + BLK * D;                // [BLK][D]
-  T* Qs = Vs + BLK * D;                // [32][D]
-  T* dOs = Qs + kRowChunk * D;         // [32][D]
-  float* rb2 = reinterpret_cast<float*>(dOs + kRowChunk * D);  // [32] bias, log2; -inf: row skips the block
-  float* rl2 = rb2 + kRowChunk;  // [32] row log-sum-exp, log2
-  float* rdd = rl2 + kRowChunk;  // [32] dout . out
-  float* rdz = rdd + kRowChunk;  // [32] dL/dz of (row, block) for this head
-  int* es = reinterpret_cast<int*>(rdz + kRowChunk);  // [BLK] entry of the block in each row's list
-  float* dss = reinterpret_cast<float*>(es + BLK);    // [D]
-  float* dkb = dss + D;                                // [D]
+  T* Qs = Vs + BLK * D;                // [2][32][D] (double buffer)
+  T* dOs = Qs + 2 * RC * D;            // [2][32][D]
+  // per row of a chunk, raw: [2][4][32] = log p_bar entry, lse, dout . out, dL/dz
+  float* raw = reinterpret_cast<float*>(dOs + 2 * RC * D);
+  int* es = reinterpret_cast<int*>(raw + 2 * 4 * RC);  // [BLK] entry of the block in each row's list
+  float* dss = reinterpret_cast<float*>(es + BLK);     // [D]
+  float* dkb = dss + D;                                 // [D]
   __shared__ int chunk_any[NRC];
 
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -522,6 +560,7 @@ __global__ void __launch_bounds__(2 * BLK) bwd_key_kernel(BwdParams p) {
   const float sc = rsqrtf((float)D) * kLog2e;
   const int kw = warp * 16;
   const uint32_t ks_b = smem_u32(Ks), vs_b = smem_u32(Vs), qs_b = smem_u32(Qs), do_b = smem_u32(dOs);
+  constexpr uint32_t kBufBytes = RC * D * sizeof(T);
   cp_async_wait<0>();
   __syncthreads();
 
@@ -533,7 +572,7 @@ __global__ void __launch_bounds__(2 * BLK) bwd_key_kernel(BwdParams p) {
     }
     const int row0 = t * BLK;
     const int nrows = min(BLK, S - row0);
-    __syncthreads();  // es / chunk_any of the previous query block are no longer read
+    __syncthreads();  // es / chunk_any / buffers of the previous query block are no longer read
     if (tid < NRC) chunk_any[tid] = 0;
     __syncthreads();
     for (int r = tid; r < BLK; r += NTH) {
@@ -555,64 +594,96 @@ __global__ void __launch_bounds__(2 * BLK) bwd_key_kernel(BwdParams p) {
         }
       }
       es[r] = e;
-      if (e != -1) chunk_any[r / kRowChunk] = 1;
+      if (e != -1) chunk_any[r / RC] = 1;
     }
     __syncthreads();
     const float beta2 = diag_bias2(p.sigma, p.causal ? t : p.n_qblocks - 1);
-    for (int hh = 0; hh < G; ++hh) {
-      const int h = g * G + hh;
-      const int64_t hrow = ((int64_t)b * p.H + h) * S;
-      for (int rc = 0; rc < nrows; rc += kRowChunk) {
-        if (!chunk_any[rc / kRowChunk]) continue;
-        const int nv = min(kRowChunk, nrows - rc);
-        __syncthreads();  // the previous chunk's readers are done with Qs / dOs / row data
-        load_rows<T, D>(Qs, static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb + (int64_t)(row0 + rc) * p.q.ss +
-                                (int64_t)h * p.q.sh,
-                        p.q.ss, nv, kRowChunk, tid, NTH);
-        load_rows<T, D>(dOs, static_cast<const T*>(p.dout.data) + (int64_t)b * p.dout.sb +
-                                 (int64_t)(row0 + rc) * p.dout.ss + (int64_t)h * p.dout.sh,
-                        p.dout.ss, nv, kRowChunk, tid, NTH);
-        cp_async_commit();
-        for (int r = tid; r < kRowChunk; r += NTH) {
+
+    // items (head, 32-row chunk) of this query block, in order; chunks no row
+    // of which selected the block are skipped.  Item i + 1 streams in while
+    // item i is computed.
+    const int n_items = G * NRC;
+    auto item_ok = [&](int i) -> bool {
+      const int rcn = i % NRC;
+      return rcn * RC < nrows && chunk_any[rcn];
+    };
+    auto next_ok = [&](int i) -> int {
+      while (i < n_items && !item_ok(i)) ++i;
+      return i;
+    };
+    auto issue = [&](int i, int bf) {
+      if (i < n_items) {
+        const int h = g * G + i / NRC, rc = (i % NRC) * RC;
+        const int nv = min(RC, nrows - rc);
+        load_rows<T, D>(Qs + bf * RC * D, static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb +
+                                              (int64_t)(row0 + rc) * p.q.ss + (int64_t)h * p.q.sh,
+                        p.q.ss, nv, RC, tid, NTH);
+        load_rows<T, D>(dOs + bf * RC * D, static_cast<const T*>(p.dout.data) + (int64_t)b * p.dout.sb +
+                                               (int64_t)(row0 + rc) * p.dout.ss + (int64_t)h * p.dout.sh,
+                        p.dout.ss, nv, RC, tid, NTH);
+        if (tid < 4 * RC) {
+          const int which = tid / RC, r = tid % RC;
           const int e = r < nv ? es[rc + r] : -1;
           const int64_t ra = row0 + rc + r;
-          float bias = kNegInf, l2 = 0.f, dd = 0.f, dzv = 0.f;
-          if (e != -1) {
-            bias = e == -2 ? beta2 : p.sigma * p.logp[(rowbase + ra) * tc + e] * kLog2e;
-            l2 = p.lse[hrow + ra];
-            dd = p.dd[hrow + ra];
-            if (e >= 0) dzv = p.dz[((rowbase + ra) * tc + e) * G + hh];
+          const int64_t hrow = ((int64_t)b * p.H + h) * S;
+          const float* src = p.lse;  // any readable address when nothing is copied
+          bool ok = false;
+          if (which == 0) {
+            ok = e >= 0;
+            if (ok) src = p.logp + (rowbase + ra) * tc + e;
+          } else if (which == 1 || which == 2) {
+            ok = e != -1;
+            if (ok) src = (which == 1 ? p.lse : p.dd) + hrow + ra;
+          } else {
+            ok = e >= 0;
+            if (ok) src = p.dz + ((rowbase + ra) * tc + e) * G + (i / NRC);
           }
-          rb2[r] = bias;
-          rl2[r] = l2;
-          rdd[r] = dd;
-          rdz[r] = dzv;
-        }
-        cp_async_wait<0>();
-        __syncthreads();
-        // S^T and dP^T for the warp's 16 keys x 32 rows
-        float s[4][4], dp[4][4];
-        tile_abt<T, D, 2>(ks_b, kw, qs_b, lane, s);
-        tile_abt<T, D, 2>(vs_b, kw, do_b, lane, dp);
-#pragma unroll
-        for (int n = 0; n < 4; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int key = key0 + kw + gq + (e >> 1) * 8;
-            const int r = n * 8 + 2 * tq + (e & 1);
-            const float bias = rb2[r];
-            const bool ok = key < S && bias != kNegInf && (!diag || !p.causal || key <= row0 + rc + r);
-            const float pr = ok ? exp2f(fmaf(s[n][e], sc, bias) - rl2[r]) : 0.f;
-            s[n][e] = pr;
-            dp[n][e] = pr * (dp[n][e] - rdd[r]);
-          }
-        tile_xb<T, D, 2>(s, do_b, lane, dv);
-        tile_xb<T, D, 2>(dp, qs_b, lane, dk);
-        if (!diag && tid < D) {
-          for (int r = 0; r < nv; ++r) dsacc = fmaf(rdz[r], Elt<T>::load1(Qs + swz<D>(r, tid)), dsacc);
+          cp_async4(raw + (bf * 4 + which) * RC + r, src, ok);
         }
       }
+      cp_async_commit();
+    };
+
+    int bf = 0;
+    issue(next_ok(0), 0);
+    for (int i = next_ok(0); i < n_items; i = next_ok(i + 1)) {
+      const int rc = (i % NRC) * RC;
+      const int nv = min(RC, nrows - rc);
+      __syncthreads();  // the other buffer's readers are done
+      issue(next_ok(i + 1), bf ^ 1);
+      cp_async_wait<1>();
+      __syncthreads();
+      const uint32_t qb = qs_b + bf * kBufBytes, ob = do_b + bf * kBufBytes;
+      const float* rlp = raw + (bf * 4 + 0) * RC;
+      const float* rl2 = raw + (bf * 4 + 1) * RC;
+      const float* rdd = raw + (bf * 4 + 2) * RC;
+      const float* rdz = raw + (bf * 4 + 3) * RC;
+      // S^T and dP^T for the warp's 16 keys x 32 rows
+      float s[4][4], dp[4][4];
+      tile_abt<T, D, 2>(ks_b, kw, qb, lane, s);
+      tile_abt<T, D, 2>(vs_b, kw, ob, lane, dp);
+#pragma unroll
+      for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key0 + kw + gq + (e >> 1) * 8;
+          const int r = n * 8 + 2 * tq + (e & 1);
+          const int en = r < nv ? es[rc + r] : -1;
+          const float bias = en == -2 ? beta2 : (en >= 0 ? p.sigma * rlp[r] * kLog2e : kNegInf);
+          const bool ok = key < S && en != -1 && (!diag || !p.causal || key <= row0 + rc + r);
+          const float pr = ok ? exp2f(fmaf(s[n][e], sc, bias) - rl2[r]) : 0.f;
+          s[n][e] = pr;
+          dp[n][e] = pr * (dp[n][e] - rdd[r]);
+        }
+      tile_xb<T, D, 2>(s, ob, lane, dv);
+      tile_xb<T, D, 2>(dp, qb, lane, dk);
+      if (!diag && tid < D) {
+        const T* qrow = Qs + bf * RC * D;
+        for (int r = 0; r < nv; ++r) dsacc = fmaf(rdz[r], Elt<T>::load1(qrow + swz<D>(r, tid)), dsacc);
+      }
+      bf ^= 1;
     }
+    cp_async_wait<0>();
   }
 
   // stage 0: s_c = kbar_c W_s, so dkbar_c = ds_c W_s^T, spread over the block's keys
@@ -668,7 +739,7 @@ __global__ void bwd_ws_kernel(const float* __restrict__ kbar, const float* __res
 
 template <typename T, int D, int BLK>
 cudaError_t launch_typed(const BwdParams& p, cudaStream_t stream) {
-  const size_t row_smem = (size_t)(2 * BLK * D + 2 * kKeyChunk * D) * sizeof(T) + BLK * 4 +
+  const size_t row_smem = (size_t)(2 * BLK * D + 4 * kKeyChunk * D) * sizeof(T) + BLK * 4 +
                           (size_t)(p.n_words + p.t_cap + 1) * 4;
   cudaError_t e = cudaFuncSetAttribute(bwd_row_kernel<T, D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)row_smem);
@@ -691,7 +762,8 @@ cudaError_t launch_typed(const BwdParams& p, cudaStream_t stream) {
   }
   if (e != cudaSuccess) return e;
 
-  const size_t key_smem = (size_t)(2 * BLK * D + 2 * kRowChunk * D) * sizeof(T) + 4 * kRowChunk * 4 + BLK * 4 + 2 * D * 4;
+  const size_t key_smem =
+      (size_t)(2 * BLK * D + 4 * kRowChunk * D) * sizeof(T) + 2 * 4 * kRowChunk * 4 + BLK * 4 + 2 * D * 4;
   e = cudaFuncSetAttribute(bwd_key_kernel<T, D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)key_smem);
   if (e != cudaSuccess) return e;
   bwd_key_kernel<T, D, BLK><<<dim3((unsigned)p.t_cap, p.Hkv, p.B), 2 * BLK, key_smem, stream>>>(p);
