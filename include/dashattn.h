@@ -382,7 +382,7 @@ dash_status_t dash_attn_decode_noalloc(const dash_tensor_t* q, const dash_tensor
 /*
  * Synchronises `stream`, then reads the device status word of a workspace
  * last used by dash_attn_fwd / dash_attn_decode / dash_attn_sparse /
- * dash_attn_route (each call clears it when it starts).  Returns DASH_OK,
+ * dash_attn_route / dash_attn_bwd (each call clears it when it starts).  Returns DASH_OK,
  * DASH_ERR_DEVICE_TIMEOUT (a bounded device wait expired; outputs of that
  * call are not valid), DASH_ERR_INVALID_ARGUMENT (a device-side value such
  * as seqlens[b] was out of range; it was clamped) or DASH_ERR_CUDA.
