@@ -326,7 +326,7 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk, do_backward=True):
     # step i-1's download overlap step i's kernels.
     e2e_ms, h2d, d2h = run_e2e(dash, cfg, q, k, v, w, ws, steps, warmup, world)
     del ws
-    bwd = run_backward(dash, cfg, q, k, v, w, out, min(steps, 5), warmup, flops) if do_backward else None
+    bwd = run_backward(dash, cfg, q, k, v, w, out, min(steps, 5), warmup, flops, world) if do_backward else None
 
     return {
         "ms": ms, "tokens": B * S, "status": status, "seg_ms": seg.tolist(), "sparse_ms": sparse_ms, "flops": flops,
@@ -336,7 +336,7 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk, do_backward=True):
     }
 
 
-def run_backward(dash, cfg, q, k, v, w, out, steps, warmup, fwd_flops):
+def run_backward(dash, cfg, q, k, v, w, out, steps, warmup, fwd_flops, world):
     """The backward pass (dash_attn_bwd) on the same inputs, timed with CUDA events.
 
     Algorithmic work: 2.5x the forward's selected FLOPs (the scores S = QK^T
@@ -358,13 +358,16 @@ def run_backward(dash, cfg, q, k, v, w, out, steps, warmup, fwd_flops):
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1) / steps
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, world)
     status = dash.device_status(ws)
     del ws
     return {"ms": ms, "flops": 2.5 * fwd_flops, "steps": steps, "status": status}
