@@ -78,7 +78,8 @@ def _attended(r: dict, pos: int, n_tokens: int, block: int, causal: bool, sigma:
 
 
 def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: np.ndarray, dout_group: np.ndarray,
-                 pos: int, n_tokens: int, block: int, alpha: float, causal: bool = True, sigma: float = 1.0) -> dict:
+                 pos: int, n_tokens: int, block: int, alpha: float, causal: bool = True, sigma: float = 1.0,
+                 out_group: np.ndarray | None = None) -> dict:
     """The contribution of one query position of one KV group to the gradients.
 
     q_group, dout_group: [G, d]; k, v: [L, d] of the KV head; summaries: all
@@ -87,11 +88,16 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
     dk / dv contributions [len(tok), d], and the candidate ids ``cand`` with
     their summary gradients ds [len(cand), d].
 
+    out_group: the forward output [G, d] as an attention backward consumes
+    it, D = dout . out (the softmax-gradient shortcut for sum_j P_j dP_j).
+    None takes the exact output, which makes every gradient the exact
+    derivative; a given (e.g. rounded) output changes D and nothing else.
+
     Also returns, for error bounds of reduced-precision implementations, the
-    magnitudes the gradients are sums of (elementwise absolute values, not
-    derivatives): dq_abs [G, d], dk_abs_tok and dv_abs_tok.  A product whose
-    operand dS (or P) carries a relative rounding error u is off by at most
-    u times these; dq and dk also count the term through D = dout . out.
+    sizes of the terms the gradients are sums of (not derivatives): the
+    sums of squares dq_ss [G, d], dk_ss_tok, dv_ss_tok of the products whose
+    operand dS (dq, dk) or P (dv) a tensor-core implementation rounds, and
+    the sums of absolute values dq_abs, dk_abs_tok, dv_abs_tok of all terms.
     """
     q_group = np.asarray(q_group, dtype=np.float64)
     dout_group = np.asarray(dout_group, dtype=np.float64)
@@ -106,13 +112,16 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
     dq_abs = np.zeros((G, d))
     dk_abs = np.zeros((len(tok), d))
     dv_abs = np.zeros((len(tok), d))
+    dq_ss = np.zeros((G, d))
+    dk_ss = np.zeros((len(tok), d))
+    dv_ss = np.zeros((len(tok), d))
     dlogp = np.zeros(len(r["blocks"]))
     dlogp_abs = np.zeros(len(r["blocks"]))
     for h in range(G):
         logits = k[tok] @ q_group[h] * scale + bias
         w = np.exp(logits - logits.max())
         P = w / w.sum()
-        o = P @ v[tok]
+        o = P @ v[tok] if out_group is None else np.asarray(out_group[h], dtype=np.float64)
         dP = v[tok] @ dout_group[h]
         dS = P * (dP - dout_group[h] @ o)
         dq[h] += scale * (dS @ k[tok])
@@ -122,6 +131,9 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
         dq_abs[h] += scale * (mag @ np.abs(k[tok]))
         dk_abs += scale * np.outer(mag, np.abs(q_group[h]))
         dv_abs += np.outer(P, np.abs(dout_group[h]))
+        dq_ss[h] += scale * scale * ((dS * dS) @ (k[tok] * k[tok]))
+        dk_ss += scale * scale * np.outer(dS * dS, q_group[h] * q_group[h])
+        dv_ss += np.outer(P * P, dout_group[h] * dout_group[h])
         for e in range(len(dlogp)):
             dlogp[e] += sigma * dS[owner == e].sum()
             dlogp_abs[e] += sigma * mag[owner == e].sum()
@@ -144,21 +156,27 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
             dq_abs[h] += gamma * (dz_abs @ np.abs(summaries[cand]))
             ds_abs += gamma * np.outer(dz_abs, np.abs(q_group[h]))
     return {"dq": dq, "tok": tok, "dk_tok": dk_tok, "dv_tok": dv_tok, "cand": cand, "ds": ds,
-            "dq_abs": dq_abs, "dk_abs_tok": dk_abs, "dv_abs_tok": dv_abs, "ds_abs": ds_abs}
+            "dq_abs": dq_abs, "dk_abs_tok": dk_abs, "dv_abs_tok": dv_abs, "ds_abs": ds_abs,
+            "dq_ss": dq_ss, "dk_ss_tok": dk_ss, "dv_ss_tok": dv_ss}
 
 
 def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout: np.ndarray, alpha: float,
-             block: int, causal: bool = True, sigma: float = 1.0) -> dict:
+             block: int, causal: bool = True, sigma: float = 1.0, out: np.ndarray | None = None) -> dict:
     """Gradients of L = sum(dout * out) for one batch element of the prefill forward.
 
     q, dout: [S, H, d]; k, v: [S, Hkv, d]; w_s: [d, d].  Inputs are promoted
-    to fp64.  Returns dq, dk, dv (shapes of q, k, v) and dw_s [d, d].
+    to fp64.  out: the forward output [S, H, d] the backward consumes for
+    D = dout . out (None: the exact output; see backward_row).  Returns dq,
+    dk, dv (shapes of q, k, v) and dw_s [d, d], plus the term sizes of
+    backward_row summed over the rows (dq_abs, dk_abs, dv_abs and the root
+    sums of squares dq_rss, dk_rss, dv_rss).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     w_s = np.asarray(w_s, dtype=np.float64)
     dout = np.asarray(dout, dtype=np.float64)
+    out = None if out is None else np.asarray(out, dtype=np.float64)
     S, H, d = q.shape
     Hkv = k.shape[1]
     G = H // Hkv
@@ -166,7 +184,8 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     dw_s = np.zeros_like(w_s)
-    mags = {"dq_abs": np.zeros_like(q), "dk_abs": np.zeros_like(k), "dv_abs": np.zeros_like(v)}
+    mags = {"dq_abs": np.zeros_like(q), "dk_abs": np.zeros_like(k), "dv_abs": np.zeros_like(v),
+            "dq_rss": np.zeros_like(q), "dk_rss": np.zeros_like(k), "dv_rss": np.zeros_like(v)}
     n_blocks = -(-S // block)
     for g in range(Hkv):
         kg, vg = k[:, g], v[:, g]
@@ -175,7 +194,8 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
         ds_abs = np.zeros((n_blocks, d))
         for pos in range(S):
             hs = slice(g * G, (g + 1) * G)
-            rb = backward_row(q[pos, hs], kg, vg, summ, dout[pos, hs], pos, S, block, alpha, causal, sigma)
+            rb = backward_row(q[pos, hs], kg, vg, summ, dout[pos, hs], pos, S, block, alpha, causal, sigma,
+                              None if out is None else out[pos, hs])
             dq[pos, hs] = rb["dq"]
             dk[rb["tok"], g] += rb["dk_tok"]
             dv[rb["tok"], g] += rb["dv_tok"]
@@ -184,6 +204,9 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
             mags["dq_abs"][pos, hs] = rb["dq_abs"]
             mags["dk_abs"][rb["tok"], g] += rb["dk_abs_tok"]
             mags["dv_abs"][rb["tok"], g] += rb["dv_abs_tok"]
+            mags["dq_rss"][pos, hs] = rb["dq_ss"]
+            mags["dk_rss"][rb["tok"], g] += rb["dk_ss_tok"]
+            mags["dv_rss"][rb["tok"], g] += rb["dv_ss_tok"]
         # stage 0: s_c = kbar_c W_s over the c's valid tokens
         for c in range(n_blocks):
             lo, hi = c * block, min(S, (c + 1) * block)
@@ -191,6 +214,8 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
             dw_s += np.outer(kbar, ds[c])
             dk[lo:hi, g] += (w_s @ ds[c]) / (hi - lo)
             mags["dk_abs"][lo:hi, g] += (np.abs(w_s) @ ds_abs[c]) / (hi - lo)
+    for name in ("dq_rss", "dk_rss", "dv_rss"):
+        mags[name] = np.sqrt(mags[name])
     return {"dq": dq, "dk": dk, "dv": dv, "dw_s": dw_s, **mags}
 
 

@@ -10,18 +10,20 @@ when every key of a KV head moves by one vector (softmax and entmax are
 shift invariant), so sum_j dk_j = 0; each softmax row sums to one, so
 sum_j dv_j = sum of dout over the rows and the group's heads.
 
-Tolerance, derived from the arithmetic: both sides read the same rounded
-inputs; the kernel rounds P and dS once each to the input type as
-tensor-core operands (unit roundoff u = 2^-8 for bf16, 2^-11 for f16), takes
-D = dout . out from the stored (rounded) forward output, and accumulates in
-fp32.  Each gradient element is a sum of such products, so its error is at
-most about u times the sum of the magnitudes of its terms, which the oracle
-returns alongside the gradients (dq_abs, dk_abs, dv_abs).  The bound is
-2 u times that magnitude (plus 1e-6 of its largest value) element by element.
-It is not a fixed fraction of the gradient: where dS nearly cancels against
-key components shared by a block (sum_j dS_j = 0 exactly), |dq| is much
-smaller than the sum it comes from.  dW_s comes out of the fp32 routing
-gradient and is held to 2e-2 normwise.
+Tolerance, derived from the arithmetic.  Both sides read the same inputs,
+the forward output included: the oracle takes the kernel's forward output
+for D = dout . out, as the backward API does.  What remains is the kernel
+rounding P (for dv) and dS (for dq, dk) once each to the input type as
+tensor-core operands (unit roundoff u = 2^-8 for bf16, 2^-11 for f16), with
+fp32 accumulation.  Round-to-nearest errors of different terms are
+independent and unbiased, so an element's error has a standard deviation of
+at most u / sqrt(3) times the root sum of squares of its rounded terms,
+which the oracle returns (dq_rss, dk_rss, dv_rss).  The bound is 3.5 u times
+that (six standard deviations), plus 2^-16 times the sum of the terms'
+absolute values for fp32 accumulation and the fp32 routing gradient.  An
+emulation of those roundings on the b64_g4 case stays within 3.2 standard
+deviations over 4e5 elements.  dW_s comes out of the fp32 routing gradient
+and is held to 2e-2 normwise.
 """
 
 import numpy as np
@@ -65,13 +67,13 @@ def _close(name, got, ref):
     assert err <= NORM_TOL, f"{name}: normwise {err:.3g}"
 
 
-def _within(name, got, ref, mag, u):
+def _within(name, got, ref, rss, absum, u):
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
-    bound = 2.0 * u * mag + 1e-6 * mag.max()
+    bound = 3.5 * u * rss + 2.0 ** -16 * absum + 1e-7 * absum.max()
     excess = np.abs(got - ref) / bound
     worst = np.unravel_index(np.argmax(excess), excess.shape)
     assert excess.max() <= 1.0, (f"{name}: error {abs(got - ref)[worst]:.3g} at {worst} above the bound "
-                                 f"{bound[worst]:.3g} (magnitude {mag[worst]:.3g})")
+                                 f"{bound[worst]:.3g} (gradient {ref[worst]:.3g})")
 
 
 @pytest.mark.parametrize("case", list(CASES))
@@ -87,9 +89,10 @@ def test_backward_matches_oracle(cuda_lib, case):
     dw_ref = np.zeros((cfg.head_dim, cfg.head_dim))
     for b in range(cfg.batch):
         ref = backward(_np(q[b]), _np(k[b]), _np(v[b]), _np(w_s), _np(dout[b]), cfg.alpha, cfg.block, cfg.causal,
-                       sigma)
+                       sigma, out=_np(out[b]))
         for name in ("dq", "dk", "dv"):
-            _within(f"{case} b{b} {name}", _np(g[name][b]), ref[name], ref[name + "_abs"], UNIT_ROUNDOFF[q.dtype])
+            _within(f"{case} b{b} {name}", _np(g[name][b]), ref[name], ref[name + "_rss"], ref[name + "_abs"],
+                    UNIT_ROUNDOFF[q.dtype])
         dw_ref += ref["dw_s"]
     if cfg.seq > cfg.block:
         _close(f"{case} dw_s", _np(g["dw_s"]), dw_ref)
@@ -142,6 +145,6 @@ def test_backward_full_prefill(cuda_lib):
         for pos in (0, 63, 64, 1000, 16385, cfg.seq - 1):
             hs = slice(kv * G, (kv + 1) * G)
             rb = backward_row(_np(q[0, pos, hs]), kg, vg, summ, _np(dout[0, pos, hs]), pos, cfg.seq, cfg.block,
-                              cfg.alpha, True)
-            _within(f"dq row {pos} KV head {kv}", _np(g["dq"][0, pos, hs]), rb["dq"], rb["dq_abs"],
-                    UNIT_ROUNDOFF[q.dtype])
+                              cfg.alpha, True, out_group=_np(out[0, pos, hs]))
+            _within(f"dq row {pos} KV head {kv}", _np(g["dq"][0, pos, hs]), rb["dq"], np.sqrt(rb["dq_ss"]),
+                    rb["dq_abs"], UNIT_ROUNDOFF[q.dtype])

@@ -174,3 +174,17 @@ def test_backward_magnitudes_bound_the_gradients():
     for name in ("dq", "dk", "dv"):
         assert np.all(g[name + "_abs"] >= np.abs(g[name]) - 1e-12), name
         assert g[name + "_abs"].min() >= 0.0
+
+
+def test_backward_given_exact_output_is_unchanged():
+    # D = dout . out with the exact forward output is the softmax-gradient
+    # identity sum_j P_j dP_j, so passing that output changes nothing; the
+    # root sums of squares are below the absolute sums of the rounded terms
+    q, k, v, w_s, dout = _tiny(17, S=40, H=4, Hkv=2, d=8)
+    out = forward(q, k, v, w_s, 1.5, 8, True)["out"]
+    g0 = backward(q, k, v, w_s, dout, 1.5, 8, True)
+    g1 = backward(q, k, v, w_s, dout, 1.5, 8, True, out=out)
+    for name in ("dq", "dk", "dv", "dw_s"):
+        np.testing.assert_allclose(g1[name], g0[name], atol=1e-12)
+    for name in ("dq", "dv"):
+        assert np.all(g0[name + "_rss"] <= g0[name + "_abs"] + 1e-15)
