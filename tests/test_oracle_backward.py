@@ -188,3 +188,47 @@ def test_backward_given_exact_output_is_unchanged():
         np.testing.assert_allclose(g1[name], g0[name], atol=1e-12)
     for name in ("dq", "dv"):
         assert np.all(g0[name + "_rss"] <= g0[name + "_abs"] + 1e-15)
+
+
+def test_rounding_error_model_behind_the_gpu_tolerance():
+    # The GPU backward rounds P (for dv) and dS (for dq, dk) to bf16 as
+    # tensor-core operands.  Rounding those operands here, in the oracle's
+    # own stage-2 sums, must stay inside the bound the GPU parity test uses:
+    # 3.5 u times the root sum of squares of the rounded terms (u = 2^-8),
+    # i.e. about six standard deviations of independent round-to-nearest errors.
+    from oracle.backward import _attended
+    from oracle.dash_oracle import block_summaries, forward_row
+
+    def bf16(x):
+        return torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+
+    rng = np.random.default_rng(8)
+    S, H, Hkv, d, block = 96, 4, 2, 32, 16
+    q = bf16(rng.normal(scale=0.5, size=(S, H, d)))
+    k = bf16(rng.normal(scale=0.5, size=(S, Hkv, d)))
+    v = bf16(rng.normal(size=(S, Hkv, d)))
+    dout = bf16(rng.normal(size=(S, H, d)))
+    w_s = np.eye(d) + 0.1 * rng.normal(size=(d, d))
+    G, scale, u = H // Hkv, 1.0 / math.sqrt(d), 2.0 ** -8
+    out = bf16(forward(q, k, v, w_s, 1.5, block, True)["out"])
+    ref = backward(q, k, v, w_s, dout, 1.5, block, True, out=out)
+    rounded = {n: np.zeros_like(a) for n, a in (("dq", q), ("dk", k), ("dv", v))}
+    exact = {n: np.zeros_like(a) for n, a in (("dq", q), ("dk", k), ("dv", v))}
+    for g in range(Hkv):
+        summ = block_summaries(k[:, g], w_s, block, S)
+        for pos in range(S):
+            r = forward_row(q[pos, g * G:(g + 1) * G], k[:, g], v[:, g], summ, pos, S, block, 1.5, True)
+            tok, bias, _ = _attended(r, pos, S, block, True, 1.0)
+            for h in range(g * G, (g + 1) * G):
+                lg = k[tok, g] @ q[pos, h] * scale + bias
+                P = np.exp(lg - lg.max())
+                P /= P.sum()
+                dS = P * (v[tok, g] @ dout[pos, h] - dout[pos, h] @ out[pos, h])
+                for acc, Pm, dSm in ((rounded, bf16(P), bf16(dS)), (exact, P, dS)):
+                    acc["dq"][pos, h] += scale * dSm @ k[tok, g]
+                    acc["dk"][tok, g] += scale * np.outer(dSm, q[pos, h])
+                    acc["dv"][tok, g] += np.outer(Pm, dout[pos, h])
+    for name in ("dq", "dk", "dv"):
+        err = np.abs(rounded[name] - exact[name])
+        assert err.max() > 0.0
+        assert np.all(err <= 3.5 * u * ref[name + "_rss"] + 1e-12), name
