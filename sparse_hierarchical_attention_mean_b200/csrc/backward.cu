@@ -31,7 +31,9 @@
 //              the block and stores the block mean for dW_s.
 //   bwd_ws     dW_s = sum over blocks of kbar^T ds.
 // Tiles in shared memory are XOR-swizzled by row (mma_sync.cuh) and filled by
-// cp.async with zero fill past the sequence end.
+// cp.async with zero fill past the sequence end; bwd_row and bwd_key
+// double-buffer what they stream (the next K/V chunk, the next (head, row
+// chunk) item with its rows' statistics) so the copies overlap the MMAs.
 #include "common.cuh"
 #include "internal.h"
 #include "mma_sync.cuh"
