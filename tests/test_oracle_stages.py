@@ -298,3 +298,63 @@ def test_decode_pair_zero_w_s_is_attention_over_context():
     ref = (w / w.sum(axis=1, keepdims=True)) @ v[:L]
     np.testing.assert_allclose(r["out"], ref, atol=1e-12)
     assert len(r["cand"]) == (L - 1) // B
+
+
+def _prior_mask_reference(q_group, k, v, summ, pos, n_tokens, block, alpha, causal, sigma, shift=0):
+    """torch fp64 SDPA with an additive float mask that carries the prior token by token.
+
+    p_bar comes from route_row (pinned on its own) over the candidates' summaries; entry i of
+    that vector belongs to block cand[i].  ``shift`` = 1 instead attaches it to block i, the
+    mistake this reference must catch (it differs from cand[i] once i passes the query's own
+    block in non-causal mode)."""
+    t = pos // block
+    n_blocks = -(-n_tokens // block)
+    cand = list(range(t)) if causal else [c for c in range(n_blocks) if c != t]
+    r = route_row(q_group, summ[cand], alpha)
+    mask = np.full(n_tokens, -np.inf)
+    for i, c in enumerate(cand):
+        owner = i if shift else c
+        if r["pbar"][i] > 0.0:
+            lo, hi = owner * block, min(n_tokens, (owner + 1) * block)
+            mask[lo:hi] = sigma * math.log(r["pbar"][i])
+    last = pos if causal else min(n_tokens, (t + 1) * block) - 1
+    mask[t * block:last + 1] = sigma * (math.log(1.0 / len(cand)) if cand else 0.0)
+    G, d = q_group.shape
+    qq = torch.from_numpy(q_group)[:, None, :]
+    kk = torch.from_numpy(k)[None].expand(G, n_tokens, d)
+    vv = torch.from_numpy(v)[None].expand(G, n_tokens, d)
+    am = torch.from_numpy(mask)[None, None, :].expand(G, 1, n_tokens)
+    return F.scaled_dot_product_attention(qq, kk, vv, attn_mask=am)[:, 0].numpy(), r
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("sigma", [0.5, 1.0, 2.0])
+def test_non_uniform_prior_lands_on_its_block(causal, sigma):
+    """The prior of "Stage 2: prior-induced sparse softmax" with a sparse, non-uniform p_bar:
+    every token of selected block c carries sigma * log p_bar_c, the diagonal block carries
+    sigma * log(1/N), every other token is masked.  forward_row must equal fp64 SDPA with that
+    additive mask, built here by block id from route_row's p_bar."""
+    rng = np.random.default_rng(11)
+    S, G, d, B = 610, 2, 16, 32  # 20 blocks, ragged tail of 2 tokens
+    k, v = rng.normal(size=(S, d)), rng.normal(size=(S, d))
+    dirs = np.linalg.qr(rng.normal(size=(d, 4)))[0].T
+    # planted blocks of graded strength on both sides of the query blocks used below
+    for c, (e, s) in {1: (0, 2.0), 4: (0, 3.0), 6: (1, 2.5), 11: (0, 2.2), 15: (1, 3.5), 17: (0, 2.8)}.items():
+        k[c * B:(c + 1) * B] += s * dirs[e]
+    w = np.eye(d) + 0.1 * rng.normal(size=(d, d))
+    summ = block_summaries(k, w, B, S)
+    q = rng.normal(size=(S, G, d))
+    q[:, 0] += 4.0 * dirs[0]
+    q[:, 1] += 4.0 * dirs[1]
+    checked = 0
+    for pos in (100, 300, 333, 420, 609):
+        r = forward_row(q[pos], k, v, summ, pos, S, B, 1.5, causal, sigma=sigma)
+        ref, rr = _prior_mask_reference(q[pos], k, v, summ, pos, S, B, 1.5, causal, sigma)
+        np.testing.assert_allclose(r["out"], ref, atol=1e-12)
+        sel = rr["pbar"][rr["pbar"] > 0]
+        if len(sel) >= 2 and len(sel) < len(rr["pbar"]) and np.ptp(sel) > 1e-3:
+            checked += 1  # a sparse and non-uniform prior
+            if not causal and pos // B < int(np.nonzero(rr["pbar"])[0].max()) + 1:
+                wrong, _ = _prior_mask_reference(q[pos], k, v, summ, pos, S, B, 1.5, causal, sigma, shift=1)
+                assert np.abs(wrong - ref).max() > 1e-3  # the reference tells the two placements apart
+    assert checked >= 3
