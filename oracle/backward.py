@@ -41,7 +41,7 @@ import math
 
 import numpy as np
 
-from .dash_oracle import block_summaries, forward, forward_row
+from .dash_oracle import block_summaries, candidate_blocks, forward, forward_row, route_row
 
 
 def entmax_vjp(p: np.ndarray, g: np.ndarray, alpha: float) -> np.ndarray:
@@ -79,7 +79,7 @@ def _attended(r: dict, pos: int, n_tokens: int, block: int, causal: bool, sigma:
 
 def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: np.ndarray, dout_group: np.ndarray,
                  pos: int, n_tokens: int, block: int, alpha: float, causal: bool = True, sigma: float = 1.0,
-                 out_group: np.ndarray | None = None) -> dict:
+                 out_group: np.ndarray | None = None, key_span: tuple[int, int] | None = None) -> dict:
     """The contribution of one query position of one KV group to the gradients.
 
     q_group, dout_group: [G, d]; k, v: [L, d] of the KV head; summaries: all
@@ -92,6 +92,11 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
     it, D = dout . out (the softmax-gradient shortcut for sum_j P_j dP_j).
     None takes the exact output, which makes every gradient the exact
     derivative; a given (e.g. rounded) output changes D and nothing else.
+
+    key_span: (lo, hi) to return the dk / dv contributions (and their term
+    sizes) of the attended tokens in [lo, hi) only; None returns all.  The
+    softmax still runs over every attended token, so what is returned is the
+    same as the matching rows of the full result.
 
     Also returns, for error bounds of reduced-precision implementations, the
     sizes of the terms the gradients are sums of (not derivatives): the
@@ -106,37 +111,40 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
     gamma = 1.0 / math.sqrt(d)
     r = forward_row(q_group, k, v, summaries, pos, n_tokens, block, alpha, causal, sigma)
     tok, bias, owner = _attended(r, pos, n_tokens, block, causal, sigma)
+    kt = np.arange(len(tok)) if key_span is None else np.nonzero((tok >= key_span[0]) & (tok < key_span[1]))[0]
     dq = np.zeros((G, d))
-    dk_tok = np.zeros((len(tok), d))
-    dv_tok = np.zeros((len(tok), d))
+    dk_tok = np.zeros((len(kt), d))
+    dv_tok = np.zeros((len(kt), d))
     dq_abs = np.zeros((G, d))
-    dk_abs = np.zeros((len(tok), d))
-    dv_abs = np.zeros((len(tok), d))
+    dk_abs = np.zeros((len(kt), d))
+    dv_abs = np.zeros((len(kt), d))
     dq_ss = np.zeros((G, d))
-    dk_ss = np.zeros((len(tok), d))
-    dv_ss = np.zeros((len(tok), d))
+    dk_ss = np.zeros((len(kt), d))
+    dv_ss = np.zeros((len(kt), d))
     dlogp = np.zeros(len(r["blocks"]))
     dlogp_abs = np.zeros(len(r["blocks"]))
+    k_t, v_t = k[tok], v[tok]  # the attended keys and values, gathered once
+    k_abs, k_sq = np.abs(k_t), k_t * k_t
     for h in range(G):
-        logits = k[tok] @ q_group[h] * scale + bias
+        logits = k_t @ q_group[h] * scale + bias
         w = np.exp(logits - logits.max())
         P = w / w.sum()
-        o = P @ v[tok] if out_group is None else np.asarray(out_group[h], dtype=np.float64)
-        dP = v[tok] @ dout_group[h]
+        o = P @ v_t if out_group is None else np.asarray(out_group[h], dtype=np.float64)
+        dP = v_t @ dout_group[h]
         dS = P * (dP - dout_group[h] @ o)
-        dq[h] += scale * (dS @ k[tok])
-        dk_tok += scale * np.outer(dS, q_group[h])
-        dv_tok += np.outer(P, dout_group[h])
+        dq[h] += scale * (dS @ k_t)
+        dk_tok += scale * np.outer(dS[kt], q_group[h])
+        dv_tok += np.outer(P[kt], dout_group[h])
         mag = np.abs(dS) + P * (np.abs(dout_group[h]) @ np.abs(o))
-        dq_abs[h] += scale * (mag @ np.abs(k[tok]))
-        dk_abs += scale * np.outer(mag, np.abs(q_group[h]))
-        dv_abs += np.outer(P, np.abs(dout_group[h]))
-        dq_ss[h] += scale * scale * ((dS * dS) @ (k[tok] * k[tok]))
-        dk_ss += scale * scale * np.outer(dS * dS, q_group[h] * q_group[h])
-        dv_ss += np.outer(P * P, dout_group[h] * dout_group[h])
-        for e in range(len(dlogp)):
-            dlogp[e] += sigma * dS[owner == e].sum()
-            dlogp_abs[e] += sigma * mag[owner == e].sum()
+        dq_abs[h] += scale * (mag @ k_abs)
+        dk_abs += scale * np.outer(mag[kt], np.abs(q_group[h]))
+        dv_abs += np.outer(P[kt], np.abs(dout_group[h]))
+        dq_ss[h] += scale * scale * ((dS * dS) @ k_sq)
+        dk_ss += scale * scale * np.outer(dS[kt] * dS[kt], q_group[h] * q_group[h])
+        dv_ss += np.outer(P[kt] * P[kt], dout_group[h] * dout_group[h])
+        listed = owner >= 0  # per list entry: the sum over the tokens of its block
+        dlogp += sigma * np.bincount(owner[listed], weights=dS[listed], minlength=len(dlogp))
+        dlogp_abs += sigma * np.bincount(owner[listed], weights=mag[listed], minlength=len(dlogp))
     cand = np.asarray(r["cand"], dtype=np.int64)
     ds = np.zeros((len(cand), d))
     ds_abs = np.zeros((len(cand), d))
@@ -155,7 +163,7 @@ def backward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: n
             dz_abs = u * (gp_abs + (u @ gp_abs) / max(u.sum(), 1e-300))
             dq_abs[h] += gamma * (dz_abs @ np.abs(summaries[cand]))
             ds_abs += gamma * np.outer(dz_abs, np.abs(q_group[h]))
-    return {"dq": dq, "tok": tok, "dk_tok": dk_tok, "dv_tok": dv_tok, "cand": cand, "ds": ds,
+    return {"dq": dq, "tok": tok[kt], "dk_tok": dk_tok, "dv_tok": dv_tok, "cand": cand, "ds": ds,
             "dq_abs": dq_abs, "dk_abs_tok": dk_abs, "dv_abs_tok": dv_abs, "ds_abs": ds_abs,
             "dq_ss": dq_ss, "dk_ss_tok": dk_ss, "dv_ss_tok": dv_ss}
 
@@ -217,6 +225,79 @@ def backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout:
     for name in ("dq_rss", "dk_rss", "dv_rss"):
         mags[name] = np.sqrt(mags[name])
     return {"dq": dq, "dk": dk, "dv": dv, "dw_s": dw_s, **mags}
+
+
+def key_block_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, w_s: np.ndarray, dout: np.ndarray,
+                       out: np.ndarray | None, blocks, block: int, alpha: float, causal: bool = True,
+                       sigma: float = 1.0, rows=None) -> dict:
+    """dk and dv of the tokens of some key blocks of one KV group, from every row that reaches them.
+
+    q, dout (and out, or None for the exact output): [S, G, d] of one KV
+    group; k, v: [S, d].  A key of block c receives gradient from the rows
+    that attend to it (c selected, i.e. p_bar_c > 0, or c the row's own
+    block) and, through stage 0, from the rows whose routing weight of c is
+    non-zero (the same rows: the entmax Jacobian vanishes off the support).
+    Every other row contributes exactly zero, so this is the same sum as
+    :func:`backward` restricted to those tokens.  Rows are routed with
+    route_row first to find the ones that reach a block.
+
+    rows: the query positions to take into account (default: all).  Every
+    returned quantity is a sum over rows, so the results of disjoint row sets
+    add up to the result over their union (callers may split the rows over
+    processes).
+
+    Returns {c: {"dk", "dv", "dk_abs", "dv_abs", "dk_ss", "dv_ss"}}, each
+    [tokens of c, d] (the ``_ss`` entries are the sums of squares of the
+    rounded terms, whose square roots are :func:`backward`'s ``_rss``), and
+    "rows": the number of rows that reached each block.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    w_s = np.asarray(w_s, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    S, G, d = q.shape
+    summ = block_summaries(k, w_s, block, S)
+    res, reached = {}, {}
+    for c in blocks:
+        n = min(S, (c + 1) * block) - c * block
+        res[c] = {name: np.zeros((n, d)) for name in ("dk", "dv", "dk_abs", "dv_abs", "dk_ss", "dv_ss")}
+        res[c]["ds"] = np.zeros(d)
+        res[c]["ds_abs"] = np.zeros(d)
+        reached[c] = 0
+    for pos in (range(S) if rows is None else rows):
+        t, cand = candidate_blocks(pos, block, S, causal)
+        reach = [c for c in blocks if c == t]
+        if any(c in cand for c in blocks):
+            r = route_row(q[pos], summ[cand], alpha)
+            reach += [c for c in blocks if c in cand and r["pbar"][cand.index(c)] > 0.0]
+        if not reach:
+            continue
+        lo, hi = min(reach) * block, min(S, (max(reach) + 1) * block)
+        rb = backward_row(q[pos], k, v, summ, dout[pos], pos, S, block, alpha, causal, sigma,
+                          None if out is None else out[pos], key_span=(lo, hi))
+        for c in reach:
+            reached[c] += 1
+            sel = (rb["tok"] >= c * block) & (rb["tok"] < (c + 1) * block)
+            off = rb["tok"][sel] - c * block
+            rc = res[c]
+            rc["dk"][off] += rb["dk_tok"][sel]
+            rc["dv"][off] += rb["dv_tok"][sel]
+            rc["dk_abs"][off] += rb["dk_abs_tok"][sel]
+            rc["dv_abs"][off] += rb["dv_abs_tok"][sel]
+            rc["dk_ss"][off] += rb["dk_ss_tok"][sel]
+            rc["dv_ss"][off] += rb["dv_ss_tok"][sel]
+            ci = np.nonzero(rb["cand"] == c)[0]
+            if len(ci):
+                rc["ds"] += rb["ds"][ci[0]]
+                rc["ds_abs"] += rb["ds_abs"][ci[0]]
+    for c in blocks:
+        rc = res[c]
+        lo, hi = c * block, min(S, (c + 1) * block)
+        rc["dk"] += (w_s @ rc["ds"]) / (hi - lo)
+        rc["dk_abs"] += (np.abs(w_s) @ rc["ds_abs"]) / (hi - lo)
+    res["rows"] = reached
+    return res
 
 
 def loss(q, k, v, w_s, dout, alpha, block, causal=True, sigma=1.0) -> float:

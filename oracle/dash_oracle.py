@@ -307,7 +307,8 @@ def forward_row(q_group: np.ndarray, k: np.ndarray, v: np.ndarray, summaries: np
     bias.append(np.full(len(span), sigma * beta))
     tok = np.concatenate(tok)
     bias = np.concatenate(bias)
-    out = np.stack([prior_softmax_attend(q_group[h], k[tok], v[tok], bias) for h in range(len(q_group))])
+    k_t, v_t = k[tok], v[tok]  # the attended keys and values, gathered once for the G heads
+    out = np.stack([prior_softmax_attend(q_group[h], k_t, v_t, bias) for h in range(len(q_group))])
     r.update({"blocks": np.array(sel, dtype=np.int64), "cand": cand, "beta": beta, "out": out})
     return r
 

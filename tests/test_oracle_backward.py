@@ -232,3 +232,34 @@ def test_rounding_error_model_behind_the_gpu_tolerance():
         err = np.abs(rounded[name] - exact[name])
         assert err.max() > 0.0
         assert np.all(err <= 3.5 * u * ref[name + "_rss"] + 1e-12), name
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_key_block_backward_is_the_whole_backward_restricted(causal):
+    # the per-block form sums the same row contributions as backward(); rows
+    # that do not reach a block add exactly nothing, so the two agree on the
+    # block's tokens (dk with its stage-0 term, dv, and the term sizes)
+    from oracle.backward import key_block_backward
+
+    S, H, Hkv, d, block = 75, 4, 2, 8, 8  # ragged tail: 75 = 9 * 8 + 3
+    q, k, v, w_s, dout = _tiny(31, S=S, H=H, Hkv=Hkv, d=d)
+    full = backward(q, k, v, w_s, dout, 1.5, block, causal, sigma=1.2)
+    G = H // Hkv
+    for g in range(Hkv):
+        hs = slice(g * G, (g + 1) * G)
+        blocks = [0, 4, 9]
+        kb = key_block_backward(q[:, hs], k[:, g], v[:, g], w_s, dout[:, hs], None, blocks, block, 1.5, causal,
+                                sigma=1.2)
+        for c in blocks:
+            lo, hi = c * block, min(S, (c + 1) * block)
+            for name in ("dk", "dv", "dk_abs", "dv_abs"):
+                np.testing.assert_allclose(kb[c][name], full[name][lo:hi, g], atol=1e-12, err_msg=f"{name} c={c}")
+            for name in ("dk", "dv"):
+                np.testing.assert_allclose(np.sqrt(kb[c][name + "_ss"]), full[name + "_rss"][lo:hi, g], atol=1e-12)
+        assert kb["rows"][0] >= block  # block 0 is reached by its own rows at least
+        # disjoint row sets add up to the whole
+        parts = [key_block_backward(q[:, hs], k[:, g], v[:, g], w_s, dout[:, hs], None, blocks, block, 1.5, causal,
+                                    sigma=1.2, rows=range(r0, S, 3)) for r0 in range(3)]
+        for c in blocks:
+            for name in ("dk", "dv", "dk_ss", "dv_abs"):
+                np.testing.assert_allclose(sum(p[c][name] for p in parts), kb[c][name], atol=1e-12)
