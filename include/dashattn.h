@@ -89,6 +89,21 @@ const char* dash_attn_last_error(void);
 size_t dash_attn_fwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t* k, int block);
 
 /*
+ * Where a dash_attn_fwd / dash_attn_fwd_ex call leaves its stage-0 summaries
+ * and routing lists in its workspace (same q, k and block as the call): byte
+ * offsets from the workspace base of
+ *   summaries [B, Hkv, T, d] fp32,
+ *   idx       [B, Hkv, S, T] int32, each row's selected block ids ascending,
+ *   logp      [B, Hkv, S, T] fp32, log p_bar of those blocks,
+ *   cnt       [B, Hkv, S] int32, the number of valid entries of each row,
+ * with T = ceil(S / block).  Entries of idx / logp past cnt are undefined.
+ * Any offset pointer may be NULL.  Host-only; launches nothing.
+ */
+dash_status_t dash_attn_fwd_workspace_lists(const dash_tensor_t* q, const dash_tensor_t* k, int block,
+                                            size_t* summ_offset, size_t* idx_offset, size_t* logp_offset,
+                                            size_t* cnt_offset);
+
+/*
  * Full prefill forward: stages 0, 1 and 2 ("Stage 0" to "Stage 2" of the
  * cited technical summary) over q [B, S, H, d], k, v [B, S, Hkv, d].
  *   w_s       device fp32 [d, d] row-major; summaries are mean(k) @ w_s.
@@ -100,8 +115,9 @@ size_t dash_attn_fwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t*
  *             its valid tokens) and the own block is included whole.
  *   out       [B, S, H, d], same dtype as q; written once per element.
  *   workspace device buffer of at least dash_attn_fwd_workspace_size()
- *             bytes, 256-byte aligned; its contents on return are the
- *             routing lists of the call (readable with the layout above).
+ *             bytes, 256-byte aligned; on return it holds the call's
+ *             summaries and routing lists, at the offsets that
+ *             dash_attn_fwd_workspace_lists gives.
  */
 dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
                             const float* w_s, float alpha, int block, int causal, dash_tensor_t* out,
@@ -277,6 +293,17 @@ dash_status_t dash_attn_lists_to_mask(const int32_t* idx, const int32_t* cnt, in
  */
 size_t dash_attn_decode_workspace_size(const dash_tensor_t* q, const dash_tensor_t* kcache, int block,
                                        int64_t t_cap);
+
+/*
+ * Where a dash_attn_decode / dash_attn_decode_ex call leaves the routing of
+ * its step in its workspace (same q, kcache, block and t_cap as the call):
+ * byte offsets of idx [B, Hkv, t_cap] int32 (ascending), logp
+ * [B, Hkv, t_cap] fp32 and cnt [B, Hkv] int32.  Any pointer may be NULL.
+ * Host-only; launches nothing.
+ */
+dash_status_t dash_attn_decode_workspace_lists(const dash_tensor_t* q, const dash_tensor_t* kcache, int block,
+                                               int64_t t_cap, size_t* idx_offset, size_t* logp_offset,
+                                               size_t* cnt_offset);
 
 /*
  * One decode step (stages 1 and 2 for a single new query token per

@@ -35,6 +35,8 @@ EXPORTED = (
     "dash_attn_version",
     "dash_attn_last_error",
     "dash_attn_fwd_workspace_size",
+    "dash_attn_fwd_workspace_lists",
+    "dash_attn_decode_workspace_lists",
     "dash_attn_fwd",
     "dash_attn_summarize",
     "dash_attn_summarize_sdpa",
@@ -99,6 +101,8 @@ def _load() -> ctypes.CDLL:
         "dash_attn_version": (i32, []),
         "dash_attn_last_error": (ctypes.c_char_p, []),
         "dash_attn_fwd_workspace_size": (sz, [T, T, i32]),
+        "dash_attn_fwd_workspace_lists": (i32, [T, T, i32, vp, vp, vp, vp]),
+        "dash_attn_decode_workspace_lists": (i32, [T, T, i32, i64, vp, vp, vp]),
         "dash_attn_fwd": (i32, [T, T, T, vp, f32, i32, i32, T, vp, sz, vp]),
         "dash_attn_summarize": (i32, [T, vp, vp, i32, vp, i64, i64, vp]),
         "dash_attn_summarize_sdpa": (i32, [T, vp, vp, vp, i32, vp, i64, i64, vp]),
@@ -332,6 +336,28 @@ def fwd(q, k, v, w_s, alpha: float, block: int, causal: bool = True, out=None, w
     return out
 
 
+def _view(ws: torch.Tensor, offset: int, shape, dtype) -> torch.Tensor:
+    n = 1
+    for e in shape:
+        n *= e
+    nbytes = n * torch.tensor([], dtype=dtype).element_size()
+    return ws[offset:offset + nbytes].view(dtype).view(*shape)
+
+
+def fwd_lists(workspace: torch.Tensor, q: torch.Tensor, k: torch.Tensor, block: int) -> dict:
+    """Views into a fwd workspace of the call's summaries and routing lists (dash_attn_fwd_workspace_lists)."""
+    qd, kd = _desc(q), _desc(k)
+    off = [ctypes.c_size_t() for _ in range(4)]
+    _check(_lib.dash_attn_fwd_workspace_lists(ctypes.byref(qd), ctypes.byref(kd), block,
+                                              *[ctypes.byref(o) for o in off]))
+    B, S, _, d = q.shape
+    Hkv, T = k.shape[2], n_blocks(S, block)
+    return {"summaries": _view(workspace, off[0].value, (B, Hkv, T, d), torch.float32),
+            "idx": _view(workspace, off[1].value, (B, Hkv, S, T), torch.int32),
+            "logp": _view(workspace, off[2].value, (B, Hkv, S, T), torch.float32),
+            "cnt": _view(workspace, off[3].value, (B, Hkv, S), torch.int32)}
+
+
 # ------------------------------------------------------------------ backward
 
 
@@ -414,6 +440,18 @@ def decode(q, kcache, vcache, seqlens, summaries, alpha: float, block: int, out=
     else:
         _check(_lib.dash_attn_decode_ex(*args, opts, _stream(stream)))
     return out
+
+
+def decode_lists(workspace: torch.Tensor, q: torch.Tensor, kcache: torch.Tensor, block: int, t_cap: int) -> dict:
+    """Views into a decode workspace of the step's routing lists (dash_attn_decode_workspace_lists)."""
+    qd, kd = _desc(q), _desc(kcache)
+    off = [ctypes.c_size_t() for _ in range(3)]
+    _check(_lib.dash_attn_decode_workspace_lists(ctypes.byref(qd), ctypes.byref(kd), block, t_cap,
+                                                 *[ctypes.byref(o) for o in off]))
+    B, Hkv = q.shape[0], kcache.shape[2]
+    return {"idx": _view(workspace, off[0].value, (B, Hkv, t_cap), torch.int32),
+            "logp": _view(workspace, off[1].value, (B, Hkv, t_cap), torch.float32),
+            "cnt": _view(workspace, off[2].value, (B, Hkv), torch.int32)}
 
 
 def decode_noalloc(q, kcache, vcache, seqlens, summaries, alpha: float, block: int, out=None,

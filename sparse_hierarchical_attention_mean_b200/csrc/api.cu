@@ -279,6 +279,20 @@ size_t dash_attn_fwd_workspace_size(const dash_tensor_t* q, const dash_tensor_t*
   return fwd_layout(q->b, q->s, q->h, k->h, q->d, block).total;
 }
 
+dash_status_t dash_attn_fwd_workspace_lists(const dash_tensor_t* q, const dash_tensor_t* k, int block,
+                                            size_t* summ_offset, size_t* idx_offset, size_t* logp_offset,
+                                            size_t* cnt_offset) {
+  dash_status_t st;
+  if ((st = check_tensor(q, "q")) || (st = check_tensor(k, "k")) || (st = check_group(q->h, k->h))) return st;
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  const FwdLayout L = fwd_layout(q->b, q->s, q->h, k->h, q->d, block);
+  if (summ_offset) *summ_offset = L.summ;
+  if (idx_offset) *idx_offset = L.idx;
+  if (logp_offset) *logp_offset = L.logp;
+  if (cnt_offset) *cnt_offset = L.cnt;
+  return ok();
+}
+
 dash_status_t dash_attn_summarize(const dash_tensor_t* k, const int32_t* seqlens, const float* w_s, int block,
                                   float* summaries, int64_t t_cap, int64_t first_block, dash_stream_t stream) {
   return dash_attn_summarize_sdpa(k, seqlens, w_s, nullptr, block, summaries, t_cap, first_block, stream);
@@ -746,6 +760,21 @@ size_t dash_attn_decode_workspace_size(const dash_tensor_t* q, const dash_tensor
       check_group(q->h, kcache->h) || t_cap <= 0)
     return 0;
   return decode_layout(q->b, q->h, kcache->h, q->d, block, t_cap).total;
+}
+
+dash_status_t dash_attn_decode_workspace_lists(const dash_tensor_t* q, const dash_tensor_t* kcache, int block,
+                                               int64_t t_cap, size_t* idx_offset, size_t* logp_offset,
+                                               size_t* cnt_offset) {
+  dash_status_t st;
+  if ((st = check_tensor(q, "q")) || (st = check_tensor(kcache, "kcache")) || (st = check_group(q->h, kcache->h)))
+    return st;
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  if (t_cap <= 0) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap must be positive");
+  const DecodeLayout L = decode_layout(q->b, q->h, kcache->h, q->d, block, t_cap);
+  if (idx_offset) *idx_offset = L.idx;
+  if (logp_offset) *logp_offset = L.logp;
+  if (cnt_offset) *cnt_offset = L.cnt;
+  return ok();
 }
 
 dash_status_t dash_attn_decode(const dash_tensor_t* q, const dash_tensor_t* kcache, const dash_tensor_t* vcache,

@@ -1,0 +1,83 @@
+"""Runs oracle row sums in worker processes (spawned, so they never inherit a CUDA context).
+
+Test infrastructure: the workers read the stored inputs from .npy files
+(memory-mapped) and call the oracle on a subset of the query rows; the oracle
+functions used here return sums over rows, which the caller adds up.
+"""
+
+from __future__ import annotations
+
+import multiprocessing as mp
+import os
+
+import numpy as np
+
+
+def _key_block_part(args):
+    from oracle.backward import key_block_backward
+
+    paths, blocks, block, alpha, causal, sigma, rows = args
+    arr = {name: np.load(path, mmap_mode="r") for name, path in paths.items()}
+    return key_block_backward(arr["q"], arr["k"], arr["v"], arr["w_s"], arr["dout"], arr.get("out"), blocks, block,
+                              alpha, causal, sigma, rows=rows)
+
+
+def key_block_backward_pooled(tmpdir, arrays: dict, blocks, block, alpha, causal=True, sigma=1.0, workers=None):
+    """oracle.backward.key_block_backward over all rows, the rows split over spawned processes.
+
+    arrays: q, k, v, w_s, dout and optionally out (numpy, one KV group, see the oracle).
+    Returns the same dict as the oracle, summed over the workers' row sets.
+    """
+    paths = {}
+    for name, a in arrays.items():
+        paths[name] = os.path.join(str(tmpdir), f"{name}.npy")
+        np.save(paths[name], np.ascontiguousarray(a))
+    S = arrays["q"].shape[0]
+    n = workers or max(1, min(24, (os.cpu_count() or 2) - 1))
+    chunks = [range(r0, S, n) for r0 in range(n)]  # interleaved, so late (long) rows spread evenly
+    with mp.get_context("spawn").Pool(n) as pool:
+        parts = pool.map(_key_block_part, [(paths, list(blocks), block, alpha, causal, sigma, ch) for ch in chunks])
+    total = parts[0]
+    for p in parts[1:]:
+        for c in blocks:
+            for name, val in p[c].items():
+                total[c][name] = total[c][name] + val
+            total["rows"][c] += p["rows"][c]
+    return total
+
+
+def _oracle_head_part(args):
+    from tests._parity import oracle_head
+
+    cfg, plan, b, g, rows, kw = args
+    return (b, g), oracle_head(cfg, plan, b, g, rows, **kw)
+
+
+def _oracle_decode_part(args):
+    from tests._parity import oracle_decode_pair
+
+    cfg, plan, b, g, kw = args
+    return (b, g), oracle_decode_pair(cfg, plan, b, g, **kw)
+
+
+def _pool_size(n_tasks: int) -> int:
+    return max(1, min(n_tasks, 24, (os.cpu_count() or 2) - 1))
+
+
+def oracle_heads_pooled(cfg, plan, pairs, rows, qbar_of=None, **kw) -> dict:
+    """tests._parity.oracle_head for every (batch, KV group) in ``pairs``, one task per pair,
+    in spawned processes.  qbar_of: optional {g: learned summary query of KV head g}.
+    Returns {(b, g): (records, summaries)}."""
+    tasks = [(cfg, plan, b, g, list(rows), dict(kw, **({"qbar": qbar_of[g]} if qbar_of else {}))) for b, g in pairs]
+    if len(tasks) == 1:
+        return dict([_oracle_head_part(tasks[0])])
+    with mp.get_context("spawn").Pool(_pool_size(len(tasks))) as pool:
+        return dict(pool.map(_oracle_head_part, tasks, chunksize=1))
+
+
+def oracle_decode_pooled(cfg, plan, pairs, **kw) -> dict:
+    """tests._parity.oracle_decode_pair for every (sequence, KV group) in ``pairs``, in spawned
+    processes.  Returns {(b, g): (record, summaries)}."""
+    tasks = [(cfg, plan, b, g, kw) for b, g in pairs]
+    with mp.get_context("spawn").Pool(_pool_size(len(tasks))) as pool:
+        return dict(pool.map(_oracle_decode_part, tasks, chunksize=1))

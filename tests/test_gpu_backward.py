@@ -4,15 +4,20 @@ Small cases run the whole oracle backward and compare every gradient; they
 span several query and key blocks with a ragged tail, every group size, both
 head dims and block sizes, the three alphas, sigma != 1, non-causal routing,
 a batch of two and a single partial block.  At the full prefill size the
-query gradients of sampled rows are compared with the oracle row by row, and
-dk / dv with two identities that hold at any size: the loss does not change
+query gradients of sampled rows are compared with the oracle row by row, dk
+and dv of the first, a middle and the last key block of one KV head element
+by element (the oracle sums every row that reaches those blocks), and dk / dv
+of every head with two identities that hold at any size: the loss does not change
 when every key of a KV head moves by one vector (softmax and entmax are
 shift invariant), so sum_j dk_j = 0; each softmax row sums to one, so
 sum_j dv_j = sum of dout over the rows and the group's heads.
 
 Tolerance, derived from the arithmetic.  Both sides read the same inputs,
-the forward output included: the oracle takes the kernel's forward output
-for D = dout . out, as the backward API does.  What remains is the kernel
+the forward output included: the backward API takes the forward output as an
+input (it enters D = dout . out), and the oracle is given the same one.  One
+test gives both sides the oracle's own forward output, rounded to the input
+type, so that no value from the GPU enters the oracle; the others give both
+the kernel's forward output, as a user of the API does.  What remains is the kernel
 rounding P (for dv) and dS (for dq, dk) once each to the input type as
 tensor-core operands (unit roundoff u = 2^-8 for bf16, 2^-11 for f16), with
 fp32 accumulation.  Round-to-nearest errors of different terms are
@@ -31,8 +36,10 @@ import pytest
 import torch
 
 from gen import full_inputs, get_config
-from oracle.backward import backward, backward_row
+from oracle.backward import _forward_sigma, backward, backward_row
 from oracle.dash_oracle import block_summaries
+
+from tests._oracle_pool import key_block_backward_pooled
 
 pytestmark = pytest.mark.gpu
 
@@ -100,6 +107,31 @@ def test_backward_matches_oracle(cuda_lib, case):
         assert torch.all(g["dw_s"] == 0)
 
 
+@pytest.mark.parametrize("case", ["b64_g4", "b128_g8_d64_f16_noncausal"])
+def test_backward_on_oracle_forward_output(cuda_lib, case):
+    # the forward output both sides consume is the oracle's (fp64, rounded to
+    # the input type), so nothing computed on the GPU enters the oracle
+    dash = cuda_lib
+    cfg, sigma = CASES[case]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w_s = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    dout = _dout(q)
+    for b in range(cfg.batch):
+        ref_out = _forward_sigma(_np(q[b]), _np(k[b]), _np(v[b]), _np(w_s), cfg.alpha, cfg.block, cfg.causal, sigma)
+        out_b = torch.from_numpy(ref_out).to(q.dtype)
+        out = torch.zeros_like(q)
+        out[b] = out_b.to(q.device)
+        g = dash.bwd(q, k, v, w_s, out, dout, cfg.alpha, cfg.block, cfg.causal, sigma=sigma)
+        torch.cuda.synchronize()
+        ref = backward(_np(q[b]), _np(k[b]), _np(v[b]), _np(w_s), _np(dout[b]), cfg.alpha, cfg.block, cfg.causal,
+                       sigma, out=out_b.double().numpy())
+        for name in ("dq", "dk", "dv"):
+            _within(f"{case} b{b} {name}", _np(g[name][b]), ref[name], ref[name + "_rss"], ref[name + "_abs"],
+                    UNIT_ROUNDOFF[q.dtype])
+        if cfg.batch == 1 and cfg.seq > cfg.block:
+            _close(f"{case} dw_s", _np(g["dw_s"]), ref["dw_s"])
+
+
 def test_backward_autograd_wrapper(cuda_lib):
     # torch.autograd through the library: the wrapper returns the same gradients
     dash = cuda_lib
@@ -118,9 +150,10 @@ def test_backward_autograd_wrapper(cuda_lib):
     assert torch.equal(w_s.grad, g["dw_s"])
 
 
-def test_backward_full_prefill(cuda_lib):
-    # the full prefill workload: sampled rows' dq against the oracle, and the
-    # two identities for dk and dv over every KV head
+def test_backward_full_prefill(cuda_lib, tmp_path):
+    # the full prefill workload: sampled rows' dq against the oracle, dk / dv
+    # of three key blocks of KV head 0 element by element, and the two
+    # identities for dk and dv over every KV head
     dash = cuda_lib
     cfg = get_config("prefill")
     inp = full_inputs(cfg, device="cuda")
@@ -148,3 +181,17 @@ def test_backward_full_prefill(cuda_lib):
                               cfg.alpha, True, out_group=_np(out[0, pos, hs]))
             _within(f"dq row {pos} KV head {kv}", _np(g["dq"][0, pos, hs]), rb["dq"], np.sqrt(rb["dq_ss"]),
                     rb["dq_abs"], UNIT_ROUNDOFF[q.dtype])
+    # dk / dv of the first, a middle and the last key block of KV head 0, from
+    # every row that reaches them (the same forward output on both sides)
+    kv, hs = 0, slice(0, G)
+    blocks = [0, cfg.n_blocks // 2, cfg.n_blocks - 1]
+    arrays = {"q": _np(q[0, :, hs]).astype(np.float32), "k": _np(k[0, :, kv]).astype(np.float32),
+              "v": _np(v[0, :, kv]).astype(np.float32), "w_s": _np(w_s), "dout": _np(dout[0, :, hs]).astype(np.float32),
+              "out": _np(out[0, :, hs]).astype(np.float32)}
+    kb = key_block_backward_pooled(tmp_path, arrays, blocks, cfg.block, cfg.alpha, True)
+    assert kb["rows"][blocks[-1]] == cfg.block and kb["rows"][0] > cfg.block
+    for c in blocks:
+        lo, hi = c * cfg.block, (c + 1) * cfg.block
+        for name in ("dk", "dv"):
+            _within(f"{name} key block {c} KV head {kv}", _np(g[name][0, lo:hi, kv]), kb[c][name],
+                    np.sqrt(kb[c][name + "_ss"]), kb[c][name + "_abs"], UNIT_ROUNDOFF[q.dtype])

@@ -1,15 +1,17 @@
 """GPU parity at the full workload sizes, in the launch configuration the
 benchmark times (one ``fwd`` / ``decode`` call over the whole batch with a
 caller-owned workspace), checked on sampled rows that the fp64 oracle
-computes one by one:
+computes one by one.  The summaries and routing lists checked are the ones
+the timed call itself produced and left in its workspace (read at the
+offsets the library reports), not those of a separate routing call:
 
   * prefill 32K (B=1, 32/8 heads, d=128, bf16, block 64): every 97th row,
     the first and last two blocks whole, the first and last row of every
     block, for the first and last KV group;
   * long prefill 128K (block 128, diffuse and needle KV heads): a sparser
     sample, one diffuse and one needle group;
-  * decode (64 sequences, 64K..128K context): a spread of (sequence, KV head)
-    pairs;
+  * decode (64 sequences, 64K..128K context): 40 (sequence, KV head) pairs
+    spread over the batch and every KV head;
   * the alpha x plant-strength sweep (B=4, 16/16 heads, d=64, f16).
 
 Same rules as the small-size tests: identical selected sets outside the
@@ -21,7 +23,8 @@ import pytest
 import torch
 
 from gen import full_inputs, get_config, sample_rows, sweep_configs
-from tests._parity import OUT_TOL, check_route_row, max_abs, oracle_decode_pair, oracle_head
+from tests._oracle_pool import oracle_decode_pooled, oracle_heads_pooled
+from tests._parity import OUT_TOL, check_route_row, max_abs
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -39,27 +42,27 @@ def _bench_fwd(dash, cfg, inp):
     dash.fwd(q, k, v, w, cfg.alpha, cfg.block, cfg.causal, out=out, workspace=ws)
     torch.cuda.synchronize()
     assert dash.device_status(ws) == 0
-    return out
+    return out, ws
 
 
 def _check_prefill(dash, cfg, batches, groups, rows):
     inp = full_inputs(cfg, device="cuda")
-    out = _bench_fwd(dash, cfg, inp)
-    summ = dash.summarize(inp["k"], inp["w_s"], cfg.block)
-    rt = dash.route(inp["q"], summ, cfg.alpha, cfg.block, cfg.causal)
-    torch.cuda.synchronize()
+    out, ws = _bench_fwd(dash, cfg, inp)
+    lists = dash.fwd_lists(ws, inp["q"], inp["k"], cfg.block)  # what the timed call routed with
+    summ, idx_all, logp_all, cnt_all = lists["summaries"], lists["idx"], lists["logp"], lists["cnt"]
     rsel = torch.tensor(rows, device="cuda")
     G = cfg.group
     tol = OUT_TOL[cfg.dtype]
     worst = 0.0
+    ref = oracle_heads_pooled(cfg, inp["plan"], [(b, g) for b in batches for g in groups], rows)
     for b in batches:
         for g in groups:
-            recs, summ_o = oracle_head(cfg, inp["plan"], b, g, rows)
+            recs, summ_o = ref[(b, g)]
             serr = np.abs(summ[b, g, : len(summ_o)].cpu().numpy() - summ_o).max()
             assert serr <= 2e-5 * max(1.0, np.abs(summ_o).max()), f"{cfg.name}: summary error {serr:.3g}"
-            idx = rt["idx"][b, g].index_select(0, rsel).cpu().numpy()
-            logp = rt["logp"][b, g].index_select(0, rsel).cpu().numpy()
-            cnt = rt["cnt"][b, g].index_select(0, rsel).cpu().numpy()
+            idx = idx_all[b, g].index_select(0, rsel).cpu().numpy()
+            logp = logp_all[b, g].index_select(0, rsel).cpu().numpy()
+            cnt = cnt_all[b, g].index_select(0, rsel).cpu().numpy()
             o = out[b, :, g * G:(g + 1) * G].index_select(0, rsel).double().cpu().numpy()
             for i, (pos, rec) in enumerate(zip(rows, recs)):
                 where = f"{cfg.name} b{b} g{g} pos{pos}"
@@ -67,7 +70,7 @@ def _check_prefill(dash, cfg, batches, groups, rows):
                 err = max_abs(o[i], rec["out"])
                 worst = max(worst, err)
                 assert err <= tol, f"{where}: output error {err:.3g} > {tol}"
-    del inp, out, summ, rt
+    del inp, out, ws, lists, summ, idx_all, logp_all, cnt_all
     torch.cuda.empty_cache()
     return worst
 
@@ -109,19 +112,23 @@ def test_decode_full_sampled(dash):
     out = torch.empty_like(q)
     ws = torch.empty(dash.decode_workspace_size(q, k, cfg.block, T), dtype=torch.uint8, device="cuda")
     dash.decode(q, k, v, sl, summ, cfg.alpha, cfg.block, out=out, workspace=ws)
-    rt = dash.route(q, summ, cfg.alpha, cfg.block, True, seqlens=sl)
     torch.cuda.synchronize()
     assert dash.device_status(ws) == 0
+    lists = dash.decode_lists(ws, q, k, cfg.block, T)  # the routing the timed step used
     G = cfg.group
     tol = OUT_TOL[cfg.dtype]
     worst = 0.0
-    for b, g in ((0, 0), (17, 3), (42, 5), (63, 7)):
-        rec, summ_o = oracle_decode_pair(cfg, inp["plan"], b, g)
+    # 40 pairs: every KV head five times, sequences spread over the batch
+    pairs = [((7 * i + 3 * (i // cfg.kv_heads)) % cfg.batch, i % cfg.kv_heads) for i in range(40)]
+    assert len(set(pairs)) == 40
+    ref = oracle_decode_pooled(cfg, inp["plan"], pairs)
+    for b, g in pairs:
+        rec, summ_o = ref[(b, g)]
         serr = np.abs(summ[b, g, : len(summ_o)].cpu().numpy() - summ_o).max()
         assert serr <= 2e-5 * max(1.0, np.abs(summ_o).max())
         where = f"decode b{b} g{g} L{int(inp['plan'].seqlens[b])}"
-        check_route_row(rec, rt["idx"][b, g, 0].cpu().numpy(), rt["logp"][b, g, 0].cpu().numpy(),
-                        rt["cnt"][b, g, 0].cpu().numpy(), where)
+        check_route_row(rec, lists["idx"][b, g].cpu().numpy(), lists["logp"][b, g].cpu().numpy(),
+                        lists["cnt"][b, g].cpu().numpy(), where)
         err = max_abs(out[b, 0, g * G:(g + 1) * G].double().cpu().numpy(), rec["out"])
         worst = max(worst, err)
         assert err <= tol, f"{where}: output error {err:.3g}"

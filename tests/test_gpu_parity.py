@@ -13,6 +13,7 @@ import torch
 
 from gen import Config, full_inputs, get_config, kv_values, make_plan
 from oracle.dash_oracle import block_summaries, block_summaries_sdpa, lists_to_mask
+from tests._oracle_pool import oracle_heads_pooled
 from tests._parity import (
     OUT_TOL,
     check_p_dense,
@@ -45,7 +46,7 @@ for a in (1.25, 1.5, 2.0):
 
 
 def _kv_subset(cfg):
-    return sorted({0, cfg.kv_heads - 1})
+    return list(range(cfg.kv_heads))  # every KV group
 
 
 @pytest.fixture(scope="module")
@@ -56,11 +57,13 @@ def dash(cuda_lib):
 def _run_all(dash, cfg):
     inp = full_inputs(cfg, device="cuda")
     q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
-    out = dash.fwd(q, k, v, w, cfg.alpha, cfg.block, cfg.causal)
+    ws = torch.empty(dash.fwd_workspace_size(q, k, cfg.block), dtype=torch.uint8, device="cuda")
+    out = dash.fwd(q, k, v, w, cfg.alpha, cfg.block, cfg.causal, workspace=ws)
+    fl = dash.fwd_lists(ws, q, k, cfg.block)  # the lists the forward itself routed with
     summ = dash.summarize(k, w, cfg.block)
     rt = dash.route(q, summ, cfg.alpha, cfg.block, cfg.causal, want_tau=True, want_p=True)
     torch.cuda.synchronize()
-    return inp, out, summ, rt
+    return inp, out, summ, rt, fl
 
 
 def test_generator_identical_on_gpu(dash):
@@ -74,25 +77,28 @@ def test_generator_identical_on_gpu(dash):
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_forward_parity_small(dash, name):
     cfg = SMALL[name]
-    inp, out, summ, rt = _run_all(dash, cfg)
+    inp, out, summ, rt, fl = _run_all(dash, cfg)
     plan = inp["plan"]
     G = cfg.group
     tol = OUT_TOL[cfg.dtype]
     out_np = to_np(out)
     summ_np = summ.cpu().numpy()
     idx, logp, cnt = rt["idx"].cpu().numpy(), rt["logp"].cpu().numpy(), rt["cnt"].cpu().numpy()
+    f_idx, f_logp, f_cnt = fl["idx"].cpu().numpy(), fl["logp"].cpu().numpy(), fl["cnt"].cpu().numpy()
     p_dense, tau = rt["p"].cpu().numpy(), rt["tau"].cpu().numpy()
     rows = list(range(cfg.seq))
     worst_out = worst_p = 0.0
+    ref = oracle_heads_pooled(cfg, plan, [(b, g) for b in range(cfg.batch) for g in _kv_subset(cfg)], rows)
     for b in range(cfg.batch):
         for g in _kv_subset(cfg):
-            recs, summ_o = oracle_head(cfg, plan, b, g, rows)
+            recs, summ_o = ref[(b, g)]
             # stage 0
             serr = np.abs(summ_np[b, g, : len(summ_o)] - summ_o).max()
             assert serr <= 2e-5 * max(1.0, np.abs(summ_o).max()), f"{name}: summary error {serr:.3g}"
             for pos, rec in zip(rows, recs):
                 where = f"{name} b{b} g{g} pos{pos}"
                 check_route_row(rec, idx[b, g, pos], logp[b, g, pos], cnt[b, g, pos], where)
+                check_route_row(rec, f_idx[b, g, pos], f_logp[b, g, pos], f_cnt[b, g, pos], where + " (fwd)")
                 e = check_p_dense(rec, p_dense[b, g * G:(g + 1) * G, pos], tau[b, g * G:(g + 1) * G, pos], where)
                 worst_p = max(worst_p, e)
                 err = max_abs(out_np[b, pos, g * G:(g + 1) * G], rec["out"])
@@ -183,9 +189,11 @@ def test_forward_options(dash, name, sigma, qscale):
     G, tol = cfg.group, OUT_TOL[cfg.dtype]
     out_np = to_np(out)
     rows = list(range(cfg.seq))
+    ref = oracle_heads_pooled(cfg, plan, [(0, g) for g in _kv_subset(cfg)], rows, sigma=sigma,
+                              qbar_of=None if qbar is None else {g: qbar[g].double().numpy()
+                                                                 for g in _kv_subset(cfg)})
     for g in _kv_subset(cfg):
-        recs, _ = oracle_head(cfg, plan, 0, g, rows, sigma=sigma,
-                              qbar=None if qbar is None else qbar[g].double().numpy())
+        recs, _ = ref[(0, g)]
         for pos, rec in zip(rows, recs):
             err = max_abs(out_np[0, pos, g * G:(g + 1) * G], rec["out"])
             assert err <= tol, f"{name} sigma {sigma} g{g} pos{pos}: output error {err:.3g}"
