@@ -210,70 +210,103 @@ def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
 
 
 def prefill_work(cfg, cnt: torch.Tensor):
-    """Selected FLOPs and union-inflated FLOPs of stage 2 from the routing counts."""
+    """Selected stage-2 FLOPs from the routing counts cnt [B, Hkv, S] (causal):
+    4 d G (block |support| + diagonal tokens) summed over the rows."""
     S, block, d, G = cfg.seq, cfg.block, cfg.head_dim, cfg.group
     pos = torch.arange(S, device=cnt.device)
     diag = (pos - (pos // block) * block + 1).double()  # causal diagonal tokens per row
     sel_tokens = cnt.double() * block + diag  # [B, Hkv, S]
-    flops = 4.0 * d * G * float(sel_tokens.sum())
-    return flops
+    return 4.0 * d * G * float(sel_tokens.sum())
 
 
-def union_flops(cfg, idx: torch.Tensor, cnt: torch.Tensor, tile_pos: int) -> float:
+def union_flops(cfg, idx: torch.Tensor, cnt: torch.Tensor) -> float:
+    """FLOPs the tile-pair stage-2 kernel executes: each tile of 128 / G positions (128 rows)
+    runs every block in the union of its rows' lists plus its own blocks (64-token steps up
+    to its last position), for all of its rows."""
     B, Hkv, S, T = idx.shape
-    mask = torch.zeros((B, Hkv, S, T + 1), dtype=torch.bool, device=idx.device)
+    P = 128 // cfg.group
+    n_tiles = -(-S // P)
+    blk = cfg.block
+    union_blocks = 0.0
+    own_tokens = 0.0
     ar = torch.arange(T, device=idx.device)
-    valid = ar[None, None, None, :] < cnt[..., None]
-    tgt = torch.where(valid, idx.long(), torch.full_like(idx.long(), T))
-    mask.scatter_(3, tgt, True)
-    mask = mask[..., :T]
-    n_tiles = S // tile_pos
-    tiles = mask[:, :, : n_tiles * tile_pos].view(B, Hkv, n_tiles, tile_pos, T).any(3)
-    rows = tile_pos * cfg.group
-    diag_tokens = 0.0
+    chunk = max(1, 16384 // P)  # tiles per pass (bounds the temporary mask)
+    for t0 in range(0, n_tiles, chunk):
+        t1 = min(n_tiles, t0 + chunk)
+        lo, hi = t0 * P, min(S, t1 * P)
+        sub_idx, sub_cnt = idx[:, :, lo:hi], cnt[:, :, lo:hi]
+        mask = torch.zeros((B, Hkv, (t1 - t0) * P, T + 1), dtype=torch.bool, device=idx.device)
+        tgt = torch.where(ar < sub_cnt[..., None], sub_idx.long(), T)
+        mask[:, :, : hi - lo].scatter_(3, tgt, True)
+        tiles = mask[..., :T].view(B, Hkv, t1 - t0, P, T).any(3)
+        for tl in range(t0, t1):  # own blocks are counted below, once
+            a, b = tl * P, min(S, tl * P + P) - 1
+            tiles[:, :, tl - t0, a // blk:b // blk + 1] = False
+        union_blocks += float(tiles.sum())
+        del mask, tgt, tiles
     for tl in range(n_tiles):
-        last = tl * tile_pos + tile_pos - 1
-        diag_tokens += (last - (last // cfg.block) * cfg.block) // 64 * 64 + 64
-    per_bg = float(tiles.sum()) * cfg.block + B * Hkv * diag_tokens
-    return 4.0 * cfg.head_dim * rows * per_bg
+        a, b = tl * P, min(S, tl * P + P) - 1
+        for c in range(a // blk, b // blk + 1):
+            last = min(b, (c + 1) * blk - 1)
+            own_tokens += -(-(last - c * blk + 1) // 64) * 64
+    tokens = union_blocks * blk + B * Hkv * own_tokens
+    return 4.0 * cfg.head_dim * 128 * tokens
 
 
-def run_prefill(dash, cfg, steps, warmup, world, rank, pk, do_backward=True):
+def measure_forward(dash, cfg, steps, warmup, world, rank, clocks=False):
+    """Times one prefill workload through dash_attn_fwd (the whole forward, CUDA events around
+    `steps` back-to-back calls, max over ranks), then the same work stage by stage, and the
+    stage-2 entry point alone (the dominant kernel).  Work counts come from the routing lists
+    the timed forward left in its workspace."""
     inp = full_inputs(cfg, device="cuda", seed=rank_seed(cfg, rank))
     q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
     B, S, H, d = q.shape
-    T = -(-S // cfg.block)
     out = torch.empty_like(q)
     ws = torch.empty(dash.fwd_workspace_size(q, k, cfg.block), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():
-        dash.fwd(q, k, v, w, cfg.alpha, cfg.block, True, out=out, workspace=ws)
+        dash.fwd(q, k, v, w, cfg.alpha, cfg.block, cfg.causal, out=out, workspace=ws)
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for _ in range(warmup):
-            step()
-        torch.cuda.synchronize()
-        barrier(world)
-        torch.cuda.synchronize()
+    clk = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if clk:
+        clk.__enter__()
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    if clk:
         clk.mark()
-        ev0.record(stream)
-        for _ in range(steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__(None, None, None)
     barrier(world)
     torch.cuda.synchronize()
     ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, world)
     status = dash.device_status(ws)
 
-    # per-stage timing of the same work through the stage entry points
-    summ = torch.empty((B, k.shape[2], T, d), dtype=torch.float32, device="cuda")
-    idx = torch.empty((B, k.shape[2], S, T), dtype=torch.int32, device="cuda")
-    logp = torch.empty((B, k.shape[2], S, T), dtype=torch.float32, device="cuda")
-    cnt = torch.empty((B, k.shape[2], S), dtype=torch.int32, device="cuda")
+    # the routing the timed forward used (views into its workspace)
+    lists = dash.fwd_lists(ws, q, k, cfg.block)
+    summ, idx, logp, cnt = lists["summaries"], lists["idx"], lists["logp"], lists["cnt"]
+    flops = prefill_work(cfg, cnt)
+    uflops = union_flops(cfg, idx, cnt)
+    pos = torch.arange(S, device="cuda")
+    cand_row = (pos // cfg.block).double()
+    per_head_cand = float(cand_row.sum()) * B
+    per_head_sel = cnt.double().sum(dim=(0, 2))  # [Hkv]
+    head_sparsity = (1.0 - per_head_sel / per_head_cand).tolist()
+    sparsity = 1.0 - float(per_head_sel.sum()) / (per_head_cand * k.shape[2])
+
+    # stage by stage through the stage entry points, writing into the same buffers
+    T = idx.shape[-1]
     sws = torch.empty(dash.sparse_workspace_size(q, k, cfg.block, T), dtype=torch.uint8, device="cuda")
+    rws = torch.empty(dash.route_workspace_size(q, k.shape[2], T, False), dtype=torch.uint8, device="cuda")
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     seg = np.zeros(3)
 
@@ -283,10 +316,10 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk, do_backward=True):
         dash.summarize(k, w, cfg.block, summaries=summ)
         if record:
             evs[1].record(stream)
-        dash.route(q, summ, cfg.alpha, cfg.block, True, idx=idx, logp=logp, cnt=cnt)
+        dash.route(q, summ, cfg.alpha, cfg.block, cfg.causal, idx=idx, logp=logp, cnt=cnt, workspace=rws)
         if record:
             evs[2].record(stream)
-        dash.sparse(q, k, v, idx, logp, cnt, cfg.block, True, out=out, workspace=sws)
+        dash.sparse(q, k, v, idx, logp, cnt, cfg.block, cfg.causal, out=out, workspace=sws)
         if record:
             evs[3].record(stream)
 
@@ -299,41 +332,91 @@ def run_prefill(dash, cfg, steps, warmup, world, rank, pk, do_backward=True):
         seg += [evs[i].elapsed_time(evs[i + 1]) for i in range(3)]
     seg /= steps
 
-    # the dominant kernel alone: stage 2 (its pair-list kernel and the tcgen05
-    # attention kernel) launched back to back on the same stream, CUDA events
-    # around the loop, so host time between launches stays hidden
+    # the dominant kernel alone: stage 2 (pair-list kernel + tcgen05 attention kernel)
+    # launched back to back on the same stream, CUDA events around the loop
     for _ in range(warmup):
-        dash.sparse(q, k, v, idx, logp, cnt, cfg.block, True, out=out, workspace=sws)
+        dash.sparse(q, k, v, idx, logp, cnt, cfg.block, cfg.causal, out=out, workspace=sws)
     torch.cuda.synchronize()
     evs[0].record(stream)
     for _ in range(steps):
-        dash.sparse(q, k, v, idx, logp, cnt, cfg.block, True, out=out, workspace=sws)
+        dash.sparse(q, k, v, idx, logp, cnt, cfg.block, cfg.causal, out=out, workspace=sws)
     evs[1].record(stream)
     torch.cuda.synchronize()
-    sparse_ms = evs[0].elapsed_time(evs[1]) / steps
+    sparse_ms = max_over_ranks(evs[0].elapsed_time(evs[1]) / steps, world)
+    del sws, rws, lists, summ, idx, logp, cnt
+    return {"inp": inp, "out": out, "ws": ws, "ms": ms, "tokens": B * S, "status": status,
+            "seg_ms": seg.tolist(), "sparse_ms": sparse_ms, "flops": flops, "union_flops": uflops,
+            "sparsity": sparsity, "head_sparsity": head_sparsity,
+            "achieved_tflops": flops / (sparse_ms * 1e-3) / 1e12, "clocks": clk.summary() if clk else None}
 
-    flops = prefill_work(cfg, cnt)
-    tile_pos = 128 // cfg.group if 128 // cfg.group < cfg.block else cfg.block
-    uflops = union_flops(cfg, idx, cnt, tile_pos)
-    cand = float(sum((p // cfg.block) for p in range(S))) * k.shape[2] * B
-    sparsity = 1.0 - float(cnt.double().sum()) / cand
-    achieved = flops / (sparse_ms * 1e-3) / 1e12
-    traffic = profiled_traffic("sparse_prefill_tc_kernel", ["attn_prefill_tc.cu", "tc.cuh", "sparse_common.cuh", "common.cuh"])
 
+def run_prefill(dash, cfg, steps, warmup, world, rank, pk, do_backward=True):
+    m = measure_forward(dash, cfg, steps, warmup, world, rank, clocks=True)
+    q, k, v, w = m["inp"]["q"], m["inp"]["k"], m["inp"]["v"], m["inp"]["w_s"]
+    traffic = profiled_traffic("sparse_prefill_tc_kernel", ["attn_prefill_tc.cu", "tc.cuh", "sparse_common.cuh",
+                                                            "common.cuh"])
     # End to end through the public API with host buffers: every step copies
     # its inputs from pinned host memory and reads its output back.  Copies
     # run on their own streams, double-buffered, so step i+1's upload and
     # step i-1's download overlap step i's kernels.
-    e2e_ms, h2d, d2h = run_e2e(dash, cfg, q, k, v, w, ws, steps, warmup, world)
+    e2e_ms, h2d, d2h = run_e2e(dash, cfg, q, k, v, w, m["ws"], steps, warmup, world)
+    ws = m.pop("ws")
     del ws
-    bwd = run_backward(dash, cfg, q, k, v, w, out, min(steps, 5), warmup, flops, world) if do_backward else None
+    bwd = run_backward(dash, cfg, q, k, v, w, m["out"], min(steps, 5), warmup, m["flops"], world) \
+        if do_backward else None
+    m.update({"traffic": traffic, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "backward": bwd})
+    del m["inp"], m["out"]
+    return m
 
-    return {
-        "ms": ms, "tokens": B * S, "status": status, "seg_ms": seg.tolist(), "sparse_ms": sparse_ms, "flops": flops,
-        "union_flops": uflops,
-        "sparsity": sparsity, "achieved_tflops": achieved, "traffic": traffic, "clocks": clk.summary(),
-        "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "backward": bwd,
+
+def prefill_object(m, cfg, pk, world, extra=None):
+    """Summary of one measured prefill workload (tokens/s, stages, sparsity, stage-2 roofline)."""
+    peak = pk["bf16_tflops"]
+    obj = {
+        "tokens_per_s": job_throughput(m["tokens"], world, m["ms"]), "ms_per_step": m["ms"],
+        "stage_ms": {"pool": m["seg_ms"][0], "route": m["seg_ms"][1], "sparse_attention": m["seg_ms"][2]},
+        "sparsity": m["sparsity"], "union_inflation": m["union_flops"] / m["flops"],
+        "roofline": {"kernel": "stage-2 entry point (pair lists + sparse_prefill_tc_kernel) back to back",
+                     "bound": "tensor", "ms_per_launch": m["sparse_ms"], "achieved": m["achieved_tflops"],
+                     "peak": peak, "unit": "TFLOP/s", "frac": m["achieved_tflops"] / peak, "traffic": None,
+                     "selected_flops": m["flops"], "peak_source": f"{pk['source']} bf16 (burst)"},
+        "device_status": m["status"],
     }
+    if extra:
+        obj.update(extra)
+    return obj
+
+
+def run_long_prefill(dash, steps, warmup, world, rank, pk):
+    cfg = get_config("long_prefill")
+    m = measure_forward(dash, cfg, steps, warmup, world, rank)
+    hs = m["head_sparsity"]
+    obj = prefill_object(m, cfg, pk, world, {
+        "workload": "long prefill: B=1, S=131072, 32/8 heads, d=128, bf16, causal, block 128 (1024 blocks), "
+                    "alpha 1.5; KV heads 0-3 diffuse (no plant), 4-7 needle heads (1-16 planted blocks per topic)",
+        "sparsity_per_kv_head": hs,
+        "sparsity_diffuse_heads": float(np.mean(hs[:4])), "sparsity_needle_heads": float(np.mean(hs[4:])),
+        "steps": steps,
+    })
+    del m
+    torch.cuda.empty_cache()
+    return obj
+
+
+def run_sweep(dash, steps, warmup, world, rank, pk):
+    from gen import sweep_configs
+
+    points = []
+    for cfg in sweep_configs():
+        m = measure_forward(dash, cfg, steps, warmup, world, rank)
+        o = prefill_object(m, cfg, pk, world, {"alpha": cfg.alpha, "key_strength": cfg.key_strength})
+        o["roofline"]["peak_source"] = f"{pk['source']} bf16 (burst); f16 has the same dense rate"
+        points.append(o)
+        del m
+        torch.cuda.empty_cache()
+    return {"workload": "alpha / sparsity sweep: B=4, 16/16 heads, d=64, f16, S=16384, causal, block 64, "
+                        "16 topics; alpha in {1.25, 1.5, 2}, key plant strength in {0, 1, 2, 4}",
+            "steps": steps, "points": points}
 
 
 def run_backward(dash, cfg, q, k, v, w, out, steps, warmup, fwd_flops, world):
@@ -493,13 +576,14 @@ def run_decode(dash, cfg, steps, warmup, world, rank):
 # --------------------------------------------------------------------------- oracle timing
 
 
-def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0, groups=None) -> dict:
-    """Times the oracle on a bounded sample of the prefill workload on this host.
+def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0, groups=None, row_offset: int = 0) -> dict:
+    """Times the oracle on a bounded sample of the prefill workload on this host, one thread.
 
     For each sampled KV group (default: all): pooling of the whole sequence
     once, then the routing and sparse attention of ``n_rows`` evenly spread
-    query positions.  Returns the full-sequence time (all KV groups and
-    positions) extrapolated from the sample, and tokens/s.
+    query positions (shifted by ``row_offset``).  Returns the full-sequence
+    time (all KV groups and positions) extrapolated from the sample, and
+    tokens/s.
     """
     from threadpoolctl import threadpool_limits
 
@@ -507,7 +591,7 @@ def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0, groups=
 
     plan = make_plan(cfg, seed)
     G = cfg.group
-    rows = np.linspace(cfg.block, cfg.seq - 1, n_rows).astype(int).tolist()
+    rows = (np.linspace(cfg.block, cfg.seq - 1 - cfg.block, n_rows).astype(int) + row_offset % cfg.block).tolist()
     pool_t = row_t = 0.0
     n_done = 0
     t_start = time.perf_counter()
@@ -530,9 +614,57 @@ def oracle_sample_time(cfg, n_rows: int, budget_s: float, seed: int = 0, groups=
     per_row = row_t / max(n_done, 1)  # one position of one KV group (G heads)
     full_s = pool_t / len(groups) * cfg.kv_heads + per_row * cfg.seq * cfg.kv_heads
     return {"full_s": full_s, "tokens_per_s": cfg.seq / full_s, "rows": n_done, "wall_s": time.perf_counter() - t_start,
+            "pool_s": pool_t, "row_s": row_t, "n_groups": len(groups),
             "sample": f"{n_done} (position, KV group) rows spread over the {cfg.seq}-token sequence + pooling of "
                       f"{len(groups)} of {cfg.kv_heads} KV heads, extrapolated to {cfg.seq} positions x "
                       f"{cfg.kv_heads} groups"}
+
+
+def _oracle_worker(args):
+    cfg, n_rows, budget_s, seed, g, offset = args
+    return oracle_sample_time(cfg, n_rows, budget_s, seed, groups=[g], row_offset=offset)
+
+
+def host_info() -> dict:
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+class OraclePool:
+    """The oracle run by one single-threaded process per host core, up to 64 (spawned, so no worker
+    inherits a CUDA context).  Each process times its own sample (the oracle as it stands),
+    all at once, so memory-bandwidth contention between cores is part of the measurement."""
+
+    def __init__(self, workers: int | None = None):
+        import multiprocessing as mp
+
+        self.n = workers or max(1, min(64, (os.cpu_count() or 2) - 1))
+        self.pool = mp.get_context("spawn").Pool(self.n)
+
+    def sample(self, cfg, n_rows: int, budget_s: float, seed: int, step: int = 0) -> dict:
+        tasks = [(cfg, n_rows, budget_s, seed, (step * self.n + i) % cfg.kv_heads, 7 * (step * self.n + i))
+                 for i in range(self.n)]
+        parts = self.pool.map(_oracle_worker, tasks, chunksize=1)
+        rows = sum(p["rows"] for p in parts)
+        row_s = sum(p["row_s"] for p in parts)
+        pool_s = sum(p["pool_s"] for p in parts) / len(parts)
+        # the whole job spread over the n processes: per-row and per-group costs measured under load
+        full_s = (pool_s * cfg.kv_heads + row_s / rows * cfg.seq * cfg.kv_heads) / self.n
+        return {"full_s": full_s, "tokens_per_s": cfg.seq / full_s, "rows": rows,
+                "sample": f"{rows} (position, KV group) rows and {len(parts)} KV-head poolings timed at once on "
+                          f"{self.n} processes (one thread each), extrapolated to {cfg.seq} positions x "
+                          f"{cfg.kv_heads} groups shared over the {self.n} processes"}
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
 
 
 # --------------------------------------------------------------------------- main
@@ -549,6 +681,8 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=64, help="sequences in the decode workload (64 = full)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
+    ap.add_argument("--skip-long", action="store_true", help="skip the 128K long-prefill workload")
+    ap.add_argument("--skip-sweep", action="store_true", help="skip the alpha / sparsity sweep")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--seq", type=int, default=None,
                     help="prefill sequence length override (smaller cases for profiling; default 32768)")
@@ -562,25 +696,29 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:
             return
+        pool = OraclePool()
         per_step = []
         samples = None
         for i in range(warmup + args.steps):
-            # each step: one KV group (rotating), its pooling and 3 rows
-            r = oracle_sample_time(cfg, n_rows=3, budget_s=30.0, seed=cfg.seed, groups=[i % cfg.kv_heads])
+            # each step: every process samples 2 rows of one KV group (rotating) and its pooling
+            r = pool.sample(cfg, n_rows=2, budget_s=30.0, seed=cfg.seed, step=i)
             if i >= warmup:
                 per_step.append(r["full_s"])
                 samples = r
+        pool.close()
         full_s = float(np.mean(per_step))
         value = cfg.seq / full_s
+        info = host_info()
         line = {
             "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": warmup, "ms_per_step": full_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"prefill GQA bf16 inputs (B=1, S={cfg.seq}, 32/8 heads, d=128, block 64, "
                                    "alpha 1.5)",
-                       "global_batch": 1, "seq_len": cfg.seq, "parallelism": "host oracle, 1 thread"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": samples["sample"] + "; each step one such sample"},
+                       "global_batch": 1, "seq_len": cfg.seq,
+                       "parallelism": f"host oracle, {pool.n} processes x 1 thread"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": pool.n, "kind": "oracle",
+                             "sample": samples["sample"] + "; each step one such sample", **info},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
         print(json.dumps(line), flush=True)
@@ -598,11 +736,22 @@ def main():
     if not args.skip_decode:
         dec = run_decode(dash, dcfg, max(20, args.steps), warmup, world, rank)
 
+    long_obj = sweep_obj = None
+    if not args.skip_long and not args.skip_prefill:
+        long_obj = run_long_prefill(dash, max(3, min(args.steps, 5)), warmup, world, rank, pk)
+    if not args.skip_sweep and not args.skip_prefill:
+        sweep_obj = run_sweep(dash, max(3, min(args.steps, 5)), warmup, world, rank, pk)
+
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
-        c = oracle_sample_time(cfg, n_rows=6, budget_s=args.cpu_budget)
-        cpu = {"value": c["tokens_per_s"], "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": c["sample"],
-               "wall_s": round(c["wall_s"], 1)}
+        c1 = oracle_sample_time(cfg, n_rows=6, budget_s=args.cpu_budget / 2)
+        pool = OraclePool()
+        cn = pool.sample(cfg, n_rows=3, budget_s=args.cpu_budget / 2, seed=cfg.seed)
+        pool.close()
+        cpu = {"value": cn["tokens_per_s"], "unit": "tokens/s", "cores": pool.n, "kind": "oracle",
+               "sample": cn["sample"], **host_info(),
+               "one_thread": {"value": c1["tokens_per_s"], "unit": "tokens/s", "cores": 1, "sample": c1["sample"],
+                              "wall_s": round(c1["wall_s"], 1)}}
 
     if rank != 0:
         barrier(world)
@@ -651,13 +800,17 @@ def main():
         },
         "e2e": {"value": job_throughput(pre["tokens"], world, pre["e2e_ms"]), "unit": "tokens/s",
                 "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"]},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 5 * args.steps,  # per forward: pool, summary split, routing, pair lists, attention
         "clocks": pre["clocks"],
         "device_status": pre["status"],
         "cpu_baseline": cpu,
     }
     if dec is not None:
         line["decode"] = decode_object(dec, dcfg, pk)
+    if long_obj is not None:
+        line["long_prefill"] = long_obj
+    if sweep_obj is not None:
+        line["sweep"] = sweep_obj
     if pre["backward"] is not None:
         bw = pre["backward"]
         ach = bw["flops"] / (bw["ms"] * 1e-3) / 1e12

@@ -7,10 +7,33 @@ functions used here return sums over rows, which the caller adds up.
 
 from __future__ import annotations
 
+import atexit
 import multiprocessing as mp
 import os
 
 import numpy as np
+
+_POOL = None
+
+
+def _pool_size(n_tasks: int = 1 << 30) -> int:
+    return max(1, min(n_tasks, 24, (os.cpu_count() or 2) - 1))
+
+
+def shared_pool():
+    """One spawned worker pool for the whole test session (started on first use)."""
+    global _POOL
+    if _POOL is None:
+        _POOL = mp.get_context("spawn").Pool(_pool_size())
+        atexit.register(_close_pool)
+    return _POOL
+
+
+def _close_pool():
+    global _POOL
+    if _POOL is not None:
+        _POOL.terminate()
+        _POOL = None
 
 
 def _key_block_part(args):
@@ -33,10 +56,15 @@ def key_block_backward_pooled(tmpdir, arrays: dict, blocks, block, alpha, causal
         paths[name] = os.path.join(str(tmpdir), f"{name}.npy")
         np.save(paths[name], np.ascontiguousarray(a))
     S = arrays["q"].shape[0]
-    n = workers or max(1, min(24, (os.cpu_count() or 2) - 1))
-    chunks = [range(r0, S, n) for r0 in range(n)]  # interleaved, so late (long) rows spread evenly
-    with mp.get_context("spawn").Pool(n) as pool:
-        parts = pool.map(_key_block_part, [(paths, list(blocks), block, alpha, causal, sigma, ch) for ch in chunks])
+    n = workers or _pool_size()
+    n_chunks = 4 * n  # interleaved row sets, so late (long) rows spread evenly
+    chunks = [range(r0, S, n_chunks) for r0 in range(n_chunks)]
+    tasks = [(paths, list(blocks), block, alpha, causal, sigma, ch) for ch in chunks]
+    if workers:
+        with mp.get_context("spawn").Pool(n) as pool:
+            parts = pool.map(_key_block_part, tasks, chunksize=1)
+    else:
+        parts = shared_pool().map(_key_block_part, tasks, chunksize=1)
     total = parts[0]
     for p in parts[1:]:
         for c in blocks:
@@ -60,24 +88,38 @@ def _oracle_decode_part(args):
     return (b, g), oracle_decode_pair(cfg, plan, b, g, **kw)
 
 
-def _pool_size(n_tasks: int) -> int:
-    return max(1, min(n_tasks, 24, (os.cpu_count() or 2) - 1))
-
-
 def oracle_heads_pooled(cfg, plan, pairs, rows, qbar_of=None, **kw) -> dict:
-    """tests._parity.oracle_head for every (batch, KV group) in ``pairs``, one task per pair,
-    in spawned processes.  qbar_of: optional {g: learned summary query of KV head g}.
-    Returns {(b, g): (records, summaries)}."""
-    tasks = [(cfg, plan, b, g, list(rows), dict(kw, **({"qbar": qbar_of[g]} if qbar_of else {}))) for b, g in pairs]
+    """tests._parity.oracle_head for every (batch, KV group) in ``pairs``, the rows of each pair
+    split into interleaved parts so that every worker is busy, in spawned processes.
+    qbar_of: optional {g: learned summary query of KV head g}.
+    Returns {(b, g): (records in the order of ``rows``, summaries)}."""
+    rows = list(rows)
+    n_parts = max(1, min(len(rows), -(-2 * _pool_size() // max(1, len(pairs)))))
+    tasks = []
+    for b, g in pairs:
+        kwg = dict(kw, **({"qbar": qbar_of[g]} if qbar_of else {}))
+        for r0 in range(n_parts):
+            tasks.append((cfg, plan, b, g, rows[r0::n_parts], kwg))
     if len(tasks) == 1:
-        return dict([_oracle_head_part(tasks[0])])
-    with mp.get_context("spawn").Pool(_pool_size(len(tasks))) as pool:
-        return dict(pool.map(_oracle_head_part, tasks, chunksize=1))
+        parts = [_oracle_head_part(tasks[0])]
+    else:
+        parts = shared_pool().map(_oracle_head_part, tasks, chunksize=1)
+    out = {}
+    for (b, g) in pairs:
+        recs = [None] * len(rows)
+        summ = None
+        for i, ((pb, pg), (r, sm)) in enumerate(parts):
+            if (pb, pg) != (b, g):
+                continue
+            r0 = i % n_parts
+            recs[r0::n_parts] = r
+            summ = sm
+        out[(b, g)] = (recs, summ)
+    return out
 
 
 def oracle_decode_pooled(cfg, plan, pairs, **kw) -> dict:
     """tests._parity.oracle_decode_pair for every (sequence, KV group) in ``pairs``, in spawned
     processes.  Returns {(b, g): (record, summaries)}."""
     tasks = [(cfg, plan, b, g, kw) for b, g in pairs]
-    with mp.get_context("spawn").Pool(_pool_size(len(tasks))) as pool:
-        return dict(pool.map(_oracle_decode_part, tasks, chunksize=1))
+    return dict(shared_pool().map(_oracle_decode_part, tasks, chunksize=1))
