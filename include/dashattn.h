@@ -381,6 +381,29 @@ dash_status_t dash_attn_sparse_ex(const dash_tensor_t* q, const dash_tensor_t* k
                                   const dash_options_t* opts, dash_stream_t stream);
 
 /*
+ * Stage 2 on the pages' routing format ("Stage 2: prior-induced sparse
+ * softmax", implementation: the kernel iterates over the active chunks of a
+ * bit-packed mask and adds the routing bias before the softmax).  The result
+ * is that of dash_attn_sparse_ex on the lists holding the same blocks with
+ * the same log p_bar values (bit-identical).  f16/bf16 only.
+ *   mask     device uint32 [B, Hkv, S, n_words]: bit c % 32 of word c / 32 of
+ *            a row set iff block c is selected for that query position (the
+ *            layout dash_attn_lists_to_mask writes).  Bits on blocks that are
+ *            not candidates of the row (its own block; later blocks when
+ *            causal) are ignored and reported as DASH_ERR_INVALID_ARGUMENT in
+ *            the workspace status word.
+ *   n_words  words per row: n_words * 32 >= ceil(S / block), at most 128.
+ *   logp     device fp32 [B, Hkv, S, t_cap]: log p_bar of block c at column c
+ *            of the row; read only where the row's bit is set.
+ *   workspace  dash_attn_sparse_workspace_size() bytes, 256-byte aligned.
+ * Other arguments as for dash_attn_sparse_ex (opts: sigma only).
+ */
+dash_status_t dash_attn_sparse_mask(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                                    const uint32_t* mask, int64_t n_words, const float* logp, int64_t t_cap, int block,
+                                    int causal, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                                    const dash_options_t* opts, dash_stream_t stream);
+
+/*
  * dash_attn_decode without a workspace argument.  The paper has no
  * counterpart: this serves callers that may not allocate device memory
  * while they run -- code inside another engine's execution hook (a serving

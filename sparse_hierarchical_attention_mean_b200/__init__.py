@@ -42,6 +42,7 @@ EXPORTED = (
     "dash_attn_summarize_sdpa",
     "dash_attn_fwd_ex",
     "dash_attn_sparse_ex",
+    "dash_attn_sparse_mask",
     "dash_attn_decode_ex",
     "dash_attn_lists_to_mask",
     "dash_attn_cp_scores",
@@ -114,6 +115,7 @@ def _load() -> ctypes.CDLL:
         "dash_attn_sparse": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, vp]),
         "dash_attn_fwd_ex": (i32, [T, T, T, vp, f32, i32, i32, T, vp, sz, O, vp]),
         "dash_attn_sparse_ex": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, O, vp]),
+        "dash_attn_sparse_mask": (i32, [T, T, T, vp, i64, vp, i64, i32, i32, T, vp, sz, O, vp]),
         "dash_attn_decode_ex": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
         "dash_attn_lists_to_mask": (i32, [vp, vp, i64, i64, vp, i64, vp]),
         "dash_attn_cp_scores": (i32, [T, i64, vp, i64, i64, i64, vp, i64, f32, i32, vp, i64, vp]),
@@ -294,6 +296,23 @@ def sparse(q, k, v, idx, logp, cnt, block: int, causal: bool = True, out=None, w
         _check(_lib.dash_attn_sparse(*args, _stream(stream)))
     else:
         _check(_lib.dash_attn_sparse_ex(*args, opts, _stream(stream)))
+    return out
+
+
+def sparse_mask(q, k, v, mask: torch.Tensor, logp_dense: torch.Tensor, block: int, causal: bool = True, out=None,
+                workspace=None, sigma: float = 1.0, stream=None) -> torch.Tensor:
+    """Stage 2 on bit-packed masks [B, Hkv, S, n_words] (int32 bit patterns) and a dense log p_bar
+    [B, Hkv, S, t_cap] (see dash_attn_sparse_mask)."""
+    assert mask.is_contiguous() and mask.dtype == torch.int32 and logp_dense.is_contiguous()
+    assert logp_dense.dtype == torch.float32
+    out = torch.empty_like(q) if out is None else out
+    t_cap, n_words = logp_dense.shape[-1], mask.shape[-1]
+    ws = _workspace(sparse_workspace_size(q, k, block, t_cap), q.device, workspace)
+    qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
+    _check(_lib.dash_attn_sparse_mask(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), mask.data_ptr(), n_words,
+                                      logp_dense.data_ptr(), t_cap, block, 1 if causal else 0, ctypes.byref(od),
+                                      ws.data_ptr(), ws.numel(), ctypes.byref(DashOptions(float(sigma), None)),
+                                      _stream(stream)))
     return out
 
 

@@ -85,10 +85,20 @@ int num_sms() {
 
 // Workspace of dash_attn_fwd.
 struct FwdLayout {
-  size_t status, summ, split, idx, logp, cnt, ulist, umask, ucnt, usteps, plist, pmask, pcnt, psteps, total;
+  size_t status, summ, split, wide, idx, logp, cnt, ulist, umask, ucnt, usteps, plist, pmask, pcnt, psteps, total;
   int64_t T, n_tiles, n_pairs;
-  int tile_pos;
+  int tile_pos, n_slots;
 };
+
+// Scratch slots of the segmented routing kernel (tiles with more than 512
+// candidate columns): one per SM (one of its CTAs fills an SM) and 32 spare,
+// so that a CTA never waits for the release of the CTA it replaces; none when
+// no tile can be that wide.
+int wide_slots(int64_t t_cap) { return t_cap > dash::route_tc_max_cols() ? num_sms() + 32 : 0; }
+size_t wide_bytes(int64_t t_cap) {
+  const int n = wide_slots(t_cap);
+  return n ? dash::route_wide_scratch_bytes(t_cap, n) : 0;
+}
 
 FwdLayout fwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, int block) {
   FwdLayout L{};
@@ -103,6 +113,9 @@ FwdLayout fwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, in
   off = align256(off + (size_t)B * Hkv * L.T * D * 4);
   L.split = off;  // summaries split for the tensor-core routing kernel
   off = align256(off + dash::route_split_bytes(B, Hkv, L.T, (int)D));
+  L.wide = off;  // scratch slots of the segmented routing kernel
+  L.n_slots = wide_slots(L.T);
+  off = align256(off + wide_bytes(L.T));
   L.idx = off;
   off = align256(off + (size_t)B * Hkv * S * L.T * 4);
   L.logp = off;
@@ -202,8 +215,9 @@ DecodeLayout decode_layout(int64_t B, int64_t H, int64_t Hkv, int64_t D, int blo
 
 // Workspace of dash_attn_bwd.
 struct BwdLayout {
-  size_t status, summ, split, idx, logp, cnt, tau, lse, dd, dz, umask, kbar, ds, total;
+  size_t status, summ, split, wide, idx, logp, cnt, tau, lse, dd, dz, umask, kbar, ds, total;
   int64_t T, n_words;
+  int n_slots;
 };
 
 BwdLayout bwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, int block) {
@@ -219,6 +233,8 @@ BwdLayout bwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, in
   take(L.status, sizeof(dash::DeviceStatus));
   take(L.summ, (size_t)B * Hkv * L.T * D * 4);
   take(L.split, dash::route_split_bytes(B, Hkv, L.T, (int)D));
+  L.n_slots = wide_slots(L.T);
+  take(L.wide, wide_bytes(L.T));
   take(L.idx, (size_t)B * Hkv * S * L.T * 4);
   take(L.logp, (size_t)B * Hkv * S * L.T * 4);
   take(L.cnt, (size_t)B * Hkv * S * 4);
@@ -354,7 +370,7 @@ struct TileLists {
 dash_status_t run_route(const dash_tensor_t* q, const float* summaries, int64_t kv_heads, int64_t t_cap, float alpha,
                         int block, int causal, int32_t* idx, float* logp, int32_t* cnt, float* tau, float* p_dense,
                         const TileLists* tl, dash::DeviceStatus* status, cudaStream_t stream, int* first_cuda_tile,
-                        float* split_buf = nullptr) {
+                        float* split_buf = nullptr, void* wide_buf = nullptr) {
   const int G = (int)(q->h / kv_heads);
   dash::RouteParams p{};
   p.q = view(q);
@@ -381,23 +397,37 @@ dash_status_t run_route(const dash_tensor_t* q, const float* summaries, int64_t 
   const int n_blocks = (int)((q->s + block - 1) / block);
   int split = 0;
   if (q->dtype != DASH_F32) {
+    // tiles [0, narrow) fit TMEM; the rest run the segmented kernel when its
+    // scratch (and the split summaries it streams) are given, else CUDA cores
     const int max_cols = dash::route_tc_max_cols();
+    int narrow;
     if (causal) {
-      split = (int)(((int64_t)(max_cols + 1) * block) / P);
-      if (split > n_tiles) split = n_tiles;
+      narrow = (int)(((int64_t)(max_cols + 1) * block) / P);
+      if (narrow > n_tiles) narrow = n_tiles;
     } else {
-      split = n_blocks <= max_cols ? n_tiles : 0;
+      narrow = n_blocks <= max_cols ? n_tiles : 0;
     }
+    const bool wide = wide_buf && split_buf && narrow < n_tiles && n_blocks <= dash::route_tc_wide_max_cols();
     dash::TileOut to{};
     if (tl) to = dash::TileOut{tl->ulist, tl->umask, tl->ucnt, tl->usteps, n_tiles};
-    if (split_buf && split > 0) {
+    if (split_buf && (narrow > 0 || wide)) {
       cudaError_t e = dash::launch_route_split(p, split_buf, stream);
       if (e != cudaSuccess) return cuda_fail(e, "route (split summaries)");
       p.summ_split = split_buf;
     }
-    cudaError_t e = dash::launch_route_prefill_tc(p, to, 0, split, stream);
-    p.summ_split = nullptr;
+    cudaError_t e = dash::launch_route_prefill_tc(p, to, 0, narrow, stream);
     if (e != cudaSuccess) return cuda_fail(e, "route (tensor cores)");
+    split = narrow;
+    if (wide) {
+      const int n_slots = wide_slots(t_cap);
+      const dash::WideScratch w = dash::route_wide_scratch(wide_buf, t_cap, n_slots);
+      e = cudaMemsetAsync(w.locks, 0, (size_t)n_slots * 4, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "memset");
+      e = dash::launch_route_prefill_tc_wide(p, to, narrow, n_tiles - narrow, w, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "route (tensor cores, segmented)");
+      split = n_tiles;
+    }
+    p.summ_split = nullptr;
   }
   p.pos_begin = split * P;
   if (p.pos_begin < p.S) {
@@ -414,7 +444,8 @@ extern "C" {
 
 size_t dash_attn_route_workspace_size(const dash_tensor_t* q, int64_t kv_heads, int64_t t_cap, int decode) {
   if (check_tensor(q, "q") || check_group(q->h, kv_heads) || t_cap <= 0) return 0;
-  if (!decode) return dash::route_split_bytes(q->b, kv_heads, t_cap, (int)q->d);  // optional in prefill mode
+  if (!decode)  // optional in prefill mode: split summaries, then the segmented kernel's scratch
+    return align256(dash::route_split_bytes(q->b, kv_heads, t_cap, (int)q->d)) + wide_bytes(t_cap);
   return decode_layout(q->b, q->h, kv_heads, q->d, 64, t_cap).idx;  // status + per-head logits
 }
 
@@ -433,11 +464,15 @@ dash_status_t dash_attn_route(const dash_tensor_t* q, const float* summaries, in
     if (T > 4096) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per sequence");
     // a workspace, when given, holds the split summaries of the tensor-core kernel
     float* split = nullptr;
-    if (workspace && reinterpret_cast<uintptr_t>(workspace) % 256 == 0 &&
-        workspace_bytes >= dash::route_split_bytes(q->b, kv_heads, t_cap, (int)q->d))
+    void* wide = nullptr;
+    const size_t split_bytes = align256(dash::route_split_bytes(q->b, kv_heads, t_cap, (int)q->d));
+    if (workspace && reinterpret_cast<uintptr_t>(workspace) % 256 == 0 && workspace_bytes >= split_bytes) {
       split = static_cast<float*>(workspace);
+      if (wide_bytes(t_cap) && workspace_bytes >= split_bytes + wide_bytes(t_cap))
+        wide = static_cast<char*>(workspace) + split_bytes;
+    }
     st = run_route(q, summaries, kv_heads, t_cap, alpha, block, causal, idx, logp, cnt, tau, p_dense, nullptr,
-                   nullptr, (cudaStream_t)stream, nullptr, split);
+                   nullptr, (cudaStream_t)stream, nullptr, split, wide);
     return st ? st : ok();
   }
   if (q->s != 1) return fail(DASH_ERR_INVALID_ARGUMENT, "decode-mode route needs q with s == 1");
@@ -491,7 +526,8 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
                                 const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap, int block,
                                 int causal, float sigma, dash_tensor_t* out, const TileLists& tl, int tile_pos,
                                 int64_t n_tiles, int union_tile0, dash::DeviceStatus* status,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, const uint32_t* mask = nullptr, int n_words = 0,
+                                const float* logp_dense = nullptr) {
   if (q->dtype != DASH_F32 && union_tile0 < n_tiles) {
     dash::UnionParams u{};
     u.B = (int)q->b;
@@ -510,6 +546,8 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
     u.usteps = tl.usteps;
     u.causal = causal ? 1 : 0;
     u.status = status;
+    u.mask = mask;
+    u.n_words = n_words;
     cudaError_t e = dash::launch_union(u, stream);
     if (e != cudaSuccess) return cuda_fail(e, "union");
   }
@@ -561,6 +599,7 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
   p.n_tiles = (int)n_tiles;
   p.sigma = sigma;
   p.status = status;
+  p.logp_dense = logp_dense;
   cudaError_t e = dash::launch_sparse_prefill(p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
   return DASH_OK;
@@ -616,6 +655,43 @@ dash_status_t dash_attn_sparse_ex(const dash_tensor_t* q, const dash_tensor_t* k
   return st ? st : ok();
 }
 
+dash_status_t dash_attn_sparse_mask(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                                    const uint32_t* mask, int64_t n_words, const float* logp, int64_t t_cap, int block,
+                                    int causal, dash_tensor_t* out, void* workspace, size_t workspace_bytes,
+                                    const dash_options_t* opts, dash_stream_t stream) {
+  dash_status_t st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
+  if ((st = check_fwd_shapes(q, k, v, out))) return st;
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "the mask form takes f16 or bf16 inputs");
+  if (k->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "prefill needs k and q of equal length");
+  if (!mask || !logp) return fail(DASH_ERR_INVALID_ARGUMENT, "null mask or logp");
+  if (reinterpret_cast<uintptr_t>(mask) % 4 || reinterpret_cast<uintptr_t>(logp) % 4)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "mask and logp must be 4-byte aligned");
+  const int64_t T = (q->s + block - 1) / block;
+  if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block)", (long long)t_cap);
+  if (T > 4096) return fail(DASH_ERR_UNSUPPORTED, "more than 4096 blocks per sequence");
+  if (n_words * 32 < T || n_words > 128)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "n_words %lld must cover ceil(S / block) blocks, at most 128",
+                (long long)n_words);
+  const SparseLayout L = sparse_layout(q->b, q->s, q->h, k->h, block, t_cap);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < L.total)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
+                     at<int32_t>(workspace, L.usteps), at<int32_t>(workspace, L.plist), at<uint4>(workspace, L.pmask),
+                     at<int32_t>(workspace, L.pcnt), at<int32_t>(workspace, L.psteps), L.n_pairs};
+  st = run_sparse(q, k, v, nullptr, nullptr, nullptr, t_cap, block, causal, sigma, out, tl, L.tile_pos, L.n_tiles, 0,
+                  at<dash::DeviceStatus>(workspace, L.status), s, mask, (int)n_words, logp);
+  return st ? st : ok();
+}
+
 dash_status_t dash_attn_fwd(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v, const float* w_s,
                             float alpha, int block, int causal, dash_tensor_t* out, void* workspace,
                             size_t workspace_bytes, dash_stream_t stream) {
@@ -653,7 +729,7 @@ dash_status_t dash_attn_fwd_ex(const dash_tensor_t* q, const dash_tensor_t* k, c
   dash::DeviceStatus* dst = at<dash::DeviceStatus>(workspace, L.status);
   int first_cuda_tile = 0;
   if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, nullptr, nullptr, &tl, dst, s,
-                      &first_cuda_tile, at<float>(workspace, L.split))))
+                      &first_cuda_tile, at<float>(workspace, L.split), L.n_slots ? at<char>(workspace, L.wide) : nullptr)))
     return st;
   st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, sigma, out, tl, L.tile_pos, L.n_tiles, first_cuda_tile,
                   dst, s);
@@ -711,7 +787,7 @@ dash_status_t dash_attn_bwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   int32_t* cnt = at<int32_t>(workspace, L.cnt);
   float* tau = at<float>(workspace, L.tau);
   if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, tau, nullptr, nullptr, dst, s, nullptr,
-                      at<float>(workspace, L.split))))
+                      at<float>(workspace, L.split), L.n_slots ? at<char>(workspace, L.wide) : nullptr)))
     return st;
   dash::BwdParams p{};
   p.idx = idx;

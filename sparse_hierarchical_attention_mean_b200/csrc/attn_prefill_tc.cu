@@ -281,7 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;  // TMEM lane quarter
     const int r = q4 * 32 + lane;
     RowPrior row;
-    row.init(p, bg, pos0 + t * P + r / G, r / G);
+    if (p.logp_dense)
+      row.init_dense(p, bg, pos0 + t * P + r / G, r / G, plist, pcnt);
+    else
+      row.init(p, bg, pos0 + t * P + r / G, r / G);
     const int head = g * G + r % G;
     const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + t * kTileCols;
     const float qk_scale = rsqrtf((float)D) * kLog2e;

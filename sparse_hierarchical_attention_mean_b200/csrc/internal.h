@@ -77,6 +77,25 @@ int route_tc_max_cols();
 cudaError_t launch_route_prefill_tc(const RouteParams& p, const TileOut& to, int tile0, int n_tiles,
                                     cudaStream_t stream);
 
+// Tiles with more than route_tc_max_cols() logit columns (up to
+// route_tc_wide_max_cols()) run the segmented tensor-core kernel, which keeps
+// each tile's logits in a scratch slot in global memory: `n_slots` slots
+// (more than the SM count: one CTA of that kernel fills an SM) and one lock
+// word per slot, which must be zero when the kernel starts (it leaves them
+// zero).
+// Needs p.summ_split.
+struct WideScratch {
+  float* logits;   // [n_slots][slot_floats]
+  int32_t* locks;  // [n_slots]
+  int n_slots;
+  int64_t slot_floats;
+};
+int route_tc_wide_max_cols();
+size_t route_wide_scratch_bytes(int64_t t_cap, int n_slots);  // locks + slots, 256-byte aligned parts
+WideScratch route_wide_scratch(void* base, int64_t t_cap, int n_slots);
+cudaError_t launch_route_prefill_tc_wide(const RouteParams& p, const TileOut& to, int tile0, int n_tiles,
+                                         const WideScratch& w, cudaStream_t stream);
+
 // Work list of each stage-2 tile of `tile_pos` consecutive positions: the
 // union of the rows' selected blocks and the rows' own blocks, ascending.
 struct UnionParams {
@@ -91,6 +110,10 @@ struct UnionParams {
   int32_t* usteps; // [B, Hkv, n_tiles]: 64-token steps of the tile
   int causal;
   DeviceStatus* status;  // invalid list entries are skipped and reported here
+  // bit-packed form instead of idx / cnt (non-null: used): [B, Hkv, S, n_words],
+  // bit c of a row set iff block c is selected
+  const uint32_t* mask;
+  int n_words;
 };
 cudaError_t launch_union(const UnionParams& p, cudaStream_t stream);
 
@@ -111,6 +134,10 @@ struct SparseParams {
   int tile_pos, n_tiles, n_pairs;
   float sigma;  // prior strength: bias sigma * log p_bar (diagonal: sigma * log(1/N))
   DeviceStatus* status;
+  // dense prior instead of the lists (tensor-core kernel; non-null: used):
+  // [B, Hkv, S, t_cap], log p_bar of block c at column c, read only where the
+  // tile work list marks the row as selecting c
+  const float* logp_dense;
 };
 // positions per stage-2 tile (tiles are 128 rows)
 int sparse_tile_positions(int G, int block);

@@ -194,6 +194,50 @@ __global__ void __launch_bounds__(kThreads) route_prefill_kernel(RouteParams p, 
 // ascending; for each listed block, the bit mask of the tile positions that
 // selected it; and the number of 64-token steps the tile takes (the causal
 // diagonal's halves past the tile's last position are skipped).
+// Second half of the tile work list (shared by the list and mask forms):
+// pmask[c] holds the positions that selected block c; the list keeps those
+// blocks and the tile's own blocks, ascending, and counts the tile's 64-token
+// steps.  Warp 0 writes it.
+__device__ __forceinline__ void emit_tile_list(const UnionParams& p, const uint4* pmask, int64_t bg, int tile,
+                                               int pos0, int lane) {
+  const int last = min(pos0 + p.tile_pos, p.S) - 1;
+  const int own_lo = pos0 / p.block, own_hi = last / p.block;
+  const int last_needed = p.causal ? last : p.S - 1;
+  const int64_t tix = bg * p.n_tiles + tile;
+  int32_t* out = p.ulist + tix * p.t_cap;
+  uint4* mout = p.umask + tix * p.t_cap;
+  int off = 0, steps = 0;
+  for (int c0 = 0; c0 < p.t_cap; c0 += 32) {
+    const int c = c0 + lane;
+    bool keep = false;
+    uint4 m = make_uint4(0u, 0u, 0u, 0u);
+    if (c < p.t_cap) {
+      m = pmask[c];
+      keep = (m.x | m.y | m.z | m.w) != 0u || (c >= own_lo && c <= own_hi);
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    int st = 0;
+    if (keep) {
+      const int k = off + __popc(bal & ((1u << lane) - 1u));
+      out[k] = c;
+      mout[k] = m;
+      for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
+    }
+    steps += warp_sum_i(st);
+    off += __popc(bal);
+  }
+  if (lane == 0) {
+    p.ucnt[tix] = off;
+    p.usteps[tix] = steps;
+  }
+}
+
+// Is block c a routing candidate of a row in block t?  (causal: an earlier
+// block; otherwise any other block)
+__device__ __forceinline__ bool candidate(const UnionParams& p, int c, int t, int n_blocks) {
+  return c >= 0 && c != t && (p.causal ? c < t : c < n_blocks);
+}
+
 __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
   extern __shared__ uint4 pmask[];  // [t_cap]: bit p set if tile position p selected the block
   const int b = blockIdx.z, g = blockIdx.y, tile = p.tile0 + blockIdx.x;
@@ -212,9 +256,7 @@ __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
     const int32_t* idx = p.idx + row * p.t_cap;
     for (int e = lane; e < n; e += 32) {
       const int c = idx[e];
-      // a candidate is a block other than the own block (causal: an earlier one)
-      const bool ok = c >= 0 && c != t && (p.causal ? c < t : c < n_blocks);
-      if (ok) {
+      if (candidate(p, c, t, n_blocks)) {
         atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (pp >> 5), 1u << (pp & 31));
       } else {
         raise_status(p.status, 1 /* DASH_ERR_INVALID_ARGUMENT */, 200);
@@ -222,38 +264,43 @@ __global__ void __launch_bounds__(kThreads) union_kernel(UnionParams p) {
     }
   }
   __syncthreads();
-  if (warp == 0) {
-    const int last = min(pos0 + p.tile_pos, p.S) - 1;
-    const int own_lo = pos0 / p.block, own_hi = last / p.block;
-    const int last_needed = p.causal ? last : p.S - 1;
-    const int64_t tix = bg * p.n_tiles + tile;
-    int32_t* out = p.ulist + tix * p.t_cap;
-    uint4* mout = p.umask + tix * p.t_cap;
-    int off = 0, steps = 0;
-    for (int c0 = 0; c0 < p.t_cap; c0 += 32) {
-      const int c = c0 + lane;
-      bool keep = false;
-      uint4 m = make_uint4(0u, 0u, 0u, 0u);
-      if (c < p.t_cap) {
-        m = pmask[c];
-        keep = (m.x | m.y | m.z | m.w) != 0u || (c >= own_lo && c <= own_hi);
+  if (warp == 0) emit_tile_list(p, pmask, bg, tile, pos0, lane);
+}
+
+// The same work list from bit-packed active-block masks (the pages' stage-2
+// kernel iterates over such a mask): one warp per tile position walks its
+// row's mask words, a lane per word, visiting the set bits with
+// find-first-set; a set bit on a block that is not a candidate of the row (its
+// own block, or a later one when causal) is skipped and reported.
+__global__ void __launch_bounds__(kThreads) union_mask_kernel(UnionParams p) {
+  extern __shared__ uint4 pmask[];
+  const int b = blockIdx.z, g = blockIdx.y, tile = p.tile0 + blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int c = tid; c < p.t_cap; c += kThreads) pmask[c] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const int pos0 = tile * p.tile_pos;
+  const int n_blocks = (p.S + p.block - 1) / p.block;
+  for (int pp = warp; pp < p.tile_pos; pp += kThreads / 32) {
+    const int pos = pos0 + pp;
+    if (pos >= p.S) break;
+    const int t = pos / p.block;
+    const uint32_t* words = p.mask + (bg * p.S + pos) * p.n_words;
+    for (int w = lane; w < p.n_words; w += 32) {
+      uint32_t word = __ldg(words + w);
+      while (word) {
+        const int c = 32 * w + __ffs(word) - 1;
+        word &= word - 1u;
+        if (c < p.t_cap && candidate(p, c, t, n_blocks)) {
+          atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (pp >> 5), 1u << (pp & 31));
+        } else {
+          raise_status(p.status, 1 /* DASH_ERR_INVALID_ARGUMENT */, 201);
+        }
       }
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      int st = 0;
-      if (keep) {
-        const int k = off + __popc(bal & ((1u << lane) - 1u));
-        out[k] = c;
-        mout[k] = m;
-        for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
-      }
-      steps += warp_sum_i(st);
-      off += __popc(bal);
-    }
-    if (lane == 0) {
-      p.ucnt[tix] = off;
-      p.usteps[tix] = steps;
     }
   }
+  __syncthreads();
+  if (warp == 0) emit_tile_list(p, pmask, bg, tile, pos0, lane);
 }
 
 // Work list of a pair of adjacent stage-2 tiles (see internal.h).
@@ -353,11 +400,12 @@ cudaError_t launch_route_prefill(const RouteParams& p, cudaStream_t stream) {
 
 cudaError_t launch_union(const UnionParams& p, cudaStream_t stream) {
   const size_t smem = (size_t)p.t_cap * sizeof(uint4);
-  cudaError_t e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = p.mask ? union_mask_kernel : union_kernel;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (p.n_tiles - p.tile0 <= 0) return cudaSuccess;
   dim3 grid(p.n_tiles - p.tile0, p.Hkv, p.B);
-  union_kernel<<<grid, kThreads, smem, stream>>>(p);
+  kern<<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

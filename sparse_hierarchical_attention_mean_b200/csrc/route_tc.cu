@@ -230,10 +230,169 @@ __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride,
   entmax_newton_rows<RW, 2>(x, stride, n, pw, kind, lane, tau, done);
 }
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RouteParams p, TileOut to, int tile0) {
+// Thresholds, GQA mean and ascending per-position lists for the tile rows
+// [row_base, row_base + round_rows), one warp per task of RW rows (RW / G
+// positions x G heads) solved in lockstep.  Tile row r's logits (scaled,
+// non-candidates -inf, readable up to the column count rounded up to 64) are
+// X[(r - row_base) * xstride + c]; its seed values are
+// seed[(r - row_base) * kSeed + l].  Marks in pmask[c] the tile positions
+// that selected block c.
+template <int G>
+__device__ __forceinline__ void solve_and_compact(const RouteParams& p, const float* X, int xstride, const float* seed,
+                                                  uint4* pmask, int row_base, int round_rows, int b, int g, int pos0,
+                                                  int n_blocks, int warp, int lane) {
   constexpr int RW = G > 4 ? G : 4;  // rows solved together by one warp
   constexpr int PPT = RW / G;        // positions per warp task
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const float pw = 1.0f / (p.alpha - 1.0f);
+  const int kind = entmax_kind(p.alpha);
+  const int n_tasks = round_rows / RW;
+  for (int task = warp; task < n_tasks; task += kWorkWarps) {
+    const int rr0 = task * RW;                 // first row within the round
+    const int tp0 = (row_base + rr0) / G;      // first tile position
+    const int pos = pos0 + tp0;
+    const int t = pos / p.block;  // the task's positions share their block
+    const int ncol = p.causal ? t : n_blocks;
+    float tau[RW];
+    // thresholds four rows at a time (register budget)
+#pragma unroll
+    for (int r4 = 0; r4 < RW; r4 += 4) {
+      if (ncol > 0) {
+        warp_entmax_tau_rows<4>(X + (rr0 + r4) * xstride, xstride, ncol, seed + (rr0 + r4) * kSeed, p.alpha, kind,
+                                lane, tau + r4);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tau[r4 + i] = 0.f;  // no candidates (nothing was copied)
+      }
+    }
+#pragma unroll
+    for (int pp = 0; pp < PPT; ++pp) {
+      const int tp = tp0 + pp;
+      const int qpos = pos0 + tp;
+      if (qpos >= p.S) continue;
+      const int n_row = p.causal ? t : n_blocks - 1;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (n_row == 0) tau[pp * G + h] = 0.f;
+        if (p.tau && lane == 0) p.tau[((int64_t)b * p.H + g * G + h) * p.S + qpos] = tau[pp * G + h];
+      }
+      const int64_t row = bg * p.S + qpos;
+      int32_t* idx = p.idx + row * p.t_cap;
+      float* logp = p.logp + row * p.t_cap;
+      int off = 0;
+      for (int c0 = 0; c0 < ncol && n_row > 0; c0 += 32) {
+        const int c = c0 + lane;
+        float pbar = 0.f;
+        if (c < ncol) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float u = X[(rr0 + pp * G + h) * xstride + c] - tau[pp * G + h];
+            const float ph = u > 0.f ? pow_pw(u, pw, kind) : 0.f;
+            pbar += ph;
+            if (p.p_dense) p.p_dense[(((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap + c] = ph;
+          }
+          pbar *= 1.0f / (float)G;
+        }
+        const bool sel = pbar > 0.f;
+        const unsigned m = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+          const int o = off + __popc(m & ((1u << lane) - 1u));
+          idx[o] = c;
+          logp[o] = logf(pbar);
+          atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (tp >> 5), 1u << (tp & 31));
+        }
+        off += __popc(m);
+      }
+      if (lane == 0) p.cnt[row] = off;
+      if (p.p_dense) {
+        const int from = n_row > 0 ? ncol : 0;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float* pd = p.p_dense + (((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap;
+          for (int c = from + lane; c < p.t_cap; c += 32) pd[c] = 0.f;
+        }
+      }
+    }
+  }
+}
+
+// The tile's stage-2 work list: the union of its positions' blocks plus the
+// tile's own blocks, ascending, each with the mask of positions that
+// selected it, and the tile's number of 64-token steps.  One warp per
+// 32-column chunk counts, then every chunk writes at its prefix offset.
+// pmask[c] (c < pmask_cap) holds the positions that selected block c; lcnt
+// and lsteps have one entry per 32-column chunk.  Called by every thread of
+// the CTA (it contains a CTA barrier).
+__device__ __forceinline__ void write_tile_list(const RouteParams& p, const TileOut& to, const uint4* pmask,
+                                                int pmask_cap, int* lcnt, int* lsteps, int64_t bg, int tile, int pos0,
+                                                int last, int t_last, int n_cols, int warp, int lane) {
+  const int own_lo = pos0 / p.block, own_hi = t_last;
+  const int last_needed = p.causal ? last : p.S - 1;
+  const int span = max(n_cols, own_hi + 1);
+  const int n_lch = (span + 31) / 32;
+  auto chunk = [&](int ch, uint4& m, unsigned& bal, int& st) {
+    const int c = ch * 32 + lane;
+    bool keep = false;
+    m = make_uint4(0u, 0u, 0u, 0u);
+    st = 0;
+    if (c < span) {
+      if (c < pmask_cap) m = pmask[c];
+      keep = (m.x | m.y | m.z | m.w) != 0u || (c >= own_lo && c <= own_hi);
+      if (keep)
+        for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
+    }
+    bal = __ballot_sync(0xffffffffu, keep);
+    return keep;
+  };
+  if (warp < kWorkWarps) {
+    for (int ch = warp; ch < n_lch; ch += kWorkWarps) {
+      uint4 m;
+      unsigned bal;
+      int st;
+      chunk(ch, m, bal, st);
+      st = warp_sum_i(st);
+      if (lane == 0) {
+        lcnt[ch] = __popc(bal);
+        lsteps[ch] = st;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp < kWorkWarps) {
+    const int64_t tix = bg * to.n_tiles + tile;
+    int32_t* out = to.ulist + tix * p.t_cap;
+    uint4* mout = to.umask + tix * p.t_cap;
+    for (int ch = warp; ch < n_lch; ch += kWorkWarps) {
+      uint4 m;
+      unsigned bal;
+      int st;
+      const bool keep = chunk(ch, m, bal, st);
+      int off = 0;
+      for (int k = 0; k < ch; ++k) off += lcnt[k];
+      if (keep) {
+        const int k = off + __popc(bal & ((1u << lane) - 1u));
+        out[k] = ch * 32 + lane;
+        mout[k] = m;
+      }
+    }
+    if (warp == 0) {
+      int n = 0, steps = 0;
+      for (int k = lane; k < n_lch; k += 32) {
+        n += lcnt[k];
+        steps += lsteps[k];
+      }
+      n = warp_sum_i(n);
+      steps = warp_sum_i(steps);
+      if (lane == 0) {
+        to.ucnt[tix] = n;
+        to.usteps[tix] = steps;
+      }
+    }
+  }
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RouteParams p, TileOut to, int tile0) {
   using L = RLayout<D>;
   constexpr uint32_t kIdesc = idesc_tf32(kRows, kChunk);
   extern __shared__ uint8_t smem_raw[];
@@ -254,8 +413,6 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   const int n_chunks = (n_cols + kChunk - 1) / kChunk;
   const int64_t bg = (int64_t)b * p.Hkv + g;
   const float coef = (p.alpha - 1.0f) * rsqrtf((float)D);
-  const float pw = 1.0f / (p.alpha - 1.0f);
-  const int kind = entmax_kind(p.alpha);
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars->a_full, kWork);
@@ -451,78 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
       }
     }
     __syncthreads();
-    if (warp < kWorkWarps) {
-      // one warp per task of RW rows (PPT positions x G heads): thresholds in
-      // lockstep, then the GQA mean and the ascending list of each position
-      const int n_tasks = round_rows / RW;
-      for (int task = warp; task < n_tasks; task += kWorkWarps) {
-        const int rr0 = task * RW;                       // first row within the round
-        const int tp0 = (half * round_rows + rr0) / G;  // first tile position
-        const int pos = pos0 + tp0;
-        const int t = pos / p.block;  // the task's positions share their block
-        const int ncol = p.causal ? t : n_blocks;
-        float tau[RW];
-        // thresholds four rows at a time (register budget)
-#pragma unroll
-        for (int r4 = 0; r4 < RW; r4 += 4) {
-          if (ncol > 0) {
-            warp_entmax_tau_rows<4>(X + (rr0 + r4) * xstride, xstride, ncol, seed + (rr0 + r4) * kSeed, p.alpha,
-                                    kind, lane, tau + r4);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) tau[r4 + i] = 0.f;  // no candidates (nothing was copied)
-          }
-        }
-#pragma unroll
-        for (int pp = 0; pp < PPT; ++pp) {
-          const int tp = tp0 + pp;
-          const int qpos = pos0 + tp;
-          if (qpos >= p.S) continue;
-          const int n_row = p.causal ? t : n_blocks - 1;
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            if (n_row == 0) tau[pp * G + h] = 0.f;
-            if (p.tau && lane == 0) p.tau[((int64_t)b * p.H + g * G + h) * p.S + qpos] = tau[pp * G + h];
-          }
-          const int64_t row = bg * p.S + qpos;
-          int32_t* idx = p.idx + row * p.t_cap;
-          float* logp = p.logp + row * p.t_cap;
-          int off = 0;
-          for (int c0 = 0; c0 < ncol && n_row > 0; c0 += 32) {
-            const int c = c0 + lane;
-            float pbar = 0.f;
-            if (c < ncol) {
-#pragma unroll
-              for (int h = 0; h < G; ++h) {
-                const float u = X[(rr0 + pp * G + h) * xstride + c] - tau[pp * G + h];
-                const float ph = u > 0.f ? pow_pw(u, pw, kind) : 0.f;
-                pbar += ph;
-                if (p.p_dense) p.p_dense[(((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap + c] = ph;
-              }
-              pbar *= 1.0f / (float)G;
-            }
-            const bool sel = pbar > 0.f;
-            const unsigned m = __ballot_sync(0xffffffffu, sel);
-            if (sel) {
-              const int o = off + __popc(m & ((1u << lane) - 1u));
-              idx[o] = c;
-              logp[o] = logf(pbar);
-              atomicOr(reinterpret_cast<uint32_t*>(&pmask[c]) + (tp >> 5), 1u << (tp & 31));
-            }
-            off += __popc(m);
-          }
-          if (lane == 0) p.cnt[row] = off;
-          if (p.p_dense) {
-            const int from = n_row > 0 ? ncol : 0;
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              float* pd = p.p_dense + (((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap;
-              for (int c = from + lane; c < p.t_cap; c += 32) pd[c] = 0.f;
-            }
-          }
-        }
-      }
-    }
+    if (warp < kWorkWarps)
+      solve_and_compact<G>(p, X, xstride, seed, pmask, half * round_rows, round_rows, b, g, pos0, n_blocks, warp, lane);
     __syncthreads();
   }
 
@@ -532,74 +619,297 @@ __global__ void __launch_bounds__(kThreads, 1) route_prefill_tc_kernel(RoutePara
   tc::fence_before_sync();
   if (to.ulist) {
     int* lcnt = reinterpret_cast<int*>(smem + L::kOffList);
-    int* lsteps = lcnt + 32;
-    const int own_lo = pos0 / p.block, own_hi = t_last;
-    const int last_needed = p.causal ? last : p.S - 1;
-    const int span = max(n_cols, own_hi + 1);
-    const int n_lch = (span + 31) / 32;
-    auto chunk = [&](int ch, uint4& m, unsigned& bal, int& st) {
-      const int c = ch * 32 + lane;
-      bool keep = false;
-      m = make_uint4(0u, 0u, 0u, 0u);
-      st = 0;
-      if (c < span) {
-        if (c < kMaxCols) m = pmask[c];
-        keep = (m.x | m.y | m.z | m.w) != 0u || (c >= own_lo && c <= own_hi);
-        if (keep)
-          for (int h = 0; h < p.block / 64; ++h) st += (c * p.block + h * 64 <= last_needed) ? 1 : 0;
-      }
-      bal = __ballot_sync(0xffffffffu, keep);
-      return keep;
-    };
-    if (warp < kWorkWarps) {
-      for (int ch = warp; ch < n_lch; ch += kWorkWarps) {
-        uint4 m;
-        unsigned bal;
-        int st;
-        chunk(ch, m, bal, st);
-        st = warp_sum_i(st);
-        if (lane == 0) {
-          lcnt[ch] = __popc(bal);
-          lsteps[ch] = st;
-        }
-      }
-    }
-    __syncthreads();
-    if (warp < kWorkWarps) {
-      const int64_t tix = bg * to.n_tiles + tile;
-      int32_t* out = to.ulist + tix * p.t_cap;
-      uint4* mout = to.umask + tix * p.t_cap;
-      for (int ch = warp; ch < n_lch; ch += kWorkWarps) {
-        uint4 m;
-        unsigned bal;
-        int st;
-        const bool keep = chunk(ch, m, bal, st);
-        int off = 0;
-        for (int k = 0; k < ch; ++k) off += lcnt[k];
-        if (keep) {
-          const int k = off + __popc(bal & ((1u << lane) - 1u));
-          out[k] = ch * 32 + lane;
-          mout[k] = m;
-        }
-      }
-      if (warp == 0) {
-        int n = 0, steps = 0;
-        for (int k = lane; k < n_lch; k += 32) {
-          n += lcnt[k];
-          steps += lsteps[k];
-        }
-        n = warp_sum_i(n);
-        steps = warp_sum_i(steps);
-        if (lane == 0) {
-          to.ucnt[tix] = n;
-          to.usteps[tix] = steps;
-        }
-      }
-    }
+    write_tile_list(p, to, pmask, kMaxCols, lcnt, lcnt + 32, bg, tile, pos0, last, t_last, n_cols, warp, lane);
   }
   if (warp == kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kMaxCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tiles with more candidate columns than TMEM holds (long contexts, up to
+// 4096 blocks).  The logits are computed in segments of 512 columns; after
+// each segment the work warps move it from TMEM into this CTA's scratch slot
+// in global memory (128 rows x the tile's columns in fp32, at most 2 MB; the
+// slots of the CTAs in flight stay in L2), scaled and masked as above, and
+// keep one seed value per row and 32-column chunk slot (the running maximum
+// of the chunks that map to it: still a subset of the row, so its threshold
+// is still a lower bound).  Thresholds, lists and the tile's work list are
+// then solved over the slot by the same code as the narrow kernel.  A CTA
+// claims a free slot with a compare-and-swap on its lock word (there are
+// more slots than CTAs of this kernel can be resident, one per SM) and frees
+// it before it exits.
+
+constexpr int kWideMaxCols = 4096;
+constexpr int kSegChunks = kMaxCols / kChunk;  // GEMM chunks per 512-column segment
+constexpr int kWideListCap = kWideMaxCols / 32 + 8;
+constexpr int kOffWideList = kWideMaxCols * 16;  // after the [4096] uint4 position masks
+
+struct WBars {
+  uint64_t a_full;
+  uint64_t b_full[2];
+  uint64_t b_empty[2];
+  uint64_t x_ready;    // one phase per segment: its MMAs are complete
+  uint64_t tmem_free;  // one phase per segment: every work warp has read it
+  uint64_t drain;      // every MMA issued is complete
+  uint32_t tmem_base;
+  int abort;
+  int slot;
+};
+static_assert(sizeof(WBars) <= 128, "barriers must fit the reserved bytes");
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    route_prefill_tc_wide_kernel(RouteParams p, TileOut to, int tile0, WideScratch wsc) {
+  using L = RLayout<D>;
+  static_assert(kOffWideList + 2 * kWideListCap * 4 <= L::kGemmBytes, "wide-tile lists must fit over the operands");
+  constexpr uint32_t kIdesc = idesc_tf32(kRows, kChunk);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  WBars* bars = reinterpret_cast<WBars*>(smem + L::kOffBar);
+  float* seed = reinterpret_cast<float*>(smem + L::kOffSeed);  // [kRows][kSeed]
+  uint4* pmask = reinterpret_cast<uint4*>(smem);               // over the operands, once the GEMMs are done
+  int* lcnt = reinterpret_cast<int*>(smem + kOffWideList);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, g = blockIdx.y, tile = tile0 + blockIdx.x;
+  constexpr int P = kRows / G;
+  const int pos0 = tile * P;
+  const int n_blocks = (p.S + p.block - 1) / p.block;
+  const int last = min(pos0 + P, p.S) - 1;
+  const int t_last = last / p.block;
+  const int n_cols = p.causal ? t_last : n_blocks;
+  const int n_chunks = (n_cols + kChunk - 1) / kChunk;
+  const int n_seg = (n_chunks + kSegChunks - 1) / kSegChunks;
+  const int n_wch = 2 * n_chunks;  // 32-column chunks, an even number
+  const int xstride = n_wch * 32 + 4;
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const float coef = (p.alpha - 1.0f) * rsqrtf((float)D);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bars->a_full, kWork);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->b_full[s], 1);
+      tc::mbar_init(&bars->b_empty[s], 1);
+    }
+    tc::mbar_init(&bars->x_ready, 1);
+    tc::mbar_init(&bars->tmem_free, kWorkWarps);
+    tc::mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    tc::fence_barrier_init();
+    // There are more slots than CTAs of this kernel can be resident, so one
+    // is free; sweeps repeat (bounded) because the release of the CTA this one
+    // replaces may still be on its way to memory.
+    int slot = -1;
+    const int64_t cta = blockIdx.x + (int64_t)gridDim.x * (blockIdx.y + (int64_t)gridDim.y * blockIdx.z);
+    const int start = (int)(cta % wsc.n_slots);
+    const long long t0 = clock64();
+    for (int sweep = 0; slot < 0; ++sweep) {
+      for (int i = 0; i < wsc.n_slots && slot < 0; ++i) {
+        const int s = (start + i) % wsc.n_slots;
+        if (atomicCAS(&wsc.locks[s], 0, 1) == 0) slot = s;
+      }
+      if (slot < 0 && clock64() - t0 > (1ll << 26)) break;
+    }
+    bars->slot = slot;
+    if (slot < 0) raise_status(p.status, 4 /* DASH_ERR_CUDA */, 23);
+  }
+  for (int i = threadIdx.x; i < kRows * kSeed; i += kThreads) seed[i] = kNegInf;
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(&bars->tmem_base, kMaxCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+  const int slot = bars->slot;
+  const bool live = slot >= 0 && n_chunks > 0;
+  float* X = live ? wsc.logits + (int64_t)slot * wsc.slot_floats : nullptr;
+
+  if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (live) {
+      bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->a_full, 0));
+      const uint64_t adesc0 = tc::smem_desc_sw128(smem + L::kOffA, 16, 1024);
+      const uint64_t bdesc0 = tc::smem_desc_sw128(smem + L::kOffB, 16, 1024);
+      for (int s = 0; ok && s < n_seg; ++s) {
+        if (s > 0) {
+          // the work warps have moved the previous segment out of TMEM
+          if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->tmem_free, (s - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+        }
+        const int j_end = min(n_chunks, (s + 1) * kSegChunks);
+        for (int j = s * kSegChunks; j < j_end; ++j) {
+          const int st = j & 1;
+          if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->b_full[st], (j >> 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+#pragma unroll
+          for (int term = 0; term < 2; ++term) {
+            const uint64_t bd = bdesc0 + (uint64_t)(((st * 2 + term) * L::kBTerm) >> 4);
+#pragma unroll
+            for (int kc = 0; kc < L::KC; ++kc) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_tf32_w(tmem + (j - s * kSegChunks) * kChunk,
+                           adesc0 + (uint64_t)((kc * L::kAChunk + k * 32) >> 4),
+                           bd + (uint64_t)((kc * L::kBChunk + k * 32) >> 4), kIdesc, (term | kc | k) ? 1u : 0u);
+            }
+          }
+          tc::mma_commit_w(&bars->b_empty[st]);
+        }
+        if (!ok) break;
+        tc::mma_commit_w(&bars->x_ready);
+      }
+      if (!ok) {
+        raise_status(p.status, 5 /* DASH_ERR_DEVICE_TIMEOUT */, 24);
+        atomicExch(&bars->abort, 1);
+      }
+      tc::mma_commit_w(&bars->drain);
+      tc::mbar_wait(&bars->drain, 0);
+    }
+  } else if (live) {
+    // ------------------------------------------------------------ operands and segment copies
+    if (threadIdx.x < kRows) {
+      // A: query row r in fp32, 128-byte swizzled
+      const int r = threadIdx.x;
+      const int pos = pos0 + r / G, head = g * G + r % G;
+      const bool valid = pos < p.S;
+      constexpr int EPV = 8;
+      const T* src = static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb + (int64_t)(valid ? pos : 0) * p.q.ss +
+                     (int64_t)head * p.q.sh;
+#pragma unroll
+      for (int v = 0; v < D / EPV; ++v) {
+        float f[EPV];
+        if (valid) {
+          Elt<T>::to_float(__ldg(reinterpret_cast<const uint4*>(src + v * EPV)), f);
+        } else {
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) f[e] = 0.f;
+        }
+        const int kc = (v * EPV) / 32, u0 = ((v * EPV) % 32) / 4;
+        uint8_t* base = smem + L::kOffA + kc * L::kAChunk;
+        *reinterpret_cast<float4*>(base + sw128(r, u0)) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(base + sw128(r, u0 + 1)) = make_float4(f[4], f[5], f[6], f[7]);
+      }
+    }
+    tc::fence_proxy_async_smem();
+    tc::mbar_arrive(&bars->a_full);
+
+    const bool loader = warp == kWorkWarps - 1 && lane == 0;
+    const uint8_t* split = reinterpret_cast<const uint8_t*>(p.summ_split) +
+                           bg * (int64_t)((p.t_cap + kChunk - 1) / kChunk) * 2 * L::kBTerm;
+    int issued = 0;
+    bool lok = true;
+    bool ok = true;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // tile row = TMEM lane
+    const int pos = pos0 + r / G;
+    const int t = pos / p.block;
+    const bool valid = pos < p.S;
+    float* xr = X + (int64_t)r * xstride;
+    float* sr = seed + r * kSeed;
+    for (int s = 0; s < n_seg; ++s) {
+      if (loader) {
+        // this segment's chunks and the first two of the next (their stages
+        // free up without waiting for this segment's copy)
+        const int j_end = min(n_chunks, (s + 1) * kSegChunks + 2);
+        for (; lok && issued < j_end; ++issued) {
+          const int j = issued, st = j & 1;
+          if (j >= 2 && !tc::mbar_wait(&bars->b_empty[st], ((j >> 1) - 1) & 1)) {
+            lok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&bars->b_full[st], 2 * L::kBTerm);
+          tc::bulk_load(smem + L::kOffB + (st * 2) * L::kBTerm, split + (int64_t)j * 2 * L::kBTerm, 2 * L::kBTerm,
+                        &bars->b_full[st]);
+        }
+      }
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->x_ready, s & 1));
+      if (!ok) break;
+      tc::fence_after_sync();
+      const int ch0 = s * (kMaxCols / 32), ch1 = min(n_wch, ch0 + kMaxCols / 32);
+      for (int ch = ch0 + (warp >> 2); ch < ch1; ch += kWorkWarps / 4) {
+        uint32_t v[32];
+        tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + (ch - ch0) * 32, v);
+        tc::tmem_wait_ld();
+        float m1 = kNegInf;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          float y[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = ch * 32 + j + e;
+            y[e] = (valid && is_cand(c, t, n_blocks, p.causal)) ? coef * __uint_as_float(v[j + e]) : kNegInf;
+            m1 = fmaxf(m1, y[e]);
+          }
+          *reinterpret_cast<float4*>(xr + ch * 32 + j) = make_float4(y[0], y[1], y[2], y[3]);
+        }
+        sr[ch & 31] = fmaxf(sr[ch & 31], m1);
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->tmem_free);
+    }
+    if (!ok) {
+      raise_status(p.status, 5 /* DASH_ERR_DEVICE_TIMEOUT */, 25);
+      atomicExch(&bars->abort, 1);
+    }
+    if (loader) {
+      // no bulk copy may still be landing in shared memory past this point
+      for (int j = max(0, issued - 2); j < issued; ++j) tc::mbar_wait(&bars->b_full[j & 1], (j >> 1) & 1);
+    }
+  }
+  __syncthreads();  // segments done: the slot holds the logits, the operand memory is free
+
+  const bool run = live && bars->abort == 0;
+  if (run)
+    for (int c = threadIdx.x; c < n_wch * 32; c += kThreads) pmask[c] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if (run && warp < kWorkWarps)
+    solve_and_compact<G>(p, X, xstride, seed, pmask, 0, kRows, b, g, pos0, n_blocks, warp, lane);
+  __syncthreads();
+  if (threadIdx.x == 0 && slot >= 0) {
+    __threadfence();  // this CTA's reads of the slot are done before another CTA may claim it
+    atomicExch(&wsc.locks[slot], 0);
+  }
+  if (run && to.ulist)
+    write_tile_list(p, to, pmask, n_wch * 32, lcnt, lcnt + kWideListCap, bg, tile, pos0, last, t_last, n_cols,
+                    warp, lane);
+  if (warp == kMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kMaxCols);
+  }
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_wide_g(const RouteParams& p, const TileOut& to, int tile0, int n_tiles, const WideScratch& w,
+                          cudaStream_t stream) {
+  using L = RLayout<D>;
+  auto kern = route_prefill_tc_wide_kernel<T, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_tiles, p.Hkv, p.B);
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(p, to, tile0, w);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_wide_t(const RouteParams& p, const TileOut& to, int tile0, int n_tiles, const WideScratch& w,
+                          cudaStream_t stream) {
+  switch (p.G) {
+    case 1: return launch_wide_g<T, D, 1>(p, to, tile0, n_tiles, w, stream);
+    case 2: return launch_wide_g<T, D, 2>(p, to, tile0, n_tiles, w, stream);
+    case 4: return launch_wide_g<T, D, 4>(p, to, tile0, n_tiles, w, stream);
+    default: return launch_wide_g<T, D, 8>(p, to, tile0, n_tiles, w, stream);
   }
 }
 
@@ -652,6 +962,36 @@ __global__ void __launch_bounds__(256) route_split_kernel(const float* summaries
 }  // namespace
 
 int route_tc_max_cols() { return kMaxCols; }
+
+int route_tc_wide_max_cols() { return kWideMaxCols; }
+
+size_t route_wide_scratch_bytes(int64_t t_cap, int n_slots) {
+  const int64_t slot_floats = (int64_t)kRows * (((t_cap + 63) / 64) * 64 + 4);
+  const size_t locks = ((size_t)n_slots * 4 + 255) & ~size_t(255);
+  return locks + (size_t)n_slots * (size_t)slot_floats * 4;
+}
+
+WideScratch route_wide_scratch(void* base, int64_t t_cap, int n_slots) {
+  WideScratch w{};
+  const size_t locks = ((size_t)n_slots * 4 + 255) & ~size_t(255);
+  w.locks = static_cast<int32_t*>(base);
+  w.logits = reinterpret_cast<float*>(static_cast<char*>(base) + locks);
+  w.n_slots = n_slots;
+  w.slot_floats = (int64_t)kRows * (((t_cap + 63) / 64) * 64 + 4);
+  return w;
+}
+
+cudaError_t launch_route_prefill_tc_wide(const RouteParams& p, const TileOut& to, int tile0, int n_tiles,
+                                         const WideScratch& w, cudaStream_t stream) {
+  if (n_tiles <= 0) return cudaSuccess;
+  if (!p.summ_split || !w.locks || w.n_slots <= 0) return cudaErrorInvalidValue;
+  if (p.D == 128) {
+    if (p.dtype == 1) return launch_wide_t<__half, 128>(p, to, tile0, n_tiles, w, stream);
+    return launch_wide_t<__nv_bfloat16, 128>(p, to, tile0, n_tiles, w, stream);
+  }
+  if (p.dtype == 1) return launch_wide_t<__half, 64>(p, to, tile0, n_tiles, w, stream);
+  return launch_wide_t<__nv_bfloat16, 64>(p, to, tile0, n_tiles, w, stream);
+}
 
 size_t route_split_bytes(int64_t B, int64_t Hkv, int64_t t_cap, int D) {
   return (size_t)(B * Hkv) * (size_t)((t_cap + kChunk - 1) / kChunk) * 2 * (size_t)(D / 32) * kChunk * 128;

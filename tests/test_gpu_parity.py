@@ -287,3 +287,125 @@ def test_device_status_and_bad_seqlens(dash):
     assert dash.device_status(ws) == 1
     dash.decode(q, k, v, sl, summ, cfg.alpha, cfg.block, workspace=ws)
     assert dash.device_status(ws) == 0
+
+
+# Tiles with more candidate blocks than TMEM holds logit columns (512) run the
+# segmented routing kernel (logits through a scratch slot in global memory).
+# Rows are sampled across the sequence, densely around the first such tile,
+# and at the end.
+WIDE = {
+    "wide_g4": _BASE.with_(name="wide_g4", heads=8, kv_heads=2, seq=36000),
+    "wide_g8_d64_f16": _BASE.with_(name="wide_g8_d64_f16", heads=16, kv_heads=2, head_dim=64, dtype="f16",
+                                   seq=34000),
+    "wide_g1_alpha2": _BASE.with_(name="wide_g1_alpha2", heads=2, kv_heads=2, seq=33500, alpha=2.0),
+    "wide_noncausal": _BASE.with_(name="wide_noncausal", heads=8, kv_heads=2, seq=33000, causal=False),
+    "wide_b128_g2_alpha125": _BASE.with_(name="wide_b128_g2_alpha125", heads=4, kv_heads=2, block=128, seq=70000,
+                                         alpha=1.25),
+}
+
+
+def _wide_rows(cfg):
+    P = 128 // cfg.group
+    first_wide = ((512 + 1) * cfg.block) // P * P if cfg.causal else 0
+    rows = set(range(0, cfg.seq, 211))
+    rows.update(range(max(0, first_wide - 48), min(cfg.seq, first_wide + 48), 3))
+    rows.update(range(cfg.seq - 70, cfg.seq))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name", sorted(WIDE))
+def test_wide_tile_routing_parity(dash, name):
+    cfg = WIDE[name]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    ws = torch.empty(dash.fwd_workspace_size(q, k, cfg.block), dtype=torch.uint8, device="cuda")
+    out = dash.fwd(q, k, v, w, cfg.alpha, cfg.block, cfg.causal, workspace=ws)
+    fl = dash.fwd_lists(ws, q, k, cfg.block)
+    summ = dash.summarize(k, w, cfg.block)
+    rt = dash.route(q, summ, cfg.alpha, cfg.block, cfg.causal, want_tau=True, want_p=True)
+    torch.cuda.synchronize()
+    assert dash.device_status(ws) == 0
+    assert -(-cfg.seq // cfg.block) > 512  # some tiles exceed TMEM's 512 columns
+    rows = _wide_rows(cfg)
+    rsel = torch.tensor(rows, device="cuda")
+    G, tol = cfg.group, OUT_TOL[cfg.dtype]
+    ref = oracle_heads_pooled(cfg, inp["plan"], [(0, g) for g in range(cfg.kv_heads)], rows)
+    worst = 0.0
+    for g in range(cfg.kv_heads):
+        recs, summ_o = ref[(0, g)]
+        serr = np.abs(fl["summaries"][0, g, : len(summ_o)].cpu().numpy() - summ_o).max()
+        assert serr <= 2e-5 * max(1.0, np.abs(summ_o).max()), f"{name}: summary error {serr:.3g}"
+        sel = {n: [t[0, g].index_select(0, rsel).cpu().numpy() for t in (src["idx"], src["logp"], src["cnt"])]
+               for n, src in (("fwd", fl), ("route", rt))}
+        p_rows = rt["p"][0, g * G:(g + 1) * G].index_select(1, rsel).cpu().numpy()
+        tau_rows = rt["tau"][0, g * G:(g + 1) * G].index_select(1, rsel).cpu().numpy()
+        o = out[0, :, g * G:(g + 1) * G].index_select(0, rsel).double().cpu().numpy()
+        for i, (pos, rec) in enumerate(zip(rows, recs)):
+            where = f"{name} g{g} pos{pos}"
+            for n, (idx, logp, cnt) in sel.items():
+                check_route_row(rec, idx[i], logp[i], cnt[i], f"{where} ({n})")
+            check_p_dense(rec, p_rows[:, i], tau_rows[:, i], where)
+            err = max_abs(o[i], rec["out"])
+            worst = max(worst, err)
+            assert err <= tol, f"{where}: output error {err:.3g} > {tol}"
+    print(f"{name}: max |out err| {worst:.3g}")
+
+
+def _dense_prior(idx, logp, cnt, fill=float("nan")):
+    """[..., t_cap] log p_bar at column c from ascending lists; `fill` elsewhere (never read)."""
+    T = idx.shape[-1]
+    dense = torch.full(idx.shape, fill, dtype=torch.float32, device=idx.device)
+    valid = torch.arange(T, device=idx.device) < cnt[..., None]
+    cols = torch.where(valid, idx.long(), torch.full_like(idx.long(), T))
+    padded = torch.cat([dense, torch.zeros(dense.shape[:-1] + (1,), device=idx.device)], dim=-1)
+    padded.scatter_(-1, cols, torch.where(valid, logp, torch.zeros_like(logp)))
+    return padded[..., :T].contiguous()
+
+
+@pytest.mark.parametrize("name,sigma", [("prefill_small", 1.0), ("g8_small", 1.0), ("g2_d64", 0.5),
+                                        ("g1_b128", 2.0), ("noncausal", 1.0), ("long_small", 1.0)])
+def test_sparse_on_bit_packed_mask(dash, name, sigma):
+    """dash_attn_sparse_mask (the pages' mask form) equals the list form bit for bit on the same
+    routing, and the oracle within the output tolerance; the dense prior is NaN wherever the
+    mask has no bit, so a read outside the selection would show."""
+    cfg = SMALL[name]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    summ = dash.summarize(k, w, cfg.block)
+    rt = dash.route(q, summ, cfg.alpha, cfg.block, cfg.causal)
+    mask = dash.lists_to_mask(rt["idx"], rt["cnt"])
+    dense = _dense_prior(rt["idx"], rt["logp"], rt["cnt"])
+    ref = dash.sparse(q, k, v, rt["idx"], rt["logp"], rt["cnt"], cfg.block, cfg.causal, sigma=sigma)
+    ws = torch.empty(dash.sparse_workspace_size(q, k, cfg.block, summ.shape[2]), dtype=torch.uint8, device="cuda")
+    got = dash.sparse_mask(q, k, v, mask, dense, cfg.block, cfg.causal, workspace=ws, sigma=sigma)
+    torch.cuda.synchronize()
+    assert dash.device_status(ws) == 0
+    assert torch.equal(got, ref)
+    # against the oracle on every KV group, a spread of rows
+    rows = sorted(set(range(0, cfg.seq, 7)) | {cfg.seq - 1})
+    oref = oracle_heads_pooled(cfg, inp["plan"], [(0, g) for g in range(cfg.kv_heads)], rows, sigma=sigma)
+    G, tol = cfg.group, OUT_TOL[cfg.dtype]
+    o = to_np(got)
+    for g in range(cfg.kv_heads):
+        for pos, rec in zip(rows, oref[(0, g)][0]):
+            err = max_abs(o[0, pos, g * G:(g + 1) * G], rec["out"])
+            assert err <= tol, f"{name} g{g} pos{pos}: output error {err:.3g}"
+
+
+def test_sparse_mask_ignores_and_reports_non_candidate_bits(dash):
+    cfg = SMALL["prefill_small"]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    summ = dash.summarize(k, w, cfg.block)
+    rt = dash.route(q, summ, cfg.alpha, cfg.block, True)
+    mask = dash.lists_to_mask(rt["idx"], rt["cnt"])
+    dense = _dense_prior(rt["idx"], rt["logp"], rt["cnt"])
+    ref = dash.sparse(q, k, v, rt["idx"], rt["logp"], rt["cnt"], cfg.block, True)
+    bad = mask.clone()
+    pos = 700  # block 10: set the bit of its own block, not a candidate
+    t = pos // cfg.block
+    bad[0, 1, pos, t // 32] |= (1 << (t % 32)) if t % 32 < 31 else -(1 << 31)
+    ws = torch.empty(dash.sparse_workspace_size(q, k, cfg.block, summ.shape[2]), dtype=torch.uint8, device="cuda")
+    got = dash.sparse_mask(q, k, v, bad, dense, cfg.block, True, workspace=ws)
+    assert dash.device_status(ws) == 1
+    assert torch.equal(got, ref)
