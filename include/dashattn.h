@@ -421,13 +421,43 @@ dash_status_t dash_attn_sparse_mask(const dash_tensor_t* q, const dash_tensor_t*
  *  - The first call on each device looks up the array's address; make that
  *    first call before any stream capture.
  *  - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
- *  - The status word it uses is the array's; dash_attn_get_device_status
- *    cannot read it, so seqlens must be valid (1 <= seqlens[b] <= Lmax).
+ *  - The status word it uses is the array's: read it with
+ *    dash_attn_decode_noalloc_status (a seqlens entry out of range is clamped
+ *    and reported there as DASH_ERR_INVALID_ARGUMENT).
+ *  - The address looked up by the first call stays valid for the life of the
+ *    device's context; after cudaDeviceReset this entry point must not be
+ *    called on that device again.
  */
 dash_status_t dash_attn_decode_noalloc(const dash_tensor_t* q, const dash_tensor_t* kcache,
                                        const dash_tensor_t* vcache, const int32_t* seqlens, const float* summaries,
                                        int64_t t_cap, float alpha, int block, dash_tensor_t* out,
                                        dash_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the status word of the last
+ * dash_attn_decode_noalloc call on the current device (kept in its scratch
+ * array), like dash_attn_get_device_status does for a workspace.  Returns
+ * DASH_ERR_INVALID_ARGUMENT when no such call has been made on this device.
+ * Allocates nothing.
+ */
+dash_status_t dash_attn_decode_noalloc_status(dash_stream_t stream);
+
+/*
+ * Test of the device-side timeout path (the paper has no counterpart): runs
+ * the stage-2 tensor-core kernel of dash_attn_sparse on the same arguments,
+ * but with its copy-issuing warp withholding every copy and every other wait
+ * for a hand-off bounded by `wait_cycles` SM cycles (1024 .. 2^31) instead of
+ * about a second.  Every such wait runs out; the kernel records
+ * DASH_ERR_DEVICE_TIMEOUT in the workspace status word, frees its tensor
+ * memory and returns, so the context stays usable and the next call on the
+ * same workspace starts clean.  `out` is not written.  Nothing is left in
+ * flight: waits that drain issued copies or MMAs keep the default bound.
+ * f16/bf16 only.
+ */
+dash_status_t dash_attn_debug_sparse_stalled(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                                             const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap,
+                                             int block, int causal, dash_tensor_t* out, void* workspace,
+                                             size_t workspace_bytes, int64_t wait_cycles, dash_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads the device status word of a workspace

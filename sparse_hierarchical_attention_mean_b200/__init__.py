@@ -43,6 +43,7 @@ EXPORTED = (
     "dash_attn_fwd_ex",
     "dash_attn_sparse_ex",
     "dash_attn_sparse_mask",
+    "dash_attn_debug_sparse_stalled",
     "dash_attn_decode_ex",
     "dash_attn_lists_to_mask",
     "dash_attn_cp_scores",
@@ -59,6 +60,7 @@ EXPORTED = (
     "dash_attn_sparse",
     "dash_attn_get_device_status",
     "dash_attn_decode_noalloc",
+    "dash_attn_decode_noalloc_status",
     "dash_attn_bwd_workspace_size",
     "dash_attn_bwd",
 )
@@ -116,6 +118,7 @@ def _load() -> ctypes.CDLL:
         "dash_attn_fwd_ex": (i32, [T, T, T, vp, f32, i32, i32, T, vp, sz, O, vp]),
         "dash_attn_sparse_ex": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, O, vp]),
         "dash_attn_sparse_mask": (i32, [T, T, T, vp, i64, vp, i64, i32, i32, T, vp, sz, O, vp]),
+        "dash_attn_debug_sparse_stalled": (i32, [T, T, T, vp, vp, vp, i64, i32, i32, T, vp, sz, i64, vp]),
         "dash_attn_decode_ex": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
         "dash_attn_lists_to_mask": (i32, [vp, vp, i64, i64, vp, i64, vp]),
         "dash_attn_cp_scores": (i32, [T, i64, vp, i64, i64, i64, vp, i64, f32, i32, vp, i64, vp]),
@@ -126,6 +129,7 @@ def _load() -> ctypes.CDLL:
         "dash_attn_decode_paged": (i32, [T, T, T, vp, i64, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
         "dash_attn_get_device_status": (i32, [vp, vp]),
         "dash_attn_decode_noalloc": (i32, [T, T, T, vp, vp, i64, f32, i32, T, vp]),
+        "dash_attn_decode_noalloc_status": (i32, [vp]),
         "dash_attn_bwd_workspace_size": (sz, [T, T, i32]),
         "dash_attn_bwd": (i32, [T, T, T, vp, T, T, f32, i32, i32, O, T, T, T, vp, vp, sz, vp]),
     }
@@ -316,6 +320,17 @@ def sparse_mask(q, k, v, mask: torch.Tensor, logp_dense: torch.Tensor, block: in
     return out
 
 
+def debug_sparse_stalled(q, k, v, idx, logp, cnt, block: int, causal: bool, out, workspace, wait_cycles: int,
+                         stream=None) -> None:
+    """Stage 2 with its copies withheld and short waits (see dash_attn_debug_sparse_stalled): a test of
+    the timeout path; the workspace status word then reads DASH_ERR_DEVICE_TIMEOUT."""
+    qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
+    _check(_lib.dash_attn_debug_sparse_stalled(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), idx.data_ptr(),
+                                               logp.data_ptr(), cnt.data_ptr(), idx.shape[-1], block,
+                                               1 if causal else 0, ctypes.byref(od), workspace.data_ptr(),
+                                               workspace.numel(), wait_cycles, _stream(stream)))
+
+
 def lists_to_mask(idx: torch.Tensor, cnt: torch.Tensor, n_words: int | None = None, stream=None) -> torch.Tensor:
     """Bit-packed active-block masks [..., n_words] (int32 bit patterns) from lists idx [..., t_cap], cnt [...]."""
     t_cap = idx.shape[-1]
@@ -487,6 +502,11 @@ def decode_noalloc(q, kcache, vcache, seqlens, summaries, alpha: float, block: i
                                          summaries.data_ptr(), summaries.shape[2], alpha, block, ctypes.byref(od),
                                          _stream(stream)))
     return out
+
+
+def decode_noalloc_status(stream=None) -> int:
+    """Status word of the last decode_noalloc call on the current device (synchronises)."""
+    return _lib.dash_attn_decode_noalloc_status(_stream(stream))
 
 
 def device_status(workspace: torch.Tensor, stream=None) -> int:

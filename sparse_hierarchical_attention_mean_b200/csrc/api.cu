@@ -527,7 +527,8 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
                                 int causal, float sigma, dash_tensor_t* out, const TileLists& tl, int tile_pos,
                                 int64_t n_tiles, int union_tile0, dash::DeviceStatus* status,
                                 cudaStream_t stream, const uint32_t* mask = nullptr, int n_words = 0,
-                                const float* logp_dense = nullptr) {
+                                const float* logp_dense = nullptr, long long wait_cycles = 0,
+                                int stall_producer = 0) {
   if (q->dtype != DASH_F32 && union_tile0 < n_tiles) {
     dash::UnionParams u{};
     u.B = (int)q->b;
@@ -600,6 +601,8 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
   p.sigma = sigma;
   p.status = status;
   p.logp_dense = logp_dense;
+  p.wait_cycles = wait_cycles;
+  p.stall_producer = stall_producer;
   cudaError_t e = dash::launch_sparse_prefill(p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
   return DASH_OK;
@@ -652,6 +655,36 @@ dash_status_t dash_attn_sparse_ex(const dash_tensor_t* q, const dash_tensor_t* k
                      at<int32_t>(workspace, L.pcnt), at<int32_t>(workspace, L.psteps), L.n_pairs};
   st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, sigma, out, tl, L.tile_pos, L.n_tiles, 0,
                   at<dash::DeviceStatus>(workspace, L.status), s);
+  return st ? st : ok();
+}
+
+dash_status_t dash_attn_debug_sparse_stalled(const dash_tensor_t* q, const dash_tensor_t* k, const dash_tensor_t* v,
+                                             const int32_t* idx, const float* logp, const int32_t* cnt, int64_t t_cap,
+                                             int block, int causal, dash_tensor_t* out, void* workspace,
+                                             size_t workspace_bytes, int64_t wait_cycles, dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_fwd_shapes(q, k, v, out))) return st;
+  if (block != 64 && block != 128) return fail(DASH_ERR_UNSUPPORTED, "block %d not in {64, 128}", block);
+  if (q->dtype == DASH_F32) return fail(DASH_ERR_UNSUPPORTED, "the stalled stage 2 is the f16/bf16 kernel");
+  if (k->s != q->s) return fail(DASH_ERR_INVALID_ARGUMENT, "prefill needs k and q of equal length");
+  if (!idx || !logp || !cnt) return fail(DASH_ERR_INVALID_ARGUMENT, "null routing lists");
+  if (wait_cycles < 1024 || wait_cycles > (1ll << 31))
+    return fail(DASH_ERR_INVALID_ARGUMENT, "wait_cycles must be in [1024, 2^31]");
+  const int64_t T = (q->s + block - 1) / block;
+  if (t_cap < T) return fail(DASH_ERR_INVALID_ARGUMENT, "t_cap %lld < ceil(S / block)", (long long)t_cap);
+  const SparseLayout L = sparse_layout(q->b, q->s, q->h, k->h, block, t_cap);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < L.total)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.status), 0, sizeof(dash::DeviceStatus), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  const TileLists tl{at<int32_t>(workspace, L.ulist), at<uint4>(workspace, L.umask), at<int32_t>(workspace, L.ucnt),
+                     at<int32_t>(workspace, L.usteps), at<int32_t>(workspace, L.plist), at<uint4>(workspace, L.pmask),
+                     at<int32_t>(workspace, L.pcnt), at<int32_t>(workspace, L.psteps), L.n_pairs};
+  st = run_sparse(q, k, v, idx, logp, cnt, t_cap, block, causal, 1.0f, out, tl, L.tile_pos, L.n_tiles, 0,
+                  at<dash::DeviceStatus>(workspace, L.status), s, nullptr, 0, nullptr, wait_cycles, 1);
   return st ? st : ok();
 }
 

@@ -128,6 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint4* pmask = p.pmask + pix * p.t_cap * kTiles;
   const int pcnt = p.pcnt[pix];
   const int n_steps = p.psteps[pix];
+  // how long a consumer waits for a hand-off (drains keep the default)
+  const long long budget = p.wait_cycles > 0 ? p.wait_cycles : tc::kWaitCycles;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars->q_full, kTiles * kRows);
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int last_needed = p.causal ? min(pos0 + kTiles * P, p.S) - 1 : p.S - 1;
     int i = 0;
     bool ok = true;
-    for (int u0 = 0; ok && u0 < pcnt; u0 += 32) {
+    for (int u0 = 0; ok && !p.stall_producer && u0 < pcnt; u0 += 32) {
       const bool have = u0 + lane < pcnt;
       const int my_c = have ? __ldg(plist + u0 + lane) : 0;
       const uint4 my_m0 = have ? __ldg(pmask + (u0 + lane) * kTiles) : make_uint4(0u, 0u, 0u, 0u);
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tok0 > last_needed) continue;
           if (lane == 0) {
             const int st = i % kStages;
-            if (i >= kStages && !tc::mbar_wait(&bars->kv_empty[st], ((i / kStages) - 1) & 1)) {
+            if (i >= kStages && !tc::mbar_wait(&bars->kv_empty[st], ((i / kStages) - 1) & 1, budget)) {
               fail_timeout(bars, p.status, 1);
               ok = false;
             } else {
@@ -220,7 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the issue loop (descriptors stay warp-uniform);
     // one elected lane issues each MMA and commit.
-    auto wait_all = [&](uint64_t* bar, uint32_t par) { return __all_sync(0xffffffffu, tc::mbar_wait(bar, par)); };
+    auto wait_all = [&](uint64_t* bar, uint32_t par) {
+      return __all_sync(0xffffffffu, tc::mbar_wait(bar, par, budget));
+    };
     bool ok = wait_all(&bars->q_full, 0);
     if (!ok) fail_timeout(bars, p.status, 2);
     tc::fence_after_sync();
@@ -315,14 +319,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < n_steps; ++i) {
       const int st = i % kStages;
       // the step's descriptor is published with its K/V copies
-      if (!tc::mbar_wait(&bars->kv_full[st], (i / kStages) & 1)) {
+      if (!tc::mbar_wait(&bars->kv_full[st], (i / kStages) & 1, budget)) {
         fail_timeout(bars, p.status, 10);
         ok = false;
         break;
       }
       const int c = bars->desc[st].c, tok0 = bars->desc[st].tok0;
       if (bars->desc[st].first) bias = row.bias(c, bars->desc[st].mask[t]);
-      if (!tc::mbar_wait(&bars->s_full[t], i & 1)) {
+      if (!tc::mbar_wait(&bars->s_full[t], i & 1, budget)) {
         fail_timeout(bars, p.status, 6);
         ok = false;
         break;
@@ -413,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&bars->p_full[t]);
     }
     // ---- epilogue: O / l -> out
-    if (ok && tc::mbar_wait(&bars->o_final, 0)) {
+    if (ok && tc::mbar_wait(&bars->o_final, 0, budget)) {
       tc::fence_after_sync();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
       T* dst = static_cast<T*>(const_cast<void*>(p.out.data)) + (int64_t)b * p.out.sb +

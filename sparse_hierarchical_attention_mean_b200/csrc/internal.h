@@ -138,6 +138,12 @@ struct SparseParams {
   // [B, Hkv, S, t_cap], log p_bar of block c at column c, read only where the
   // tile work list marks the row as selecting c
   const float* logp_dense;
+  // test of the timeout path (tensor-core kernel): cycles a consumer waits for
+  // a hand-off before it gives up (0: the default, about a second), and a
+  // switch that makes the producer issue no copies, so every consumer wait
+  // runs out.  Waits that drain issued copies or MMAs always use the default.
+  long long wait_cycles;
+  int stall_producer;
 };
 // positions per stage-2 tile (tiles are 128 rows)
 int sparse_tile_positions(int G, int block);

@@ -20,7 +20,15 @@
 //
 // Set-up: the first call on each device looks up the array's device address
 // with cudaGetSymbolAddress (with that device current); that first call
-// should therefore come before any stream capture.
+// should therefore come before any stream capture.  The address stays valid
+// for the life of the device's context: after cudaDeviceReset (or anything
+// else that destroys the primary context) the module is loaded again at
+// another address, so a process that resets a device must not call this
+// entry point (or dash_attn_decode_noalloc_status) on it again.
+//
+// The status word of a call (a seqlens entry out of range, a bounded device
+// wait that gave up) sits at the start of the array;
+// dash_attn_decode_noalloc_status reads it without allocating.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -74,4 +82,19 @@ extern "C" dash_status_t dash_attn_decode_noalloc(const dash_tensor_t* q, const 
   }
   return dash_attn_decode(q, kcache, vcache, seqlens, summaries, t_cap, alpha, block, out, scratch,
                           kScratchBytes, stream);
+}
+
+extern "C" dash_status_t dash_attn_decode_noalloc_status(dash_stream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return dash::set_last_error(DASH_ERR_CUDA, "dash_attn_decode_noalloc_status: no usable current device");
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    scratch = g_scratch_addr[dev];
+  }
+  if (!scratch)
+    return dash::set_last_error(DASH_ERR_INVALID_ARGUMENT,
+                                "dash_attn_decode_noalloc_status: no dash_attn_decode_noalloc call on this device yet");
+  return dash_attn_get_device_status(scratch, stream);
 }

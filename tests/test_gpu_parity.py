@@ -409,3 +409,23 @@ def test_sparse_mask_ignores_and_reports_non_candidate_bits(dash):
     got = dash.sparse_mask(q, k, v, bad, dense, cfg.block, True, workspace=ws)
     assert dash.device_status(ws) == 1
     assert torch.equal(got, ref)
+
+
+def test_bounded_wait_gives_up_and_reports(dash):
+    """A stage-2 launch whose copies never come: every bounded wait runs out after 2^20
+    cycles, the status word reads DASH_ERR_DEVICE_TIMEOUT (5) and the context stays usable;
+    the next call on the same workspace reports 0 and matches a call that never stalled."""
+    cfg = SMALL["prefill_small"]
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w = inp["q"], inp["k"], inp["v"], inp["w_s"]
+    summ = dash.summarize(k, w, cfg.block)
+    rt = dash.route(q, summ, cfg.alpha, cfg.block, True)
+    ref = dash.sparse(q, k, v, rt["idx"], rt["logp"], rt["cnt"], cfg.block, True)
+    ws = torch.empty(dash.sparse_workspace_size(q, k, cfg.block, summ.shape[2]), dtype=torch.uint8, device="cuda")
+    junk = torch.zeros_like(q)
+    dash.debug_sparse_stalled(q, k, v, rt["idx"], rt["logp"], rt["cnt"], cfg.block, True, junk, ws, 1 << 20)
+    assert dash.device_status(ws) == 5
+    out = dash.sparse(q, k, v, rt["idx"], rt["logp"], rt["cnt"], cfg.block, True, workspace=ws)
+    assert dash.device_status(ws) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
