@@ -46,3 +46,20 @@ def test_noalloc_decode_refuses_problems_beyond_its_scratch(cuda_lib):
         dash.decode_noalloc(q, kc, kc, sl, summ, 1.5, 64)
     assert e.value.status == 2
     assert "scratch" in str(e.value)
+
+
+def test_noalloc_decode_reports_bad_seqlens_through_its_status(cuda_lib):
+    # the status word lives in the library-owned array; the accessor reads it
+    # without allocating: an out-of-range context length is clamped on the
+    # device and reported, and the next valid call reports success again
+    dash = cuda_lib
+    cfg = get_config("decode").with_(batch=3, seq=2048, seqlen_lo=100, seqlen_hi=2048)
+    inp = full_inputs(cfg, device="cuda")
+    q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
+    summ = dash.summarize(k, w, cfg.block, seqlens=sl)
+    bad = sl.clone()
+    bad[1] = cfg.seq + 5
+    dash.decode_noalloc(q, k, v, bad, summ, cfg.alpha, cfg.block)
+    assert dash.decode_noalloc_status() == 1
+    dash.decode_noalloc(q, k, v, sl, summ, cfg.alpha, cfg.block)
+    assert dash.decode_noalloc_status() == 0
