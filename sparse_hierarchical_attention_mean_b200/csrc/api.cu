@@ -215,9 +215,11 @@ DecodeLayout decode_layout(int64_t B, int64_t H, int64_t Hkv, int64_t D, int blo
 
 // Workspace of dash_attn_bwd.
 struct BwdLayout {
-  size_t status, summ, split, wide, idx, logp, cnt, tau, lse, dd, dz, umask, kbar, ds, total;
+  size_t status, summ, split, wide, idx, logp, cnt, tau, lse, dd, dz, umask, kbar, ds, lists, rmask, rrank, tbits,
+      total;
   int64_t T, n_words;
   int n_slots;
+  SparseLayout sl;  // tile work lists of the stage-2 pass that takes each row's log-sum-exp
 };
 
 BwdLayout bwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, int block) {
@@ -245,6 +247,11 @@ BwdLayout bwd_layout(int64_t B, int64_t S, int64_t H, int64_t Hkv, int64_t D, in
   take(L.umask, (size_t)B * Hkv * L.T * L.n_words * 4);
   take(L.kbar, (size_t)B * Hkv * L.T * D * 4);
   take(L.ds, (size_t)B * Hkv * L.T * D * 4);
+  L.sl = sparse_layout(B, S, H, Hkv, block, L.T);
+  take(L.lists, L.sl.total);
+  take(L.rmask, (size_t)B * Hkv * S * L.n_words * 4);
+  take(L.rrank, (size_t)B * Hkv * S * L.n_words * 4);
+  take(L.tbits, (size_t)B * Hkv * L.sl.n_tiles * L.n_words * 4);
   L.total = off;
   return L;
 }
@@ -528,7 +535,7 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
                                 int64_t n_tiles, int union_tile0, dash::DeviceStatus* status,
                                 cudaStream_t stream, const uint32_t* mask = nullptr, int n_words = 0,
                                 const float* logp_dense = nullptr, long long wait_cycles = 0,
-                                int stall_producer = 0) {
+                                int stall_producer = 0, float* lse = nullptr, int skip_out = 0) {
   if (q->dtype != DASH_F32 && union_tile0 < n_tiles) {
     dash::UnionParams u{};
     u.B = (int)q->b;
@@ -603,6 +610,8 @@ static dash_status_t run_sparse(const dash_tensor_t* q, const dash_tensor_t* k, 
   p.logp_dense = logp_dense;
   p.wait_cycles = wait_cycles;
   p.stall_producer = stall_producer;
+  p.lse = lse;
+  p.skip_out = skip_out;
   cudaError_t e = dash::launch_sparse_prefill(p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention");
   return DASH_OK;
@@ -822,6 +831,29 @@ dash_status_t dash_attn_bwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   if ((st = run_route(q, summ, k->h, L.T, alpha, block, causal, idx, logp, cnt, tau, nullptr, nullptr, dst, s, nullptr,
                       at<float>(workspace, L.split), L.n_slots ? at<char>(workspace, L.wide) : nullptr)))
     return st;
+  // each row's log-sum-exp: the forward's stage-2 kernel on the same lists,
+  // without writing an output
+  float* lse = at<float>(workspace, L.lse);
+  {
+    char* lw = at<char>(workspace, L.lists);
+    const TileLists tl{at<int32_t>(lw, L.sl.ulist), at<uint4>(lw, L.sl.umask), at<int32_t>(lw, L.sl.ucnt),
+                       at<int32_t>(lw, L.sl.usteps), at<int32_t>(lw, L.sl.plist), at<uint4>(lw, L.sl.pmask),
+                       at<int32_t>(lw, L.sl.pcnt), at<int32_t>(lw, L.sl.psteps), L.sl.n_pairs};
+    dash_tensor_t scratch_out = *out;  // not written (skip_out)
+    if ((st = run_sparse(q, k, v, idx, logp, cnt, L.T, block, causal, sigma, &scratch_out, tl, L.sl.tile_pos,
+                         L.sl.n_tiles, 0, dst, s, nullptr, 0, nullptr, 0, 0, lse, 1)))
+      return st;
+    // which tiles hold which blocks, and which blocks each row selected, as bit masks
+    e = dash::launch_tile_bits(tl.ulist, tl.ucnt, q->b * k->h * L.sl.n_tiles, L.T, at<uint32_t>(workspace, L.tbits),
+                               (int)L.n_words, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tile bits");
+    e = dash::launch_lists_to_mask(idx, cnt, q->b * k->h * q->s, L.T, at<uint32_t>(workspace, L.rmask),
+                                   (int)L.n_words, s);
+    if (e != cudaSuccess) return cuda_fail(e, "row masks");
+    e = dash::launch_row_ranks(at<uint32_t>(workspace, L.rmask), q->b * k->h * q->s, (int)L.n_words,
+                               at<int32_t>(workspace, L.rrank), s);
+    if (e != cudaSuccess) return cuda_fail(e, "row ranks");
+  }
   dash::BwdParams p{};
   p.idx = idx;
   p.logp = logp;
@@ -851,7 +883,7 @@ dash_status_t dash_attn_bwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   p.t_cap = L.T;
   p.n_qblocks = (int)L.T;
   p.n_words = (int)L.n_words;
-  p.lse = at<float>(workspace, L.lse);
+  p.lse = lse;
   p.dd = at<float>(workspace, L.dd);
   p.dz = at<float>(workspace, L.dz);
   p.umask = at<uint32_t>(workspace, L.umask);
@@ -859,6 +891,10 @@ dash_status_t dash_attn_bwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   p.ds = at<float>(workspace, L.ds);
   p.dw_s = dw_s;
   p.status = dst;
+  p.tbits = at<uint32_t>(workspace, L.tbits);
+  p.rmask = at<uint32_t>(workspace, L.rmask);
+  p.rrank = at<int32_t>(workspace, L.rrank);
+  p.n_tiles = (int)L.sl.n_tiles;
   e = dash::launch_bwd(p, s);
   if (e != cudaSuccess) return cuda_fail(e, "backward");
   return ok();

@@ -416,8 +416,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->p_full[t]);
     }
-    // ---- epilogue: O / l -> out
-    if (ok && tc::mbar_wait(&bars->o_final, 0, budget)) {
+    // ---- epilogue: the row's log-sum-exp (log2 units) if wanted, O / l -> out
+    if (ok && p.lse && row.valid) p.lse[((int64_t)b * p.H + head) * p.S + row.pos] = m_used + log2f(lsum);
+    if (p.skip_out) {
+      // nothing to read back; the MMA warp drains its MMAs before TMEM is freed
+    } else if (ok && tc::mbar_wait(&bars->o_final, 0, budget)) {
       tc::fence_after_sync();
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
       T* dst = static_cast<T*>(const_cast<void*>(p.out.data)) + (int64_t)b * p.out.sb +
@@ -452,8 +455,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------ host side
 
+namespace {
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -466,8 +472,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D map over a [B, S, H, D] view (innermost first: D, H, S, B), 128-byte
-// swizzle, box {64, box_h, box_s, 1}.
+}  // namespace
+
 bool make_map(CUtensorMap* map, const View& v, int dtype, int64_t B, int64_t S, int64_t H, int D, int box_h,
               int box_s) {
   auto fn = encode_fn();
@@ -483,6 +489,8 @@ bool make_map(CUtensorMap* map, const View& v, int dtype, int64_t B, int64_t S, 
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <typename T, int D>
 cudaError_t launch_tc(const SparseParams& p, cudaStream_t stream) {

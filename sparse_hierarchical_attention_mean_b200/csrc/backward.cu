@@ -11,14 +11,15 @@
 //
 // Four kernels, all on the forward's lists (the union of a query block's
 // lists is rebuilt here):
-//   bwd_row    one CTA per (query block, head); warp w owns 16 rows.  Two
-//              passes over the 64-key chunks of the union of the rows'
-//              selected blocks and the diagonal block: the first takes the
-//              row log-sum-exp, the second P, dP = dout V^T, dS = P (dP - D)
-//              and dq = dS K / sqrt(d), plus each row's d log p_bar of every
-//              selected block (the row sum of dS over the block).  All three
-//              products are warp-level MMAs (m16n8k16, fp32 accumulate); dS
-//              is the accumulator re-packed as the A operand.
+//   bwd_row    one CTA per (query block, head); warp w owns 16 rows.  One
+//              pass over the 64-key chunks of the union of the rows'
+//              selected blocks and the diagonal block, with each row's
+//              log-sum-exp from the forward's stage-2 kernel: P, dP = dout
+//              V^T, dS = P (dP - D) and dq = dS K / sqrt(d), plus each row's
+//              d log p_bar of every selected block (the row sum of dS over the
+//              block).  All three products are warp-level MMAs (m16n8k16,
+//              fp32 accumulate); dS is the accumulator re-packed as the A
+//              operand.
 //   bwd_route  one CTA per (row, KV head): the entmax vector-Jacobian
 //              product per head from the recomputed scores and the
 //              forward's thresholds, and dq += gamma dz S.
@@ -43,7 +44,6 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kKeyChunk = 64;  // keys per step of bwd_row
-constexpr int kRowChunk = 32;  // query rows per step of bwd_key
 
 // rows [0, n_rows) of a [n_rows][D] tile from `g` (row stride `stride`
 // elements); rows >= n_valid are zero-filled.  Requires n_valid >= 1.
@@ -114,10 +114,6 @@ __device__ __forceinline__ void tile_xb(const float (*x)[4], uint32_t bbase, int
 __device__ __forceinline__ float quad_sum(float x) {
   x += __shfl_xor_sync(kFull, x, 1);
   return x + __shfl_xor_sync(kFull, x, 2);
-}
-__device__ __forceinline__ float quad_max(float x) {
-  x = fmaxf(x, __shfl_xor_sync(kFull, x, 1));
-  return fmaxf(x, __shfl_xor_sync(kFull, x, 2));
 }
 
 // prior of the diagonal block, log2 units: sigma * log(1/N), 0 when N = 0
@@ -285,61 +281,10 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
   };
   constexpr uint32_t kBufBytes = kKeyChunk * D * sizeof(T);
 
-  // pass 1: log-sum-exp of every row.  The next chunk's K streams in while
-  // this one is reduced.
-  float m_a = kNegInf, m_b = kNegInf, l_a = 0.f, l_b = 0.f;
+  // each row's log-sum-exp (log2 units) comes from the forward's stage-2 kernel
   int buf = 0;
-  issue(next_ok(0), 0, false);
-  for (int ch = 0; ch < nchunks; ++ch) {
-    const int bi = ch / SPB, sub = ch - bi * SPB;
-    const int c = ulist[bi];
-    const bool diag = bi == nu;
-    const int key0 = c * BLK + sub * kKeyChunk;
-    float ba, bb;
-    int ea, eb;
-    row_bias(c, diag, sub, ba, bb, ea, eb);
-    if (!chunk_ok(ch)) continue;
-    __syncthreads();  // the other buffer's readers are done
-    issue(next_ok(ch + 1), buf ^ 1, false);
-    cp_async_wait<1>();
-    __syncthreads();
-    float s[8][4];
-    tile_abt<T, D, 4>(qs_b, warp * 16, ks_b + buf * kBufBytes, lane, s);
-    logits(s, key0, diag, ba, bb);
-    float mx_a = kNegInf, mx_b = kNegInf;
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      mx_a = fmaxf(mx_a, fmaxf(s[n][0], s[n][1]));
-      mx_b = fmaxf(mx_b, fmaxf(s[n][2], s[n][3]));
-    }
-    mx_a = quad_max(mx_a);
-    mx_b = quad_max(mx_b);
-    if (mx_a > m_a) {
-      l_a *= exp2f(m_a - mx_a);
-      m_a = mx_a;
-    }
-    if (mx_b > m_b) {
-      l_b *= exp2f(m_b - mx_b);
-      m_b = mx_b;
-    }
-    if (m_a != kNegInf)
-#pragma unroll
-      for (int n = 0; n < 8; ++n) l_a += exp2f(s[n][0] - m_a) + exp2f(s[n][1] - m_a);
-    if (m_b != kNegInf)
-#pragma unroll
-      for (int n = 0; n < 8; ++n) l_b += exp2f(s[n][2] - m_b) + exp2f(s[n][3] - m_b);
-    buf ^= 1;
-  }
-  cp_async_wait<0>();
-  l_a = quad_sum(l_a);
-  l_b = quad_sum(l_b);
-  // every valid row attends at least its own token, so m and l are finite
-  const float lse_a = va ? m_a + log2f(l_a) : 0.f;
-  const float lse_b = vb ? m_b + log2f(l_b) : 0.f;
-  if (tq == 0) {
-    if (va) p.lse[((int64_t)b * p.H + h) * S + pa] = lse_a;
-    if (vb) p.lse[((int64_t)b * p.H + h) * S + pb] = lse_b;
-  }
+  const float lse_a = va ? p.lse[((int64_t)b * p.H + h) * S + pa] : 0.f;
+  const float lse_b = vb ? p.lse[((int64_t)b * p.H + h) * S + pb] : 0.f;
   const float d_a = Dsm[ra], d_b = Dsm[rb];
 
   // pass 2: dS, dq and d log p_bar, with the same prefetch of K and V
@@ -347,11 +292,8 @@ __global__ void __launch_bounds__(2 * BLK) bwd_row_kernel(BwdParams p) {
 #pragma unroll
   for (int n = 0; n < NT; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
   float dl_a = 0.f, dl_b = 0.f;
-  cur_a = cur_b = 0;
   float* dz_a = p.dz + (rowbase + (va ? pa : row0)) * tc * p.G + hh;
   float* dz_b = p.dz + (rowbase + (vb ? pb : row0)) * tc * p.G + hh;
-  __syncthreads();  // pass 1's readers are done with both buffers
-  buf = 0;
   issue(next_ok(0), 0, true);
   for (int ch = 0; ch < nchunks; ++ch) {
     const int bi = ch / SPB, sub = ch - bi * SPB;
@@ -509,222 +451,6 @@ __global__ void __launch_bounds__(128) bwd_route_kernel(BwdParams p) {
   }
 }
 
-// ------------------------------------------------------------------ bwd_key
-// 4-byte cp.async (zero fill when !valid; `gmem` must still be a readable address)
-__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(smem)), "l"(gmem),
-               "r"(valid ? 4 : 0)
-               : "memory");
-}
-
-template <typename T, int D, int BLK>
-__global__ void __launch_bounds__(2 * BLK, BLK == 64 ? 3 : 1) bwd_key_kernel(BwdParams p) {
-  constexpr int NW = BLK / 16, NTH = NW * 32;
-  constexpr int NT = D / 8;
-  constexpr int NRC = BLK / kRowChunk;
-  constexpr int RC = kRowChunk;
-  extern __shared__ __align__(128) uint8_t smem[];
-  T* Ks = reinterpret_cast<T*>(smem);  // [BLK][D]
-  T* Vs = Ks + BLK * D;                // [BLK][D]
-  T* Qs = Vs + BLK * D;                // [2][32][D] (double buffer)
-  T* dOs = Qs + 2 * RC * D;            // [2][32][D]
-  // per row of a chunk, raw: [2][4][32] = log p_bar entry, lse, dout . out, dL/dz
-  float* raw = reinterpret_cast<float*>(dOs + 2 * RC * D);
-  int* es = reinterpret_cast<int*>(raw + 2 * 4 * RC);  // [BLK] entry of the block in each row's list
-  float* dss = reinterpret_cast<float*>(es + BLK);     // [D]
-  float* dkb = dss + D;                                 // [D]
-  __shared__ int chunk_any[NRC];
-
-  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, tq = lane & 3;
-  const int S = p.S;
-  const int64_t tc = p.t_cap;
-  const int G = p.G;
-  const int key0 = c * BLK;
-  const int nkeys = min(BLK, S - key0);
-  if (nkeys <= 0) return;
-  const int64_t bg = (int64_t)b * p.Hkv + g;
-  const int64_t rowbase = bg * S;
-  const T* kg = static_cast<const T*>(p.k.data) + (int64_t)b * p.k.sb + (int64_t)g * p.k.sh;
-  const T* vg = static_cast<const T*>(p.v.data) + (int64_t)b * p.v.sb + (int64_t)g * p.v.sh;
-  load_rows<T, D>(Ks, kg + (int64_t)key0 * p.k.ss, p.k.ss, nkeys, BLK, tid, NTH);
-  load_rows<T, D>(Vs, vg + (int64_t)key0 * p.v.ss, p.v.ss, nkeys, BLK, tid, NTH);
-  cp_async_commit();
-
-  float dk[NT][4], dv[NT][4];
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    dk[n][0] = dk[n][1] = dk[n][2] = dk[n][3] = 0.f;
-    dv[n][0] = dv[n][1] = dv[n][2] = dv[n][3] = 0.f;
-  }
-  float dsacc = 0.f;  // column tid of sum dz q (tid < D)
-  const float sc = rsqrtf((float)D) * kLog2e;
-  const int kw = warp * 16;
-  const uint32_t ks_b = smem_u32(Ks), vs_b = smem_u32(Vs), qs_b = smem_u32(Qs), do_b = smem_u32(dOs);
-  constexpr uint32_t kBufBytes = RC * D * sizeof(T);
-  cp_async_wait<0>();
-  __syncthreads();
-
-  for (int t = p.causal ? c : 0; t < p.n_qblocks; ++t) {
-    const bool diag = t == c;
-    if (!diag) {
-      const uint32_t w = p.umask[(bg * p.n_qblocks + t) * p.n_words + (c >> 5)];
-      if (!((w >> (c & 31)) & 1u)) continue;
-    }
-    const int row0 = t * BLK;
-    const int nrows = min(BLK, S - row0);
-    __syncthreads();  // es / chunk_any / buffers of the previous query block are no longer read
-    if (tid < NRC) chunk_any[tid] = 0;
-    __syncthreads();
-    for (int r = tid; r < BLK; r += NTH) {
-      int e = -1;
-      if (r < nrows) {
-        if (diag) {
-          e = -2;
-        } else {
-          const int64_t row = rowbase + row0 + r;
-          const int n = p.cnt[row];
-          const int32_t* list = p.idx + row * tc;
-          int lo = 0, hi = n;
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (list[mid] < c) lo = mid + 1;
-            else hi = mid;
-          }
-          if (lo < n && list[lo] == c) e = lo;
-        }
-      }
-      es[r] = e;
-      if (e != -1) chunk_any[r / RC] = 1;
-    }
-    __syncthreads();
-    const float beta2 = diag_bias2(p.sigma, p.causal ? t : p.n_qblocks - 1);
-
-    // items (head, 32-row chunk) of this query block, in order; chunks no row
-    // of which selected the block are skipped.  Item i + 1 streams in while
-    // item i is computed.
-    const int n_items = G * NRC;
-    auto item_ok = [&](int i) -> bool {
-      const int rcn = i % NRC;
-      return rcn * RC < nrows && chunk_any[rcn];
-    };
-    auto next_ok = [&](int i) -> int {
-      while (i < n_items && !item_ok(i)) ++i;
-      return i;
-    };
-    auto issue = [&](int i, int bf) {
-      if (i < n_items) {
-        const int h = g * G + i / NRC, rc = (i % NRC) * RC;
-        const int nv = min(RC, nrows - rc);
-        load_rows<T, D>(Qs + bf * RC * D, static_cast<const T*>(p.q.data) + (int64_t)b * p.q.sb +
-                                              (int64_t)(row0 + rc) * p.q.ss + (int64_t)h * p.q.sh,
-                        p.q.ss, nv, RC, tid, NTH);
-        load_rows<T, D>(dOs + bf * RC * D, static_cast<const T*>(p.dout.data) + (int64_t)b * p.dout.sb +
-                                               (int64_t)(row0 + rc) * p.dout.ss + (int64_t)h * p.dout.sh,
-                        p.dout.ss, nv, RC, tid, NTH);
-        if (tid < 4 * RC) {
-          const int which = tid / RC, r = tid % RC;
-          const int e = r < nv ? es[rc + r] : -1;
-          const int64_t ra = row0 + rc + r;
-          const int64_t hrow = ((int64_t)b * p.H + h) * S;
-          const float* src = p.lse;  // any readable address when nothing is copied
-          bool ok = false;
-          if (which == 0) {
-            ok = e >= 0;
-            if (ok) src = p.logp + (rowbase + ra) * tc + e;
-          } else if (which == 1 || which == 2) {
-            ok = e != -1;
-            if (ok) src = (which == 1 ? p.lse : p.dd) + hrow + ra;
-          } else {
-            ok = e >= 0;
-            if (ok) src = p.dz + ((rowbase + ra) * tc + e) * G + (i / NRC);
-          }
-          cp_async4(raw + (bf * 4 + which) * RC + r, src, ok);
-        }
-      }
-      cp_async_commit();
-    };
-
-    int bf = 0;
-    issue(next_ok(0), 0);
-    for (int i = next_ok(0); i < n_items; i = next_ok(i + 1)) {
-      const int rc = (i % NRC) * RC;
-      const int nv = min(RC, nrows - rc);
-      __syncthreads();  // the other buffer's readers are done
-      issue(next_ok(i + 1), bf ^ 1);
-      cp_async_wait<1>();
-      __syncthreads();
-      const uint32_t qb = qs_b + bf * kBufBytes, ob = do_b + bf * kBufBytes;
-      const float* rlp = raw + (bf * 4 + 0) * RC;
-      const float* rl2 = raw + (bf * 4 + 1) * RC;
-      const float* rdd = raw + (bf * 4 + 2) * RC;
-      const float* rdz = raw + (bf * 4 + 3) * RC;
-      // S^T and dP^T for the warp's 16 keys x 32 rows
-      float s[4][4], dp[4][4];
-      tile_abt<T, D, 2>(ks_b, kw, qb, lane, s);
-      tile_abt<T, D, 2>(vs_b, kw, ob, lane, dp);
-#pragma unroll
-      for (int n = 0; n < 4; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = key0 + kw + gq + (e >> 1) * 8;
-          const int r = n * 8 + 2 * tq + (e & 1);
-          const int en = r < nv ? es[rc + r] : -1;
-          const float bias = en == -2 ? beta2 : (en >= 0 ? p.sigma * rlp[r] * kLog2e : kNegInf);
-          const bool ok = key < S && en != -1 && (!diag || !p.causal || key <= row0 + rc + r);
-          const float pr = ok ? exp2f(fmaf(s[n][e], sc, bias) - rl2[r]) : 0.f;
-          s[n][e] = pr;
-          dp[n][e] = pr * (dp[n][e] - rdd[r]);
-        }
-      tile_xb<T, D, 2>(s, ob, lane, dv);
-      tile_xb<T, D, 2>(dp, qb, lane, dk);
-      if (!diag && tid < D) {
-        const T* qrow = Qs + bf * RC * D;
-        for (int r = 0; r < nv; ++r) dsacc = fmaf(rdz[r], Elt<T>::load1(qrow + swz<D>(r, tid)), dsacc);
-      }
-      bf ^= 1;
-    }
-    cp_async_wait<0>();
-  }
-
-  // stage 0: s_c = kbar_c W_s, so dkbar_c = ds_c W_s^T, spread over the block's keys
-  __syncthreads();
-  const float gam = rsqrtf((float)D);
-  if (tid < D) {
-    float kb = 0.f;
-    for (int j = 0; j < nkeys; ++j) kb += Elt<T>::load1(Ks + swz<D>(j, tid));
-    const float dsv = gam * dsacc;
-    p.kbar[(bg * tc + c) * D + tid] = kb / (float)nkeys;
-    p.ds[(bg * tc + c) * D + tid] = dsv;
-    dss[tid] = dsv;
-  }
-  __syncthreads();
-  if (tid < D) {
-    const float* wr = p.w_s + (int64_t)tid * D;
-    float a = 0.f;
-    for (int j = 0; j < D; ++j) a = fmaf(__ldg(wr + j), dss[j], a);
-    dkb[tid] = a / (float)nkeys;
-  }
-  __syncthreads();
-  const float ksc = rsqrtf((float)D);
-  float* dkg = static_cast<float*>(const_cast<void*>(p.dk.data)) + (int64_t)b * p.dk.sb + (int64_t)g * p.dk.sh;
-  float* dvg = static_cast<float*>(const_cast<void*>(p.dv.data)) + (int64_t)b * p.dv.sb + (int64_t)g * p.dv.sh;
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const int col = n * 8 + 2 * tq;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int key = key0 + kw + gq + half * 8;
-      if (key < S) {
-        *reinterpret_cast<float2*>(dkg + (int64_t)key * p.dk.ss + col) =
-            make_float2(fmaf(dk[n][2 * half], ksc, dkb[col]), fmaf(dk[n][2 * half + 1], ksc, dkb[col + 1]));
-        *reinterpret_cast<float2*>(dvg + (int64_t)key * p.dv.ss + col) = make_float2(dv[n][2 * half], dv[n][2 * half + 1]);
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------ bwd_ws
 // dW_s[a][col] = sum over blocks i of kbar[i][a] ds[i][col]; one CTA per row a.
 __global__ void bwd_ws_kernel(const float* __restrict__ kbar, const float* __restrict__ ds, int64_t n, int D,
@@ -764,12 +490,8 @@ cudaError_t launch_typed(const BwdParams& p, cudaStream_t stream) {
   }
   if (e != cudaSuccess) return e;
 
-  const size_t key_smem =
-      (size_t)(2 * BLK * D + 4 * kRowChunk * D) * sizeof(T) + 2 * 4 * kRowChunk * 4 + BLK * 4 + 2 * D * 4;
-  e = cudaFuncSetAttribute(bwd_key_kernel<T, D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)key_smem);
-  if (e != cudaSuccess) return e;
-  bwd_key_kernel<T, D, BLK><<<dim3((unsigned)p.t_cap, p.Hkv, p.B), 2 * BLK, key_smem, stream>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // dk, dv, the summary gradient and the block means on the tensor cores
+  if ((e = launch_bwd_key_tc(p, stream)) != cudaSuccess) return e;
 
   bwd_ws_kernel<<<D, D, 0, stream>>>(p.kbar, p.ds, (int64_t)p.B * p.Hkv * p.t_cap, D, p.dw_s);
   return cudaGetLastError();

@@ -1,6 +1,7 @@
 // Internal launch interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -144,6 +145,10 @@ struct SparseParams {
   // runs out.  Waits that drain issued copies or MMAs always use the default.
   long long wait_cycles;
   int stall_producer;
+  // tensor-core kernel: per-row log-sum-exp of the biased logits in log2
+  // units, [B, H, S] (null: not written); skip_out: do not write `out`
+  float* lse;
+  int skip_out;
 };
 // positions per stage-2 tile (tiles are 128 rows)
 int sparse_tile_positions(int G, int block);
@@ -165,6 +170,10 @@ struct PairParams {
   int32_t* psteps;
 };
 cudaError_t launch_pairs(const PairParams& p, cudaStream_t stream);
+// 4-D TMA map over a [B, S, H, D] f16/bf16 view (innermost first: D, H, S,
+// B), 128-byte swizzle, box {64, box_h, box_s, 1}; no multicast.
+bool make_map(CUtensorMap* map, const View& v, int dtype, int64_t B, int64_t S, int64_t H, int D, int box_h,
+              int box_s);
 cudaError_t launch_sparse_prefill(const SparseParams& p, cudaStream_t stream);
 cudaError_t launch_sparse_prefill_tc(const SparseParams& p, cudaStream_t stream);
 
@@ -246,7 +255,7 @@ struct BwdParams {
   const float* logp;       // [B, Hkv, S, t_cap]
   const int32_t* cnt;      // [B, Hkv, S]
   const float* tau;        // [B, H, S]
-  float* lse;              // [B, H, S] log-sum-exp of the logits, log2 units
+  const float* lse;        // [B, H, S] log-sum-exp of the logits, log2 units (from the forward kernel)
   float* dd;               // [B, H, S] dout . out
   float* dz;               // [B, Hkv, S, t_cap, G]: d log p_bar per head, then dL/dz
   uint32_t* umask;         // [B, Hkv, n_qblocks, n_words]: blocks some row of the query block selected
@@ -254,7 +263,19 @@ struct BwdParams {
   float* ds;               // [B, Hkv, t_cap, D] dL/d(summary)
   float* dw_s;             // [D, D]
   DeviceStatus* status;
+  // key-centric tensor-core kernel: the stage-2 tiles (128 / G positions x G
+  // heads) whose work lists hold each block, and each row's selection
+  const uint32_t* tbits;   // [B, Hkv, n_tiles, n_words]: bit c set iff block c is in the tile's work list
+  const uint32_t* rmask;   // [B, Hkv, S, n_words]: bit c set iff the row selected block c
+  const int32_t* rrank;    // [B, Hkv, S, n_words]: the row's selections below block 32 w
+  int n_tiles;
 };
 cudaError_t launch_bwd(const BwdParams& p, cudaStream_t stream);
+// the key-centric backward kernel alone (dk, dv, ds, kbar), and the tile bit
+// masks it reads, from the tiles' work lists ulist / ucnt ([n_lists][t_cap])
+cudaError_t launch_bwd_key_tc(const BwdParams& p, cudaStream_t stream);
+cudaError_t launch_row_ranks(const uint32_t* mask, int64_t rows, int n_words, int32_t* rank, cudaStream_t stream);
+cudaError_t launch_tile_bits(const int32_t* ulist, const int32_t* ucnt, int64_t n_lists, int64_t t_cap, uint32_t* bits,
+                             int n_words, cudaStream_t stream);
 
 }  // namespace dash

@@ -14,17 +14,30 @@ import os
 import numpy as np
 
 _POOL = None
+_LIMIT = None
 
 
 def _pool_size(n_tasks: int = 1 << 30) -> int:
     return max(1, min(n_tasks, 24, (os.cpu_count() or 2) - 1))
 
 
+def _one_thread():
+    """Worker start-up: one BLAS / OpenMP thread per process (the pool supplies the parallelism)."""
+    from threadpoolctl import threadpool_limits
+
+    global _LIMIT
+    _LIMIT = threadpool_limits(1)
+
+
+def _spawn_pool(n: int):
+    return mp.get_context("spawn").Pool(n, initializer=_one_thread)
+
+
 def shared_pool():
     """One spawned worker pool for the whole test session (started on first use)."""
     global _POOL
     if _POOL is None:
-        _POOL = mp.get_context("spawn").Pool(_pool_size())
+        _POOL = _spawn_pool(_pool_size())
         atexit.register(_close_pool)
     return _POOL
 
@@ -61,7 +74,7 @@ def key_block_backward_pooled(tmpdir, arrays: dict, blocks, block, alpha, causal
     chunks = [range(r0, S, n_chunks) for r0 in range(n_chunks)]
     tasks = [(paths, list(blocks), block, alpha, causal, sigma, ch) for ch in chunks]
     if workers:
-        with mp.get_context("spawn").Pool(n) as pool:
+        with _spawn_pool(n) as pool:
             parts = pool.map(_key_block_part, tasks, chunksize=1)
     else:
         parts = shared_pool().map(_key_block_part, tasks, chunksize=1)
