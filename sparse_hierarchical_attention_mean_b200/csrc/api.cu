@@ -895,6 +895,13 @@ dash_status_t dash_attn_bwd(const dash_tensor_t* q, const dash_tensor_t* k, cons
   p.rmask = at<uint32_t>(workspace, L.rmask);
   p.rrank = at<int32_t>(workspace, L.rrank);
   p.n_tiles = (int)L.sl.n_tiles;
+  {
+    char* lw = at<char>(workspace, L.lists);
+    p.ulist = at<int32_t>(lw, L.sl.ulist);
+    p.tmask = at<uint4>(lw, L.sl.umask);
+    p.ucnt = at<int32_t>(lw, L.sl.ucnt);
+    p.usteps = at<int32_t>(lw, L.sl.usteps);
+  }
   e = dash::launch_bwd(p, s);
   if (e != cudaSuccess) return cuda_fail(e, "backward");
   return ok();

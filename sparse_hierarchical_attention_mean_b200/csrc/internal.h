@@ -269,11 +269,19 @@ struct BwdParams {
   const uint32_t* rmask;   // [B, Hkv, S, n_words]: bit c set iff the row selected block c
   const int32_t* rrank;    // [B, Hkv, S, n_words]: the row's selections below block 32 w
   int n_tiles;
+  // row-centric tensor-core kernel: the stage-2 tiles' work lists ([B, Hkv, n_tiles] lists of
+  // t_cap entries: blocks ascending, the mask of tile positions that selected each, counts, steps)
+  const int32_t* ulist;
+  const uint4* tmask;
+  const int32_t* ucnt;
+  const int32_t* usteps;
 };
 cudaError_t launch_bwd(const BwdParams& p, cudaStream_t stream);
 // the key-centric backward kernel alone (dk, dv, ds, kbar), and the tile bit
 // masks it reads, from the tiles' work lists ulist / ucnt ([n_lists][t_cap])
 cudaError_t launch_bwd_key_tc(const BwdParams& p, cudaStream_t stream);
+// the row-centric backward kernel alone (dq of stage 2, d log p_bar per head into dz, D into dd)
+cudaError_t launch_bwd_row_tc(const BwdParams& p, cudaStream_t stream);
 cudaError_t launch_row_ranks(const uint32_t* mask, int64_t rows, int n_words, int32_t* rank, cudaStream_t stream);
 cudaError_t launch_tile_bits(const int32_t* ulist, const int32_t* ucnt, int64_t n_lists, int64_t t_cap, uint32_t* bits,
                              int n_words, cudaStream_t stream);
