@@ -817,8 +817,8 @@ def main():
         line["backward"] = {
             "workload": "gradients of the prefill workload above (dq, dk, dv fp32 and dW_s), dout ~ N(0, 1)",
             "ms": bw["ms"], "steps": bw["steps"], "device_status": bw["status"],
-            "roofline": {"kernels": "the whole backward call: pooling, routing, bwd_row, bwd_route, bwd_key, "
-                                    "bwd_ws (warp-level MMAs)",
+            "roofline": {"kernels": "the whole backward call: pooling, routing, the stage-2 log-sum-exp pass, "
+                                    "row masks, bwd_row_tc and bwd_key_tc (tcgen05), bwd_route, bwd_ws",
                          "bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
                          "traffic": None, "algorithmic_flops": bw["flops"],
                          "peak_source": f"{pk['source']} bf16 (burst)"},
