@@ -22,7 +22,16 @@ def _pool_size(n_tasks: int = 1 << 30) -> int:
 
 
 def _one_thread():
-    """Worker start-up: one BLAS / OpenMP thread per process (the pool supplies the parallelism)."""
+    """Worker start-up: one BLAS / OpenMP thread per process (the pool supplies the parallelism).
+
+    The limits are set before torch (whose CPU ops generate the inputs) starts its thread pool,
+    and applied again to every numerical library loaded by then."""
+    os.environ["OMP_NUM_THREADS"] = "1"
+    os.environ["MKL_NUM_THREADS"] = "1"
+    import torch
+
+    torch.set_num_threads(1)
+    torch.set_num_interop_threads(1)
     from threadpoolctl import threadpool_limits
 
     global _LIMIT
