@@ -27,8 +27,9 @@ constexpr int kMaxBpc = 32;
 // One CTA: up to kMaxBpc consecutive blocks of one (batch, KV head).
 //   Pooling: each warp takes whole blocks (w, w + 8, ...); a lane owns one
 //   16-byte column vector of a row group and sums its rows in registers with
-//   eight loads in flight, then the lanes holding the same columns combine by
-//   shuffles.  No barrier per block.
+//   sixteen loads in flight (mean pooling; eight with the learned query),
+//   then the lanes holding the same columns combine by shuffles.  No barrier
+//   per block.
 //   Projection: means[nb][D] x W_s[D][D] with a 4 x 4 (blocks x columns)
 //   register tile per thread; W_s rows are read as float4 through L1.
 template <typename T, int D, bool SDPA>
@@ -41,11 +42,16 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
   constexpr int BPT = kMaxBpc / BG;        // blocks per thread in the projection
   __shared__ __align__(16) float means[kMaxBpc][D];
 
-  const int b = blockIdx.z, g = blockIdx.y;
+  // consecutive CTAs take the same blocks of consecutive KV heads: the heads'
+  // rows of a token are adjacent in memory, so the CTAs in flight together
+  // read whole rows of the cache and each DRAM page is opened once
+  const int b = blockIdx.z;
+  const int g = (int)(blockIdx.x % (unsigned)p.Hkv);
+  const int chunk = (int)(blockIdx.x / (unsigned)p.Hkv);
   int n_tok = p.S;
   if (p.seqlens) n_tok = min(max(p.seqlens[b], 0), p.S);
   const int64_t nblk = (n_tok + p.block - 1) / p.block;
-  const int64_t c_begin = p.first_block + (int64_t)blockIdx.x * bpc;
+  const int64_t c_begin = p.first_block + (int64_t)chunk * bpc;
   if (c_begin >= nblk) return;
   const int nb = (int)(nblk - c_begin < bpc ? nblk - c_begin : bpc);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -65,15 +71,15 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolParams p, int bpc) {
       float acc[EPV];
 #pragma unroll
       for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
-      for (int64_t j0 = lo; j0 < hi; j0 += 8 * RPL) {
-        uint4 v[8];
+      for (int64_t j0 = lo; j0 < hi; j0 += 16 * RPL) {
+        uint4 v[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 16; ++u) {
           const int64_t j = j0 + u * RPL + vrow;
           v[u] = j < hi ? __ldg(reinterpret_cast<const uint4*>(kb + (j - lo) * p.k.ss)) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 16; ++u) {
           float f[EPV];
           Elt<T>::to_float(v[u], f);
 #pragma unroll
@@ -212,7 +218,7 @@ cudaError_t launch_typed(const PoolParams& p, cudaStream_t stream) {
   // as many blocks per CTA as keep about four CTAs per SM busy
   int bpc = kMaxBpc;
   while (bpc > kWarpsP && total / bpc < 148 * 4) bpc /= 2;
-  dim3 grid((unsigned)((span + bpc - 1) / bpc), p.Hkv, p.B);
+  dim3 grid((unsigned)((span + bpc - 1) / bpc * p.Hkv), 1, p.B);
   if (p.qbar)
     pool_kernel<T, D, true><<<grid, kThreads, 0, stream>>>(p, bpc);
   else
