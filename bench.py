@@ -573,6 +573,67 @@ def run_decode(dash, cfg, steps, warmup, world, rank):
             "status": status, "clocks": clk.summary()}
 
 
+def run_cp_decode(dash, cfg, steps, warmup, rank, ranks=4):
+    """Context-parallel decode on the decode workload, `ranks` block-aligned shards of every
+    sequence's cache run one after another on this GPU (what the ranks of a context-parallel
+    group do at once): shard scores, their sum (the all-reduce), lists, shard attention, and
+    the log-sum-exp merge of the stacked partials (the all-gather).  The shards are views of
+    the cache; each has its own summaries, built once outside the timed steps."""
+    inp = full_inputs(cfg, device="cuda", seed=rank_seed(cfg, rank))
+    q, k, v, w, sl = inp["q"], inp["k"], inp["v"], inp["w_s"], inp["seqlens"]
+    B, lmax, Hkv, d = k.shape
+    G, blk = cfg.group, cfg.block
+    t_cap = -(-lmax // blk)
+    bounds = [((lmax // blk) * r // ranks) * blk for r in range(ranks)] + [lmax]
+    shards = []
+    for r in range(ranks):
+        lo, hi = bounds[r], bounds[r + 1]
+        ks, vs = k[:, lo:hi], v[:, lo:hi]
+        sl_r = (sl - lo).clamp(0, hi - lo).to(torch.int32)
+        shards.append((lo, hi, ks, vs, dash.summarize(ks, w, blk, seqlens=sl_r)))
+    scores = torch.zeros((B, Hkv, G, t_cap), dtype=torch.float32, device="cuda")
+    part_scores = torch.zeros_like(scores)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    attend_ms = 0.0
+
+    def step(record):
+        scores.zero_()
+        for lo, hi, ks, vs, summ_r in shards:
+            part_scores.zero_()
+            dash.cp_scores(q, summ_r, lo // blk, hi // blk, sl, lmax, cfg.alpha, blk, part_scores)
+            scores.add_(part_scores)
+        lists = dash.cp_lists(q, Hkv, scores, sl, lmax, cfg.alpha, blk)
+        if record:
+            ev[2].record(stream)
+        parts = [dash.cp_attend(q, ks, vs, lo, sl, lmax, lists, blk) for lo, hi, ks, vs, _ in shards]
+        if record:
+            ev[3].record(stream)
+        dash.cp_merge(torch.stack(parts).contiguous(), out)
+        return lists
+
+    for _ in range(warmup):
+        step(False)
+    torch.cuda.synchronize()
+    total = 0.0
+    for _ in range(steps):
+        ev[0].record(stream)
+        lists = step(True)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        total += ev[0].elapsed_time(ev[1])
+        attend_ms += ev[2].elapsed_time(ev[3])
+    # bytes the shard attention reads: the selected and diagonal K/V (each read once over the shards)
+    cnt = lists["cnt"].double()
+    pos = sl.double() - 1
+    diag = pos - torch.floor(pos / blk) * blk + 1
+    kv_bytes = float((cnt * blk * d * 4).sum()) + float((diag * d * 4).sum()) * Hkv
+    attend_us = attend_ms / steps * 1e3
+    return {"ranks": ranks, "us_per_step": total / steps * 1e3, "attend_us": attend_us,
+            "attend_gbs": kv_bytes / (attend_us * 1e-6) / 1e9, "kv_bytes": kv_bytes}
+
+
 # --------------------------------------------------------------------------- oracle timing
 
 
@@ -683,6 +744,7 @@ def main():
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-long", action="store_true", help="skip the 128K long-prefill workload")
     ap.add_argument("--skip-sweep", action="store_true", help="skip the alpha / sparsity sweep")
+    ap.add_argument("--skip-cp", action="store_true", help="skip the context-parallel decode emulation")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--seq", type=int, default=None,
                     help="prefill sequence length override (smaller cases for profiling; default 32768)")
@@ -731,10 +793,14 @@ def main():
     pk = peaks()
     pre = None if args.skip_prefill else run_prefill(dash, cfg, args.steps, warmup, world, rank, pk,
                                                          not args.skip_backward)
-    dec = None
+    dec = cpd = None
     dcfg = get_config("decode").with_(batch=args.decode_batch)
     if not args.skip_decode:
         dec = run_decode(dash, dcfg, max(20, args.steps), warmup, world, rank)
+        torch.cuda.empty_cache()
+        if not args.skip_cp:
+            cpd = run_cp_decode(dash, dcfg, max(5, min(args.steps, 10)), warmup, rank)
+            torch.cuda.empty_cache()
 
     long_obj = sweep_obj = None
     if not args.skip_long and not args.skip_prefill:
@@ -807,6 +873,16 @@ def main():
     }
     if dec is not None:
         line["decode"] = decode_object(dec, dcfg, pk)
+    if cpd is not None:
+        line["cp_decode"] = {
+            "workload": f"decode workload above, each sequence's cache split into {cpd['ranks']} block-aligned "
+                        "shards run one after another on this GPU (shard scores, their sum, lists, shard "
+                        "attention, log-sum-exp merge)",
+            "us_per_step_all_shards": cpd["us_per_step"], "shard_attention_us": cpd["attend_us"],
+            "shard_attention": {"bound": "hbm", "achieved": cpd["attend_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                "frac": cpd["attend_gbs"] / pk["hbm_gbs"], "bytes": cpd["kv_bytes"],
+                                "peak_source": f"{pk['source']} HBM copy"},
+        }
     if long_obj is not None:
         line["long_prefill"] = long_obj
     if sweep_obj is not None:
