@@ -591,8 +591,11 @@ def run_cp_decode(dash, cfg, steps, warmup, rank, ranks=4):
         ks, vs = k[:, lo:hi], v[:, lo:hi]
         sl_r = (sl - lo).clamp(0, hi - lo).to(torch.int32)
         shards.append((lo, hi, ks, vs, dash.summarize(ks, w, blk, seqlens=sl_r)))
+    H = q.shape[2]
     scores = torch.zeros((B, Hkv, G, t_cap), dtype=torch.float32, device="cuda")
     part_scores = torch.zeros_like(scores)
+    parts = torch.empty((ranks, B, H, d + 2), dtype=torch.float32, device="cuda")
+    ws = torch.empty(dash.cp_attend_workspace_size(B, H, Hkv, d, blk, t_cap), dtype=torch.uint8, device="cuda")
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -607,10 +610,11 @@ def run_cp_decode(dash, cfg, steps, warmup, rank, ranks=4):
         lists = dash.cp_lists(q, Hkv, scores, sl, lmax, cfg.alpha, blk)
         if record:
             ev[2].record(stream)
-        parts = [dash.cp_attend(q, ks, vs, lo, sl, lmax, lists, blk) for lo, hi, ks, vs, _ in shards]
+        for r, (lo, hi, ks, vs, _) in enumerate(shards):
+            dash.cp_attend_ex(q, ks, vs, lo, sl, lmax, lists, blk, part=parts[r], workspace=ws)
         if record:
             ev[3].record(stream)
-        dash.cp_merge(torch.stack(parts).contiguous(), out)
+        dash.cp_merge(parts, out)
         return lists
 
     for _ in range(warmup):
@@ -624,14 +628,40 @@ def run_cp_decode(dash, cfg, steps, warmup, rank, ranks=4):
         torch.cuda.synchronize()
         total += ev[0].elapsed_time(ev[1])
         attend_ms += ev[2].elapsed_time(ev[3])
+    # the CUDA-core shard attention (no workspace) on the same lists, for comparison
+    core_ms = 0.0
+    for _ in range(steps):
+        ev[2].record(stream)
+        for r, (lo, hi, ks, vs, _) in enumerate(shards):
+            dash.cp_attend(q, ks, vs, lo, sl, lmax, lists, blk, part=parts[r])
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        core_ms += ev[2].elapsed_time(ev[3])
     # bytes the shard attention reads: the selected and diagonal K/V (each read once over the shards)
     cnt = lists["cnt"].double()
     pos = sl.double() - 1
     diag = pos - torch.floor(pos / blk) * blk + 1
     kv_bytes = float((cnt * blk * d * 4).sum()) + float((diag * d * 4).sum()) * Hkv
     attend_us = attend_ms / steps * 1e3
+    core_us = core_ms / steps * 1e3
     return {"ranks": ranks, "us_per_step": total / steps * 1e3, "attend_us": attend_us,
-            "attend_gbs": kv_bytes / (attend_us * 1e-6) / 1e9, "kv_bytes": kv_bytes}
+            "attend_gbs": kv_bytes / (attend_us * 1e-6) / 1e9, "kv_bytes": kv_bytes,
+            "attend_kernel": "split-KV tensor-core path (dash_attn_cp_attend_ex)",
+            "attend_cuda_cores_us": core_us, "attend_cuda_cores_gbs": kv_bytes / (core_us * 1e-6) / 1e9}
+
+
+def cp_object(cpd, pk) -> dict:
+    return {
+        "workload": f"decode workload above, each sequence's cache split into {cpd['ranks']} block-aligned "
+                    "shards run one after another on this GPU (shard scores, their sum, lists, shard "
+                    "attention, log-sum-exp merge)",
+        "us_per_step_all_shards": cpd["us_per_step"], "shard_attention_us": cpd["attend_us"],
+        "shard_attention": {"bound": "hbm", "achieved": cpd["attend_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                            "frac": cpd["attend_gbs"] / pk["hbm_gbs"], "bytes": cpd["kv_bytes"],
+                            "kernel": cpd["attend_kernel"], "peak_source": f"{pk['source']} HBM copy"},
+        "shard_attention_cuda_cores": {"us": cpd["attend_cuda_cores_us"], "achieved": cpd["attend_cuda_cores_gbs"],
+                                       "unit": "GB/s", "frac": cpd["attend_cuda_cores_gbs"] / pk["hbm_gbs"]},
+    }
 
 
 # --------------------------------------------------------------------------- oracle timing
@@ -825,7 +855,8 @@ def main():
         return
     if pre is None:
         print(json.dumps({"decode_only": True, "us_per_step": None if dec is None else dec["us"],
-                          "decode": None if dec is None else decode_object(dec, dcfg, pk)}), flush=True)
+                          "decode": None if dec is None else decode_object(dec, dcfg, pk),
+                          "cp_decode": None if cpd is None else cp_object(cpd, pk)}), flush=True)
         barrier(world)
         finish(world)
         return
@@ -874,15 +905,7 @@ def main():
     if dec is not None:
         line["decode"] = decode_object(dec, dcfg, pk)
     if cpd is not None:
-        line["cp_decode"] = {
-            "workload": f"decode workload above, each sequence's cache split into {cpd['ranks']} block-aligned "
-                        "shards run one after another on this GPU (shard scores, their sum, lists, shard "
-                        "attention, log-sum-exp merge)",
-            "us_per_step_all_shards": cpd["us_per_step"], "shard_attention_us": cpd["attend_us"],
-            "shard_attention": {"bound": "hbm", "achieved": cpd["attend_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                "frac": cpd["attend_gbs"] / pk["hbm_gbs"], "bytes": cpd["kv_bytes"],
-                                "peak_source": f"{pk['source']} HBM copy"},
-        }
+        line["cp_decode"] = cp_object(cpd, pk)
     if long_obj is not None:
         line["long_prefill"] = long_obj
     if sweep_obj is not None:

@@ -271,6 +271,26 @@ dash_status_t dash_attn_cp_attend(const dash_tensor_t* q, const dash_tensor_t* k
                                   int64_t tok_lo, const int32_t* seqlens, int64_t lmax, const int32_t* idx,
                                   const float* logp, const int32_t* cnt, int64_t t_cap, int block,
                                   const dash_options_t* opts, float* part, dash_stream_t stream);
+/*
+ * dash_attn_cp_attend_ex: step 4 on the tensor-core split-KV path of
+ * dash_attn_decode_ex.  Same arguments and partials as dash_attn_cp_attend;
+ * the range of each (b, KV head)'s ascending list that falls in the shard's
+ * blocks, plus the diagonal block when the shard holds it, is cut into work
+ * items that the whole GPU shares.  Partials are the same up to rounding
+ * order.
+ *   workspace  256-byte aligned device pointer of at least
+ *              dash_attn_cp_attend_workspace_size(B, H, Hkv, d, block, t_cap)
+ *              bytes, owned by the caller; the call may use it until the
+ *              stream reaches its end.  Too small: DASH_ERR_WORKSPACE_TOO_SMALL.
+ * dash_attn_cp_attend_workspace_size returns 0 for invalid sizes.
+ */
+size_t dash_attn_cp_attend_workspace_size(int64_t batch, int64_t heads, int64_t kv_heads, int64_t head_dim, int block,
+                                          int64_t t_cap);
+dash_status_t dash_attn_cp_attend_ex(const dash_tensor_t* q, const dash_tensor_t* kshard, const dash_tensor_t* vshard,
+                                     int64_t tok_lo, const int32_t* seqlens, int64_t lmax, const int32_t* idx,
+                                     const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                                     const dash_options_t* opts, float* part, void* workspace, size_t workspace_bytes,
+                                     dash_stream_t stream);
 /*   parts  device fp32 [n_parts, B, H, d + 2]; out [B, 1, H, d] (f16/bf16). */
 dash_status_t dash_attn_cp_merge(const float* parts, int64_t n_parts, dash_tensor_t* out, dash_stream_t stream);
 

@@ -49,6 +49,8 @@ EXPORTED = (
     "dash_attn_cp_scores",
     "dash_attn_cp_lists",
     "dash_attn_cp_attend",
+    "dash_attn_cp_attend_workspace_size",
+    "dash_attn_cp_attend_ex",
     "dash_attn_cp_merge",
     "dash_attn_summarize_paged",
     "dash_attn_decode_paged",
@@ -124,6 +126,8 @@ def _load() -> ctypes.CDLL:
         "dash_attn_cp_scores": (i32, [T, i64, vp, i64, i64, i64, vp, i64, f32, i32, vp, i64, vp]),
         "dash_attn_cp_lists": (i32, [T, i64, vp, vp, i64, f32, i32, vp, vp, vp, i64, vp]),
         "dash_attn_cp_attend": (i32, [T, T, T, i64, vp, i64, vp, vp, vp, i64, i32, O, vp, vp]),
+        "dash_attn_cp_attend_workspace_size": (sz, [i64, i64, i64, i64, i32, i64]),
+        "dash_attn_cp_attend_ex": (i32, [T, T, T, i64, vp, i64, vp, vp, vp, i64, i32, O, vp, vp, sz, vp]),
         "dash_attn_cp_merge": (i32, [vp, i64, T, vp]),
         "dash_attn_summarize_paged": (i32, [T, vp, i64, i64, vp, vp, vp, i32, vp, i64, i64, vp]),
         "dash_attn_decode_paged": (i32, [T, T, T, vp, i64, vp, vp, i64, f32, i32, T, vp, sz, O, vp]),
@@ -552,6 +556,30 @@ def cp_attend(q, kshard, vshard, tok_lo: int, seqlens, lmax: int, lists: dict, b
     _check(_lib.dash_attn_cp_attend(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), tok_lo, seqlens.data_ptr(),
                                     lmax, lists["idx"].data_ptr(), lists["logp"].data_ptr(), lists["cnt"].data_ptr(),
                                     t_cap, block, _options(sigma, None), part.data_ptr(), _stream(stream)))
+    return part
+
+
+def cp_attend_workspace_size(B: int, H: int, Hkv: int, d: int, block: int, t_cap: int) -> int:
+    """Bytes of workspace dash_attn_cp_attend_ex needs."""
+    return int(_lib.dash_attn_cp_attend_workspace_size(B, H, Hkv, d, block, t_cap))
+
+
+def cp_attend_ex(q, kshard, vshard, tok_lo: int, seqlens, lmax: int, lists: dict, block: int, sigma: float = 1.0,
+                 part=None, workspace=None, stream=None) -> torch.Tensor:
+    """Partials [B, H, d + 2] of this rank's tokens on the split-KV path (see dash_attn_cp_attend_ex)."""
+    B, _, H, d = q.shape
+    Hkv = kshard.shape[2]
+    t_cap = lists["idx"].shape[-1]
+    part = torch.empty((B, H, d + 2), dtype=torch.float32, device=q.device) if part is None else part
+    n_ws = cp_attend_workspace_size(B, H, Hkv, d, block, t_cap)
+    if workspace is None:
+        workspace = torch.empty(n_ws, dtype=torch.uint8, device=q.device)
+    qd, kd, vd = _desc(q), _desc(kshard), _desc(vshard)
+    _check(_lib.dash_attn_cp_attend_ex(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), tok_lo,
+                                       seqlens.data_ptr(), lmax, lists["idx"].data_ptr(), lists["logp"].data_ptr(),
+                                       lists["cnt"].data_ptr(), t_cap, block, _options(sigma, None), part.data_ptr(),
+                                       workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))
     return part
 
 

@@ -23,7 +23,7 @@ from __future__ import annotations
 
 import torch
 
-from . import cp_attend, cp_lists, cp_merge, cp_scores
+from . import cp_attend_ex, cp_lists, cp_merge, cp_scores
 
 
 class CudaOps:
@@ -43,7 +43,8 @@ class CudaOps:
 
     @staticmethod
     def attend(q, kshard, vshard, tok_lo, seqlens, lmax, lists, block, sigma):
-        return cp_attend(q, kshard, vshard, tok_lo, seqlens, lmax, lists, block, sigma)
+        # the split-KV tensor-core path (its workspace allocated per call)
+        return cp_attend_ex(q, kshard, vshard, tok_lo, seqlens, lmax, lists, block, sigma)
 
     @staticmethod
     def merge(parts, q):

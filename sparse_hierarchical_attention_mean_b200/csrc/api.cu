@@ -1205,6 +1205,92 @@ dash_status_t dash_attn_cp_attend(const dash_tensor_t* q, const dash_tensor_t* k
   return ok();
 }
 
+// Workspace of the split-KV shard attention: per (b, g) the shard's entry
+// range, the work items and their per-item partials.
+struct CpAttendLayout {
+  size_t shard, items, n_items, pair_base, part_o, part_ml, total;
+  int64_t max_items;
+  int chunk;
+};
+
+static CpAttendLayout cp_attend_layout(int64_t B, int64_t H, int64_t Hkv, int64_t D, int block, int64_t t_cap) {
+  CpAttendLayout L{};
+  const int64_t G = H / Hkv;
+  L.chunk = block == 64 ? 16 : 8;
+  L.max_items = dash::decode_max_items(B, Hkv, t_cap, L.chunk);
+  size_t off = 0;
+  L.shard = off;
+  off = align256(off + (size_t)B * Hkv * 4 * 4);
+  L.items = off;
+  off = align256(off + (size_t)L.max_items * 2 * 4);
+  L.n_items = off;
+  off = align256(off + 4);
+  L.pair_base = off;
+  off = align256(off + (size_t)B * Hkv * 4);
+  L.part_o = off;
+  off = align256(off + (size_t)L.max_items * G * D * 4);
+  L.part_ml = off;
+  off = align256(off + (size_t)L.max_items * G * 2 * 4);
+  L.total = off;
+  return L;
+}
+
+size_t dash_attn_cp_attend_workspace_size(int64_t batch, int64_t heads, int64_t kv_heads, int64_t head_dim, int block,
+                                          int64_t t_cap) {
+  if (batch < 1 || kv_heads < 1 || heads < kv_heads || heads % kv_heads || head_dim < 1 || block < 1 || t_cap < 1)
+    return 0;
+  return cp_attend_layout(batch, heads, kv_heads, head_dim, block, t_cap).total;
+}
+
+dash_status_t dash_attn_cp_attend_ex(const dash_tensor_t* q, const dash_tensor_t* kshard, const dash_tensor_t* vshard,
+                                     int64_t tok_lo, const int32_t* seqlens, int64_t lmax, const int32_t* idx,
+                                     const float* logp, const int32_t* cnt, int64_t t_cap, int block,
+                                     const dash_options_t* opts, float* part, void* workspace, size_t workspace_bytes,
+                                     dash_stream_t stream) {
+  dash_status_t st;
+  if ((st = check_tensor(kshard, "kshard")) || (st = check_tensor(vshard, "vshard"))) return st;
+  if ((st = cp_common(q, kshard->h, seqlens, lmax, block, t_cap))) return st;
+  float sigma;
+  const float* qbar;
+  if ((st = read_options(opts, false, &sigma, &qbar))) return st;
+  if (q->dtype != kshard->dtype || q->dtype != vshard->dtype) return fail(DASH_ERR_INVALID_ARGUMENT, "dtype mismatch");
+  if (kshard->b != q->b || vshard->b != q->b || kshard->d != q->d || vshard->d != q->d || vshard->h != kshard->h ||
+      vshard->s != kshard->s)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "shard shapes do not match q");
+  if (tok_lo < 0 || tok_lo % block || kshard->s % block)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "shard start and length must be multiples of the block");
+  if (!idx || !logp || !cnt || !part) return fail(DASH_ERR_INVALID_ARGUMENT, "null lists or partials");
+  const CpAttendLayout L = cp_attend_layout(q->b, q->h, kshard->h, q->d, block, t_cap);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(DASH_ERR_INVALID_ARGUMENT, "workspace must be a 256-byte aligned device pointer");
+  if (workspace_bytes < L.total)
+    return fail(DASH_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(at<char>(workspace, L.n_items), 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  dash::DecodeParams p = cp_params(q, kshard->h, seqlens, lmax, block, t_cap);
+  p.k = view(kshard);
+  p.v = view(vshard);
+  p.sigma = sigma;
+  p.idx = const_cast<int32_t*>(idx);
+  p.logp = const_cast<float*>(logp);
+  p.cnt = const_cast<int32_t*>(cnt);
+  p.tok_lo = (int)tok_lo;
+  p.tok_n = (int)kshard->s;
+  p.part = part;
+  p.shard = at<int32_t>(workspace, L.shard);
+  p.items = at<int32_t>(workspace, L.items);
+  p.n_items = at<int32_t>(workspace, L.n_items);
+  p.pair_base = at<int32_t>(workspace, L.pair_base);
+  p.part_o = at<float>(workspace, L.part_o);
+  p.part_ml = at<float>(workspace, L.part_ml);
+  p.max_items = L.max_items;
+  p.chunk_blocks = L.chunk;
+  e = dash::launch_cp_attend_mma(p, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "context-parallel attention (split-KV)");
+  return ok();
+}
+
 dash_status_t dash_attn_cp_merge(const float* parts, int64_t n_parts, dash_tensor_t* out, dash_stream_t stream) {
   dash_status_t st;
   if ((st = check_tensor(out, "out"))) return st;

@@ -23,7 +23,11 @@
 //                    4 warps merge into one (m, l, o) partial per item.
 //  combine_decode    log-sum-exp merge of the partials of each (b, g).
 //  attend_shard, cp_merge  context parallelism: stage 2 over one rank's
-//                    tokens into per-head partials, and their merge.
+//                    tokens into per-head partials (CUDA cores, no
+//                    workspace), and their merge.
+//  shard_items, combine_partial  context parallelism on the split-KV path:
+//                    the shard's range of each list cut into work items for
+//                    attend_decode_mma, and its per-head partials.
 #include <type_traits>
 
 #include "common.cuh"
@@ -229,10 +233,17 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
     const int pos = L - 1;
     const int t = pos / p.block;
     const int N = t;
-    const int cnt = p.cnt[bg];
-    const int e_begin = chunk * p.chunk_blocks;
-    const int e_end = min(e_begin + p.chunk_blocks, cnt + 1);
-    const bool has_diag = e_end == cnt + 1;
+    // list entries [e_lo, e_hi) and, when held, the diagonal block (entry e_hi)
+    int e_lo = 0, e_hi = p.cnt[bg];
+    bool diag_held = true;
+    if (p.shard) {
+      e_lo = p.shard[4 * bg];
+      e_hi = p.shard[4 * bg + 1];
+      diag_held = p.shard[4 * bg + 2] != 0;
+    }
+    const int e_begin = e_lo + chunk * p.chunk_blocks;
+    const int e_end = min(e_begin + p.chunk_blocks, diag_held ? e_hi + 1 : e_hi);
+    const bool has_diag = diag_held && e_end == e_hi + 1;
     const int spb = p.block / kStep;
     const int n_diag = has_diag ? (pos - t * p.block) / kStep + 1 : 0;
     const int n_sel = (has_diag ? e_end - 1 : e_end) - e_begin;
@@ -249,7 +260,10 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
     };
     auto load = [&](int s) {
       if (s < n_sub) {
-        const int tok0 = sub_tok0(s);
+        int tok0 = sub_tok0(s);
+        // a shard reads only its own rows (ascending lists keep every step
+        // inside it; anything else is zero-filled)
+        const bool in_shard = !p.shard || (tok0 >= p.tok_lo && tok0 + kStep <= p.tok_lo + p.tok_n);
         // first row of the step: a step never crosses a block, so a paged
         // cache needs one page lookup per step
         int64_t kr0, vr0;
@@ -258,14 +272,15 @@ __global__ void __launch_bounds__(kWarps * 32) attend_decode_mma_kernel(DecodePa
           kr0 = page * p.k.sb + (int64_t)(tok0 % p.block) * p.k.ss;
           vr0 = page * p.v.sb + (int64_t)(tok0 % p.block) * p.v.ss;
         } else {
-          kr0 = (int64_t)b * p.k.sb + (int64_t)tok0 * p.k.ss;
-          vr0 = (int64_t)b * p.v.sb + (int64_t)tok0 * p.v.ss;
+          const int row0 = in_shard ? tok0 - p.tok_lo : 0;
+          kr0 = (int64_t)b * p.k.sb + (int64_t)row0 * p.k.ss;
+          vr0 = (int64_t)b * p.v.sb + (int64_t)row0 * p.v.ss;
         }
         T* kd = Ks + (s % kDStages) * kStageElems;
         T* vd = Vs + (s % kDStages) * kStageElems;
         for (int i = tid; i < kStep * NCH; i += kWarps * 32) {
           const int r = i / NCH, c = i % NCH;
-          const bool ok = tok0 + r < L;  // rows past the context are zero-filled
+          const bool ok = in_shard && tok0 + r < L;  // rows past the context are zero-filled
           const int pc = c ^ (r & 7);
           const int rr = ok ? r : 0;
           cp_async16(kd + r * D + pc * 8, kg + kr0 + (int64_t)rr * p.k.ss + c * 8, ok);
@@ -667,6 +682,75 @@ __global__ void __launch_bounds__(256) combine_decode_kernel(DecodeParams p) {
   }
 }
 
+// Context parallelism on the split-KV path: the part of each (sequence, KV
+// head)'s ascending list that falls in this shard's blocks [block_lo,
+// block_hi) is a contiguous entry range; with the diagonal block when the
+// shard holds it, it is cut into work items of chunk_blocks entries as in
+// the regular decode (one warp per (b, g)).
+__global__ void __launch_bounds__(256) shard_items_kernel(DecodeParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t bg = (int64_t)blockIdx.x * 8 + warp;
+  if (bg >= (int64_t)p.B * p.Hkv) return;
+  const int b = (int)(bg / p.Hkv);
+  const int L = clamp_len(p.seqlens, b, p.Lmax, nullptr);
+  const int t = (L - 1) / p.block;
+  const int block_lo = p.tok_lo / p.block, block_hi = (p.tok_lo + p.tok_n) / p.block;
+  const int cnt = min(max(p.cnt[bg], 0), (int)p.t_cap);
+  const int32_t* idx = p.idx + bg * p.t_cap;
+  int below_lo = 0, below_hi = 0;  // entries before the shard's first block / past its last
+  for (int e = lane; e < cnt; e += 32) {
+    const int c = idx[e];
+    below_lo += c < block_lo ? 1 : 0;
+    below_hi += c < block_hi ? 1 : 0;
+  }
+  below_lo = warp_sum_i(below_lo);
+  below_hi = warp_sum_i(below_hi);
+  if (lane == 0) {
+    const int diag = (t >= block_lo && t < block_hi) ? 1 : 0;
+    const int n_entries = below_hi - below_lo + diag;
+    const int n_it = (n_entries + p.chunk_blocks - 1) / p.chunk_blocks;
+    const int base = n_it > 0 ? atomicAdd(p.n_items, n_it) : 0;
+    p.pair_base[bg] = base;
+    p.shard[4 * bg] = below_lo;
+    p.shard[4 * bg + 1] = below_hi;
+    p.shard[4 * bg + 2] = diag;
+    p.shard[4 * bg + 3] = n_it;
+    for (int k = 0; k < n_it; ++k) {
+      p.items[2 * (base + k)] = (int32_t)bg;
+      p.items[2 * (base + k) + 1] = k;
+    }
+  }
+}
+
+// The shard's per-head partial of each (b, g): log-sum-exp merge of its
+// items' partials, left unnormalised for the merge across shards (o relative
+// to the reference max m, m in log2 units, l); no items: m = -inf, l = 0.
+template <int D>
+__global__ void __launch_bounds__(256) combine_partial_kernel(DecodeParams p) {
+  const int b = blockIdx.y, g = blockIdx.x;
+  const int64_t bg = (int64_t)b * p.Hkv + g;
+  const int n_it = p.shard[4 * bg + 3];
+  const int64_t base = p.pair_base[bg];
+  for (int i = threadIdx.x; i < p.G * D; i += blockDim.x) {
+    const int h = i / D, e = i % D;
+    float M = kNegInf;
+    for (int k = 0; k < n_it; ++k) M = fmaxf(M, p.part_ml[((base + k) * p.G + h) * 2]);
+    const float Mu = M == kNegInf ? 0.f : M;
+    float acc = 0.f, lsum = 0.f;
+    for (int k = 0; k < n_it; ++k) {
+      const float f = exp2f(p.part_ml[((base + k) * p.G + h) * 2] - Mu);
+      acc += f * p.part_o[((base + k) * p.G + h) * D + e];
+      lsum += f * p.part_ml[((base + k) * p.G + h) * 2 + 1];
+    }
+    float* part = p.part + ((int64_t)b * p.H + g * p.G + h) * (D + 2);
+    part[e] = acc;
+    if (e == 0) {
+      part[D] = M;
+      part[D + 1] = lsum;
+    }
+  }
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_route_t(const DecodeParams& p, cudaStream_t stream) {
   dim3 grid((unsigned)((p.t_cap + 63) / 64), p.Hkv, p.B);
@@ -681,7 +765,7 @@ cudaError_t launch_route_t(const DecodeParams& p, cudaStream_t stream) {
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_attend_t(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+cudaError_t launch_attend_t(const DecodeParams& p, int num_sms, cudaStream_t stream, bool partial = false) {
   const size_t smem =
       (size_t)2 * kDStages * kStep * D * sizeof(T) + (size_t)(2 * kWarps * G + kWarps * G * D) * sizeof(float);
   auto kern = attend_decode_mma_kernel<T, D, G>;
@@ -694,7 +778,10 @@ cudaError_t launch_attend_t(const DecodeParams& p, int num_sms, cudaStream_t str
   kern<<<num_sms * per_sm, kWarps * 32, smem, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  combine_decode_kernel<T, D><<<dim3(p.Hkv, p.B), 256, 0, stream>>>(p);
+  if (partial)
+    combine_partial_kernel<D><<<dim3(p.Hkv, p.B), 256, 0, stream>>>(p);
+  else
+    combine_decode_kernel<T, D><<<dim3(p.Hkv, p.B), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -708,12 +795,12 @@ cudaError_t route_d(const DecodeParams& p, cudaStream_t s) {
   }
 }
 template <typename T, int D>
-cudaError_t attend_d(const DecodeParams& p, int n, cudaStream_t s) {
+cudaError_t attend_d(const DecodeParams& p, int n, cudaStream_t s, bool partial = false) {
   switch (p.G) {
-    case 1: return launch_attend_t<T, D, 1>(p, n, s);
-    case 2: return launch_attend_t<T, D, 2>(p, n, s);
-    case 4: return launch_attend_t<T, D, 4>(p, n, s);
-    default: return launch_attend_t<T, D, 8>(p, n, s);
+    case 1: return launch_attend_t<T, D, 1>(p, n, s, partial);
+    case 2: return launch_attend_t<T, D, 2>(p, n, s, partial);
+    case 4: return launch_attend_t<T, D, 4>(p, n, s, partial);
+    default: return launch_attend_t<T, D, 8>(p, n, s, partial);
   }
 }
 
@@ -785,6 +872,20 @@ cudaError_t launch_cp_lists(const DecodeParams& p, cudaStream_t stream) {
 cudaError_t launch_cp_attend(const DecodeParams& p, cudaStream_t stream) {
   if (p.D == 128) return p.dtype == 1 ? cp_attend_d<__half, 128>(p, stream) : cp_attend_d<__nv_bfloat16, 128>(p, stream);
   return p.dtype == 1 ? cp_attend_d<__half, 64>(p, stream) : cp_attend_d<__nv_bfloat16, 64>(p, stream);
+}
+
+cudaError_t launch_cp_attend_mma(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+  if (p.dtype == 0 || !p.shard) return cudaErrorInvalidValue;
+  const int64_t n_bg = (int64_t)p.B * p.Hkv;
+  shard_items_kernel<<<(unsigned)((n_bg + 7) / 8), 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (p.D == 128) {
+    if (p.dtype == 1) return attend_d<__half, 128>(p, num_sms, stream, true);
+    return attend_d<__nv_bfloat16, 128>(p, num_sms, stream, true);
+  }
+  if (p.dtype == 1) return attend_d<__half, 64>(p, num_sms, stream, true);
+  return attend_d<__nv_bfloat16, 64>(p, num_sms, stream, true);
 }
 
 cudaError_t launch_cp_merge(const float* parts, int n_parts, int B, int H, int D, const View& out, int dtype,

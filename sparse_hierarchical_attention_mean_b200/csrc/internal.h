@@ -212,6 +212,11 @@ struct DecodeParams {
   // block_table[b * max_blocks + c] of k / v (sb = page stride); null: dense
   const int32_t* block_table;
   int max_blocks;
+  // split-KV attention over one shard of the cache (context parallelism):
+  // per (b, g) four ints {first list entry, end entry, diagonal held, items};
+  // the shard's k / v rows start at token tok_lo.  Null: the whole list and
+  // the diagonal block (the regular decode step).
+  int32_t* shard;
   // optional route outputs (dash_attn_route in decode mode)
   float* tau;      // [B, H]
   float* p_dense;  // [B, H, t_cap]
@@ -230,6 +235,10 @@ cudaError_t launch_cp_lists(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_cp_attend(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_cp_merge(const float* parts, int n_parts, int B, int H, int D, const View& out, int dtype,
                             cudaStream_t stream);
+// context parallelism on the split-KV tensor-core path: the shard's work
+// items (p.shard, p.items, p.n_items zeroed, p.pair_base), the split-KV
+// kernel over them and a combine into per-head partials p.part [B, H, D + 2]
+cudaError_t launch_cp_attend_mma(const DecodeParams& p, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- backward
 // Gradients of sum(dout * out) for the prefill forward (f16/bf16 inputs,

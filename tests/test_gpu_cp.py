@@ -1,7 +1,9 @@
 """Context-parallel decode on one GPU: R ranks emulated one after the other
 (the score all-reduce is a sum of the ranks' buffers, the all-gather a stack
 of their partials).  Checked against the whole-cache decode (identical
-lists; outputs within the decode tolerance of each other) and the oracle."""
+lists; outputs within the decode tolerance of each other) and the oracle;
+both shard-attention paths (CUDA cores, and the split-KV tensor-core path
+with a workspace) give the same partials."""
 
 import pytest
 import torch
@@ -55,6 +57,11 @@ def test_context_parallel_decode(dash, name):
     lists = dash.cp_lists(q, Hkv, scores, sl, lmax, cfg.alpha, blk)
     parts = torch.stack([dash.cp_attend(q, ks, vs, lo, sl, lmax, lists, blk, sigma=sigma) for lo, ks, vs in shards])
     out = dash.cp_merge(parts.contiguous(), torch.empty_like(q))
+    # the same shards on the split-KV tensor-core path, one workspace reused
+    ws = torch.empty(dash.cp_attend_workspace_size(B, H, Hkv, d, blk, t_cap), dtype=torch.uint8, device="cuda")
+    parts_x = torch.stack([dash.cp_attend_ex(q, ks, vs, lo, sl, lmax, lists, blk, sigma=sigma, workspace=ws)
+                           for lo, ks, vs in shards])
+    out_x = dash.cp_merge(parts_x.contiguous(), torch.empty_like(q))
     torch.cuda.synchronize()
     # the routing is the whole cache's, bit for bit
     assert torch.equal(lists["cnt"], rt["cnt"][:, :, 0])
@@ -65,11 +72,26 @@ def test_context_parallel_decode(dash, name):
             assert torch.equal(lists["logp"][b, g, :n], rt["logp"][b, g, 0, :n])
     tol = OUT_TOL[cfg.dtype]
     assert max_abs(to_np(out), to_np(ref)) <= tol
+    assert max_abs(to_np(out_x), to_np(ref)) <= tol
+    # per shard and head: the two paths find the same mass (l = 0 exactly
+    # where the shard holds none of the head's blocks) and the same
+    # normalised partial output
+    l, lx = parts[..., d + 1], parts_x[..., d + 1]
+    assert torch.equal(l == 0, lx == 0)
+    held = l > 0
+    o_n = parts[..., :d] / l.clamp_min(1e-30)[..., None]
+    ox_n = parts_x[..., :d] / lx.clamp_min(1e-30)[..., None]
+    assert (o_n - ox_n)[held].abs().max().item() <= tol
+    # l relative to each path's own reference max m: l * 2^m agrees
+    lm = torch.log2(l[held]) + parts[..., d][held]
+    lmx = torch.log2(lx[held]) + parts_x[..., d][held]
+    assert (lm - lmx).abs().max().item() <= 1e-2
     for b in range(B):
         for g in sorted({0, Hkv - 1}):
             rec, _ = oracle_decode_pair(cfg, inp["plan"], b, g, sigma=sigma)
-            err = max_abs(to_np(out)[b, 0, g * G:(g + 1) * G], rec["out"])
-            assert err <= tol, f"{name} b{b} g{g}: {err:.3g}"
+            for o_, tag in ((out, "cuda cores"), (out_x, "split-KV")):
+                err = max_abs(to_np(o_)[b, 0, g * G:(g + 1) * G], rec["out"])
+                assert err <= tol, f"{name} {tag} b{b} g{g}: {err:.3g}"
 
 
 @pytest.mark.parametrize("block,dtype,qscale", [(64, "bf16", None), (128, "f16", 3.0)])
