@@ -112,23 +112,26 @@ __device__ __forceinline__ bool is_cand(int c, int t, int n_blocks, int causal) 
 // (32 values per row); COLS = 2: row i's values are x[i * stride + c], read 64
 // columns per iteration for c < n (readable, -inf, up to n rounded up to 64).
 // tau[i] must be a lower bound of the root (F >= 1); rows with done[i] set are
-// left alone.
-template <int RW, int COLS>
-__device__ __forceinline__ void entmax_newton_rows(const float* x, int stride, int n, float pw, int kind, int lane,
-                                                   float* tau, bool* done) {
+// left alone.  KIND: 0 alpha = 2, 1 alpha = 1.5, 2 any other alpha.  The
+// support size is summed and the smallest positive u taken over the warp
+// with one redux each (u > 0, so its bits order as unsigned integers).
+template <int RW, int COLS, int KIND>
+__device__ __forceinline__ void entmax_newton_rows(const float* x, int stride, int n, float pw, int lane, float* tau,
+                                                   bool* done) {
   for (int it = 0; it < 100; ++it) {
-    float f[RW], a[RW], k[RW], umin[RW], fd[RW];
+    float f[RW], a[RW], umin[RW], fd[RW];
+    int k[RW];
 #pragma unroll
-    for (int i = 0; i < RW; ++i) f[i] = a[i] = k[i] = fd[i] = 0.f, umin[i] = 3.0e38f;
+    for (int i = 0; i < RW; ++i) f[i] = a[i] = fd[i] = 0.f, umin[i] = 3.0e38f, k[i] = 0;
     auto add = [&](int i, float xv) {
       const float u = xv - tau[i];
       if (u > 0.f) {
-        k[i] += 1.f;
+        k[i] += 1;
         a[i] += u;
         umin[i] = fminf(umin[i], u);
-        if (kind == 0) {
+        if constexpr (KIND == 0) {
           f[i] += u;
-        } else if (kind == 1) {
+        } else if constexpr (KIND == 1) {
           f[i] = fmaf(u, u, f[i]);
         } else {
           const float up = exp2f((pw - 1.0f) * log2f(u));
@@ -158,16 +161,19 @@ __device__ __forceinline__ void entmax_newton_rows(const float* x, int stride, i
       for (int i = 0; i < RW; ++i) {
         f[i] += __shfl_xor_sync(0xffffffffu, f[i], o);
         a[i] += __shfl_xor_sync(0xffffffffu, a[i], o);
-        k[i] += __shfl_xor_sync(0xffffffffu, k[i], o);
-        umin[i] = fminf(umin[i], __shfl_xor_sync(0xffffffffu, umin[i], o));
-        if (kind == 2) fd[i] += __shfl_xor_sync(0xffffffffu, fd[i], o);
+        if constexpr (KIND == 2) fd[i] += __shfl_xor_sync(0xffffffffu, fd[i], o);
       }
+    }
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+      k[i] = (int)__reduce_add_sync(0xffffffffu, (unsigned)k[i]);
+      umin[i] = __uint_as_float(__reduce_min_sync(0xffffffffu, __float_as_uint(umin[i])));
     }
     bool all = true;
 #pragma unroll
     for (int i = 0; i < RW; ++i) {
       if (!done[i]) {
-        if (kind == 0) {
+        if constexpr (KIND == 0) {
           const float delta = (f[i] - 1.0f) / k[i];
           if (delta < umin[i]) {
             tau[i] += fmaxf(delta, 0.0f);
@@ -175,7 +181,7 @@ __device__ __forceinline__ void entmax_newton_rows(const float* x, int stride, i
           } else {
             tau[i] += delta;
           }
-        } else if (kind == 1) {
+        } else if constexpr (KIND == 1) {
           const float disc = a[i] * a[i] - k[i] * (f[i] - 1.0f);
           float delta = 3.0e38f;
           if (disc >= 0.f) delta = (f[i] - 1.0f) / (a[i] + sqrtf(disc));
@@ -205,9 +211,9 @@ __device__ __forceinline__ void entmax_newton_rows(const float* x, int stride, i
 // threshold, solved first in registers, is a lower bound on the row's (F
 // over the row >= F over any subset), so the passes over the row start there
 // instead of at max - 1 and usually find the exact support at once.
-template <int RW>
+template <int RW, int KIND>
 __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride, int n, const float* seed,
-                                                     float alpha, int kind, int lane, float* tau) {
+                                                     float alpha, int lane, float* tau) {
   static_assert(kSeed == 32, "one seed value per lane");
   const float pw = 1.0f / (alpha - 1.0f);
   float sv[RW], mx[RW];
@@ -224,10 +230,10 @@ __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride,
     tau[i] = mx[i] - 1.0f;
     done[i] = mx[i] == kNegInf;
   }
-  entmax_newton_rows<RW, 1>(sv, 0, 32, pw, kind, lane, tau, done);
+  entmax_newton_rows<RW, 1, KIND>(sv, 0, 32, pw, lane, tau, done);
 #pragma unroll
   for (int i = 0; i < RW; ++i) done[i] = mx[i] == kNegInf;
-  entmax_newton_rows<RW, 2>(x, stride, n, pw, kind, lane, tau, done);
+  entmax_newton_rows<RW, 2, KIND>(x, stride, n, pw, lane, tau, done);
 }
 
 // Thresholds, GQA mean and ascending per-position lists for the tile rows
@@ -236,16 +242,15 @@ __device__ __forceinline__ void warp_entmax_tau_rows(const float* x, int stride,
 // non-candidates -inf, readable up to the column count rounded up to 64) are
 // X[(r - row_base) * xstride + c]; its seed values are
 // seed[(r - row_base) * kSeed + l].  Marks in pmask[c] the tile positions
-// that selected block c.
-template <int G>
-__device__ __forceinline__ void solve_and_compact(const RouteParams& p, const float* X, int xstride, const float* seed,
-                                                  uint4* pmask, int row_base, int round_rows, int b, int g, int pos0,
-                                                  int n_blocks, int warp, int lane) {
+// that selected block c.  KIND is entmax_kind(p.alpha).
+template <int G, int KIND>
+__device__ __forceinline__ void solve_and_compact_k(const RouteParams& p, const float* X, int xstride,
+                                                    const float* seed, uint4* pmask, int row_base, int round_rows,
+                                                    int b, int g, int pos0, int n_blocks, int warp, int lane) {
   constexpr int RW = G > 4 ? G : 4;  // rows solved together by one warp
   constexpr int PPT = RW / G;        // positions per warp task
   const int64_t bg = (int64_t)b * p.Hkv + g;
   const float pw = 1.0f / (p.alpha - 1.0f);
-  const int kind = entmax_kind(p.alpha);
   const int n_tasks = round_rows / RW;
   for (int task = warp; task < n_tasks; task += kWorkWarps) {
     const int rr0 = task * RW;                 // first row within the round
@@ -258,8 +263,8 @@ __device__ __forceinline__ void solve_and_compact(const RouteParams& p, const fl
 #pragma unroll
     for (int r4 = 0; r4 < RW; r4 += 4) {
       if (ncol > 0) {
-        warp_entmax_tau_rows<4>(X + (rr0 + r4) * xstride, xstride, ncol, seed + (rr0 + r4) * kSeed, p.alpha, kind,
-                                lane, tau + r4);
+        warp_entmax_tau_rows<4, KIND>(X + (rr0 + r4) * xstride, xstride, ncol, seed + (rr0 + r4) * kSeed, p.alpha,
+                                      lane, tau + r4);
       } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) tau[r4 + i] = 0.f;  // no candidates (nothing was copied)
@@ -287,7 +292,7 @@ __device__ __forceinline__ void solve_and_compact(const RouteParams& p, const fl
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const float u = X[(rr0 + pp * G + h) * xstride + c] - tau[pp * G + h];
-            const float ph = u > 0.f ? pow_pw(u, pw, kind) : 0.f;
+            const float ph = u > 0.f ? pow_pw(u, pw, KIND) : 0.f;
             pbar += ph;
             if (p.p_dense) p.p_dense[(((int64_t)b * p.H + g * G + h) * p.S + qpos) * p.t_cap + c] = ph;
           }
@@ -313,6 +318,22 @@ __device__ __forceinline__ void solve_and_compact(const RouteParams& p, const fl
         }
       }
     }
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void solve_and_compact(const RouteParams& p, const float* X, int xstride, const float* seed,
+                                                  uint4* pmask, int row_base, int round_rows, int b, int g, int pos0,
+                                                  int n_blocks, int warp, int lane) {
+  switch (entmax_kind(p.alpha)) {
+    case 0:
+      solve_and_compact_k<G, 0>(p, X, xstride, seed, pmask, row_base, round_rows, b, g, pos0, n_blocks, warp, lane);
+      break;
+    case 1:
+      solve_and_compact_k<G, 1>(p, X, xstride, seed, pmask, row_base, round_rows, b, g, pos0, n_blocks, warp, lane);
+      break;
+    default:
+      solve_and_compact_k<G, 2>(p, X, xstride, seed, pmask, row_base, round_rows, b, g, pos0, n_blocks, warp, lane);
   }
 }
 
