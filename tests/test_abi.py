@@ -181,6 +181,40 @@ def test_paged_and_context_parallel_reject_bad_arguments():
     assert st == 2
 
 
+def test_context_parallel_split_kv_workspace_checks():
+    """dash_attn_cp_attend_ex: its workspace size, and the host checks of the shard and the workspace."""
+    lib = dash.load()
+    B, H, Hkv, d, blk, t_cap = 4, 8, 2, 128, 64, 64
+    n = lib.dash_attn_cp_attend_workspace_size(B, H, Hkv, d, blk, t_cap)
+    # shard ranges [4 ints], work items of 16 blocks (block 64) with G heads' partials each
+    items = B * Hkv * (-(-(t_cap + 1) // 16))
+    assert n >= B * Hkv * 16 + items * 8 + B * Hkv * 4 + items * (H // Hkv) * (d + 2) * 4
+    assert n % 256 == 0
+    assert lib.dash_attn_cp_attend_workspace_size(B, H, Hkv, d, 128, t_cap) > n  # 8-block items: more of them
+    assert lib.dash_attn_cp_attend_workspace_size(B, H, 3, d, blk, t_cap) == 0  # H not a multiple of Hkv
+    assert lib.dash_attn_cp_attend_workspace_size(0, H, Hkv, d, blk, t_cap) == 0
+    q = tensor(B, 1, H, d)
+    shard = tensor(B, 1024, Hkv, d)
+
+    def call(shard_t=shard, tok_lo=1024, ws=FAKE, ws_bytes=n):
+        st = lib.dash_attn_cp_attend_ex(ctypes.byref(q), ctypes.byref(shard_t), ctypes.byref(shard_t), tok_lo, FAKE,
+                                        4096, FAKE, FAKE, FAKE, t_cap, blk, None, FAKE, ws, ws_bytes, None)
+        return st, lib.dash_attn_last_error().decode()
+
+    st, msg = call(tok_lo=1000)
+    assert st == 1 and "multiples of the block" in msg
+    st, msg = call(shard_t=tensor(B, 1000, Hkv, d))
+    assert st == 1 and "multiples of the block" in msg
+    st, msg = call(ws=None)
+    assert st == 1 and "256-byte aligned" in msg
+    st, msg = call(ws=FAKE + 128)
+    assert st == 1 and "256-byte aligned" in msg
+    st, msg = call(ws_bytes=n - 1)
+    assert st == 3 and "workspace" in msg
+    st, msg = call(shard_t=tensor(B, 1024, Hkv, d, dtype=1))
+    assert st == 1 and "dtype" in msg
+
+
 def test_binding_refuses_host_tensors():
     import torch
 
