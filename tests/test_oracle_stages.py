@@ -358,3 +358,20 @@ def test_non_uniform_prior_lands_on_its_block(causal, sigma):
                 wrong, _ = _prior_mask_reference(q[pos], k, v, summ, pos, S, B, 1.5, causal, sigma, shift=1)
                 assert np.abs(wrong - ref).max() > 1e-3  # the reference tells the two placements apart
     assert checked >= 3
+
+
+def test_candidate_blocks_enumerated():
+    """Candidates of "Stage 1": causal rows score the complete blocks before
+    their own; non-causal rows every other block, the ragged last one included."""
+    from oracle.dash_oracle import candidate_blocks
+
+    assert candidate_blocks(0, 64, 1000, True) == (0, [])
+    assert candidate_blocks(63, 64, 1000, True) == (0, [])
+    assert candidate_blocks(64, 64, 1000, True) == (1, [0])
+    assert candidate_blocks(130, 64, 200, True) == (2, [0, 1])
+    # 200 tokens in blocks of 64: blocks 0, 1, 2 full, block 3 holds tokens 192..199
+    assert candidate_blocks(130, 64, 200, False) == (2, [0, 1, 3])
+    assert candidate_blocks(199, 64, 200, False) == (3, [0, 1, 2])
+    assert candidate_blocks(5, 64, 200, False) == (0, [1, 2, 3])
+    assert candidate_blocks(5, 64, 64, False) == (0, [])
+    assert candidate_blocks(300, 128, 1024, True) == (2, [0, 1])
